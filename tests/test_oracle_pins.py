@@ -1,0 +1,524 @@
+"""Pins for the fp64 oracle: closed forms, library routines, brute force and
+invariants -- never the oracle against itself.
+
+Each test names the plain fact it checks.  A plausible slip in the oracle (a
+dropped term, a wrong sign or index, a transposed operand, a wrong page or
+head mapping, a wrong rounding rule) fails at least one of them.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixed_length_paged_b200 import workloads as W
+from tests.helpers import bf16_values, bits16, dense_attention, dense_kv
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- bf16 codec
+
+def test_bf16_decode_matches_float32_view():
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 1 << 16, size=4096, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.bf16_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(ours[ok], ref[ok])
+
+
+def test_bf16_round_matches_torch_rne_on_float32_values():
+    # For values exactly representable in fp32, fp64->bf16 RNE equals torch's
+    # fp32->bf16 RNE cast (a library routine).
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(3000).astype(np.float32),
+                        (rng.standard_normal(500) * 1e-38).astype(np.float32),   # subnormal range
+                        (rng.standard_normal(500) * 1e30).astype(np.float32)])
+    ours = oracle.bf16_from_f64(x.astype(np.float64))
+    ref = bits16(torch.from_numpy(x).to(torch.bfloat16))
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_bf16_round_ties_to_even():
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even mantissa (1.0).
+    assert oracle.bf16_from_f64(1.0 + 2.0 ** -8) == 0x3F80
+    # 1 + 3*2^-8 is halfway between 1+2^-7 (odd) and 1+2^-6 (even) -> 1+2^-6
+    assert oracle.bf16_from_f64(1.0 + 3 * 2.0 ** -8) == 0x3F82
+    # just above the tie rounds up
+    assert oracle.bf16_from_f64(1.0 + 2.0 ** -8 + 2.0 ** -30) == 0x3F81
+
+
+# ---------------------------------------------------------------- e4m3 codec
+
+def _golden_e4m3():
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_table.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            kind, code, val = line.split()
+            rows.append((kind, int(code, 16), float(val)))
+    return rows
+
+
+def test_e4m3_golden_table():
+    for kind, code, val in _golden_e4m3():
+        if kind == "decode":
+            got = oracle.e4m3_decode([code])[0]
+            if math.isnan(val):
+                assert math.isnan(got), hex(code)
+            else:
+                assert got == val and math.copysign(1, got) == math.copysign(1, val), hex(code)
+        else:
+            assert oracle.e4m3_encode([val])[0] == code, (val, hex(code))
+
+
+def test_e4m3_decode_all_codes_closed_form():
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_decode(codes)
+    for c in range(256):
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        if e == 15 and m == 7:
+            assert math.isnan(got[c])
+            continue
+        mag = m * 2.0 ** -9 if e == 0 else (8 + m) * 2.0 ** (e - 10)
+        assert got[c] == (-mag if s else mag), hex(c)
+
+
+def test_e4m3_decode_matches_torch_float8():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_decode(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+
+
+def test_e4m3_encode_roundtrips_every_finite_code():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    np.testing.assert_array_equal(oracle.e4m3_encode(vals), codes)
+
+
+def test_e4m3_encode_midpoints_brute_force():
+    # Every midpoint between adjacent non-negative finite values rounds to the
+    # neighbour with an even code (even mantissa); just off the midpoint rounds
+    # to the nearer one.
+    pos = [c for c in range(0x7F)]
+    vals = oracle.e4m3_decode(np.array(pos, dtype=np.uint8))
+    for a, b in zip(pos[:-1], pos[1:]):
+        va, vb = vals[a], vals[b]
+        mid = (va + vb) / 2
+        even = a if a % 2 == 0 else b
+        assert oracle.e4m3_encode([mid])[0] == even, (hex(a), hex(b))
+        eps = (vb - va) * 1e-6
+        assert oracle.e4m3_encode([mid - eps])[0] == a
+        assert oracle.e4m3_encode([mid + eps])[0] == b
+        assert oracle.e4m3_encode([-(mid + eps)])[0] == (0x80 | b)
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    rng = np.random.default_rng(2)
+    x = np.concatenate([rng.standard_normal(4000) * 50, rng.standard_normal(1000) * 0.01])
+    x = np.clip(x, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_encode(x.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_quantizer_scale_and_error_bound():
+    shape = W.DecodeShape("q", 4, 2, 16, kv_dtype="fp8_e4m3")
+    batch = W.make_batch(shape, [70, 5], seed=3)
+    vals = batch.k_cache.numpy()
+    live = batch.live.numpy()
+    codes, scales = oracle.quantize_kv_e4m3(vals, live, dead_code=0x7F)
+    for p in range(vals.shape[0]):
+        for g in range(vals.shape[1]):
+            n = live[p]
+            if n == 0:
+                assert scales[p, g] == 1.0
+                assert np.all(codes[p, g] == 0x7F)
+                continue
+            blk = vals[p, g, :n].astype(np.float64)
+            amax = np.abs(blk).max()
+            assert scales[p, g] == np.float32(amax / 448.0)
+            dec = oracle.e4m3_decode(codes[p, g, :n]) * float(scales[p, g])
+            # RNE with 3 mantissa bits: relative error <= 2^-4 for normals,
+            # absolute error <= 2^-10 * scale in the subnormal range.
+            err = np.abs(dec - blk)
+            bound = np.maximum(np.abs(blk) * 2.0 ** -4, 2.0 ** -10 * float(scales[p, g]))
+            assert np.all(err <= bound * (1 + 1e-12))
+            # the amax element lands on +-448
+            i = np.unravel_index(np.abs(blk).argmax(), blk.shape)
+            assert abs(oracle.e4m3_decode([codes[p, g][i]])[0]) == 448.0
+            assert np.all(codes[p, g, n:] == 0x7F)
+
+
+# ---------------------------------------------------------------- RMSNorm / RoPE
+
+def test_rmsnorm_closed_form():
+    # x = (3, 4): mean square 12.5, y = x / sqrt(12.5) * gamma
+    y = oracle.rmsnorm([3.0, 4.0], [1.0, 2.0], 0.0)
+    np.testing.assert_allclose(y, [3 * math.sqrt(2) / 5, 2 * 4 * math.sqrt(2) / 5], rtol=1e-15)
+
+
+def test_rmsnorm_unit_rms_scale_invariance_and_eps():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal(128)
+    y = oracle.rmsnorm(x, np.ones(128), 0.0)
+    assert abs(math.sqrt(np.mean(y * y)) - 1.0) < 1e-14
+    np.testing.assert_allclose(oracle.rmsnorm(7.5 * x, np.ones(128), 0.0), y, rtol=1e-14)
+    ms = np.mean(x * x)
+    ye = oracle.rmsnorm(x, np.ones(128), 1e-6)
+    assert abs(math.sqrt(np.mean(ye * ye)) - math.sqrt(ms / (ms + 1e-6))) < 1e-14
+    g = rng.uniform(0.5, 1.5, 128)
+    np.testing.assert_allclose(oracle.rmsnorm(x, g, 0.0), y * g, rtol=1e-14)
+
+
+def test_rope_position_zero_is_identity():
+    x = np.random.default_rng(5).standard_normal(128)
+    np.testing.assert_array_equal(oracle.rope(x, 0, 10000.0), x)
+
+
+def test_rope_matches_complex_rotation():
+    # Rotate-half RoPE == multiplying z_i = x_i + i x_{i+D/2} by e^{i pos w_i},
+    # w_i = theta^(-2i/D), evaluated with numpy's complex exponential.
+    rng = np.random.default_rng(6)
+    D, theta = 128, 10000.0
+    x = rng.standard_normal(D)
+    for pos in [1, 7, 4095, 65536]:
+        i = np.arange(D // 2)
+        w = theta ** (-2.0 * i / D)
+        z = (x[:D // 2] + 1j * x[D // 2:]) * np.exp(1j * pos * w)
+        y = oracle.rope(x, pos, theta)
+        np.testing.assert_allclose(y[:D // 2], z.real, atol=1e-12)
+        np.testing.assert_allclose(y[D // 2:], z.imag, atol=1e-12)
+
+
+def test_rope_quarter_turn_and_invariants():
+    # D = 2: one pair with w_0 = 1; pos = pi/2 maps (a, b) to (-b, a).
+    y = oracle.rope([0.3, -1.7], math.pi / 2, 10000.0)
+    np.testing.assert_allclose(y, [1.7, 0.3], atol=1e-15)
+    rng = np.random.default_rng(7)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for m, n, t in [(5, 2, 11), (1000, 37, 4096), (65536, 3, 17)]:
+        yq = oracle.rope(q, m, 10000.0)
+        # every (i, i+D/2) pair keeps its norm
+        np.testing.assert_allclose(yq[:32] ** 2 + yq[32:] ** 2, q[:32] ** 2 + q[32:] ** 2,
+                                   rtol=1e-12)
+        # <R(m)q, R(n)k> depends only on m - n
+        a = np.dot(yq, oracle.rope(k, n, 10000.0))
+        b = np.dot(oracle.rope(q, m + t, 10000.0), oracle.rope(k, n + t, 10000.0))
+        assert abs(a - b) < 1e-10
+
+
+# ---------------------------------------------------------------- attention
+
+def _tiny(seed=0, lens=(37, 200), Hq=8, Hkv=2, D=64):
+    shape = W.DecodeShape("t", Hq, Hkv, D)
+    return W.make_batch(shape, list(lens), seed=seed)
+
+
+def _run(batch, **kw):
+    D = batch.shape.head_dim
+    return oracle.paged_decode(bits16(batch.q), bits16(batch.k_cache), bits16(batch.v_cache),
+                               batch.page_table.numpy(), batch.seq_lens.numpy(),
+                               batch.shape.num_kv_heads, 1.0 / math.sqrt(D), **kw)
+
+
+def test_attention_golden_equal_logits():
+    with open(os.path.join(GOLDEN, "attention_equal_logits.json")) as f:
+        g = json.load(f)
+
+    def arr(x):
+        return np.array(x, dtype=np.float64)
+
+    q = arr(g["q"])
+    kc = oracle.bf16_from_f64(arr(g["k_cache"]))
+    vc = oracle.bf16_from_f64(arr(g["v_cache"]))
+    out = oracle.paged_decode(q, kc, vc, np.array(g["page_table"], dtype=np.int32),
+                              np.array(g["seq_lens"], dtype=np.int32), g["num_kv_heads"],
+                              g["scale"], page_size=g["page_size"])
+    np.testing.assert_allclose(out, arr(g["expected"]), rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("seed,lens,Hq,Hkv,D", [
+    (0, (37, 200), 8, 2, 64),
+    (1, (1, 64, 65, 129), 8, 8, 32),
+    (2, (300, 7), 16, 2, 128),
+    (3, (128,), 4, 1, 16),
+])
+def test_attention_matches_dense_brute_force(seed, lens, Hq, Hkv, D):
+    batch = _tiny(seed, lens, Hq, Hkv, D)
+    out = _run(batch)
+    kv = bf16_values(bits16(batch.k_cache))
+    vv = bf16_values(bits16(batch.v_cache))
+    qv = bf16_values(bits16(batch.q))
+    pt = batch.page_table.numpy()
+    for b, L in enumerate(lens):
+        ref = dense_attention(qv[b], dense_kv(kv, pt, b, L), dense_kv(vv, pt, b, L),
+                              1.0 / math.sqrt(D))
+        np.testing.assert_allclose(out[b], ref, rtol=0, atol=1e-12)
+
+
+def test_attention_length_one_returns_v():
+    batch = _tiny(4, (1, 1), 8, 2, 64)
+    out = _run(batch)
+    vv = bf16_values(bits16(batch.v_cache))
+    pt = batch.page_table.numpy()
+    for b in range(2):
+        for h in range(8):
+            np.testing.assert_array_equal(out[b, h], vv[pt[b, 0], h // 4, 0])
+
+
+def test_attention_zero_query_is_mean_of_v():
+    batch = _tiny(5, (37, 200), 8, 2, 64)
+    batch.q.zero_()
+    out = _run(batch)
+    vv = bf16_values(bits16(batch.v_cache))
+    pt = batch.page_table.numpy()
+    for b, L in enumerate((37, 200)):
+        V = dense_kv(vv, pt, b, L)
+        for h in range(8):
+            np.testing.assert_allclose(out[b, h], V[:, h // 4, :].mean(axis=0), atol=1e-14)
+
+
+def test_attention_invariant_under_page_permutation():
+    batch = _tiny(6, (37, 200), 8, 2, 64)
+    out = _run(batch)
+    rng = np.random.default_rng(99)
+    P = batch.num_pages
+    perm = rng.permutation(P)               # new physical id of old page p
+    kc = np.empty_like(bits16(batch.k_cache))
+    vc = np.empty_like(kc)
+    kc[perm] = bits16(batch.k_cache)
+    vc[perm] = bits16(batch.v_cache)
+    pt = batch.page_table.numpy().copy()
+    pt[pt >= 0] = perm[pt[pt >= 0]]
+    out2 = oracle.paged_decode(bits16(batch.q), kc, vc, pt, batch.seq_lens.numpy(), 2, 1 / 8)
+    np.testing.assert_array_equal(out, out2)
+
+
+def test_split_and_lse_merge_equals_unsplit():
+    batch = _tiny(7, (37, 200), 8, 2, 64)
+    out = _run(batch)
+    q, kc, vc = bits16(batch.q), bits16(batch.k_cache), bits16(batch.v_cache)
+    pt = batch.page_table.numpy()
+    rng = np.random.default_rng(8)
+    for b, L in enumerate((37, 200)):
+        for h in (0, 5):
+            for nsplit in (1, 2, 3, 7):
+                cuts = np.sort(rng.choice(np.arange(1, L), size=nsplit - 1, replace=False)) \
+                    if nsplit > 1 else np.array([], dtype=int)
+                edges = [0, *cuts.tolist(), L]
+                parts = [oracle.partial(q, kc, vc, pt, 2, 1 / 8, b, h, a, e)
+                         for a, e in zip(edges[:-1], edges[1:])]
+                acc = np.stack([p[0] for p in parts])
+                m = np.array([p[1] for p in parts])
+                l = np.array([p[2] for p in parts])
+                np.testing.assert_allclose(oracle.lse_merge(acc, m, l), out[b, h], atol=1e-12)
+            # an empty partial contributes nothing
+            a0, m0, l0 = oracle.partial(q, kc, vc, pt, 2, 1 / 8, b, h, 0, 0)
+            assert m0 == -math.inf and l0 == 0.0
+            a1, m1, l1 = oracle.partial(q, kc, vc, pt, 2, 1 / 8, b, h, 0, L)
+            np.testing.assert_allclose(
+                oracle.lse_merge(np.stack([a0, a1]), [m0, m1], [l0, l1]), out[b, h], atol=1e-15)
+
+
+def test_needle_in_128k_tokens():
+    # A key planted as c * q / |q| at a random position of a 131072-token
+    # sequence takes essentially all the softmax mass: o ~= V[needle].
+    D, Hkv, Hq, L = 128, 1, 2, 131072
+    shape = W.DecodeShape("needle", Hq, Hkv, D)
+    batch = W.make_batch(shape, [L], seed=9, spare_pages=1)
+    q = bf16_values(bits16(batch.q))[0, 0]
+    j = int(np.random.default_rng(10).integers(0, L))
+    pt = batch.page_table.numpy()
+    page, slot = pt[0, j // 64], j % 64
+    batch.k_cache[page, 0, slot] = torch.from_numpy(40.0 * q / np.linalg.norm(q)).to(torch.bfloat16)
+    out = _run(batch, num_threads=0)
+    vv = bf16_values(bits16(batch.v_cache))
+    np.testing.assert_allclose(out[0, 0], vv[page, 0, slot], atol=1e-6)
+    # the other head of the group does not see the needle
+    assert np.abs(out[0, 1] - vv[page, 0, slot]).max() > 0.1
+
+
+def test_zero_length_sequence_gives_zero_output():
+    batch = _tiny(11, (0, 5), 8, 2, 64)
+    out = _run(batch)
+    assert np.all(out[0] == 0.0)
+    assert np.all(np.isfinite(out[1]))
+
+
+def test_rows_subset_matches_full():
+    batch = _tiny(12, (37, 200, 90), 8, 2, 64)
+    full = _run(batch)
+    sub = _run(batch, rows=np.array([2, 0], dtype=np.int32))
+    np.testing.assert_array_equal(sub[[0, 2]], full[[0, 2]])
+    assert np.all(sub[1] == 0)
+
+
+def test_fp8_attention_matches_dense_on_dequantised_values():
+    shape = W.DecodeShape("f", 8, 2, 64, kv_dtype="fp8_e4m3")
+    lens = (70, 130)
+    batch = W.make_batch(shape, list(lens), seed=13)
+    kcode, ks = oracle.quantize_kv_e4m3(batch.k_cache.numpy(), batch.live.numpy())
+    vcode, vs = oracle.quantize_kv_e4m3(batch.v_cache.numpy(), batch.live.numpy())
+    pt = batch.page_table.numpy()
+    out = oracle.paged_decode(bits16(batch.q), kcode, vcode, pt, batch.seq_lens.numpy(), 2,
+                              1 / 8, kv_fp8=True, k_scale=ks, v_scale=vs)
+    # dequantise with torch's float8 decoder (library) and the scales
+    kd = torch.from_numpy(kcode).view(torch.float8_e4m3fn).to(torch.float64).numpy() \
+        * ks[:, :, None, None]
+    vd = torch.from_numpy(vcode).view(torch.float8_e4m3fn).to(torch.float64).numpy() \
+        * vs[:, :, None, None]
+    qv = bf16_values(bits16(batch.q))
+    for b, L in enumerate(lens):
+        ref = dense_attention(qv[b], dense_kv(kd, pt, b, L), dense_kv(vd, pt, b, L), 1 / 8)
+        np.testing.assert_allclose(out[b], ref, atol=1e-12)
+
+
+# ---------------------------------------------------------------- prologue
+
+def test_prologue_slot_write_and_values():
+    shape = W.DecodeShape("p", 8, 2, 64, prologue=True)
+    lens = [63, 64, 130, 0]
+    batch = W.make_batch(shape, lens, seed=14)
+    kc0, vc0 = bits16(batch.k_cache), bits16(batch.v_cache)
+    kc, vc = kc0.copy(), vc0.copy()
+    pt = batch.page_table.numpy()
+    eps, theta = 1e-6, 10000.0
+    q_out = oracle.prologue(bits16(batch.q_raw), bits16(batch.k_raw), bits16(batch.v_raw),
+                            batch.q_gamma.numpy(), batch.k_gamma.numpy(), eps, theta,
+                            batch.positions.numpy(), pt, kc, vc)
+    touched = np.zeros(kc.shape[:3], dtype=bool)
+    qg = batch.q_gamma.numpy().astype(np.float64)
+    kg = batch.k_gamma.numpy().astype(np.float64)
+    for b, pos in enumerate(lens):
+        page, slot = pt[b, pos // 64], pos % 64
+        for g in range(2):
+            touched[page, g, slot] = True
+            kraw = bf16_values(bits16(batch.k_raw))[b, g]
+            # RMSNorm (closed form, numpy) then rotation (numpy complex form)
+            x = kraw / math.sqrt(np.mean(kraw * kraw) + eps) * kg
+            w = theta ** (-2.0 * np.arange(32) / 64)
+            z = (x[:32] + 1j * x[32:]) * np.exp(1j * pos * w)
+            ref = np.concatenate([z.real, z.imag])
+            got = bf16_values(kc[page, g, slot])
+            # fp64 RNE of nearly the same value: equal, or 1 ulp apart at a tie
+            ulp = np.abs(got) * 2.0 ** -7
+            assert np.all(np.abs(got - ref) <= ulp * 0.5000001 + 1e-300)
+            np.testing.assert_array_equal(vc[page, g, slot], bits16(batch.v_raw)[b, g])
+        for h in range(8):
+            qraw = bf16_values(bits16(batch.q_raw))[b, h]
+            x = qraw / math.sqrt(np.mean(qraw * qraw) + eps) * qg
+            w = theta ** (-2.0 * np.arange(32) / 64)
+            z = (x[:32] + 1j * x[32:]) * np.exp(1j * pos * w)
+            np.testing.assert_allclose(q_out[b, h], np.concatenate([z.real, z.imag]), atol=1e-12)
+    # nothing else in either cache changed (NaN-aware byte comparison)
+    np.testing.assert_array_equal(kc[~touched], kc0[~touched])
+    np.testing.assert_array_equal(vc[~touched], vc0[~touched])
+
+
+# ---------------------------------------------------------------- planner
+
+def _units(lens, Hkv):
+    """Global unit list (b, g, t) in seq-major, kv-head, tile order."""
+    out = []
+    for b, L in enumerate(lens):
+        n = (max(0, L) + 63) // 64
+        for g in range(Hkv):
+            for t in range(n):
+                out.append((b, g, t))
+    return out
+
+
+def _check_plan_invariants(p, lens, Hkv, kind):
+    units = _units(lens, Hkv)
+    U = len(units)
+    assert p["n_units"] == U
+    cta = p["cta"]
+    # ordered, contiguous, disjoint, covering [0, U) exactly once
+    cover = np.zeros(U, dtype=int)
+    prev_end = 0
+    for c in range(p["grid"]):
+        a, e = int(cta[c, 0]), int(cta[c, 1])
+        assert 0 <= a <= e <= U
+        if a < e:
+            assert a == prev_end
+            prev_end = e
+        cover[a:e] += 1
+    assert prev_end == U and np.all(cover == 1)
+    # split counts and first-split indices, recounted with Python sets
+    holders = {}
+    for c in range(p["grid"]):
+        a, e = int(cta[c, 0]), int(cta[c, 1])
+        segs = []
+        for u in range(a, e):
+            s = units[u][0] * Hkv + units[u][1]
+            if not segs or segs[-1] != s:
+                segs.append(s)
+        for i, s in enumerate(segs):
+            if i == 0:
+                assert cta[c, 2] == len(holders.get(s, []))
+            holders.setdefault(s, []).append(c)
+        if not segs:
+            assert cta[c, 2] == 0
+    S = len(lens) * Hkv
+    base = 0
+    for s in range(S):
+        n = len(holders.get(s, []))
+        assert p["split_count"][s] == n
+        assert p["partial_base"][s] == base
+        if n > 1:
+            base += n
+    if kind == 0:
+        sizes = [int(cta[c, 1] - cta[c, 0]) for c in range(p["grid"])]
+        active = [s for s in sizes if s > 0]
+        assert len(active) == min(p["grid"], U)
+        if active:
+            assert max(active) - min(active) <= 1
+
+
+@pytest.mark.parametrize("lens,Hkv,P", [
+    ([131072] + [4096] * 31, 8, 148),
+    ([512] * 64, 8, 148),
+    ([37, 200], 2, 148),
+    ([37, 200], 2, 3),
+    ([0, 5, 0, 64, 65], 4, 7),
+    ([1], 1, 148),
+    ([0, 0], 2, 5),
+])
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_planner_invariants(lens, Hkv, P, kind):
+    p = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P,
+                    max_seq_len=max(lens), capacity_tokens=max(64, max(lens)))
+    _check_plan_invariants(p, lens, Hkv, kind)
+
+
+def test_planner_static_shapes():
+    lens = [131072] + [4096] * 31
+    pA = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=1, num_ctas=148, max_seq_len=131072,
+                     capacity_tokens=131072)
+    assert pA["grid"] == 32 * 8  # ceil(148 / 256) = 1 split per (seq, kv head)
+    pB = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=2, num_ctas=148, max_seq_len=131072,
+                     capacity_tokens=131072)
+    # chunk = ceil(2048 / ceil(148 / 8)) = 108 tiles; 19 chunks per segment
+    assert pB["grid"] == 32 * 8 * 19
+    sizes = pB["cta"][:, 1] - pB["cta"][:, 0]
+    assert sizes.max() == 108 and (sizes == 0).sum() == 31 * 8 * 18
+
+
+def test_planner_clamps_lengths_to_capacity():
+    p = oracle.plan(np.array([-5, 1000, 64], dtype=np.int32), 2, kind=0, num_ctas=4,
+                    capacity_tokens=128)
+    np.testing.assert_array_equal(p["lens"], [0, 128, 64])
+    np.testing.assert_array_equal(p["tile_start"], [0, 0, 2, 3])
