@@ -1,0 +1,429 @@
+"""Decode-step benchmark: KV-cache GB/s and us per step on the skewed batch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = hpa_decode_plan + hpa_decode_run (the whole decode path for a batch
+without a prologue) over the skewed workload: 1 x 131072 + 31 x 4096 KV
+tokens, 64 query heads, 8 KV heads, head_dim 128, bf16 cache, 64-token pages
+shuffled over HBM (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section, the
+1 x 128K + 31 x 4K case).  Inputs are synthetic (seeded N(0,1)) and resident
+in HBM; 1.06 GB of live KV per step is far above the 126 MB L2, so no flush
+is needed between steps.
+
+Printed (rank 0, one JSON line): value = live KV bytes per step / step time
+(whole job over N GPUs: each rank runs its own batch, weak scaling), the run
+kernel's roofline against the measured HBM copy bandwidth, an end-to-end
+figure through the public API with host buffers, the fp64 oracle timed on a
+bounded sample on the host cores, the static split-KV plans fed to the same
+kernel, and SM clocks sampled during the timed region.
+
+--impl reference times the oracle (the plain fp64 CPU implementation) on the
+host cores on a bounded sample of the same workload and prints the same line
+with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV-cache GB/s (% of HBM peak), µs/decode step, skewed 1x128K+31x4K"
+WORKLOAD = "skewed"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_run_skewed_ncu.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "mixed_length_paged_b200", "csrc", f)
+                  for f in ("decode.cu", "hpa_common.cuh")]
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the static-plan comparison and the e2e leg")
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic():
+    """DRAM bytes per launch of the run kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    kv = {}
+    for line in text.splitlines():
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            kv[k.strip()] = v.strip().strip("`")
+    if kv.get("kernel_source_sha256_16") != _kernel_hash():
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch_full_workload"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _smi_index(local_rank: int) -> str:
+    """nvidia-smi id of this rank's GPU (honours CUDA_VISIBLE_DEVICES)."""
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    return vis[local_rank] if local_rank < len(vis) else str(local_rank)
+
+
+def _cpu_baseline_sample(batch_host, rows):
+    """Time the oracle (as it stands) on sequences `rows` of the workload."""
+    import numpy as np
+
+    import oracle
+    D = batch_host["D"]
+    t0 = time.perf_counter()
+    oracle.paged_decode(batch_host["q"], batch_host["k"], batch_host["v"], batch_host["pt"],
+                        batch_host["sl"], batch_host["Hkv"], 1.0 / math.sqrt(D),
+                        rows=np.array(rows, dtype=np.int32))
+    dt = time.perf_counter() - t0
+    toks = int(sum(int(batch_host["sl"][b]) for b in rows))
+    nbytes = toks * 2 * batch_host["Hkv"] * D * 2
+    return nbytes / dt / 1e9, dt, toks
+
+
+def _host_sample(batch, rows):
+    """Host (numpy) copy of the sampled sequences only, pages renumbered."""
+    import numpy as np
+    import torch
+    pt = batch.page_table.cpu().numpy()
+    sl = batch.seq_lens.cpu().numpy()
+    used = []
+    new_pt = np.full((len(rows), pt.shape[1]), -1, dtype=np.int32)
+    for i, b in enumerate(rows):
+        n = (int(sl[b]) + 63) // 64
+        new_pt[i, :n] = np.arange(len(used), len(used) + n)
+        used.extend(pt[b, :n].tolist())
+    idx = torch.tensor(used, dtype=torch.long, device=batch.k_cache.device)
+
+    def bits(t):
+        return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    return {"q": bits(batch.q[rows]), "k": bits(batch.k_cache.index_select(0, idx)),
+            "v": bits(batch.v_cache.index_select(0, idx)), "pt": new_pt,
+            "sl": sl[rows].astype(np.int32), "Hkv": batch.shape.num_kv_heads,
+            "D": batch.shape.head_dim}
+
+
+# sample for the CPU legs: the 31 short sequences (126,976 tokens x 8 kv heads)
+CPU_SAMPLE_ROWS = list(range(1, 32))
+CPU_SAMPLE_DESC = ("oracle (fp64, OpenMP over (sequence, head)) on the 31 x 4096-token "
+                   "sequences of the skewed batch (126,976 KV tokens, 12% of a step's KV)")
+
+
+def run_reference(args, rank: int):
+    """--impl reference: the oracle on the host cores, bounded sample per step."""
+    if rank != 0:
+        return
+    import torch
+
+    import oracle
+    from mixed_length_paged_b200 import workloads as W
+    batch = W.build(args.workload, device="cpu")
+    host = _host_sample(batch, CPU_SAMPLE_ROWS)
+    cores = oracle.num_threads()
+    for _ in range(max(0, min(args.warmup, 1))):
+        _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))
+    times, gbs = [], []
+    for _ in range(args.steps):
+        g, dt, toks = _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))
+        times.append(dt)
+        gbs.append(g)
+    value = statistics.median(gbs)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "skewed 1x131072+31x4096 sample", "sample": CPU_SAMPLE_DESC},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": CPU_SAMPLE_DESC},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del torch
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import mixed_length_paged_b200 as hpa
+    from mixed_length_paged_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hpa.lib()
+    batch = W.build(args.workload, device=dev, seed=0)
+    shape = batch.shape
+    B, Hq, Hkv, D = batch.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim
+    lens = batch.seq_lens.cpu().numpy()
+    kv_bytes = W.live_kv_bytes(lens, Hkv, D, 2)
+    tiles = int(((lens + 63) // 64).sum())
+    # algorithmic bytes of one run launch: live KV + q + out + page-table entries read
+    run_bytes = kv_bytes + 2 * B * Hq * D * 2 + tiles * 4
+    scale = 1.0 / math.sqrt(D)
+    num_ctas = hpa.default_num_ctas(local_rank)
+    stream = torch.cuda.current_stream()
+    dec = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, num_ctas=num_ctas, device=dev)
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    seq_lens = batch.seq_lens
+
+    def step():
+        dec.plan(seq_lens)
+        dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * K)]
+    sampler = ClockSampler(_smi_index(local_rank))
+    sampler.start()
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(K):
+        ev[3 * i].record(stream)
+        dec.plan(seq_lens)
+        ev[3 * i + 1].record(stream)
+        dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale)
+        ev[3 * i + 2].record(stream)
+    end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(end)
+    run_ms = [ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(K)]
+    plan_ms = [ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(K)]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    status = dec.status()
+
+    # static split-KV comparators: the same run kernel fed the static plans
+    extras = {}
+    if not args.no_extras:
+        for name, kind in (("static_nsplit", hpa.PLAN_STATIC_NSPLIT),
+                           ("static_chunk", hpa.PLAN_STATIC_CHUNK)):
+            sd = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, kind=kind, num_ctas=num_ctas,
+                                  max_seq_len=int(lens.max()), device=dev)
+            for _ in range(3):
+                sd(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale)
+            torch.cuda.synchronize()
+            n = max(10, min(200, K))
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                sd(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / n
+            extras[name] = {"us_per_step": 1e3 * ms, "GB_s": kv_bytes / (ms * 1e-3) / 1e9,
+                            "grid": sd.grid}
+        best_static = min(extras[k]["us_per_step"] for k in extras)
+        extras["dynamic_speedup_vs_best_static"] = best_static / (1e3 * ms_per_step)
+
+    # end to end through the public API: pinned host inputs -> device, step,
+    # result -> pinned host, all inside the timed region
+    e2e = None
+    if not args.no_extras:
+        q_h = batch.q.cpu().pin_memory()
+        sl_h = batch.seq_lens.cpu().pin_memory()
+        pt_h = batch.page_table.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        q_d, sl_d, pt_d = torch.empty_like(batch.q), torch.empty_like(seq_lens), \
+            torch.empty_like(batch.page_table)
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            sl_d.copy_(sl_h, non_blocking=True)
+            pt_d.copy_(pt_h, non_blocking=True)
+            dec.plan(sl_d)
+            dec.run(q_d, batch.k_cache, batch.v_cache, pt_d, out, scale)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        n = max(10, min(500, K))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        e_ms = a.elapsed_time(b) / n
+        et = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e_ms = float(et.item())
+        h2d = q_h.numel() * 2 + sl_h.numel() * 4 + pt_h.numel() * 4
+        e2e = {"value": world * kv_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "us_per_step": 1e3 * e_ms, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(out_h.numel() * 2)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        host = _host_sample(batch, CPU_SAMPLE_ROWS)
+        _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))  # warm-up
+        g, dt, toks = _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))
+        cpu = {"value": g, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": CPU_SAMPLE_DESC, "seconds": dt}
+
+    if rank != 0:
+        return
+    peak, peak_kind = _peaks()
+    run_avg_ms = statistics.mean(run_ms)
+    achieved = run_bytes / (run_avg_ms * 1e-3) / 1e9
+    traffic = _profiled_traffic()
+    value = world * kv_bytes / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "us_per_step": 1e3 * ms_per_step,
+        "pct_of_hbm_peak": 100.0 * (kv_bytes / (ms_per_step * 1e-3) / 1e9) / peak,
+        "config": {
+            "workload": "skewed decode: 1 x 131072 + 31 x 4096 KV tokens, 64 q heads, 8 kv heads, "
+                        "head_dim 128, bf16 KV, 64-token pages shuffled; dynamic plan",
+            "batch": B, "kv_bytes_per_step_per_gpu": kv_bytes, "num_ctas": num_ctas,
+            "l2": "no flush: 1.06 GB of KV per step is larger than the 126 MB L2",
+            "parallelism": f"data-parallel replicas x{world} (independent batches, no collective)",
+        },
+        "breakdown_us": {"plan": 1e3 * statistics.mean(plan_ms), "run": 1e3 * run_avg_ms},
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel (hpa_decode_run)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "traffic": traffic, "algorithmic_bytes_per_launch": run_bytes},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+        "static_splitkv": extras or None,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,233 @@
+/*
+ * hpa.h -- paged mixed-length decode attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libhpa.so.  One decode step of one attention layer is
+ *
+ *     hpa_kv_prologue   (optional: RMSNorm + RoPE of the new token's q/k and
+ *                        the K/V write into its cache slot)
+ *     hpa_decode_plan   (per-step tile plan from the device-side lengths)
+ *     hpa_decode_run    (persistent paged GQA decode + log-sum-exp merge)
+ *
+ * all asynchronous on one CUDA stream, with no host synchronisation in
+ * between, so a step can be captured in a CUDA graph.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device (or managed) pointers owned by
+ *     the caller; the library never allocates, frees or retains them past the
+ *     call.  Host pointers are read or written before the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued on it; the call returns without waiting.
+ *   - Arguments are validated on the host before anything is enqueued; a bad
+ *     argument returns an error and enqueues nothing.  Values that only the
+ *     device sees (lengths, page ids, positions) are checked by the kernels,
+ *     which never trap: they skip the offending access and set a bit in a
+ *     device status word (HPA_DEVICE_*), read back with hpa_read_status.
+ *   - Shapes: head_dim D in {64, 128}; page (tile) size 64 tokens; GQA group
+ *     G = num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
+ *
+ * Tensor layouts (row-major, innermost last):
+ *   q, q_raw, out        [batch][num_q_heads][D]
+ *   k_raw, v_raw         [batch][num_kv_heads][D]
+ *   k_cache, v_cache     [num_pages][num_kv_heads][64][D]   one (page, kv head)
+ *                        tile is one contiguous 64 x D block
+ *   k_scale, v_scale     [num_pages][num_kv_heads] fp32      (FP8 caches only)
+ *   page_table           [batch][pt_stride] int32: physical page of tile t of
+ *                        sequence b; entries past a sequence's last tile are
+ *                        never read
+ *   seq_lens             [batch] int32: tokens attended this step (after the
+ *                        prologue appended the new one)
+ *   positions            [batch] int32: 0-based index of the new token (the
+ *                        length before the append)
+ *   Token j of sequence b lives in row j % 64 of page page_table[b][j / 64].
+ *
+ * Sources.  The method is the HPC-Ops attention backend as reported on the
+ * web pages this library restates: xiaodao.ai "HPC-Ops TPOT -48.8%"
+ * (Attention section: live KV cut into 64-token tiles, the global task list
+ * spread as evenly as possible over persistent CTAs, versus static split-KV
+ * with a fixed split count or a fixed split size), bitbyai.com "vLLM x
+ * HPC-Ops" (Attention Backend: per-step load-balanced scheduler; RoPE,
+ * query-key normalisation and KV-write fused into a prologue), openai-hub.com
+ * news/688 (the illustrative paged attention call) and aipuzi.cn "HPC-Ops"
+ * (section 2.3: native BF16/FP8).
+ */
+#ifndef HPA_H
+#define HPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HPA_API __attribute__((visibility("default")))
+#else
+#define HPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HPA_OK = 0,
+  HPA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shapes */
+  HPA_ERR_UNSUPPORTED = 2,  /* a shape outside the supported set (see above) */
+  HPA_ERR_WORKSPACE = 3,    /* workspace too small or misaligned */
+  HPA_ERR_CUDA = 4          /* a CUDA runtime/driver call or launch failed;
+                               hpa_last_cuda_error() names it */
+} hpa_status;
+
+typedef enum { HPA_KV_BF16 = 0, HPA_KV_FP8_E4M3 = 1 } hpa_kv_dtype;
+typedef enum { HPA_OUT_BF16 = 0, HPA_OUT_F32 = 1 } hpa_out_dtype;
+
+/* Plan kinds.  DYNAMIC is the method; the two STATIC kinds are the static
+ * split-KV schedules it is measured against, fed to the same run kernel
+ * (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section). */
+typedef enum {
+  HPA_PLAN_DYNAMIC = 0,        /* param unused */
+  HPA_PLAN_STATIC_NSPLIT = 1,  /* param = splits per (seq, kv head); 0 = ceil(num_ctas / (B Hkv)) */
+  HPA_PLAN_STATIC_CHUNK = 2    /* param = tiles per split; 0 = ceil(T_max / ceil(num_ctas / Hkv)) */
+} hpa_plan_kind;
+
+/* Bits of the device status word (hpa_read_status). */
+#define HPA_DEVICE_LEN_CLAMPED 0x1  /* a seq_len < 0 or > pt_stride * 64 was clamped */
+#define HPA_DEVICE_BAD_PAGE 0x2     /* a page id outside [0, num_pages) was skipped  */
+#define HPA_DEVICE_BAD_PLAN 0x4     /* run found no plan, or one for other shapes    */
+#define HPA_DEVICE_BAD_POSITION 0x8 /* prologue: position outside the page table     */
+#define HPA_DEVICE_TIMEOUT 0x10     /* a pipeline wait gave up after 2 s (results void) */
+
+/* Human-readable name of a status code (static string, never NULL). */
+HPA_API const char* hpa_status_string(hpa_status status);
+
+/* Text of the last CUDA error seen by a call on this host thread ("" if none). */
+HPA_API const char* hpa_last_cuda_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+HPA_API int hpa_version(void);
+
+/* Number of persistent CTAs for `device`: one per SM (148 on B200).
+ * Returns -1 if the device cannot be queried. */
+HPA_API int hpa_default_num_ctas(int device);
+
+/* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC,
+ * B * Hkv * S for STATIC_NSPLIT, B * Hkv * ceil(T_max / C) for STATIC_CHUNK
+ * (T_max = ceil(max_seq_len / 64), S and C the resolved params).  Host only;
+ * returns -1 on invalid arguments. */
+HPA_API int hpa_plan_grid(hpa_plan_kind kind, int batch, int num_kv_heads, int num_ctas, int param,
+                  int max_seq_len);
+
+/* Bytes of device workspace that a plan of `grid` CTAs and the matching run
+ * need.  Host only; returns 0 on invalid arguments. */
+HPA_API size_t hpa_decode_workspace_size(int batch, int num_kv_heads, int num_q_heads, int head_dim,
+                                 int grid);
+
+/* Byte offsets of the workspace regions, for inspection by tests and tools:
+ * offsets[0..8] = header, lens, tile_start, cta_desc (int32 x4 per CTA:
+ * u_begin, u_end, first_split, 0), split_count, partial_base, arrive,
+ * partial (m, l), partial acc; offsets[9] = total size.  Returns HPA_OK or
+ * HPA_ERR_INVALID_ARG. */
+HPA_API hpa_status hpa_workspace_layout(int batch, int num_kv_heads, int num_q_heads, int head_dim,
+                                int grid, size_t offsets[10]);
+
+/*
+ * hpa_decode_plan -- per-step tile plan (xiaodao.ai "HPC-Ops TPOT -48.8%",
+ * Attention section; bitbyai.com "vLLM x HPC-Ops", Attention Backend).
+ *
+ * Cuts every sequence's live KV into 64-token tiles.  A unit is one
+ * (sequence b, kv head g, tile t); the global list orders units by b, g, t.
+ * DYNAMIC gives CTA c the units [floor(c U / P'), floor((c+1) U / P')) with
+ * P' = min(num_ctas, U): contiguous, equal to within one unit, so a short
+ * sequence lands whole in one CTA and a long one is spread over many.  The
+ * STATIC kinds give one CTA per (segment, split) instead.
+ *
+ *   seq_lens     device [batch] int32; values are clamped to [0, pt_stride*64]
+ *                (HPA_DEVICE_LEN_CLAMPED).  A sequence of length 0 gets a zero
+ *                output row from hpa_decode_run.
+ *   num_ctas     persistent CTA count (hpa_default_num_ctas), >= 1.
+ *   max_seq_len  host upper bound on every seq_len; sizes the STATIC_CHUNK
+ *                grid (ignored otherwise, may be 0).
+ *   workspace    device, >= hpa_decode_workspace_size(..., grid) bytes,
+ *                256-byte aligned.  The plan overwrites it entirely.
+ *   grid_out     host; receives the grid hpa_decode_run must be given.
+ *
+ * Recompute the plan whenever seq_lens change (every decode step).  A run
+ * must use the workspace of the plan made for its step; two steps in flight
+ * at once need two workspaces.
+ */
+HPA_API hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int num_kv_heads,
+                           int num_q_heads, int head_dim, int pt_stride, hpa_plan_kind kind,
+                           int num_ctas, int param, int max_seq_len, void* workspace,
+                           size_t ws_bytes, int* grid_out, void* stream);
+
+/*
+ * hpa_decode_run -- persistent paged GQA decode attention with split-KV
+ * log-sum-exp merge (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section:
+ * persistent CTAs consume 64-token tiles; a sequence split over CTAs is
+ * merged from per-split partials).
+ *
+ * For sequence b and query head h (kv head g = h / G):
+ *     out[b][h] = sum_j softmax_j(softmax_scale * <q[b][h], K_b[j, g]>) V_b[j, g]
+ * over j < seq_lens[b] as captured by the plan.  Computed in fp32 with
+ * bf16 (or f16 for FP8 caches) tensor-core products.
+ *
+ *   q            device bf16 [batch][num_q_heads][D]
+ *   k_cache, v_cache  device [num_pages][num_kv_heads][64][D]; bf16, or e4m3
+ *                codes when kv_dtype = HPA_KV_FP8_E4M3.  16-byte aligned.
+ *   k_scale, v_scale  device fp32 [num_pages][num_kv_heads] dequantisation
+ *                scales (value = code * scale); NULL for bf16 caches.
+ *   page_table   device int32 [batch][pt_stride]; ids outside
+ *                [0, num_pages) are skipped (HPA_DEVICE_BAD_PAGE).
+ *   out          device [batch][num_q_heads][D], bf16 or fp32 (out_dtype).
+ *   grid         the grid_out of the plan that filled `workspace`.
+ *   workspace    the plan's workspace; its partial and arrival regions are
+ *                rewritten by the run.
+ * Partial slots are merged by the last CTA to finish a sequence's kv head,
+ * in split order, so results do not depend on CTA timing.
+ */
+HPA_API hpa_status hpa_decode_run(const void* q, const void* k_cache, const void* v_cache,
+                          const float* k_scale, const float* v_scale, hpa_kv_dtype kv_dtype,
+                          const int32_t* page_table, int pt_stride, int num_pages, void* out,
+                          hpa_out_dtype out_dtype, int batch, int num_q_heads,
+                          int num_kv_heads, int head_dim, float softmax_scale, int grid,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hpa_kv_prologue -- fused RMSNorm + RoPE + KV write for the new token of
+ * each sequence (bitbyai.com "vLLM x HPC-Ops", Attention Backend: RoPE,
+ * query-key normalisation and KV-write fused into one prologue).
+ *
+ * For sequence b at position p = positions[b]:
+ *   q_out[b][h]  = RoPE(RMSNorm(q_raw[b][h]; q_gamma), p)       for every h
+ *   K slot (b,g) = RoPE(RMSNorm(k_raw[b][g]; k_gamma), p)       rounded to bf16
+ *   V slot (b,g) = v_raw[b][g]                                  bit copy
+ * with RMSNorm(x; w)_i = x_i / sqrt(mean(x^2) + eps) * w_i over one head's D
+ * elements and rotate-half RoPE over the full head: for i < D/2,
+ * phi = p * theta^(-2i/D), (x_i, x_{i+D/2}) -> (x_i cos phi - x_{i+D/2} sin phi,
+ * x_{i+D/2} cos phi + x_i sin phi).  The slot is row p % 64 of page
+ * page_table[b][p / 64], kv head g.  The step then attends p + 1 tokens.
+ *
+ *   q_raw, k_raw, v_raw  device bf16, layouts above.
+ *   q_gamma, k_gamma     device fp32 [D], shared by all heads.
+ *   positions            device int32 [batch]; a position whose page-table
+ *                        entry is missing or out of range skips the K/V write
+ *                        and sets HPA_DEVICE_BAD_POSITION in *status.
+ *   k_cache, v_cache     device bf16 caches, written in place (one row per
+ *                        (b, g); nothing else is touched).
+ *   q_out                device bf16 [batch][num_q_heads][D].
+ *   status               device int32 word ORed with HPA_DEVICE_* bits, or NULL.
+ */
+HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
+                           const float* q_gamma, const float* k_gamma, float eps,
+                           float rope_theta, const int32_t* positions,
+                           const int32_t* page_table, int pt_stride, void* k_cache,
+                           void* v_cache, void* q_out, int batch, int num_q_heads,
+                           int num_kv_heads, int head_dim, int num_pages, int32_t* status,
+                           void* stream);
+
+/* Copies the device status word of a plan's workspace to *status_out (host)
+ * after the work queued on `stream` so far; synchronises the stream. */
+HPA_API hpa_status hpa_read_status(const void* workspace, int32_t* status_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HPA_H */

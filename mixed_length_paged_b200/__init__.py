@@ -1,0 +1,278 @@
+"""Python binding of libhpa.so: paged mixed-length decode attention on B200.
+
+Argument marshalling only -- every step of the decode path (prologue, plan,
+run, split merge) executes in the library's CUDA kernels.  PyTorch supplies
+device memory and streams.  The library must have been built
+(``python -m mixed_length_paged_b200.build``); importing the binding without
+it raises ``HpaLibraryMissing`` -- there is no fallback implementation.
+
+The functions mirror the C ABI in ``include/hpa.h``:
+
+    decode_workspace_size, plan_grid, default_num_ctas, workspace_layout,
+    decode_plan, decode_run, kv_prologue, read_status
+
+and ``PagedDecoder`` bundles a workspace with plan + run for callers who do
+not want to manage it.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+__all__ = [
+    "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
+    "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
+    "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
+    "default_num_ctas", "workspace_layout", "decode_plan", "decode_run", "kv_prologue",
+    "read_status", "PagedDecoder", "version",
+]
+
+PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2
+KV_BF16, KV_FP8_E4M3 = 0, 1
+OUT_BF16, OUT_F32 = 0, 1
+DEVICE_LEN_CLAMPED, DEVICE_BAD_PAGE, DEVICE_BAD_PLAN = 0x1, 0x2, 0x4
+DEVICE_BAD_POSITION, DEVICE_TIMEOUT = 0x8, 0x10
+PAGE_SIZE = 64
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libhpa.so")
+
+
+class HpaError(RuntimeError):
+    pass
+
+
+class HpaLibraryMissing(ImportError):
+    pass
+
+
+_STATUS = {0: "HPA_OK", 1: "HPA_ERR_INVALID_ARG", 2: "HPA_ERR_UNSUPPORTED",
+           3: "HPA_ERR_WORKSPACE", 4: "HPA_ERR_CUDA"}
+_lib = None
+
+_V, _I, _F, _Z = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+
+
+def lib():
+    """The loaded libhpa.so (loaded on first use; raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise HpaLibraryMissing(
+                f"{library_path} not found; build it with `python -m mixed_length_paged_b200.build`")
+        L = C.CDLL(library_path)
+        L.hpa_status_string.restype = C.c_char_p
+        L.hpa_status_string.argtypes = [_I]
+        L.hpa_last_cuda_error.restype = C.c_char_p
+        L.hpa_last_cuda_error.argtypes = []
+        L.hpa_version.restype = _I
+        L.hpa_version.argtypes = []
+        L.hpa_default_num_ctas.restype = _I
+        L.hpa_default_num_ctas.argtypes = [_I]
+        L.hpa_plan_grid.restype = _I
+        L.hpa_plan_grid.argtypes = [_I, _I, _I, _I, _I, _I]
+        L.hpa_decode_workspace_size.restype = _Z
+        L.hpa_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+        L.hpa_workspace_layout.restype = _I
+        L.hpa_workspace_layout.argtypes = [_I, _I, _I, _I, _I, C.POINTER(_Z)]
+        L.hpa_decode_plan.restype = _I
+        L.hpa_decode_plan.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V, _Z,
+                                      C.POINTER(_I), _V]
+        L.hpa_decode_run.restype = _I
+        L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
+                                     _F, _I, _V, _Z, _V]
+        L.hpa_kv_prologue.restype = _I
+        L.hpa_kv_prologue.argtypes = [_V, _V, _V, _V, _V, _F, _F, _V, _V, _I, _V, _V, _V, _I, _I,
+                                      _I, _I, _I, _V, _V]
+        L.hpa_read_status.restype = _I
+        L.hpa_read_status.argtypes = [_V, C.POINTER(C.c_int32), _V]
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = f"{what} failed: {_STATUS.get(rc, rc)}"
+        if rc == 4:
+            msg += " (" + lib().hpa_last_cuda_error().decode() + ")"
+        raise HpaError(msg)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, name: str, dtypes, ndim=None):
+    if not t.is_cuda:
+        raise HpaError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise HpaError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise HpaError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise HpaError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def version() -> int:
+    return int(lib().hpa_version())
+
+
+def default_num_ctas(device: int | None = None) -> int:
+    d = torch.cuda.current_device() if device is None else device
+    n = lib().hpa_default_num_ctas(d)
+    if n < 1:
+        raise HpaError("hpa_default_num_ctas: " + lib().hpa_last_cuda_error().decode())
+    return n
+
+
+def plan_grid(kind: int, batch: int, num_kv_heads: int, num_ctas: int, param: int = 0,
+              max_seq_len: int = 0) -> int:
+    g = lib().hpa_plan_grid(kind, batch, num_kv_heads, num_ctas, param, max_seq_len)
+    if g < 1:
+        raise HpaError("hpa_plan_grid: invalid arguments")
+    return g
+
+
+def decode_workspace_size(batch: int, num_kv_heads: int, num_q_heads: int, head_dim: int,
+                          grid: int) -> int:
+    n = lib().hpa_decode_workspace_size(batch, num_kv_heads, num_q_heads, head_dim, grid)
+    if n == 0:
+        raise HpaError("hpa_decode_workspace_size: invalid arguments")
+    return int(n)
+
+
+def workspace_layout(batch, num_kv_heads, num_q_heads, head_dim, grid) -> dict:
+    off = (_Z * 10)()
+    _check(lib().hpa_workspace_layout(batch, num_kv_heads, num_q_heads, head_dim, grid, off),
+           "hpa_workspace_layout")
+    names = ["header", "lens", "tile_start", "cta_desc", "split_count", "part_base", "arrive",
+             "part_ml", "part_acc", "total"]
+    return {n: int(v) for n, v in zip(names, off)}
+
+
+def decode_plan(seq_lens: torch.Tensor, *, num_kv_heads: int, num_q_heads: int, head_dim: int,
+                pt_stride: int, workspace: torch.Tensor, kind: int = PLAN_DYNAMIC,
+                num_ctas: int | None = None, param: int = 0, max_seq_len: int = 0,
+                stream=None) -> int:
+    """Enqueue the tile plan; returns the grid to pass to decode_run."""
+    _dev(seq_lens, "seq_lens", (torch.int32,), 1)
+    _dev(workspace, "workspace", (torch.uint8,))
+    if num_ctas is None:
+        num_ctas = default_num_ctas(seq_lens.device.index)
+    grid = C.c_int(0)
+    rc = lib().hpa_decode_plan(_ptr(seq_lens), seq_lens.shape[0], num_kv_heads, num_q_heads,
+                               head_dim, pt_stride, kind, num_ctas, param, max_seq_len,
+                               _ptr(workspace), workspace.numel(), C.byref(grid), _stream(stream))
+    _check(rc, "hpa_decode_plan")
+    return grid.value
+
+
+def decode_run(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+               page_table: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, grid: int,
+               softmax_scale: float, *, k_scale: torch.Tensor | None = None,
+               v_scale: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Enqueue the persistent decode kernel; writes and returns ``out``.
+
+    k_cache/v_cache: bf16, or uint8 / float8_e4m3fn codes with k_scale/v_scale."""
+    _dev(q, "q", (torch.bfloat16,), 3)
+    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
+    cache_types = (torch.uint8, torch.float8_e4m3fn) if fp8 else (torch.bfloat16,)
+    _dev(k_cache, "k_cache", cache_types, 4)
+    _dev(v_cache, "v_cache", cache_types, 4)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    _dev(out, "out", (torch.bfloat16, torch.float32), 3)
+    _dev(workspace, "workspace", (torch.uint8,))
+    if fp8:
+        if k_scale is None or v_scale is None:
+            raise HpaError("FP8 caches need k_scale and v_scale")
+        _dev(k_scale, "k_scale", (torch.float32,), 2)
+        _dev(v_scale, "v_scale", (torch.float32,), 2)
+    B, Hq, D = q.shape
+    num_pages, Hkv, S, Dk = k_cache.shape
+    if S != PAGE_SIZE or Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or tuple(out.shape) != tuple(q.shape) or page_table.shape[0] != B:
+        raise HpaError("decode_run: inconsistent shapes")
+    rc = lib().hpa_decode_run(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                              _ptr(v_scale), KV_FP8_E4M3 if fp8 else KV_BF16, _ptr(page_table),
+                              page_table.shape[1], num_pages, _ptr(out),
+                              OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, Hq, Hkv, D,
+                              float(softmax_scale), grid, _ptr(workspace), workspace.numel(),
+                              _stream(stream))
+    _check(rc, "hpa_decode_run")
+    return out
+
+
+def kv_prologue(q_raw, k_raw, v_raw, q_gamma, k_gamma, positions, page_table, k_cache, v_cache,
+                q_out, *, eps: float = 1e-6, rope_theta: float = 10000.0, status=None,
+                stream=None) -> torch.Tensor:
+    """Enqueue the fused RMSNorm + RoPE + KV-write prologue; returns q_out."""
+    for t, n, nd in ((q_raw, "q_raw", 3), (k_raw, "k_raw", 3), (v_raw, "v_raw", 3),
+                     (q_out, "q_out", 3), (k_cache, "k_cache", 4), (v_cache, "v_cache", 4)):
+        _dev(t, n, (torch.bfloat16,), nd)
+    _dev(q_gamma, "q_gamma", (torch.float32,), 1)
+    _dev(k_gamma, "k_gamma", (torch.float32,), 1)
+    _dev(positions, "positions", (torch.int32,), 1)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    if status is not None:
+        _dev(status, "status", (torch.int32,))
+    B, Hq, D = q_raw.shape
+    Hkv = k_raw.shape[1]
+    rc = lib().hpa_kv_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(q_gamma),
+                               _ptr(k_gamma), float(eps), float(rope_theta), _ptr(positions),
+                               _ptr(page_table), page_table.shape[1], _ptr(k_cache),
+                               _ptr(v_cache), _ptr(q_out), B, Hq, Hkv, D, k_cache.shape[0],
+                               _ptr(status), _stream(stream))
+    _check(rc, "hpa_kv_prologue")
+    return q_out
+
+
+def read_status(workspace: torch.Tensor, stream=None) -> int:
+    """Device status word of a plan's workspace (synchronises the stream)."""
+    v = C.c_int32(0)
+    _check(lib().hpa_read_status(_ptr(workspace), C.byref(v), _stream(stream)), "hpa_read_status")
+    return int(v.value)
+
+
+class PagedDecoder:
+    """A workspace sized for one batch shape, plus plan + run in one call."""
+
+    def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                 pt_stride: int, *, kind: int = PLAN_DYNAMIC, num_ctas: int | None = None,
+                 param: int = 0, max_seq_len: int = 0, device=None):
+        self.device = torch.device("cuda" if device is None else device)
+        self.num_ctas = num_ctas or default_num_ctas(self.device.index or 0)
+        self.kind, self.param, self.max_seq_len = kind, param, max_seq_len
+        self.shape = (batch, num_q_heads, num_kv_heads, head_dim, pt_stride)
+        grid = plan_grid(kind, batch, num_kv_heads, self.num_ctas, param, max_seq_len)
+        self.workspace = torch.empty(decode_workspace_size(batch, num_kv_heads, num_q_heads,
+                                                           head_dim, grid),
+                                     dtype=torch.uint8, device=self.device)
+        self.grid = grid
+
+    def plan(self, seq_lens: torch.Tensor, stream=None) -> int:
+        B, Hq, Hkv, D, pts = self.shape
+        self.grid = decode_plan(seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
+                                pt_stride=pts, workspace=self.workspace, kind=self.kind,
+                                num_ctas=self.num_ctas, param=self.param,
+                                max_seq_len=self.max_seq_len, stream=stream)
+        return self.grid
+
+    def run(self, q, k_cache, v_cache, page_table, out, softmax_scale, *, k_scale=None,
+            v_scale=None, stream=None):
+        return decode_run(q, k_cache, v_cache, page_table, out, self.workspace, self.grid,
+                          softmax_scale, k_scale=k_scale, v_scale=v_scale, stream=stream)
+
+    def __call__(self, q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, **kw):
+        self.plan(seq_lens, stream=kw.get("stream"))
+        return self.run(q, k_cache, v_cache, page_table, out, softmax_scale, **kw)
+
+    def status(self, stream=None) -> int:
+        return read_status(self.workspace, stream)

@@ -1,0 +1,240 @@
+// hpa_common.cuh -- shared pieces of the sm_100a kernels: the workspace layout,
+// inline-PTX wrappers (mbarrier, TMA, ldmatrix/movmatrix, mma.sync, PDL) and
+// small host helpers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hpa.h"
+
+namespace hpa {
+
+constexpr int kPageSize = 64;            // tokens per page == tokens per tile
+constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
+
+// ---------------------------------------------------------------------------
+// Workspace layout.  Every region starts on a 256-byte boundary.
+//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T
+//   lens        int32[B]     clamped lengths
+//   tile_start  int32[B+1]   exclusive prefix sum of tiles per sequence
+//   cta_desc    int4[grid]   (u_begin, u_end, first_split, 0)
+//   split_count int32[B*Hkv]
+//   part_base   int32[B*Hkv]
+//   arrive      int32[B*Hkv] arrival counters of the split merge
+//   part_ml     float2[2*grid][G]     (m, l) of each partial, log2 units
+//   part_acc    float[2*grid][G][D]   un-normalised partial outputs
+// A plan of `grid` CTAs has at most 2*(grid-1) partials (each CTA boundary
+// cuts at most one segment), so 2*grid slots always suffice.
+// ---------------------------------------------------------------------------
+enum HeaderField {
+  kHdrMagic = 0, kHdrStatus = 1, kHdrUnits = 2, kHdrGrid = 3, kHdrKind = 4,
+  kHdrBatch = 5, kHdrKvHeads = 6, kHdrGroup = 7, kHdrHeadDim = 8, kHdrTiles = 9,
+  kHdrWords = 16
+};
+
+struct WsLayout {
+  size_t header, lens, tile_start, cta_desc, split_count, part_base, arrive, part_ml, part_acc,
+      total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline bool ws_layout(int B, int Hkv, int Hq, int D, int grid, WsLayout* L) {
+  if (B <= 0 || Hkv <= 0 || Hq <= 0 || D <= 0 || grid <= 0 || Hq % Hkv) return false;
+  const size_t G = size_t(Hq / Hkv), S = size_t(B) * Hkv, slots = 2 * size_t(grid);
+  size_t off = 0;
+  L->header = off;      off = align256(off + kHdrWords * 4);
+  L->lens = off;        off = align256(off + size_t(B) * 4);
+  L->tile_start = off;  off = align256(off + (size_t(B) + 1) * 4);
+  L->cta_desc = off;    off = align256(off + size_t(grid) * 16);
+  L->split_count = off; off = align256(off + S * 4);
+  L->part_base = off;   off = align256(off + S * 4);
+  L->arrive = off;      off = align256(off + S * 4);
+  L->part_ml = off;     off = align256(off + slots * G * 8);
+  L->part_acc = off;    off = align256(off + slots * G * size_t(D) * 4);
+  L->total = off;
+  return true;
+}
+
+// Device view of a workspace.
+struct Ws {
+  int32_t* header;
+  int32_t* lens;
+  int32_t* tile_start;
+  int4* cta_desc;
+  int32_t* split_count;
+  int32_t* part_base;
+  int32_t* arrive;
+  float2* part_ml;
+  float* part_acc;
+};
+
+inline Ws ws_view(void* base, const WsLayout& L) {
+  char* p = static_cast<char*>(base);
+  return Ws{reinterpret_cast<int32_t*>(p + L.header), reinterpret_cast<int32_t*>(p + L.lens),
+            reinterpret_cast<int32_t*>(p + L.tile_start), reinterpret_cast<int4*>(p + L.cta_desc),
+            reinterpret_cast<int32_t*>(p + L.split_count),
+            reinterpret_cast<int32_t*>(p + L.part_base), reinterpret_cast<int32_t*>(p + L.arrive),
+            reinterpret_cast<float2*>(p + L.part_ml), reinterpret_cast<float*>(p + L.part_acc)};
+}
+
+// Host-side grid of a plan (must equal the oracle's definition; see hpa.h).
+inline long long plan_grid_ll(int kind, int B, int Hkv, int num_ctas, int param,
+                              int max_seq_len, long long* chunk_out) {
+  if (B <= 0 || Hkv <= 0 || num_ctas <= 0 || param < 0 || max_seq_len < 0) return -1;
+  if (chunk_out) *chunk_out = 0;
+  if (kind == HPA_PLAN_DYNAMIC) return num_ctas;
+  const long long S = (long long)B * Hkv;
+  if (kind == HPA_PLAN_STATIC_NSPLIT) {
+    long long s = param > 0 ? param : (num_ctas + S - 1) / S;
+    if (s < 1) s = 1;
+    return S * s;
+  }
+  if (kind == HPA_PLAN_STATIC_CHUNK) {
+    const long long tmax = ((long long)max_seq_len + kPageSize - 1) / kPageSize;
+    const long long per_seg = (num_ctas + Hkv - 1) / Hkv;
+    long long c = param > 0 ? param : (tmax + per_seg - 1) / per_seg;
+    if (c < 1) c = 1;
+    long long nc = (tmax + c - 1) / c;
+    if (nc < 1) nc = 1;
+    if (chunk_out) *chunk_out = c;
+    return S * nc;
+  }
+  return -1;
+}
+
+// Records a CUDA error for hpa_last_cuda_error().
+void set_cuda_error(cudaError_t e, const char* where);
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Programmatic dependent launch: wait for the preceding grid's memory, and let
+// the next grid start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: gives up after `limit` polls (each try_wait itself suspends
+// for a hardware-defined interval) and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+// 2-D TMA tile load global -> shared, completing on an mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, bf16 or f16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two fp32 -> packed bf16x2 / f16x2 (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two e4m3 codes (low byte = first) -> f16x2 (exact: every e4m3 value is an f16).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
+  return r;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+#endif  // __CUDACC__
+
+}  // namespace hpa

@@ -43,3 +43,109 @@ def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -
         P = P / P.sum(axis=1, keepdims=True)
         out[g * G:(g + 1) * G] = P @ V[:, g, :]
     return out
+
+
+# ---------------------------------------------------------------- GPU-side runners
+
+def to_device(batch, device="cuda"):
+    """Copy every tensor of a DecodeBatch to `device` (in place)."""
+    for name in ["seq_lens", "page_table", "k_cache", "v_cache", "q", "live", "q_raw", "k_raw",
+                 "v_raw", "q_gamma", "k_gamma", "positions"]:
+        t = getattr(batch, name)
+        if t is not None:
+            setattr(batch, name, t.to(device))
+    return batch
+
+
+def quantize_fp8(batch):
+    """e4m3 codes + scales of an fp8 workload, made by the oracle's quantiser on
+    the host (the decode path only consumes them)."""
+    import oracle
+    kv = batch.k_cache.float().cpu().numpy()
+    vv = batch.v_cache.float().cpu().numpy()
+    live = batch.live.cpu().numpy()
+    kc, ks = oracle.quantize_kv_e4m3(kv, live)
+    vc, vs = oracle.quantize_kv_e4m3(vv, live)
+    return kc, ks, vc, vs
+
+
+def gpu_decode(batch, *, kind=0, num_ctas=None, param=0, max_seq_len=None,
+               out_dtype=torch.bfloat16, fp8=None, q=None, return_ws=False):
+    """plan + run on the GPU through the C-ABI binding; returns the output tensor."""
+    import mixed_length_paged_b200 as hpa
+    dev = torch.device("cuda")
+    B, Hq, D = batch.batch, batch.shape.num_q_heads, batch.shape.head_dim
+    Hkv = batch.shape.num_kv_heads
+    if num_ctas is None:
+        num_ctas = hpa.default_num_ctas()
+    if max_seq_len is None:
+        max_seq_len = int(batch.seq_lens.max().item())
+    grid = hpa.plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len)
+    ws = torch.zeros(hpa.decode_workspace_size(B, Hkv, Hq, D, grid), dtype=torch.uint8, device=dev)
+    seq_lens = batch.seq_lens.to(dev)
+    g = hpa.decode_plan(seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
+                        pt_stride=batch.pt_stride, workspace=ws, kind=kind, num_ctas=num_ctas,
+                        param=param, max_seq_len=max_seq_len)
+    assert g == grid
+    q = (batch.q if q is None else q).to(dev)
+    out = torch.full((B, Hq, D), float("nan"), dtype=out_dtype, device=dev)
+    pt = batch.page_table.to(dev)
+    if fp8 is not None:
+        kc, ks, vc, vs = (torch.from_numpy(x).to(dev) for x in fp8)
+        hpa.decode_run(q, kc, vc, pt, out, ws, grid, 1.0 / D ** 0.5, k_scale=ks, v_scale=vs)
+    else:
+        hpa.decode_run(q, batch.k_cache.to(dev), batch.v_cache.to(dev), pt, out, ws, grid,
+                       1.0 / D ** 0.5)
+    torch.cuda.synchronize()
+    if return_ws:
+        return out, ws, grid
+    return out
+
+
+def oracle_decode(batch, rows=None, fp8=None, q=None):
+    """fp64 oracle output [B][Hq][D] for the sequences in `rows` (all if None)."""
+    import oracle
+    D = batch.shape.head_dim
+    pt = batch.page_table.cpu().numpy()
+    sl = batch.seq_lens.cpu().numpy()
+    qq = bits16(batch.q) if q is None else q
+    if fp8 is not None:
+        kc, ks, vc, vs = fp8
+        return oracle.paged_decode(qq, kc, vc, pt, sl, batch.shape.num_kv_heads,
+                                   1.0 / D ** 0.5, kv_fp8=True, k_scale=ks, v_scale=vs,
+                                   rows=rows)
+    return oracle.paged_decode(qq, bits16(batch.k_cache), bits16(batch.v_cache), pt, sl,
+                               batch.shape.num_kv_heads, 1.0 / D ** 0.5, rows=rows)
+
+
+def compact_rows(batch, rows):
+    """A host copy of `batch` restricted to sequences `rows`, with only their
+    pages (re-numbered), so the oracle can run on a sample of a large batch."""
+    import copy
+    pt = batch.page_table.cpu()
+    sl = batch.seq_lens.cpu()
+    used = []
+    new_pt = torch.full((len(rows), pt.shape[1]), -1, dtype=torch.int32)
+    for i, b in enumerate(rows):
+        n = (int(sl[b]) + 63) // 64
+        ids = pt[b, :n]
+        new_pt[i, :n] = torch.arange(len(used), len(used) + n, dtype=torch.int32)
+        used.extend(ids.tolist())
+    idx = torch.tensor(used, dtype=torch.long, device=batch.k_cache.device)
+    small = copy.copy(batch)
+    small.k_cache = batch.k_cache.index_select(0, idx).cpu()
+    small.v_cache = batch.v_cache.index_select(0, idx).cpu()
+    small.page_table = new_pt
+    small.seq_lens = sl[list(rows)].clone()
+    small.num_pages = len(used)
+    if batch.q is not None:
+        small.q = batch.q[list(rows)].cpu()
+    if batch.live is not None:
+        small.live = batch.live.index_select(0, idx).cpu()
+    return small
+
+
+def errors(gpu_out: torch.Tensor, ref: np.ndarray):
+    g = gpu_out.float().cpu().numpy().astype(np.float64)
+    d = np.abs(g - ref)
+    return float(d.max()), float(d.mean())

@@ -1,0 +1,173 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, its host-only arithmetic matches the oracle's definitions,
+and argument validation rejects bad calls before anything is enqueued."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import mixed_length_paged_b200 as hpa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hpa.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*HPA_API\s+(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(hpa_[a-z0-9_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mixed_length_paged_b200 import build
+    build.build()
+    return hpa.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ["hpa_decode_plan", "hpa_decode_run", "hpa_kv_prologue",
+              "hpa_decode_workspace_size", "hpa_default_num_ctas", "hpa_status_string",
+              "hpa_plan_grid", "hpa_workspace_layout", "hpa_read_status"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    missing = [n for n in _declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_only_declared_symbols_are_exported(L):
+    out = os.popen(f"nm -D --defined-only {hpa.library_path}").read()
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    ours = {s for s in exported if s.startswith("hpa_")}
+    assert ours == set(_declared_functions())
+
+
+def test_status_strings(L):
+    for code, name in [(0, b"HPA_OK"), (1, b"HPA_ERR_INVALID_ARG"), (2, b"HPA_ERR_UNSUPPORTED"),
+                       (3, b"HPA_ERR_WORKSPACE"), (4, b"HPA_ERR_CUDA")]:
+        assert L.hpa_status_string(code) == name
+    assert L.hpa_version() == 100
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("B,Hkv,P,param,maxlen", [
+    (32, 8, 148, 0, 131072), (64, 8, 148, 0, 512), (2, 2, 148, 0, 200), (2, 2, 148, 3, 200),
+    (5, 4, 7, 5, 65), (1, 1, 1, 0, 1), (256, 8, 148, 0, 16384), (3, 2, 5, 0, 0),
+])
+def test_plan_grid_matches_oracle(L, kind, B, Hkv, P, param, maxlen):
+    assert hpa.plan_grid(kind, B, Hkv, P, param, maxlen) == \
+        oracle.plan_grid(kind, B, Hkv, P, param, maxlen)
+
+
+def test_workspace_layout_is_aligned_and_ordered(L):
+    for args in [(32, 8, 64, 128, 148), (2, 2, 8, 64, 148), (256, 8, 64, 128, 4864)]:
+        lay = hpa.workspace_layout(*args)
+        offs = [lay[k] for k in ["header", "lens", "tile_start", "cta_desc", "split_count",
+                                 "part_base", "arrive", "part_ml", "part_acc", "total"]]
+        assert all(o % 256 == 0 for o in offs)
+        assert offs == sorted(offs)
+        B, Hkv, Hq, D, grid = args
+        G = Hq // Hkv
+        assert lay["part_acc"] - lay["part_ml"] >= 2 * grid * G * 8
+        assert lay["total"] - lay["part_acc"] >= 2 * grid * G * D * 4
+        assert lay["cta_desc"] - lay["tile_start"] >= (B + 1) * 4
+        assert hpa.decode_workspace_size(*args) == lay["total"]
+    assert L.hpa_decode_workspace_size(0, 8, 64, 128, 148) == 0
+    assert L.hpa_decode_workspace_size(2, 3, 8, 64, 148) == 0  # Hq % Hkv != 0
+
+
+def _plan(L, **kw):
+    a = dict(seq_lens=1, batch=2, num_kv_heads=2, num_q_heads=8, head_dim=64, pt_stride=4,
+             kind=0, num_ctas=148, param=0, max_seq_len=0, workspace=256, ws_bytes=1 << 20)
+    a.update(kw)
+    g = C.c_int(-7)
+    rc = L.hpa_decode_plan(a["seq_lens"], a["batch"], a["num_kv_heads"], a["num_q_heads"],
+                           a["head_dim"], a["pt_stride"], a["kind"], a["num_ctas"], a["param"],
+                           a["max_seq_len"], a["workspace"], a["ws_bytes"], C.byref(g), None)
+    return rc, g.value
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(seq_lens=None), 1), (dict(workspace=None), 1), (dict(batch=0), 1),
+    (dict(num_kv_heads=0), 1), (dict(num_q_heads=7), 1), (dict(pt_stride=0), 1),
+    (dict(num_ctas=0), 1), (dict(kind=3), 1), (dict(param=-1), 1), (dict(ws_bytes=16), 3),
+    (dict(workspace=256 + 8), 3),
+])
+def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
+    rc, grid = _plan(L, **bad)
+    assert rc == expect
+    assert grid == -7  # nothing reported, nothing enqueued
+
+
+def _run(L, **kw):
+    a = dict(q=256, k=256, v=256, ks=None, vs=None, kvd=0, pt=256, pts=4, pages=8, out=256,
+             outd=0, B=2, Hq=8, Hkv=2, D=64, scale=0.125, grid=148, ws=256, wsb=1 << 22)
+    a.update(kw)
+    return L.hpa_decode_run(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["kvd"], a["pt"], a["pts"],
+                            a["pages"], a["out"], a["outd"], a["B"], a["Hq"], a["Hkv"], a["D"],
+                            C.c_float(a["scale"]), a["grid"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
+    (dict(B=0), 1), (dict(Hq=6, Hkv=4), 1), (dict(kvd=5), 1), (dict(outd=2), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(kvd=1), 1),  # fp8 w/o scales
+    (dict(Hq=24, Hkv=8), 2),   # G = 3
+    (dict(Hq=64, Hkv=2), 2),   # G = 32
+    (dict(D=96), 2), (dict(D=256), 2), (dict(kvd=1, ks=256, vs=256), 2),  # fp8 needs D = 128
+    (dict(pages=1 << 26, Hkv=8, Hq=8), 2),  # rows overflow int32 TMA coordinates
+    (dict(k=256 + 8), 1), (dict(q=256 + 2), 1), (dict(out=256 + 2), 1),
+    (dict(wsb=64), 3), (dict(ws=256 + 16), 3),
+])
+def test_run_rejects_bad_arguments_without_launching(L, bad, expect):
+    assert _run(L, **bad) == expect
+
+
+def _prologue(L, **kw):
+    a = dict(qr=256, kr=256, vr=256, gq=256, gk=256, eps=1e-6, theta=1e4, pos=256, pt=256, pts=4,
+             kc=256, vc=256, qo=256, B=2, Hq=8, Hkv=2, D=64, pages=8, status=None)
+    a.update(kw)
+    return L.hpa_kv_prologue(a["qr"], a["kr"], a["vr"], a["gq"], a["gk"], C.c_float(a["eps"]),
+                             C.c_float(a["theta"]), a["pos"], a["pt"], a["pts"], a["kc"], a["vc"],
+                             a["qo"], a["B"], a["Hq"], a["Hkv"], a["D"], a["pages"], a["status"],
+                             None)
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(qr=None), 1), (dict(gk=None), 1), (dict(pos=None), 1), (dict(B=0), 1),
+    (dict(Hq=7), 1), (dict(eps=-1.0), 1), (dict(theta=0.0), 1), (dict(theta=float("inf")), 1),
+    (dict(D=80), 2),
+])
+def test_prologue_rejects_bad_arguments_without_launching(L, bad, expect):
+    assert _prologue(L, **bad) == expect
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(hpa, "_lib", None)
+    monkeypatch.setattr(hpa, "library_path", "/nonexistent/libhpa.so")
+    with pytest.raises(hpa.HpaLibraryMissing):
+        hpa.lib()
+    with pytest.raises(hpa.HpaLibraryMissing):
+        hpa.decode_workspace_size(2, 2, 8, 64, 148)
+
+
+def test_product_path_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "mixed_length_paged_b200")
+    for dirpath, _, files in os.walk(pkg):
+        if "_build" in dirpath:
+            continue
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "liboracle" not in text, f

@@ -1,0 +1,351 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (bf16 output): max-abs <= 2e-2, mean-abs <= 2e-3; FP8 caches:
+max-abs <= 5e-2.  Split schedules must agree with one another within 1e-3 in
+fp32 output; plans and slot writes are compared bit for bit.
+"""
+from __future__ import annotations
+
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mixed_length_paged_b200 as hpa
+from mixed_length_paged_b200 import workloads as W
+from tests.helpers import (bf16_values, bits16, compact_rows, errors, gpu_decode, oracle_decode,
+                           quantize_fp8, to_device)
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS, FP8_MAX_ABS, SCHED_TOL = 2e-2, 2e-3, 5e-2, 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mixed_length_paged_b200 import build
+    build.build()
+    hpa.lib()
+
+
+def _check(out, ref, max_abs=MAX_ABS, mean_abs=MEAN_ABS, rows=None):
+    if rows is not None:
+        out, ref = out[list(rows)], ref[list(rows)]
+    assert torch.isfinite(out.float()).all()
+    mx, mn = errors(out, ref)
+    assert mx <= max_abs and mn <= mean_abs, (mx, mn)
+    return mx, mn
+
+
+# ---------------------------------------------------------------- plan
+
+def _read_plan(ws, B, Hkv, Hq, D, grid):
+    lay = hpa.workspace_layout(B, Hkv, Hq, D, grid)
+    w = ws.cpu().numpy()
+
+    def i32(off, n):
+        return w[off:off + 4 * n].view(np.int32)
+
+    S = B * Hkv
+    return {
+        "header": i32(lay["header"], 16), "lens": i32(lay["lens"], B),
+        "tile_start": i32(lay["tile_start"], B + 1),
+        "cta": i32(lay["cta_desc"], 4 * grid).reshape(grid, 4),
+        "split_count": i32(lay["split_count"], S), "partial_base": i32(lay["part_base"], S),
+        "arrive": i32(lay["arrive"], S),
+    }
+
+
+@pytest.mark.parametrize("lens,Hkv,P", [
+    ([131072] + [4096] * 31, 8, 148), ([512] * 64, 8, 148), ([37, 200], 2, 148),
+    ([37, 200], 2, 3), ([0, 5, 0, 64, 65, 3000, 1], 4, 7), ([1], 1, 148), ([0, 0], 2, 5),
+    (list(range(1, 3000, 7)), 2, 148),
+])
+@pytest.mark.parametrize("kind,param", [(0, 0), (1, 0), (1, 3), (2, 0), (2, 5)])
+def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
+    B, Hq, D = len(lens), Hkv * 2, 64
+    cap = max(64, max(lens))
+    pts = (cap + 63) // 64
+    maxlen = max(lens)
+    grid = hpa.plan_grid(kind, B, Hkv, P, param, maxlen)
+    ref = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P, param=param,
+                      max_seq_len=maxlen, capacity_tokens=pts * 64)
+    assert grid == ref["grid"]
+    ws = torch.full((hpa.decode_workspace_size(B, Hkv, Hq, D, grid),), 0xAB, dtype=torch.uint8,
+                    device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    g = hpa.decode_plan(sl, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D, pt_stride=pts,
+                        workspace=ws, kind=kind, num_ctas=P, param=param, max_seq_len=maxlen)
+    torch.cuda.synchronize()
+    assert g == grid
+    got = _read_plan(ws, B, Hkv, Hq, D, grid)
+    np.testing.assert_array_equal(got["lens"], ref["lens"])
+    np.testing.assert_array_equal(got["tile_start"], ref["tile_start"])
+    np.testing.assert_array_equal(got["cta"][:, :3], ref["cta"])
+    np.testing.assert_array_equal(got["split_count"], ref["split_count"])
+    np.testing.assert_array_equal(got["partial_base"], ref["partial_base"])
+    assert np.all(got["arrive"] == 0)
+    h = got["header"]
+    assert h[2] == ref["n_units"] and h[3] == grid and h[1] == 0
+
+
+def test_plan_flags_clamped_lengths():
+    sl = torch.tensor([-3, 100, 10_000], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(hpa.decode_workspace_size(3, 2, 4, 64, 148), dtype=torch.uint8, device="cuda")
+    hpa.decode_plan(sl, num_kv_heads=2, num_q_heads=4, head_dim=64, pt_stride=4, workspace=ws,
+                    num_ctas=148)
+    assert hpa.read_status(ws) & hpa.DEVICE_LEN_CLAMPED
+    got = _read_plan(ws, 3, 2, 4, 64, 148)
+    np.testing.assert_array_equal(got["lens"], [0, 100, 256])
+
+
+# ---------------------------------------------------------------- small cases
+
+SMALL = [
+    # name, lens, Hq, Hkv, D
+    ("tiny", [37, 200], 8, 2, 64),
+    ("ragged_g4_d128", [1, 63, 64, 65, 300, 1000, 2047, 5000], 16, 4, 128),
+    ("g8", [129, 1, 700, 64], 64, 8, 128),
+    ("g1", [90, 257], 4, 4, 128),
+    ("g2_d64", [33, 400, 1], 8, 4, 64),
+    ("g16", [200, 1500], 32, 2, 128),
+    ("b1", [3333], 8, 1, 128),
+]
+
+
+@pytest.mark.parametrize("name,lens,Hq,Hkv,D", SMALL)
+@pytest.mark.parametrize("num_ctas", [None, 7, 1])
+def test_decode_matches_oracle_small(name, lens, Hq, Hkv, D, num_ctas):
+    batch = W.make_batch(W.DecodeShape(name, Hq, Hkv, D), lens, seed=zlib.crc32(name.encode()) % 1000)
+    ref = oracle_decode(batch)
+    to_device(batch)
+    out = gpu_decode(batch, num_ctas=num_ctas)
+    _check(out, ref)
+    out32 = gpu_decode(batch, num_ctas=num_ctas, out_dtype=torch.float32)
+    mx, _ = errors(out32, ref)
+    assert mx <= 5e-3, mx
+
+
+def test_tiny_workload_exact_config():
+    batch = W.build("tiny")
+    ref = oracle_decode(batch)
+    out = gpu_decode(to_device(batch))
+    _check(out, ref)
+
+
+def test_length_one_returns_v_row():
+    batch = W.make_batch(W.DecodeShape("l1", 16, 2, 128), [1, 1, 1], seed=5)
+    out = gpu_decode(to_device(batch), out_dtype=torch.float32).cpu()
+    vv = batch.v_cache.float().cpu()
+    pt = batch.page_table.cpu()
+    for b in range(3):
+        for h in range(16):
+            torch.testing.assert_close(out[b, h], vv[pt[b, 0], h // 8, 0], rtol=0, atol=0)
+
+
+def test_zero_length_sequence_gives_zeros():
+    batch = W.make_batch(W.DecodeShape("z", 8, 2, 64), [0, 100, 0], seed=6)
+    ref = oracle_decode(batch)
+    out = gpu_decode(to_device(batch))
+    assert torch.all(out[0] == 0) and torch.all(out[2] == 0)
+    _check(out, ref)
+
+
+def test_page_permutation_invariance_on_gpu():
+    batch = W.make_batch(W.DecodeShape("perm", 16, 4, 128), [700, 33, 2000], seed=8)
+    to_device(batch)
+    out1 = gpu_decode(batch, out_dtype=torch.float32)
+    perm = torch.randperm(batch.num_pages, generator=torch.Generator().manual_seed(1)).cuda()
+    k2 = torch.empty_like(batch.k_cache)
+    v2 = torch.empty_like(batch.v_cache)
+    k2[perm] = batch.k_cache
+    v2[perm] = batch.v_cache
+    pt = batch.page_table.clone()
+    m = pt >= 0
+    pt[m] = perm[pt[m].long()].int()
+    batch.k_cache, batch.v_cache, batch.page_table = k2, v2, pt
+    out2 = gpu_decode(batch, out_dtype=torch.float32)
+    assert torch.equal(out1, out2)
+
+
+def test_repeated_steps_are_deterministic():
+    batch = W.make_batch(W.DecodeShape("rep", 64, 8, 128), [5000, 64, 9000, 1], seed=9)
+    to_device(batch)
+    outs = [gpu_decode(batch, num_ctas=37, out_dtype=torch.float32) for _ in range(3)]
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+# ---------------------------------------------------------------- schedules
+
+@pytest.mark.parametrize("lens", [[131072 // 8] + [4096 // 8] * 31, [1, 63, 64, 65, 300, 5000]])
+def test_split_schedules_agree(lens):
+    batch = W.make_batch(W.DecodeShape("sched", 64, 8, 128), lens, seed=10)
+    ref = oracle_decode(batch)
+    to_device(batch)
+    U = sum((L + 63) // 64 for L in lens) * 8
+    plans = [(0, None, 0), (0, 1, 0), (0, U, 0), (0, 37, 0), (1, None, 0), (1, None, 3),
+             (2, None, 0), (2, None, 1), (2, None, 7)]
+    outs = []
+    for kind, nc, param in plans:
+        o = gpu_decode(batch, kind=kind, num_ctas=nc, param=param, out_dtype=torch.float32)
+        mx, _ = errors(o, ref)
+        assert mx <= 5e-3, (kind, nc, param, mx)
+        outs.append(o)
+    for o in outs[1:]:
+        assert (o - outs[0]).abs().max().item() <= SCHED_TOL
+
+
+# ---------------------------------------------------------------- named workloads
+
+def test_uniform_workload():
+    batch = W.build("uniform")
+    ref = oracle_decode(batch)
+    out = gpu_decode(to_device(batch))
+    _check(out, ref)
+
+
+def test_skewed_workload_sampled_rows():
+    batch = W.build("skewed", device="cuda")
+    out = gpu_decode(batch)  # dynamic plan, one CTA per SM: the benchmark's launch
+    rows = [0, 1, 17, 31]
+    small = compact_rows(batch, rows)
+    ref = oracle_decode(small)
+    _check(out[rows], ref)
+    outA = gpu_decode(batch, kind=1, out_dtype=torch.float32)
+    outD = gpu_decode(batch, out_dtype=torch.float32)
+    assert (outA - outD).abs().max().item() <= SCHED_TOL
+
+
+def test_fp8_small():
+    shape = W.DecodeShape("f8", 64, 8, 128, kv_dtype="fp8_e4m3")
+    batch = W.make_batch(shape, [1, 63, 64, 65, 700, 3000], seed=12)
+    fp8 = quantize_fp8(batch)
+    ref = oracle_decode(batch, fp8=fp8)
+    to_device(batch)
+    for nc in (None, 5):
+        out = gpu_decode(batch, fp8=fp8, num_ctas=nc)
+        _check(out, ref, max_abs=FP8_MAX_ABS, mean_abs=MEAN_ABS)
+
+
+def test_fp8_workload_sampled_rows():
+    batch = W.build("fp8", device="cuda")
+    fp8 = quantize_fp8(batch)
+    out = gpu_decode(batch, fp8=fp8)
+    L = batch.seq_lens.cpu().numpy()
+    rows = [int(np.argmax(L)), int(np.argmin(L)), 0, 100, 255]
+    ref = oracle_decode(batch, fp8=fp8, rows=np.array(rows, dtype=np.int32))
+    _check(out, ref, max_abs=FP8_MAX_ABS, rows=rows)
+
+
+# ---------------------------------------------------------------- prologue
+
+def _prologue_case(lens, Hq=32, Hkv=8, D=128, seed=13, device="cpu"):
+    shape = W.DecodeShape("pro", Hq, Hkv, D, prologue=True)
+    return W.make_batch(shape, lens, seed=seed, device=device)
+
+
+def _run_prologue(batch):
+    B, Hq, D = batch.q_raw.shape
+    q_out = torch.empty_like(batch.q_raw)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hpa.kv_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
+                    batch.positions, batch.page_table, batch.k_cache, batch.v_cache, q_out,
+                    eps=1e-6, rope_theta=10000.0, status=status)
+    torch.cuda.synchronize()
+    return q_out, int(status.item())
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_prologue_slot_writes_and_attention(D):
+    lens = [0, 63, 64, 127, 1000, 4095]
+    batch = _prologue_case(lens, Hq=16, Hkv=4, D=D)
+    kc, vc = bits16(batch.k_cache).copy(), bits16(batch.v_cache).copy()
+    pt = batch.page_table.numpy()
+    q64 = oracle.prologue(bits16(batch.q_raw), bits16(batch.k_raw), bits16(batch.v_raw),
+                          batch.q_gamma.numpy(), batch.k_gamma.numpy(), 1e-6, 1e4,
+                          batch.positions.numpy(), pt, kc, vc)
+    to_device(batch)
+    q_out, status = _run_prologue(batch)
+    assert status == 0
+    gk, gv = bits16(batch.k_cache), bits16(batch.v_cache)
+    # V slots and every untouched byte: bit-exact
+    np.testing.assert_array_equal(gv, vc)
+    diff = gk != kc
+    # K slots: equal up to one bf16 ulp (fp32 vs fp64 rounding at a tie)
+    touched = np.zeros(diff.shape[:3], dtype=bool)
+    for b, pos in enumerate(lens):
+        touched[pt[b, pos // 64], :, pos % 64] = True
+    assert not diff[~touched].any()
+    a, b_ = gk[touched].astype(np.int32), kc[touched].astype(np.int32)
+    assert np.all(np.abs(a - b_) <= 1)
+    # q_out against the oracle's fp64 prologue
+    qg = bf16_values(bits16(q_out))
+    assert np.abs(qg - q64).max() <= np.abs(q64).max() * 2.0 ** -8 + 1e-6
+    # attention over the appended token
+    ref = oracle.paged_decode(q64, kc, vc, pt, batch.seq_lens.cpu().numpy(), 4, 1 / math.sqrt(D))
+    out = gpu_decode(batch, q=q_out)
+    _check(out, ref)
+
+
+def test_prologue_bad_position_is_flagged_not_written():
+    batch = _prologue_case([10, 20], Hq=8, Hkv=2, D=64)
+    batch.positions[1] = 10_000  # beyond the page table
+    before = bits16(batch.k_cache).copy()
+    to_device(batch)
+    _, status = _run_prologue(batch)
+    assert status & hpa.DEVICE_BAD_POSITION
+    after = bits16(batch.k_cache)
+    changed = np.argwhere((after != before).any(axis=-1))
+    assert len(changed) == 2  # sequence 0's K row for its two kv heads only
+
+
+def test_mix_prologue_workload_sampled_rows():
+    batch = W.build("mix_prologue", device="cuda")
+    rows = [0, 1, 50, 127]
+    L = batch.positions.cpu().numpy()
+    rows.append(int(np.argmax(L)))
+    small = compact_rows(batch, rows)
+    small.q_raw = batch.q_raw[rows].cpu()
+    small.k_raw = batch.k_raw[rows].cpu()
+    small.v_raw = batch.v_raw[rows].cpu()
+    small.positions = batch.positions[rows].cpu()
+    kc, vc = bits16(small.k_cache).copy(), bits16(small.v_cache).copy()
+    q64 = oracle.prologue(bits16(small.q_raw), bits16(small.k_raw), bits16(small.v_raw),
+                          batch.q_gamma.cpu().numpy(), batch.k_gamma.cpu().numpy(), 1e-6, 1e4,
+                          small.positions.numpy(), small.page_table.numpy(), kc, vc)
+    ref = oracle.paged_decode(q64, kc, vc, small.page_table.numpy(), small.seq_lens.numpy(), 8,
+                              1 / math.sqrt(128))
+    q_out, status = _run_prologue(batch)
+    assert status == 0
+    out = gpu_decode(batch, q=q_out)
+    _check(out[rows], ref)
+
+
+# ---------------------------------------------------------------- device-side checks
+
+def test_bad_page_id_is_flagged():
+    batch = W.make_batch(W.DecodeShape("bad", 8, 2, 64), [100, 300], seed=14)
+    batch.page_table[1, 2] = batch.num_pages + 5
+    to_device(batch)
+    out, ws, _ = gpu_decode(batch, return_ws=True)
+    assert hpa.read_status(ws) & hpa.DEVICE_BAD_PAGE
+
+
+def test_run_without_plan_is_flagged():
+    batch = W.make_batch(W.DecodeShape("np", 8, 2, 64), [100], seed=15)
+    to_device(batch)
+    grid = 148
+    ws = torch.zeros(hpa.decode_workspace_size(1, 2, 8, 64, grid), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, 8, 64, dtype=torch.bfloat16, device="cuda")
+    hpa.decode_run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, ws, grid, 0.125)
+    assert hpa.read_status(ws) & hpa.DEVICE_BAD_PLAN
+
+
+def test_status_clean_on_normal_run():
+    batch = W.make_batch(W.DecodeShape("ok", 16, 4, 128), [700, 33], seed=16)
+    to_device(batch)
+    _, ws, _ = gpu_decode(batch, return_ws=True)
+    assert hpa.read_status(ws) == 0
