@@ -222,6 +222,40 @@ HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const v
                            int num_kv_heads, int head_dim, int num_pages, int32_t* status,
                            void* stream);
 
+/*
+ * hpa_decode_noalloc -- one decode step (plan + run, dynamic plan) for callers
+ * that must not allocate device memory while they run it: code inside a
+ * device memory pool that may not grow after start-up, code whose allocator
+ * belongs to another framework and is out of reach where the step is issued,
+ * or a plain C program that keeps cudaMalloc off its hot path.  The pages
+ * have no counterpart of this call; it exists for such integrations.
+ *
+ * Arguments are those of hpa_decode_plan + hpa_decode_run with the dynamic
+ * plan; num_ctas = 0 means one CTA per SM.  Instead of a caller workspace the
+ * step uses a library-owned static device array of HPA_NOALLOC_SCRATCH_BYTES
+ * (8 MiB), which every GPU that loads the library holds until the process
+ * exits.  A step whose workspace would exceed it (see
+ * hpa_decode_workspace_size) returns HPA_ERR_WORKSPACE before any CUDA call.
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and the SM count with that device current; make that
+ * first call before any stream capture.  All calls share the array and it
+ * keeps the last call's contents; the plan rewrites everything the run reads
+ * and zeroes the arrival counters on every call, so stale contents never
+ * reach a result, but calls that overlap on the GPU (unordered streams) race
+ * on the array.  The device status word of the array is not exposed.
+ */
+#define HPA_NOALLOC_SCRATCH_BYTES (8u << 20)
+HPA_API hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                      const float* k_scale, const float* v_scale,
+                                      hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                                      int pt_stride, int num_pages, const int32_t* seq_lens,
+                                      void* out, hpa_out_dtype out_dtype, int batch,
+                                      int num_q_heads, int num_kv_heads, int head_dim,
+                                      float softmax_scale, int num_ctas, void* stream);
+
 /* Copies the device status word of a plan's workspace to *status_out (host)
  * after the work queued on `stream` so far; synchronises the stream. */
 HPA_API hpa_status hpa_read_status(const void* workspace, int32_t* status_out, void* stream);

@@ -26,7 +26,7 @@ __all__ = [
     "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
     "default_num_ctas", "workspace_layout", "decode_plan", "decode_run", "kv_prologue",
-    "read_status", "PagedDecoder", "version",
+    "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
 PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2
@@ -35,6 +35,7 @@ OUT_BF16, OUT_F32 = 0, 1
 DEVICE_LEN_CLAMPED, DEVICE_BAD_PAGE, DEVICE_BAD_PLAN = 0x1, 0x2, 0x4
 DEVICE_BAD_POSITION, DEVICE_TIMEOUT = 0x8, 0x10
 PAGE_SIZE = 64
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libhpa.so")
@@ -86,6 +87,9 @@ def lib():
         L.hpa_kv_prologue.restype = _I
         L.hpa_kv_prologue.argtypes = [_V, _V, _V, _V, _V, _F, _F, _V, _V, _I, _V, _V, _V, _I, _I,
                                       _I, _I, _I, _V, _V]
+        L.hpa_decode_noalloc.restype = _I
+        L.hpa_decode_noalloc.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _V, _I, _I, _I,
+                                         _I, _I, _F, _I, _V]
         L.hpa_read_status.restype = _I
         L.hpa_read_status.argtypes = [_V, C.POINTER(C.c_int32), _V]
         _lib = L
@@ -232,6 +236,37 @@ def kv_prologue(q_raw, k_raw, v_raw, q_gamma, k_gamma, positions, page_table, k_
                                _ptr(status), _stream(stream))
     _check(rc, "hpa_kv_prologue")
     return q_out
+
+
+def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   page_table: torch.Tensor, seq_lens: torch.Tensor, out: torch.Tensor,
+                   softmax_scale: float, *, k_scale: torch.Tensor | None = None,
+                   v_scale: torch.Tensor | None = None, num_ctas: int = 0,
+                   stream=None) -> torch.Tensor:
+    """One decode step (dynamic plan + run) without a caller workspace.
+
+    For callers that cannot allocate device memory where the step is issued:
+    the scratch is the library's static 8 MiB device array, shared by every
+    call on the device (calls that overlap on the GPU race on it).  The first
+    call on a device looks the array up; make it before any stream capture."""
+    _dev(q, "q", (torch.bfloat16,), 3)
+    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
+    cache_types = (torch.uint8, torch.float8_e4m3fn) if fp8 else (torch.bfloat16,)
+    _dev(k_cache, "k_cache", cache_types, 4)
+    _dev(v_cache, "v_cache", cache_types, 4)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    _dev(seq_lens, "seq_lens", (torch.int32,), 1)
+    _dev(out, "out", (torch.bfloat16, torch.float32), 3)
+    B, Hq, D = q.shape
+    num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
+    rc = lib().hpa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                  _ptr(v_scale), KV_FP8_E4M3 if fp8 else KV_BF16,
+                                  _ptr(page_table), page_table.shape[1], num_pages,
+                                  _ptr(seq_lens), _ptr(out),
+                                  OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, Hq,
+                                  Hkv, D, float(softmax_scale), num_ctas, _stream(stream))
+    _check(rc, "hpa_decode_noalloc")
+    return out
 
 
 def read_status(workspace: torch.Tensor, stream=None) -> int:
