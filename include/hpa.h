@@ -103,8 +103,9 @@ HPA_API const char* hpa_last_cuda_error(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 HPA_API int hpa_version(void);
 
-/* Number of persistent CTAs for `device`: one per SM (148 on B200).
- * Returns -1 if the device cannot be queried. */
+/* Number of persistent CTAs for `device`: two per SM (296 on B200), which
+ * the run kernel executes as two co-resident CTAs per SM.  Returns -1 if the
+ * device cannot be queried. */
 HPA_API int hpa_default_num_ctas(int device);
 
 /* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC,
@@ -114,29 +115,37 @@ HPA_API int hpa_default_num_ctas(int device);
 HPA_API int hpa_plan_grid(hpa_plan_kind kind, int batch, int num_kv_heads, int num_ctas, int param,
                   int max_seq_len);
 
-/* Bytes of device workspace that a plan of `grid` CTAs and the matching run
- * need.  Host only; returns 0 on invalid arguments. */
-HPA_API size_t hpa_decode_workspace_size(int batch, int num_kv_heads, int num_q_heads, int head_dim,
-                                 int grid);
+/* Bytes of device workspace that a plan of this kind over `grid` CTAs and
+ * the matching run need.  Host only; returns 0 on invalid arguments. */
+HPA_API size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_kv_heads,
+                                         int num_q_heads, int head_dim, int grid);
 
 /* Byte offsets of the workspace regions, for inspection by tests and tools:
- * offsets[0..8] = header, lens, tile_start, cta_desc (int32 x4 per CTA:
- * u_begin, u_end, first_split, 0), split_count, partial_base, arrive,
- * partial (m, l), partial acc; offsets[9] = total size.  Returns HPA_OK or
- * HPA_ERR_INVALID_ARG. */
-HPA_API hpa_status hpa_workspace_layout(int batch, int num_kv_heads, int num_q_heads, int head_dim,
-                                int grid, size_t offsets[10]);
+ * offsets[0..7] = header (int32[16]: magic, status, units, grid, kind, batch,
+ * kv heads, group, head_dim, tiles, ranges V, ...), lens, tile_start,
+ * range descriptors (int32 x8 per range: u_begin, u_end, first_split, and the
+ * sequence, kv head, tile and tile count of its first unit), split_count,
+ * partial_base, partial (m, l), partial acc; offsets[8] = total size.
+ * Returns HPA_OK or HPA_ERR_INVALID_ARG. */
+HPA_API hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_kv_heads,
+                                        int num_q_heads, int head_dim, int grid,
+                                        size_t offsets[9]);
 
 /*
  * hpa_decode_plan -- per-step tile plan (xiaodao.ai "HPC-Ops TPOT -48.8%",
  * Attention section; bitbyai.com "vLLM x HPC-Ops", Attention Backend).
  *
  * Cuts every sequence's live KV into 64-token tiles.  A unit is one
- * (sequence b, kv head g, tile t); the global list orders units by b, g, t.
- * DYNAMIC gives CTA c the units [floor(c U / P'), floor((c+1) U / P')) with
- * P' = min(num_ctas, U): contiguous, equal to within one unit, so a short
- * sequence lands whole in one CTA and a long one is spread over many.  The
- * STATIC kinds give one CTA per (segment, split) instead.
+ * (sequence b, kv head g, tile t); the global list orders units by b, g, t,
+ * and the plan cuts it into contiguous ranges.  DYNAMIC (P = num_ctas
+ * persistent CTAs, U units): if U <= P, CTA c < U takes unit c; otherwise the
+ * last Ut = min(floor(U/8), U - P) units form M = min(4P, Ut) tail chunks
+ * [U1 + floor(jUt/M), U1 + floor((j+1)Ut/M)) and the first U1 = U - Ut units
+ * the P primary ranges [floor(cU1/P), floor((c+1)U1/P)).  CTA c runs primary
+ * range c, then takes tail chunks in order from a counter as it finishes, so
+ * CTAs that got more HBM bandwidth do more of the tail.  A short sequence
+ * lands whole in one range; a long one is spread over many.  The STATIC
+ * kinds give one CTA per (segment, split) instead.
  *
  *   seq_lens     device [batch] int32; values are clamped to [0, pt_stride*64]
  *                (HPA_DEVICE_LEN_CLAMPED).  A sequence of length 0 gets a zero
@@ -144,8 +153,9 @@ HPA_API hpa_status hpa_workspace_layout(int batch, int num_kv_heads, int num_q_h
  *   num_ctas     persistent CTA count (hpa_default_num_ctas), >= 1.
  *   max_seq_len  host upper bound on every seq_len; sizes the STATIC_CHUNK
  *                grid (ignored otherwise, may be 0).
- *   workspace    device, >= hpa_decode_workspace_size(..., grid) bytes,
- *                256-byte aligned.  The plan overwrites it entirely.
+ *   workspace    device, >= hpa_decode_workspace_size(kind, ..., grid)
+ *                bytes, 256-byte aligned.  The plan rewrites everything the
+ *                run reads.
  *   grid_out     host; receives the grid hpa_decode_run must be given.
  *
  * Recompute the plan whenever seq_lens change (every decode step).  A run
@@ -176,18 +186,20 @@ HPA_API hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int num_k
  *   page_table   device int32 [batch][pt_stride]; ids outside
  *                [0, num_pages) are skipped (HPA_DEVICE_BAD_PAGE).
  *   out          device [batch][num_q_heads][D], bf16 or fp32 (out_dtype).
- *   grid         the grid_out of the plan that filled `workspace`.
- *   workspace    the plan's workspace; its partial and arrival regions are
- *                rewritten by the run.
- * Partial slots are merged by the last CTA to finish a sequence's kv head,
- * in split order, so results do not depend on CTA timing.
+ *   kind, grid   the kind and grid_out of the plan that filled `workspace`.
+ *   workspace    the plan's workspace; its partial regions are rewritten by
+ *                the run.
+ * Splits of one (sequence, kv head) leave fp32 partials in the workspace; a
+ * second kernel launched by this call merges them in split order, so results
+ * do not depend on CTA timing.
  */
 HPA_API hpa_status hpa_decode_run(const void* q, const void* k_cache, const void* v_cache,
                           const float* k_scale, const float* v_scale, hpa_kv_dtype kv_dtype,
                           const int32_t* page_table, int pt_stride, int num_pages, void* out,
                           hpa_out_dtype out_dtype, int batch, int num_q_heads,
-                          int num_kv_heads, int head_dim, float softmax_scale, int grid,
-                          void* workspace, size_t ws_bytes, void* stream);
+                          int num_kv_heads, int head_dim, float softmax_scale,
+                          hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes,
+                          void* stream);
 
 /*
  * hpa_kv_prologue -- fused RMSNorm + RoPE + KV write for the new token of

@@ -75,15 +75,15 @@ def lib():
         L.hpa_plan_grid.restype = _I
         L.hpa_plan_grid.argtypes = [_I, _I, _I, _I, _I, _I]
         L.hpa_decode_workspace_size.restype = _Z
-        L.hpa_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+        L.hpa_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
         L.hpa_workspace_layout.restype = _I
-        L.hpa_workspace_layout.argtypes = [_I, _I, _I, _I, _I, C.POINTER(_Z)]
+        L.hpa_workspace_layout.argtypes = [_I, _I, _I, _I, _I, _I, C.POINTER(_Z)]
         L.hpa_decode_plan.restype = _I
         L.hpa_decode_plan.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V, _Z,
                                       C.POINTER(_I), _V]
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
-                                     _F, _I, _V, _Z, _V]
+                                     _F, _I, _I, _V, _Z, _V]
         L.hpa_kv_prologue.restype = _I
         L.hpa_kv_prologue.argtypes = [_V, _V, _V, _V, _V, _F, _F, _V, _V, _I, _V, _V, _V, _I, _I,
                                       _I, _I, _I, _V, _V]
@@ -145,20 +145,20 @@ def plan_grid(kind: int, batch: int, num_kv_heads: int, num_ctas: int, param: in
     return g
 
 
-def decode_workspace_size(batch: int, num_kv_heads: int, num_q_heads: int, head_dim: int,
-                          grid: int) -> int:
-    n = lib().hpa_decode_workspace_size(batch, num_kv_heads, num_q_heads, head_dim, grid)
+def decode_workspace_size(kind: int, batch: int, num_kv_heads: int, num_q_heads: int,
+                          head_dim: int, grid: int) -> int:
+    n = lib().hpa_decode_workspace_size(kind, batch, num_kv_heads, num_q_heads, head_dim, grid)
     if n == 0:
         raise HpaError("hpa_decode_workspace_size: invalid arguments")
     return int(n)
 
 
-def workspace_layout(batch, num_kv_heads, num_q_heads, head_dim, grid) -> dict:
-    off = (_Z * 10)()
-    _check(lib().hpa_workspace_layout(batch, num_kv_heads, num_q_heads, head_dim, grid, off),
+def workspace_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid) -> dict:
+    off = (_Z * 9)()
+    _check(lib().hpa_workspace_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, off),
            "hpa_workspace_layout")
-    names = ["header", "lens", "tile_start", "cta_desc", "split_count", "part_base", "arrive",
-             "part_ml", "part_acc", "total"]
+    names = ["header", "lens", "tile_start", "cta_desc", "split_count", "part_base", "part_ml",
+             "part_acc", "total"]
     return {n: int(v) for n, v in zip(names, off)}
 
 
@@ -181,9 +181,11 @@ def decode_plan(seq_lens: torch.Tensor, *, num_kv_heads: int, num_q_heads: int, 
 
 def decode_run(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                page_table: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, grid: int,
-               softmax_scale: float, *, k_scale: torch.Tensor | None = None,
-               v_scale: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Enqueue the persistent decode kernel; writes and returns ``out``.
+               softmax_scale: float, *, kind: int = PLAN_DYNAMIC,
+               k_scale: torch.Tensor | None = None, v_scale: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Enqueue the persistent decode kernel (and the split merge); writes and
+    returns ``out``.  ``kind``/``grid``: those of the plan in ``workspace``.
 
     k_cache/v_cache: bf16, or uint8 / float8_e4m3fn codes with k_scale/v_scale."""
     _dev(q, "q", (torch.bfloat16,), 3)
@@ -208,8 +210,8 @@ def decode_run(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                               _ptr(v_scale), KV_FP8_E4M3 if fp8 else KV_BF16, _ptr(page_table),
                               page_table.shape[1], num_pages, _ptr(out),
                               OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, Hq, Hkv, D,
-                              float(softmax_scale), grid, _ptr(workspace), workspace.numel(),
-                              _stream(stream))
+                              float(softmax_scale), kind, grid, _ptr(workspace),
+                              workspace.numel(), _stream(stream))
     _check(rc, "hpa_decode_run")
     return out
 
@@ -287,7 +289,7 @@ class PagedDecoder:
         self.kind, self.param, self.max_seq_len = kind, param, max_seq_len
         self.shape = (batch, num_q_heads, num_kv_heads, head_dim, pt_stride)
         grid = plan_grid(kind, batch, num_kv_heads, self.num_ctas, param, max_seq_len)
-        self.workspace = torch.empty(decode_workspace_size(batch, num_kv_heads, num_q_heads,
+        self.workspace = torch.empty(decode_workspace_size(kind, batch, num_kv_heads, num_q_heads,
                                                            head_dim, grid),
                                      dtype=torch.uint8, device=self.device)
         self.grid = grid
@@ -303,7 +305,8 @@ class PagedDecoder:
     def run(self, q, k_cache, v_cache, page_table, out, softmax_scale, *, k_scale=None,
             v_scale=None, stream=None):
         return decode_run(q, k_cache, v_cache, page_table, out, self.workspace, self.grid,
-                          softmax_scale, k_scale=k_scale, v_scale=v_scale, stream=stream)
+                          softmax_scale, kind=self.kind, k_scale=k_scale, v_scale=v_scale,
+                          stream=stream)
 
     def __call__(self, q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, **kw):
         self.plan(seq_lens, stream=kw.get("stream"))

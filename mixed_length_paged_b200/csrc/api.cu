@@ -33,6 +33,10 @@ extern "C" const char* hpa_last_cuda_error(void) { return g_last_error; }
 
 extern "C" int hpa_version(void) { return 100; }
 
+#ifndef HPA_CTAS_PER_SM
+#define HPA_CTAS_PER_SM 2
+#endif
+
 extern "C" int hpa_default_num_ctas(int device) {
   int n = 0;
   cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
@@ -40,23 +44,24 @@ extern "C" int hpa_default_num_ctas(int device) {
     set_cuda_error(e, "hpa_default_num_ctas");
     return -1;
   }
-  return n;
+  return n * HPA_CTAS_PER_SM;
 }
 
-extern "C" size_t hpa_decode_workspace_size(int batch, int num_kv_heads, int num_q_heads,
-                                            int head_dim, int grid) {
+extern "C" size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_kv_heads,
+                                            int num_q_heads, int head_dim, int grid) {
   WsLayout L;
-  if (!ws_layout(batch, num_kv_heads, num_q_heads, head_dim, grid, &L)) return 0;
+  if (!ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, &L)) return 0;
   return L.total;
 }
 
-extern "C" hpa_status hpa_workspace_layout(int batch, int num_kv_heads, int num_q_heads,
-                                           int head_dim, int grid, size_t offsets[10]) {
+extern "C" hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_kv_heads,
+                                           int num_q_heads, int head_dim, int grid,
+                                           size_t offsets[9]) {
   WsLayout L;
-  if (!offsets || !ws_layout(batch, num_kv_heads, num_q_heads, head_dim, grid, &L))
+  if (!offsets || !ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, &L))
     return HPA_ERR_INVALID_ARG;
-  const size_t v[10] = {L.header,    L.lens,   L.tile_start, L.cta_desc, L.split_count,
-                        L.part_base, L.arrive, L.part_ml,    L.part_acc, L.total};
+  const size_t v[9] = {L.header,    L.lens,    L.tile_start, L.cta_desc, L.split_count,
+                       L.part_base, L.part_ml, L.part_acc,   L.total};
   std::memcpy(offsets, v, sizeof v);
   return HPA_OK;
 }

@@ -6,13 +6,17 @@
 // log-sum-exp merge.  The pages describe a Hopper design (TMA + WGMMA); this
 // is written for sm_100a as follows.
 //
-// CTA = 4 consumer warps + 1 producer warp, one CTA per SM.
-//   producer: walks the CTA's unit range, reads page ids (32 at a time, one
-//     per lane), and for each unit issues 2-D TMA tile loads of the K and V
-//     tiles of (page, kv head) -- each a contiguous 64 x D block -- into a
-//     ring of shared-memory stages, with 128-byte swizzle so the tensor-core
-//     fragment loads below are bank-conflict free.  Loads carry an L2
-//     evict-first hint: the cache is streamed once per step.
+// CTA = 4 consumer warps + 1 producer warp + 1 epilogue warp; one CTA per SM
+// when the grid fits the SMs, two smaller co-resident CTAs per SM otherwise
+// (twice the warps to hide each other's latencies).
+//   producer: walks the CTA's unit range and resolves each unit's metadata
+//     (page id, live tokens, first/last tile of its segment, split slot, FP8
+//     scales) 32 units at a time, one per lane, so the global reads overlap.
+//     For each unit it issues 2-D TMA loads of the K and V tiles of (page, kv
+//     head) -- each a contiguous 64 x D block -- into a ring of shared-memory
+//     stages with 128-byte swizzle (bank-conflict-free fragment loads) and an
+//     L2 evict-first hint; for the first tile of a segment it also bulk-copies
+//     the segment's query rows.  The metadata rides along in the stage.
 //   consumers: warp w owns tokens [16w, 16w+16) of every tile and keeps its own
 //     online-softmax state (m, l, acc) for the tile's G query heads:
 //       S^T[16 tok x 8 heads] = K_w[16 x D] . Q^T        (mma m16n8k16, fp32 acc)
@@ -20,11 +24,17 @@
 //       O^T[D x 8 heads]    += V_w^T[D x 16] . P^T      (P^T built in registers
 //                                                       with movmatrix)
 //     The GQA group sits on the MMA N dimension (8 heads per n-tile), so no
-//     padding is needed for G = 8.  At the end of a (sequence, kv head)
-//     segment the four warps' states are combined through shared memory; a
-//     segment held whole by the CTA writes its output directly, otherwise the
-//     CTA stores an (acc, m, l) partial and the last CTA to arrive merges all
-//     partials of that segment in split order.
+//     padding is needed for G = 8.  At a segment end each warp deposits its
+//     state in a double-buffered shared-memory slot and carries on.
+//   epilogue: combines the four warps' states of each deposited segment; a
+//     segment held whole by the CTA is written directly, otherwise the CTA
+//     stores an (acc, m, l) partial.  This keeps the consumers streaming
+//     through segment boundaries.
+// A second, small kernel (chained by programmatic dependent launch) merges
+// the partials of every split segment in split order: one CTA per segment,
+// all partial rows loaded in parallel.  (Merging inside the persistent kernel
+// puts a single CTA's dependent L2 reads on the critical path: the splits of
+// a long sequence all finish together at the end of the step.)
 //
 // FP8 (e4m3) caches: K/V codes are converted in registers with
 // cvt.rn.f16x2.e4m3x2 (exact) and the products run as f16 MMAs; the
@@ -32,7 +42,7 @@
 // into its probabilities.  To keep the e4m3 -> f16 conversion on whole
 // registers, the D index inside each 16-wide MMA step is permuted (the same
 // permutation on both operands, so the dot products are unchanged) and the
-// output rows are un-permuted when stored.
+// output rows are un-permuted when deposited.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -46,11 +56,15 @@ namespace hpa {
 namespace {
 
 constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kSmemLimit = 227 * 1024;
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kEpilogueWarp = kConsumerWarps + 1;
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
+constexpr int kSmemLimit = 227 * 1024;   // per CTA
+constexpr int kSmemPerSm = 228 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any barrier wait
+constexpr int kDepBufs = 2;              // deposit slots between consumers and epilogue
 
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, int CPS>
 struct Cfg {
   static constexpr int kElt = FP8 ? 1 : 2;
   static constexpr int kRowBytes = D * kElt;           // one token row of one head
@@ -59,17 +73,25 @@ struct Cfg {
   static constexpr int kTileBytes = kPageSize * kRowBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
   static constexpr int kHeads = 8 * NT;                // MMA N (padded group)
-  static constexpr int kAccStride = D + 4;             // floats; pads merge stores off one bank
-  static constexpr int kMergeBytes = kConsumerWarps * kHeads * kAccStride * 4;
-  static constexpr int kMlBytes = kConsumerWarps * kHeads * 8;
-  static constexpr int kMisc = 1024;                   // barriers, stage info, flags
-  static constexpr int kStagesFit = (kSmemLimit - 1024 - kMergeBytes - kMlBytes - kMisc) / kStageBytes;
+  static constexpr int kQBytes = kHeads * D * 2;       // a segment's bf16 query rows
+  static constexpr int kAccStride = D + 4;             // floats; keeps deposits off one bank
+  // one deposit: acc[warp][head][D + 4] floats, then (m, l)[warp][head]
+  static constexpr int kDepAccFloats = kConsumerWarps * kHeads * kAccStride;
+  static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kHeads * 8;
+  static constexpr int kMisc = 2048;                   // barriers, stage info, flags
+  // CPS CTAs share one SM's 228 KiB (1 KiB of it reserved per CTA)
+  static constexpr int kBudget = CPS == 1 ? kSmemLimit : (kSmemPerSm / CPS - 1024);
+  static constexpr int kStagesFit =
+      (kBudget - 1024 - kDepBufs * kDepBytes - kMisc) / (kStageBytes + kQBytes);
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMergeBytes + kMlBytes + kMisc;
+  static constexpr int kSmemBytes =
+      1024 + kStages * (kStageBytes + kQBytes) + kDepBufs * kDepBytes + kMisc;
   static constexpr int kKSteps = D / 16;               // QK MMA k-steps
   static constexpr int kMTiles = D / 16;               // PV MMA m-tiles
+  static constexpr int kVec = D / 32;                  // output floats per epilogue lane
   static_assert(kRowBytes % 128 == 0, "tile rows must be whole 128-byte boxes");
   static_assert(kStages >= 2, "not enough shared memory for a pipeline");
+  static_assert(kDepBytes % 16 == 0, "deposit slots must stay 16-byte aligned");
 };
 
 struct RunParams {
@@ -82,12 +104,32 @@ struct RunParams {
   int B, Hq, Hkv, G;
   float scale_log2;         // softmax_scale * log2(e)
   Ws ws;
-  int grid;
+  int grid, kind;
+  int slots;                // 2 * V partial slots in the workspace
 };
 
-struct StageInfo {
-  float k_scale, v_scale;
+// What the producer resolved for the unit held in one stage.
+constexpr int kFirst = 1;   // first tile of its segment in this range
+constexpr int kLast = 2;    // last tile of its segment in this range
+constexpr int kEnd = 4;     // no unit: the producer has no more work
+struct alignas(16) StageInfo {
+  int32_t b, g, valid, flags;   // sequence, kv head, live tokens in the tile, kFirst|kLast
+  int32_t nsplit, slot, pbase, pad;  // split count; partial slot and first slot (if split)
+  float k_scale, v_scale, pad2, pad3;
 };
+
+// Segment handed from the consumers to the epilogue warp.
+struct alignas(16) DepDesc {
+  int32_t b, g, nsplit, slot, pbase, stop, pad0, pad1;
+};
+
+// 2^x on the SFU (ex2.approx, flush-to-zero): relative error ~2^-22, and
+// 2^-inf = +0, which the masked logits rely on.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -114,26 +156,9 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   return false;
 }
 
-// Largest b in [0, B) with tile_start[b] * Hkv <= u.
-__device__ __forceinline__ int seq_of_unit(const int32_t* ts, int B, int Hkv, int u) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if ((long long)ts[mid] * Hkv <= u) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// Walk over (b, g, t) units in global order.
+// Walk over (b, g, t) units in global order; n = tiles of sequence b.
 struct Walk {
   int b, g, t, n;
-  __device__ void init(const int32_t* ts, int B, int Hkv, int u) {
-    b = seq_of_unit(ts, B, Hkv, u);
-    n = ts[b + 1] - ts[b];
-    const int rem = u - ts[b] * Hkv;
-    g = rem / n;
-    t = rem % n;
-  }
   __device__ void next(const int32_t* ts, int Hkv) {
     if (++t < n) return;
     t = 0;
@@ -146,29 +171,50 @@ struct Walk {
   }
 };
 
-// Shared-memory byte offset of 16-byte chunk `chunk` of token row `tok` in a
-// tile stored as 128-byte-swizzled boxes of 64 rows x 128 bytes.
-__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int tok, int chunk) {
-  return tile + (chunk >> 3) * (kPageSize * 128) + tok * 128 + (((chunk & 7) ^ (tok & 7)) << 4);
+template <bool OUT_F32>
+__device__ __forceinline__ void store_out(void* out, long long i, float v) {
+  if constexpr (OUT_F32) reinterpret_cast<float*>(out)[i] = v;
+  else reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
 }
 
-template <int D, int NT, bool FP8, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 1)
+// Stores kVec consecutive outputs starting at element i (i a multiple of kVec).
+template <bool OUT_F32, int kVec>
+__device__ __forceinline__ void store_out_vec(void* out, long long i, const float (&v)[kVec]) {
+  if constexpr (OUT_F32) {
+    if constexpr (kVec == 4) *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2*>(reinterpret_cast<float*>(out) + i) = make_float2(v[0], v[1]);
+  } else {
+    if constexpr (kVec == 4) {
+      uint2 w;
+      w.x = pack_bf16(v[0], v[1]);
+      w.y = pack_bf16(v[2], v[3]);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + i) = w;
+    } else {
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(out) + i) = pack_bf16(v[0], v[1]);
+    }
+  }
+}
+
+template <int D, int NT, bool FP8, bool OUT_F32, int CPS>
+__global__ void __launch_bounds__(kThreads, CPS)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const RunParams p) {
-  using C = Cfg<D, NT, FP8>;
+  using C = Cfg<D, NT, FP8, CPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  float* red_acc = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
-  float2* red_ml = reinterpret_cast<float2*>(smem + C::kStages * C::kStageBytes + C::kMergeBytes);
-  uint8_t* misc = smem + C::kStages * C::kStageBytes + C::kMergeBytes + C::kMlBytes;
+  uint8_t* qslots = smem + C::kStages * C::kStageBytes;
+  uint8_t* deps = qslots + C::kStages * C::kQBytes;     // kDepBufs deposit slots
+  uint8_t* misc = deps + kDepBufs * C::kDepBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(misc);
   uint64_t* empty_bar = full_bar + C::kStages;
-  StageInfo* info = reinterpret_cast<StageInfo*>(empty_bar + C::kStages);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(info + C::kStages);
-  volatile int* s_last = s_abort + 1;
-  volatile int* s_plan_ok = s_abort + 2;
+  uint64_t* dep_full = empty_bar + C::kStages;
+  uint64_t* dep_empty = dep_full + kDepBufs;
+  StageInfo* info = reinterpret_cast<StageInfo*>(dep_empty + kDepBufs);
+  DepDesc* dep_desc = reinterpret_cast<DepDesc*>(info + C::kStages);
+  volatile int* s_flags = reinterpret_cast<volatile int*>(dep_desc + kDepBufs);
+  volatile int* s_abort = s_flags;
+  volatile int* s_plan_ok = s_flags + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -176,10 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), kConsumerWarps);
     }
+    for (int d = 0; d < kDepBufs; ++d) {
+      mbar_init(smem_u32(&dep_full[d]), kConsumerWarps);
+      mbar_init(smem_u32(&dep_empty[d]), 1);
+    }
     *s_abort = 0;
     fence_barrier_init();
   }
-  if (warp == kConsumerWarps && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
   }
@@ -189,7 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t* h = p.ws.header;
     const bool ok = h[kHdrMagic] == kPlanMagic && h[kHdrGrid] == p.grid &&
                     h[kHdrGrid] == (int)gridDim.x && h[kHdrBatch] == p.B &&
-                    h[kHdrKvHeads] == p.Hkv && h[kHdrGroup] == p.G && h[kHdrHeadDim] == D;
+                    h[kHdrKvHeads] == p.Hkv && h[kHdrGroup] == p.G && h[kHdrHeadDim] == D &&
+                    h[kHdrKind] == p.kind && h[kHdrRanges] >= p.grid &&
+                    h[kHdrRanges] <= plan_ranges_ll(p.kind, p.grid);
     *s_plan_ok = ok;
     if (!ok) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
   }
@@ -199,68 +251,153 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   int32_t* status = &p.ws.header[kHdrStatus];
   const int32_t* ts = p.ws.tile_start;
-  const int U = p.ws.header[kHdrUnits];
-  const int4 desc = p.ws.cta_desc[blockIdx.x];
-  const int ub = desc.x, ue = min(desc.y, U);
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    uint64_t policy = l2_policy_evict_first();
-    Walk wk;
+    const uint64_t policy = l2_policy_evict_first();
+    const int qbytes = p.G * D * 2;
+    const int U = p.ws.header[kHdrUnits];
+    const int V = p.ws.header[kHdrRanges];
+    const bool dyn = p.kind == HPA_PLAN_DYNAMIC;
     int it = 0;
-    if (ub < ue) wk.init(ts, p.B, p.Hkv, ub);
-    for (int u0 = ub; u0 < ue; u0 += 32) {
-      // lane i resolves unit u0 + i: (page, kv head) -> tile row, scales
-      int row = 0, bad = 0;
-      float ks = 1.f, vs = 1.f;
-      {
-        Walk w2 = wk;
-        for (int k = 0; k < lane && u0 + k + 1 < ue; ++k) w2.next(ts, p.Hkv);
-        if (u0 + lane < ue) {
-          const int page = p.page_table[(long long)w2.b * p.pt_stride + w2.t];
-          if (page < 0 || page >= p.num_pages) {
-            bad = 1;
-          } else {
-            row = (page * p.Hkv + w2.g) * kPageSize;
+    // This CTA's primary range first; under the dynamic plan it then takes
+    // tail chunks, reserving the next one (and reading its descriptor) while
+    // it streams the current one.
+    int v = blockIdx.x;
+    int4 d0 = p.ws.cta_desc[2 * v], d1 = p.ws.cta_desc[2 * v + 1];
+    while (true) {
+      int vn = V;
+      int4 n0 = make_int4(0, 0, 0, 0), n1 = n0;
+      if (dyn) {
+        if (lane == 0) vn = p.grid + atomicAdd(&p.ws.header[kHdrNext], 1);
+        vn = __shfl_sync(0xffffffffu, vn, 0);
+        if (vn < V) {
+          n0 = p.ws.cta_desc[2 * vn];
+          n1 = p.ws.cta_desc[2 * vn + 1];
+        }
+      }
+      const int ub = max(0, d0.x), ue = min(d0.y, U);
+      Walk wk{d0.w, d1.x, d1.y, d1.z};
+      const int b_first = d0.w, g_first = d1.x, first_split = d0.z;
+      if (ub < ue && (wk.b < 0 || wk.b >= p.B || wk.n <= 0 || wk.n != ts[wk.b + 1] - ts[wk.b] ||
+                      wk.g < 0 || wk.g >= p.Hkv || wk.t < 0 || wk.t >= wk.n)) {
+        if (lane == 0) atomicOr(status, HPA_DEVICE_BAD_PLAN);
+      } else {
+        for (int u0 = ub; u0 < ue; u0 += 32) {
+          Walk w2 = wk;
+          for (int k = 0; k < lane && u0 + k + 1 < ue; ++k) w2.next(ts, p.Hkv);
+          const int u = u0 + lane;
+          int row = 0, valid = 0, flags = 0, nsplit = 1, slot = -1, pbase = 0, bad = 0;
+          float ks = 1.f, vs = 1.f;
+          if (u < ue) {
+            const int page = __ldg(p.page_table + (long long)w2.b * p.pt_stride + w2.t);
+            const int L = p.ws.lens[w2.b];
+            valid = min(kPageSize, L - w2.t * kPageSize);
+            flags = ((w2.t == 0 || u == ub) ? kFirst : 0) | ((w2.t == w2.n - 1 || u == ue - 1) ? kLast : 0);
+            if (flags & kLast) {
+              const int sg = w2.b * p.Hkv + w2.g;
+              nsplit = p.ws.split_count[sg];
+              if (nsplit > 1) {
+                pbase = p.ws.part_base[sg];
+                const int sidx = (w2.b == b_first && w2.g == g_first) ? first_split : 0;
+                slot = pbase + sidx;
+                if (sidx >= nsplit || pbase < 0 || pbase + nsplit > p.slots) {
+                  atomicOr(status, HPA_DEVICE_BAD_PLAN);
+                  slot = -1;  // the output of this segment is void
+                }
+              }
+            }
+            if (page < 0 || page >= p.num_pages) {
+              bad = 1;
+            } else {
+              row = (page * p.Hkv + w2.g) * kPageSize;
+              if constexpr (FP8) {
+                ks = __ldg(p.k_scale + page * p.Hkv + w2.g);
+                vs = __ldg(p.v_scale + page * p.Hkv + w2.g);
+              }
+            }
+          }
+          // small fields travel packed: valid (7 bits) | flags (2) | bad (1) | g (<< 10)
+          const int packed = valid | (flags << 7) | (bad << 9) | (w2.g << 10);
+          const int cnt = min(32, ue - u0);
+          for (int k = 0; k < cnt; ++k) {
+            const int rk = __shfl_sync(0xffffffffu, row, k);
+            const int pk = __shfl_sync(0xffffffffu, packed, k);
+            StageInfo si;
+            si.b = __shfl_sync(0xffffffffu, w2.b, k);
+            si.g = pk >> 10;
+            si.valid = pk & 127;
+            si.flags = (pk >> 7) & 3;
+            const int bk = (pk >> 9) & 1;
+            si.nsplit = 1;
+            si.slot = -1;
+            si.pbase = 0;
+            if (si.flags & kLast) {  // warp-uniform: pk is the same in every lane
+              si.nsplit = __shfl_sync(0xffffffffu, nsplit, k);
+              si.slot = __shfl_sync(0xffffffffu, slot, k);
+              si.pbase = __shfl_sync(0xffffffffu, pbase, k);
+            }
+            si.pad = 0;
+            si.k_scale = si.v_scale = 1.f;
             if constexpr (FP8) {
-              ks = p.k_scale[page * p.Hkv + w2.g];
-              vs = p.v_scale[page * p.Hkv + w2.g];
+              si.k_scale = __shfl_sync(0xffffffffu, ks, k);
+              si.v_scale = __shfl_sync(0xffffffffu, vs, k);
             }
+            si.pad2 = si.pad3 = 0.f;
+            if (lane == 0) {
+              const int s = it % C::kStages;
+              const uint32_t par = ((it / C::kStages) & 1) ^ 1;
+              const uint32_t fb = smem_u32(&full_bar[s]);
+              if (wait_bar(smem_u32(&empty_bar[s]), par, s_abort, status) && !bk) {
+                info[s] = si;
+                const bool first = si.flags & kFirst;
+                mbar_arrive_expect_tx(fb, C::kStageBytes + (first ? qbytes : 0));
+                if (first)
+                  bulk_load(smem_u32(qslots + s * C::kQBytes),
+                            p.q + ((long long)si.b * p.Hq + (long long)si.g * p.G) * D, qbytes, fb);
+                const uint32_t kdst = smem_u32(stages + s * C::kStageBytes);
+                const uint32_t vdst = kdst + C::kTileBytes;
+    #pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                  const int x = bx * (128 / C::kElt);
+                  tma_load_2d(kdst + bx * C::kBoxBytes, &tm_k, x, rk, fb, policy);
+                  tma_load_2d(vdst + bx * C::kBoxBytes, &tm_v, x, rk, fb, policy);
+                }
+              } else {
+                info[s] = si;
+                if (bk) atomicOr(status, HPA_DEVICE_BAD_PAGE);
+                mbar_arrive(fb);  // release the consumers without data (result void)
+              }
+            }
+            __syncwarp();
+            ++it;
           }
+          for (int k = 0; k < cnt; ++k)
+            if (u0 + k + 1 < ue) wk.next(ts, p.Hkv);
         }
       }
-      const int cnt = min(32, ue - u0);
-      for (int k = 0; k < cnt; ++k) {
-        const int rk = __shfl_sync(0xffffffffu, row, k);
-        const int bk = __shfl_sync(0xffffffffu, bad, k);
-        const float kk = __shfl_sync(0xffffffffu, ks, k);
-        const float vv = __shfl_sync(0xffffffffu, vs, k);
-        if (lane == 0) {
-          const int s = it % C::kStages;
-          const uint32_t par = ((it / C::kStages) & 1) ^ 1;
-          const uint32_t fb = smem_u32(&full_bar[s]);
-          if (wait_bar(smem_u32(&empty_bar[s]), par, s_abort, status) && !bk) {
-            info[s].k_scale = kk;
-            info[s].v_scale = vv;
-            mbar_arrive_expect_tx(fb, C::kStageBytes);
-            const uint32_t kdst = smem_u32(stages + s * C::kStageBytes);
-            const uint32_t vdst = kdst + C::kTileBytes;
-#pragma unroll
-            for (int bx = 0; bx < C::kBoxes; ++bx) {
-              const int x = bx * (128 / C::kElt);
-              tma_load_2d(kdst + bx * C::kBoxBytes, &tm_k, x, rk, fb, policy);
-              tma_load_2d(vdst + bx * C::kBoxBytes, &tm_v, x, rk, fb, policy);
-            }
-          } else {
-            if (bk) atomicOr(status, HPA_DEVICE_BAD_PAGE);
-            mbar_arrive(fb);  // release consumers without data
-          }
-        }
-        __syncwarp();
-        ++it;
+      if (!dyn || vn >= V || *s_abort) break;
+      v = vn;
+      d0 = n0;
+      d1 = n1;
+    }
+    // end of work: a stage without data whose info says so
+    if (lane == 0) {
+      const int s = it % C::kStages;
+      const uint32_t par = ((it / C::kStages) & 1) ^ 1;
+      if (wait_bar(smem_u32(&empty_bar[s]), par, s_abort, status)) {
+        StageInfo si = {};
+        si.flags = kEnd;
+        info[s] = si;
+        mbar_arrive(smem_u32(&full_bar[s]));
       }
-      for (int k = 0; k < cnt; ++k)
-        if (u0 + k + 1 < ue) wk.next(ts, p.Hkv);
+    }
+    __syncwarp();
+    ++it;
+    // zero output rows of empty sequences (a softmax over no tokens)
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+      if (p.ws.lens[b] != 0) continue;
+      for (int i = lane; i < p.Hq * D; i += 32) store_out<OUT_F32>(p.out, (long long)b * p.Hq * D + i, 0.f);
     }
     // After an abort, make sure no copy is still landing in shared memory.
     if (lane == 0 && *s_abort) {
@@ -276,6 +413,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
+  if (warp == kEpilogueWarp) {
+    // ------------------------------------------------------------ epilogue
+    const int G = p.G;
+    constexpr int V = C::kVec;
+    for (int k = 0;; ++k) {
+      const int db = k % kDepBufs;
+      if (!wait_bar(smem_u32(&dep_full[db]), (k / kDepBufs) & 1, s_abort, status)) break;
+      DepDesc dd = dep_desc[db];
+      if (dd.stop) break;
+      // Never trust a deposit as an index without checking it.
+      if (dd.b < 0 || dd.b >= p.B || dd.g < 0 || dd.g >= p.Hkv ||
+          (dd.nsplit > 1 && (dd.slot < 0 || dd.slot >= p.slots || dd.pbase < 0 ||
+                             dd.pbase + dd.nsplit > p.slots))) {
+        if (lane == 0) atomicOr(status, HPA_DEVICE_BAD_PLAN);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&dep_empty[db]));
+        continue;
+      }
+      const float* dacc = reinterpret_cast<const float*>(deps + db * C::kDepBytes);
+      const float2* dml = reinterpret_cast<const float2*>(dacc + C::kDepAccFloats);
+      const long long out_row0 = ((long long)dd.b * p.Hq + (long long)dd.g * G) * D;
+      const int d = lane * V;
+      // combine the four warps' states, head by head
+      for (int h = 0; h < G; ++h) {
+        float2 ml[kConsumerWarps];
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          ml[w] = dml[w * C::kHeads + h];
+          M = fmaxf(M, ml[w].x);
+        }
+        float lam = 0.f, o[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) o[v] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float sc = (ml[w].x == -INFINITY) ? 0.f : fast_exp2(ml[w].x - M);
+          lam += ml[w].y * sc;
+          const float* src = dacc + (w * C::kHeads + h) * C::kAccStride + d;
+          if constexpr (V == 4) {
+            const float4 a = *reinterpret_cast<const float4*>(src);
+            o[0] += a.x * sc; o[1] += a.y * sc; o[2] += a.z * sc; o[3] += a.w * sc;
+          } else {
+            const float2 a = *reinterpret_cast<const float2*>(src);
+            o[0] += a.x * sc; o[1] += a.y * sc;
+          }
+        }
+        if (dd.nsplit <= 1) {
+          const float inv = 1.f / lam;
+#pragma unroll
+          for (int v = 0; v < V; ++v) o[v] *= inv;
+          store_out_vec<OUT_F32, V>(p.out, out_row0 + (long long)h * D + d, o);
+        } else if (dd.slot >= 0) {
+          float* dst = p.ws.part_acc + ((long long)dd.slot * G + h) * D + d;
+          if constexpr (V == 4) *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+          else *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
+          if (lane == 0) p.ws.part_ml[(long long)dd.slot * G + h] = make_float2(M, lam);
+        }
+      }
+      // the deposit slot is free again
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&dep_empty[db]));
+    }
+    return;
+  }
+
   // -------------------------------------------------------------- consumers
   const int r = lane >> 2, c = lane & 3;          // MMA fragment coordinates
   const int lm = lane >> 3, lr = lane & 7;        // ldmatrix address lane roles
@@ -285,152 +488,96 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int k_chk = lm >> 1;
   const int v_tok = FP8 ? tok0 + (lm & 1) * 8 + lr : tok0 + (lm >> 1) * 8 + lr;
   const int v_chk = FP8 ? (lm >> 1) : (lm & 1);
-
-  // zero output rows of empty sequences (a softmax over no tokens)
-  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-    if (p.ws.lens[b] != 0) continue;
-    for (int i = threadIdx.x; i < p.Hq * D; i += kConsumerWarps * 32) {
-      const long long o = (long long)b * p.Hq * D + i;
-      if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[o] = 0.f;
-      else reinterpret_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(0.f);
-    }
+  // Byte offsets (inside a tile) of this lane's ldmatrix rows for chunk 2j +
+  // chk, j = 0..3, under the 128-byte swizzle; chunk 2j + 8 + chk adds one box.
+  uint32_t koff[4], voff[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    koff[j] = k_tok * 128 + ((((2 * j + k_chk) & 7) ^ (k_tok & 7)) << 4);
+    voff[j] = v_tok * 128 + ((((2 * j + v_chk) & 7) ^ (v_tok & 7)) << 4);
   }
 
   uint32_t qf[NT][C::kKSteps][2];
   float acc[NT][C::kMTiles][4];
   float m_run[NT][2], l_run[NT][2];
+  int nseg = 0;  // segments deposited so far
 
-  Walk wk;
-  if (ub < ue) wk.init(ts, p.B, p.Hkv, ub);
-  int seg_b = -1, seg_g = 0, L = 0;
-
-  auto finish_segment = [&](int b, int g, int split_idx) {
-    // full-warp l (m is already uniform across the lanes sharing a head)
+  // Hand this warp's state of a finished segment to the epilogue warp.
+  auto deposit = [&](const StageInfo* inf) {
+    const int db = nseg % kDepBufs;
+    wait_bar(smem_u32(&dep_empty[db]), ((nseg / kDepBufs) & 1) ^ 1, s_abort, status);
+    if (inf) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float v = l_run[nt][e];
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        l_run[nt][e] = v;
-      }
-    float* my_acc = red_acc + warp * C::kHeads * C::kAccStride;
+        for (int e = 0; e < 2; ++e) {
+          float v = l_run[nt][e];
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          l_run[nt][e] = v;
+        }
+      float* dacc = reinterpret_cast<float*>(deps + db * C::kDepBytes);
+      float2* dml = reinterpret_cast<float2*>(dacc + C::kDepAccFloats);
+      float* my_acc = dacc + warp * C::kHeads * C::kAccStride;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int h0 = nt * 8 + 2 * c;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int h0 = nt * 8 + 2 * c;
 #pragma unroll
-      for (int i = 0; i < C::kMTiles; ++i) {
-        const int d0 = FP8 ? 16 * i + 2 * r : 16 * i + r;
-        const int d1 = FP8 ? d0 + 1 : d0 + 8;
-        my_acc[h0 * C::kAccStride + d0] = acc[nt][i][0];
-        my_acc[(h0 + 1) * C::kAccStride + d0] = acc[nt][i][1];
-        my_acc[h0 * C::kAccStride + d1] = acc[nt][i][2];
-        my_acc[(h0 + 1) * C::kAccStride + d1] = acc[nt][i][3];
-      }
-      if (r == 0) {
-        red_ml[warp * C::kHeads + h0] = make_float2(m_run[nt][0], l_run[nt][0]);
-        red_ml[warp * C::kHeads + h0 + 1] = make_float2(m_run[nt][1], l_run[nt][1]);
-      }
-    }
-    named_bar_sync(1, kConsumerWarps * 32);
-
-    const int s = b * p.Hkv + g;
-    const int nsplit = p.ws.split_count[s];
-    const int G = p.G;
-    const int tid = threadIdx.x;
-    const long long out_row0 = ((long long)b * p.Hq + (long long)g * G) * D;
-    int slot = -1;
-    if (nsplit > 1) {
-      slot = p.ws.part_base[s] + split_idx;
-      if (slot < 0 || slot >= 2 * p.grid || split_idx >= nsplit) {
-        if (tid == 0) atomicOr(status, HPA_DEVICE_BAD_PLAN);
-        slot = -1;
-      }
-    }
-    for (int e = tid; e < G * D; e += kConsumerWarps * 32) {
-      const int h = e / D, d = e - h * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_ml[w * C::kHeads + h].x);
-      float lam = 0.f, o = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float2 ml = red_ml[w * C::kHeads + h];
-        const float sc = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-        lam += ml.y * sc;
-        o += red_acc[(w * C::kHeads + h) * C::kAccStride + d] * sc;
-      }
-      if (nsplit <= 1) {
-        const float v = o / lam;
-        if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[out_row0 + e] = v;
-        else reinterpret_cast<__nv_bfloat16*>(p.out)[out_row0 + e] = __float2bfloat16_rn(v);
-      } else if (slot >= 0) {
-        p.ws.part_acc[((long long)slot * G + h) * D + d] = o;
-        if (d == 0) p.ws.part_ml[(long long)slot * G + h] = make_float2(M, lam);
-      }
-    }
-    if (nsplit > 1) {
-      __threadfence();
-      named_bar_sync(1, kConsumerWarps * 32);
-      if (tid == 0) {
-        const int prev = atomicAdd(&p.ws.arrive[s], 1);
-        *s_last = (prev == nsplit - 1);
-      }
-      named_bar_sync(1, kConsumerWarps * 32);
-      if (*s_last) {
-        __threadfence();
-        const int base = p.ws.part_base[s];
-        if (base >= 0 && base + nsplit <= 2 * p.grid) {
-          for (int e = tid; e < G * D; e += kConsumerWarps * 32) {
-            const int h = e / D, d = e - h * D;
-            float M = -INFINITY;
-            for (int i = 0; i < nsplit; ++i)
-              M = fmaxf(M, __ldcg(&p.ws.part_ml[(long long)(base + i) * G + h]).x);
-            float lam = 0.f, o = 0.f;
-            for (int i = 0; i < nsplit; ++i) {
-              const float2 ml = __ldcg(&p.ws.part_ml[(long long)(base + i) * G + h]);
-              const float sc = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-              lam += ml.y * sc;
-              o += __ldcg(&p.ws.part_acc[((long long)(base + i) * G + h) * D + d]) * sc;
-            }
-            const float v = o / lam;
-            if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[out_row0 + e] = v;
-            else reinterpret_cast<__nv_bfloat16*>(p.out)[out_row0 + e] = __float2bfloat16_rn(v);
-          }
+        for (int i = 0; i < C::kMTiles; ++i) {
+          const int dr0 = FP8 ? 16 * i + 2 * r : 16 * i + r;
+          const int dr1 = FP8 ? dr0 + 1 : dr0 + 8;
+          my_acc[h0 * C::kAccStride + dr0] = acc[nt][i][0];
+          my_acc[(h0 + 1) * C::kAccStride + dr0] = acc[nt][i][1];
+          my_acc[h0 * C::kAccStride + dr1] = acc[nt][i][2];
+          my_acc[(h0 + 1) * C::kAccStride + dr1] = acc[nt][i][3];
+        }
+        if (r == 0) {
+          dml[warp * C::kHeads + h0] = make_float2(m_run[nt][0], l_run[nt][0]);
+          dml[warp * C::kHeads + h0 + 1] = make_float2(m_run[nt][1], l_run[nt][1]);
         }
       }
     }
-    named_bar_sync(1, kConsumerWarps * 32);  // shared merge buffers free again
+    if (warp == 0 && lane == 0) {
+      DepDesc dd;
+      dd.b = inf ? inf->b : -1;
+      dd.g = inf ? inf->g : 0;
+      dd.nsplit = inf ? inf->nsplit : 0;
+      dd.slot = inf ? inf->slot : -1;
+      dd.pbase = inf ? inf->pbase : 0;
+      dd.stop = inf ? 0 : 1;
+      dd.pad0 = dd.pad1 = 0;
+      dep_desc[db] = dd;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&dep_full[db]));
+    ++nseg;
   };
 
-  int it = 0;
-  int split_idx = desc.z;
-  for (int u = ub; u < ue; ++u, ++it) {
-    if (seg_b < 0 || wk.t == 0) {
-      if (seg_b >= 0) {
-        finish_segment(seg_b, seg_g, split_idx);
-        split_idx = 0;
-      }
-      seg_b = wk.b;
-      seg_g = wk.g;
-      L = p.ws.lens[seg_b];
+  for (int it = 0;; ++it) {
+    const int s = it % C::kStages;
+    if (!wait_bar(smem_u32(&full_bar[s]), (it / C::kStages) & 1, s_abort, status)) break;
+    const StageInfo inf = info[s];
+    if (inf.flags & kEnd) break;
+    const uint32_t kt = smem_u32(stages + s * C::kStageBytes);
+    const uint32_t vt = kt + C::kTileBytes;
+
+    if (inf.flags & kFirst) {
       // query fragments (MMA B operand) of this kv head's G query heads
-      const uint16_t* qbase = p.q + ((long long)seg_b * p.Hq + (long long)seg_g * p.G) * D;
+      const uint16_t* qs = reinterpret_cast<const uint16_t*>(qslots + s * C::kQBytes);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int hh = nt * 8 + r;
-        const bool valid = hh < p.G;
-        const uint16_t* qrow = qbase + (long long)hh * D;
+        const bool hv = hh < p.G;
+        const uint16_t* qrow = qs + hh * D;
 #pragma unroll
         for (int ks = 0; ks < C::kKSteps; ++ks) {
           if constexpr (!FP8) {
-            qf[nt][ks][0] = valid ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
-            qf[nt][ks][1] = valid ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+            qf[nt][ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
+            qf[nt][ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
           } else {
             // permuted k index: step ks covers d = 16 ks + 4c + {0,1} and {2,3}
-            uint2 raw = valid ? *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c) : make_uint2(0, 0);
+            const uint2 raw = hv ? *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c) : make_uint2(0, 0);
             const float x0 = __uint_as_float(raw.x << 16), x1 = __uint_as_float(raw.x & 0xffff0000u);
             const float x2 = __uint_as_float(raw.y << 16), x3 = __uint_as_float(raw.y & 0xffff0000u);
             qf[nt][ks][0] = pack_f16(x0, x1);
@@ -446,108 +593,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    const int s = it % C::kStages;
-    const bool have = wait_bar(smem_u32(&full_bar[s]), (it / C::kStages) & 1, s_abort, status);
-    const uint32_t kt = smem_u32(stages + s * C::kStageBytes);
-    const uint32_t vt = kt + C::kTileBytes;
-    float ksc = 1.f, vsc = 1.f;
-    if constexpr (FP8) {
-      ksc = info[s].k_scale;
-      vsc = info[s].v_scale;
-    }
-    (void)have;
-
-    // ---- S^T = K_w . Q^T
-    float sacc[NT][4];
+    // ---- S^T = K_w . Q^T, four independent accumulation chains (k-step mod 4)
+    constexpr int kChains = 4;
+    float sch[kChains][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int q = 0; q < kChains; ++q)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sacc[nt][j] = 0.f;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sch[q][nt][j] = 0.f;
     if constexpr (!FP8) {
 #pragma unroll
       for (int ks = 0; ks < C::kKSteps; ++ks) {
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(tile_addr(kt, k_tok, 2 * ks + k_chk), a0, a1, a2, a3);
+        ldsm_x4(kt + koff[ks & 3] + (ks >> 2) * C::kBoxBytes, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16(sacc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+        for (int nt = 0; nt < NT; ++nt)
+          mma_bf16(sch[ks % kChains][nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
       }
     } else {
 #pragma unroll
       for (int kp = 0; kp < C::kKSteps / 2; ++kp) {
         uint32_t r0, r1, r2, r3;
-        ldsm_x4(tile_addr(kt, k_tok, 2 * kp + k_chk), r0, r1, r2, r3);
+        ldsm_x4(kt + koff[kp], r0, r1, r2, r3);
         const uint32_t a[2][4] = {
             {e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff), e4m3x2_to_f16x2(r0 >> 16),
              e4m3x2_to_f16x2(r1 >> 16)},
             {e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff), e4m3x2_to_f16x2(r2 >> 16),
              e4m3x2_to_f16x2(r3 >> 16)}};
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_f16(sacc[nt], a[h][0], a[h][1], a[h][2], a[h][3], qf[nt][2 * kp + h][0],
-                    qf[nt][2 * kp + h][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_f16(sch[(2 * kp) % kChains][nt], a[0][0], a[0][1], a[0][2], a[0][3],
+                  qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+          mma_f16(sch[(2 * kp + 1) % kChains][nt], a[1][0], a[1][1], a[1][2], a[1][3],
+                  qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+        }
       }
     }
-
-    // ---- online softmax (base 2)
-    const int valid = L - (wk.t * kPageSize + tok0);  // live tokens in this warp's slice
-    const float mul = p.scale_log2 * ksc;
-    uint32_t pb[NT][2];
+    float sacc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float s0 = sacc[nt][0] * mul, s1 = sacc[nt][1] * mul;
-      float s2 = sacc[nt][2] * mul, s3 = sacc[nt][3] * mul;
-      if (r >= valid) { s0 = -INFINITY; s1 = -INFINITY; }
-      if (r + 8 >= valid) { s2 = -INFINITY; s3 = -INFINITY; }
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 4));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 4));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 8));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 8));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 16));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 16));
-      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-      const float base0 = (mn0 == -INFINITY) ? 0.f : mn0;
-      const float base1 = (mn1 == -INFINITY) ? 0.f : mn1;
-      const float al0 = exp2f(m_run[nt][0] - base0), al1 = exp2f(m_run[nt][1] - base1);
-      const float p0 = exp2f(s0 - base0), p2 = exp2f(s2 - base0);
-      const float p1 = exp2f(s1 - base1), p3 = exp2f(s3 - base1);
-      l_run[nt][0] = l_run[nt][0] * al0 + p0 + p2;
-      l_run[nt][1] = l_run[nt][1] * al1 + p1 + p3;
-      m_run[nt][0] = mn0;
-      m_run[nt][1] = mn1;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < C::kMTiles; ++i) {
-        acc[nt][i][0] *= al0;
-        acc[nt][i][1] *= al1;
-        acc[nt][i][2] *= al0;
-        acc[nt][i][3] *= al1;
-      }
-      if constexpr (!FP8) {
-        pb[nt][0] = movm_t(pack_bf16(p0, p1));
-        pb[nt][1] = movm_t(pack_bf16(p2, p3));
-      } else {
-        pb[nt][0] = movm_t(pack_f16(p0 * vsc, p1 * vsc));
-        pb[nt][1] = movm_t(pack_f16(p2 * vsc, p3 * vsc));
-      }
-    }
+      for (int j = 0; j < 4; ++j)
+        sacc[nt][j] = (sch[0][nt][j] + sch[1][nt][j]) + (sch[2][nt][j] + sch[3][nt][j]);
 
-    // ---- O^T += V_w^T . P^T   (V rows past the length are zeroed in registers:
-    // their probabilities are 0 but the slot may hold NaN/Inf garbage)
-    const bool tail = valid < 16;
-    const uint32_t m_lo = (2 * c < valid ? 0x0000ffffu : 0u) | (2 * c + 1 < valid ? 0xffff0000u : 0u);
-    const uint32_t m_hi = (2 * c + 8 < valid ? 0x0000ffffu : 0u) | (2 * c + 9 < valid ? 0xffff0000u : 0u);
+    // V fragments now, so their shared-memory latency overlaps the softmax
     uint32_t va[C::kMTiles][4];
     if constexpr (!FP8) {
 #pragma unroll
       for (int i = 0; i < C::kMTiles; ++i)
-        ldsm_x4_t(tile_addr(vt, v_tok, 2 * i + v_chk), va[i][0], va[i][1], va[i][2], va[i][3]);
+        ldsm_x4_t(vt + voff[i & 3] + (i >> 2) * C::kBoxBytes, va[i][0], va[i][1], va[i][2], va[i][3]);
     } else {
 #pragma unroll
       for (int ip = 0; ip < C::kMTiles / 2; ++ip) {
         uint32_t r0, r1, r2, r3;
-        ldsm_x4_t(tile_addr(vt, v_tok, 2 * ip + v_chk), r0, r1, r2, r3);
+        ldsm_x4_t(vt + voff[ip], r0, r1, r2, r3);
         // r0/r1: tokens [0,8)/[8,16) of chunk 2ip; r2/r3: same for chunk 2ip+1.
         // Each holds bytes {V(t,d), V(t,d+1), V(t+1,d), V(t+1,d+1)}.
         va[2 * ip][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0020));
@@ -560,10 +660,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         va[2 * ip + 1][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0031));
       }
     }
-    // all shared-memory reads of this stage are done: hand it back
+    // all shared-memory reads of this stage are issued: hand it back
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
+
+    // ---- online softmax (base 2)
+    const int valid = inf.valid - tok0;  // live tokens in this warp's slice
+    const bool tail = valid < 16;        // warp-uniform
+    const float mul = p.scale_log2 * inf.k_scale;
+    uint32_t pb[NT][2];
+    float alpha[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float s0 = sacc[nt][0] * mul, s1 = sacc[nt][1] * mul;
+      float s2 = sacc[nt][2] * mul, s3 = sacc[nt][3] * mul;
+      if (tail) {
+        if (r >= valid) { s0 = -INFINITY; s1 = -INFINITY; }
+        if (r + 8 >= valid) { s2 = -INFINITY; s3 = -INFINITY; }
+      }
+      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 4));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 4));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 8));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 8));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 16));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 16));
+      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+      const float base0 = (mn0 == -INFINITY) ? 0.f : mn0;
+      const float base1 = (mn1 == -INFINITY) ? 0.f : mn1;
+      const float al0 = fast_exp2(m_run[nt][0] - base0), al1 = fast_exp2(m_run[nt][1] - base1);
+      const float p0 = fast_exp2(s0 - base0), p2 = fast_exp2(s2 - base0);
+      const float p1 = fast_exp2(s1 - base1), p3 = fast_exp2(s3 - base1);
+      l_run[nt][0] = l_run[nt][0] * al0 + p0 + p2;
+      l_run[nt][1] = l_run[nt][1] * al1 + p1 + p3;
+      m_run[nt][0] = mn0;
+      m_run[nt][1] = mn1;
+      alpha[nt][0] = al0;
+      alpha[nt][1] = al1;
+      if constexpr (!FP8) {
+        pb[nt][0] = movm_t(pack_bf16(p0, p1));
+        pb[nt][1] = movm_t(pack_bf16(p2, p3));
+      } else {
+        const float vsc = inf.v_scale;
+        pb[nt][0] = movm_t(pack_f16(p0 * vsc, p1 * vsc));
+        pb[nt][1] = movm_t(pack_f16(p2 * vsc, p3 * vsc));
+      }
+    }
+    // Rescale the accumulators only if some running max moved (once the
+    // maxima settle, almost no tile needs it).
+    bool moved = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) moved |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < C::kMTiles; ++i) {
+          acc[nt][i][0] *= alpha[nt][0];
+          acc[nt][i][1] *= alpha[nt][1];
+          acc[nt][i][2] *= alpha[nt][0];
+          acc[nt][i][3] *= alpha[nt][1];
+        }
+    }
+
+    // ---- O^T += V_w^T . P^T   (V rows past the length are zeroed in registers:
+    // their probabilities are 0 but the slot may hold NaN/Inf garbage)
     if (tail) {
+      const uint32_t m_lo = (2 * c < valid ? 0x0000ffffu : 0u) | (2 * c + 1 < valid ? 0xffff0000u : 0u);
+      const uint32_t m_hi = (2 * c + 8 < valid ? 0x0000ffffu : 0u) | (2 * c + 9 < valid ? 0xffff0000u : 0u);
 #pragma unroll
       for (int i = 0; i < C::kMTiles; ++i) {
         va[i][0] &= m_lo;
@@ -580,9 +744,102 @@ __global__ void __launch_bounds__(kThreads, 1)
         else mma_f16(acc[nt][i], va[i][0], va[i][1], va[i][2], va[i][3], pb[nt][0], pb[nt][1]);
       }
 
-    if (u + 1 < ue) wk.next(ts, p.Hkv);
+    if (inf.flags & kLast) deposit(&inf);
   }
-  if (seg_b >= 0) finish_segment(seg_b, seg_g, split_idx);
+  deposit(nullptr);  // tells the epilogue warp that this CTA is done
+}
+
+
+// ---------------------------------------------------------------------------
+// Split merge: for every segment with more than one split, the log-sum-exp
+// combination of its partials in split order,
+//   M = max_i m_i,  Lambda = sum_i l_i 2^(m_i - M),  o = sum_i acc_i 2^(m_i - M) / Lambda
+// (m in log2 units).  One CTA per (segment, head) -- grid-stride -- and one
+// thread per output element: the CTA stages the head's (m, l) of all splits
+// in shared memory in one pass, forms the weights with warp reductions, and
+// every thread then loads its element of each split's partial in batches of
+// independent loads, so the merge costs a few L2 round trips.
+// ---------------------------------------------------------------------------
+constexpr int kMergeBatch = 32;   // splits whose partial values are loaded together
+
+// L2-only load kept in program order (the batch below is issued before any
+// of its values is used).
+__device__ __forceinline__ float ld_cg(const float* p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+constexpr int kMergeStage = 1024; // (m, l) pairs staged per pass
+
+struct MergeParams {
+  Ws ws;
+  void* out;
+  int S, Hkv, G, Hq, slots;  // slots = 2 * V partial slots in the workspace
+};
+
+template <int D, bool OUT_F32>
+__global__ void __launch_bounds__(D) merge_kernel(const MergeParams p) {
+  __shared__ float s_w[kMergeStage];  // weights 2^(m_i - M) of the staged splits
+  __shared__ float s_red[2][D / 32];
+  pdl_wait();                         // the partials of the decode kernel
+  const int G = p.G;
+  const int d = threadIdx.x, warp = d >> 5, lane = d & 31;
+  for (int job = blockIdx.x; job < p.S * G; job += gridDim.x) {
+    const int s = job / G, h = job - s * G;
+    const int ns = p.ws.split_count[s];
+    if (ns <= 1) continue;
+    const int base = p.ws.part_base[s];
+    if (base < 0 || base + ns > p.slots) {
+      if (d == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
+      continue;
+    }
+    const float2* ml = p.ws.part_ml + (long long)base * G + h;
+    const float* acc = p.ws.part_acc + (long long)base * G * D + (long long)h * D + d;
+    // 1. the head's maximum over all splits
+    float M = -INFINITY;
+    for (int i = d; i < ns; i += D) M = fmaxf(M, __ldcg(&ml[(long long)i * G]).x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) s_red[0][warp] = M;
+    __syncthreads();
+    M = s_red[0][0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_red[0][w]);
+    // 2. weights (staged) and the weighted sum of the l's; 3. weighted partials
+    float lam = 0.f, o = 0.f;
+    for (int i0 = 0; i0 < ns; i0 += kMergeStage) {
+      const int n = min(kMergeStage, ns - i0);
+      __syncthreads();
+      for (int i = d; i < n; i += D) {
+        const float2 v = __ldcg(&ml[(long long)(i0 + i) * G]);
+        const float w = (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - M);
+        s_w[i] = w;
+        lam += v.y * w;
+      }
+      __syncthreads();
+      for (int j0 = 0; j0 < n; j0 += kMergeBatch) {
+        float a[kMergeBatch];
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j)
+          a[j] = (j0 + j < n) ? ld_cg(acc + (long long)(i0 + j0 + j) * G * D) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j)
+          if (j0 + j < n) o += a[j] * s_w[j0 + j];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lam += __shfl_xor_sync(0xffffffffu, lam, off);
+    __syncthreads();
+    if (lane == 0) s_red[1][warp] = lam;
+    __syncthreads();
+    lam = 0.f;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) lam += s_red[1][w];
+    const int b = s / p.Hkv, g = s - b * p.Hkv;
+    store_out<OUT_F32>(p.out, ((long long)b * p.Hq + (long long)g * G + h) * D + d, o / lam);
+    __syncthreads();  // s_red / s_w are reused by the next job
+  }
+  pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -624,11 +881,11 @@ bool make_cache_map(CUtensorMap* tm, const void* base, int num_pages, int Hkv, i
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int NT, bool FP8, bool OUT_F32>
+template <int D, int NT, bool FP8, bool OUT_F32, int CPS>
 hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams& p, int grid,
                   cudaStream_t stream) {
-  using C = Cfg<D, NT, FP8>;
-  auto kern = decode_kernel<D, NT, FP8, OUT_F32>;
+  using C = Cfg<D, NT, FP8, CPS>;
+  auto kern = decode_kernel<D, NT, FP8, OUT_F32, CPS>;
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<uint64_t> ready_mask{0};
   int dev = 0;
@@ -664,11 +921,31 @@ hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams&
   return HPA_OK;
 }
 
+// One persistent CTA per SM when the grid fits the SMs; two co-resident
+// (smaller) CTAs per SM when the grid is larger, so that twice as many
+// consumer warps hide each other's latencies.
 template <int D, bool FP8, bool OUT_F32>
-hpa_status launch_nt(int nt, const CUtensorMap& tk, const CUtensorMap& tv, const RunParams& p,
-                     int grid, cudaStream_t s) {
-  return nt == 1 ? launch<D, 1, FP8, OUT_F32>(tk, tv, p, grid, s)
-                 : launch<D, 2, FP8, OUT_F32>(tk, tv, p, grid, s);
+hpa_status launch_nt(int nt, int cps, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const RunParams& p, int grid, cudaStream_t s) {
+  if (cps == 1)
+    return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1>(tk, tv, p, grid, s)
+                   : launch<D, 2, FP8, OUT_F32, 1>(tk, tv, p, grid, s);
+  // G = 16 (two n-tiles) does not fit two CTAs per SM: it always runs one
+  return nt == 1 ? launch<D, 1, FP8, OUT_F32, 2>(tk, tv, p, grid, s)
+                 : launch<D, 2, FP8, OUT_F32, 1>(tk, tv, p, grid, s);
+}
+
+// Cached SM count of the current device (0 if unknown).
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = cache[dev].load();
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(n);
+  }
+  return n;
 }
 
 }  // namespace
@@ -682,7 +959,8 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
                                      int pt_stride, int num_pages, void* out,
                                      hpa_out_dtype out_dtype, int batch, int num_q_heads,
                                      int num_kv_heads, int head_dim, float softmax_scale,
-                                     int grid, void* workspace, size_t ws_bytes, void* stream) {
+                                     hpa_plan_kind kind, int grid, void* workspace,
+                                     size_t ws_bytes, void* stream) {
   if (!q || !k_cache || !v_cache || !page_table || !out || !workspace) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || pt_stride <= 0 || num_pages <= 0 ||
       grid <= 0)
@@ -700,10 +978,11 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
   if ((long long)num_pages * num_kv_heads * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15)
     return HPA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) & 7) || (reinterpret_cast<uintptr_t>(out) & 3))
+  if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 3))
     return HPA_ERR_INVALID_ARG;
   WsLayout L;
-  if (!ws_layout(batch, num_kv_heads, num_q_heads, head_dim, grid, &L)) return HPA_ERR_INVALID_ARG;
+  if (!ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, &L))
+    return HPA_ERR_INVALID_ARG;
   if (ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return HPA_ERR_WORKSPACE;
 
   CUtensorMap tk, tv;
@@ -727,15 +1006,53 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.ws = ws_view(workspace, L);
   p.grid = grid;
+  p.kind = kind;
+  p.slots = (int)(2 * plan_ranges_ll(kind, grid));
   const int nt = G > 8 ? 2 : 1;
+  const int sms = sm_count();
+  const int cps = (sms > 0 && grid > sms) ? 2 : 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool f32 = out_dtype == HPA_OUT_F32;
+  hpa_status st;
   if (fp8)
-    return f32 ? launch_nt<128, true, true>(nt, tk, tv, p, grid, s)
-               : launch_nt<128, true, false>(nt, tk, tv, p, grid, s);
+    st = f32 ? launch_nt<128, true, true>(nt, cps, tk, tv, p, grid, s)
+             : launch_nt<128, true, false>(nt, cps, tk, tv, p, grid, s);
+  else if (head_dim == 128)
+    st = f32 ? launch_nt<128, false, true>(nt, cps, tk, tv, p, grid, s)
+             : launch_nt<128, false, false>(nt, cps, tk, tv, p, grid, s);
+  else
+    st = f32 ? launch_nt<64, false, true>(nt, cps, tk, tv, p, grid, s)
+             : launch_nt<64, false, false>(nt, cps, tk, tv, p, grid, s);
+  if (st != HPA_OK) return st;
+
+  // split merge, chained behind the decode kernel
+  MergeParams mp;
+  mp.ws = p.ws;
+  mp.out = out;
+  mp.S = batch * num_kv_heads;
+  mp.Hkv = num_kv_heads;
+  mp.G = G;
+  mp.Hq = num_q_heads;
+  mp.slots = (int)(2 * plan_ranges_ll(kind, grid));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min<long long>((long long)mp.S * G, (long long)std::max(1, sms) * 16));
+  cfg.blockDim = dim3(head_dim);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (head_dim == 128)
-    return f32 ? launch_nt<128, false, true>(nt, tk, tv, p, grid, s)
-               : launch_nt<128, false, false>(nt, tk, tv, p, grid, s);
-  return f32 ? launch_nt<64, false, true>(nt, tk, tv, p, grid, s)
-             : launch_nt<64, false, false>(nt, tk, tv, p, grid, s);
+    e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<128, true>, mp)
+            : cudaLaunchKernelEx(&cfg, merge_kernel<128, false>, mp);
+  else
+    e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<64, true>, mp)
+            : cudaLaunchKernelEx(&cfg, merge_kernel<64, false>, mp);
+  if (e != cudaSuccess) {
+    set_cuda_error(e, "hpa_decode_run merge launch");
+    return HPA_ERR_CUDA;
+  }
+  return HPA_OK;
 }

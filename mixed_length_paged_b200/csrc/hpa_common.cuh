@@ -12,6 +12,7 @@
 namespace hpa {
 
 constexpr int kPageSize = 64;            // tokens per page == tokens per tile
+constexpr int kMaxPlanBatch = 32768;     // sequences per plan (tile offsets live in shared memory)
 constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 
 // ---------------------------------------------------------------------------
@@ -19,39 +20,60 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 //   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T
 //   lens        int32[B]     clamped lengths
 //   tile_start  int32[B+1]   exclusive prefix sum of tiles per sequence
-//   cta_desc    int4[grid]   (u_begin, u_end, first_split, 0)
+//   cta_desc    int4[2*V]    per virtual range v: (u_begin, u_end,
+//                            first_split, b0), (g0, t0, n0, 0): the unit
+//                            range, the split index of its first segment, and
+//                            the (sequence, kv head, tile, tiles of that
+//                            sequence) of its first unit.  V = grid for the
+//                            static plans; for the dynamic plan V <= 5 * grid
+//                            (grid primary ranges, then the tail chunks).
 //   split_count int32[B*Hkv]
 //   part_base   int32[B*Hkv]
-//   arrive      int32[B*Hkv] arrival counters of the split merge
 //   part_ml     float2[2*grid][G]     (m, l) of each partial, log2 units
 //   part_acc    float[2*grid][G][D]   un-normalised partial outputs
-// A plan of `grid` CTAs has at most 2*(grid-1) partials (each CTA boundary
-// cuts at most one segment), so 2*grid slots always suffice.
+// V contiguous ranges have at most 2*(V-1) partials (each range boundary
+// cuts at most one segment), so 2*V slots always suffice.
 // ---------------------------------------------------------------------------
 enum HeaderField {
   kHdrMagic = 0, kHdrStatus = 1, kHdrUnits = 2, kHdrGrid = 3, kHdrKind = 4,
   kHdrBatch = 5, kHdrKvHeads = 6, kHdrGroup = 7, kHdrHeadDim = 8, kHdrTiles = 9,
+  kHdrRanges = 10,  // virtual ranges V (grid for static plans)
+  kHdrNext = 11,    // dynamic plan: next tail chunk to hand out (run-time counter)
   kHdrWords = 16
 };
 
+// The dynamic plan gives each of its P persistent CTAs one primary range and
+// hands out up to kTailChunksPerCta * P tail chunks at run time.
+constexpr int kTailChunksPerCta = 4;
+constexpr int kTailFractionDiv = 8;  // the tail holds floor(U / 8) units (fewer if U is small)
+
+// Virtual ranges a plan of this kind and grid can describe.
+#if defined(__CUDACC__)
+__host__ __device__
+#endif
+inline long long plan_ranges_ll(int kind, int grid) {
+  return kind == HPA_PLAN_DYNAMIC ? (long long)grid * (1 + kTailChunksPerCta) : grid;
+}
+
 struct WsLayout {
-  size_t header, lens, tile_start, cta_desc, split_count, part_base, arrive, part_ml, part_acc,
-      total;
+  size_t header, lens, tile_start, cta_desc, split_count, part_base, part_ml, part_acc, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline bool ws_layout(int B, int Hkv, int Hq, int D, int grid, WsLayout* L) {
+inline bool ws_layout(int kind, int B, int Hkv, int Hq, int D, int grid, WsLayout* L) {
   if (B <= 0 || Hkv <= 0 || Hq <= 0 || D <= 0 || grid <= 0 || Hq % Hkv) return false;
-  const size_t G = size_t(Hq / Hkv), S = size_t(B) * Hkv, slots = 2 * size_t(grid);
+  if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK)
+    return false;
+  const size_t V = size_t(plan_ranges_ll(kind, grid));
+  const size_t G = size_t(Hq / Hkv), S = size_t(B) * Hkv, slots = 2 * V;
   size_t off = 0;
   L->header = off;      off = align256(off + kHdrWords * 4);
   L->lens = off;        off = align256(off + size_t(B) * 4);
   L->tile_start = off;  off = align256(off + (size_t(B) + 1) * 4);
-  L->cta_desc = off;    off = align256(off + size_t(grid) * 16);
+  L->cta_desc = off;    off = align256(off + V * 32);
   L->split_count = off; off = align256(off + S * 4);
   L->part_base = off;   off = align256(off + S * 4);
-  L->arrive = off;      off = align256(off + S * 4);
   L->part_ml = off;     off = align256(off + slots * G * 8);
   L->part_acc = off;    off = align256(off + slots * G * size_t(D) * 4);
   L->total = off;
@@ -66,7 +88,6 @@ struct Ws {
   int4* cta_desc;
   int32_t* split_count;
   int32_t* part_base;
-  int32_t* arrive;
   float2* part_ml;
   float* part_acc;
 };
@@ -76,8 +97,8 @@ inline Ws ws_view(void* base, const WsLayout& L) {
   return Ws{reinterpret_cast<int32_t*>(p + L.header), reinterpret_cast<int32_t*>(p + L.lens),
             reinterpret_cast<int32_t*>(p + L.tile_start), reinterpret_cast<int4*>(p + L.cta_desc),
             reinterpret_cast<int32_t*>(p + L.split_count),
-            reinterpret_cast<int32_t*>(p + L.part_base), reinterpret_cast<int32_t*>(p + L.arrive),
-            reinterpret_cast<float2*>(p + L.part_ml), reinterpret_cast<float*>(p + L.part_acc)};
+            reinterpret_cast<int32_t*>(p + L.part_base), reinterpret_cast<float2*>(p + L.part_ml),
+            reinterpret_cast<float*>(p + L.part_acc)};
 }
 
 // Host-side grid of a plan (must equal the oracle's definition; see hpa.h).
@@ -149,12 +170,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` polls (each try_wait itself suspends
-// for a hardware-defined interval) and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm) {

@@ -88,7 +88,7 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
   if (!(softmax_scale > 0.f) || softmax_scale == INFINITY) return HPA_ERR_INVALID_ARG;
   if (kv_dtype == HPA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return HPA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15 ||
-      (reinterpret_cast<uintptr_t>(q) & 7) || (reinterpret_cast<uintptr_t>(out) & 3))
+      (reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 3))
     return HPA_ERR_INVALID_ARG;
   {
     const int G = num_q_heads / num_kv_heads;
@@ -101,7 +101,8 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
   // any CUDA call.
   if (num_ctas > 0) {
     const size_t need =
-        hpa_decode_workspace_size(batch, num_kv_heads, num_q_heads, head_dim, num_ctas);
+        hpa_decode_workspace_size(HPA_PLAN_DYNAMIC, batch, num_kv_heads, num_q_heads, head_dim,
+                                  num_ctas);
     if (need == 0) return HPA_ERR_INVALID_ARG;
     if (need > HPA_NOALLOC_SCRATCH_BYTES) return HPA_ERR_WORKSPACE;
   }
@@ -110,7 +111,8 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
   hpa_status st = device_setup(&dev, &scratch, &sms);
   if (st != HPA_OK) return st;
   const int ctas = num_ctas > 0 ? num_ctas : sms;
-  const size_t need = hpa_decode_workspace_size(batch, num_kv_heads, num_q_heads, head_dim, ctas);
+  const size_t need = hpa_decode_workspace_size(HPA_PLAN_DYNAMIC, batch, num_kv_heads, num_q_heads,
+                                                head_dim, ctas);
   if (need == 0) return HPA_ERR_INVALID_ARG;
   if (need > HPA_NOALLOC_SCRATCH_BYTES) return HPA_ERR_WORKSPACE;
   int grid = 0;
@@ -120,5 +122,6 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
   if (st != HPA_OK) return st;
   return hpa_decode_run(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
                         num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
-                        softmax_scale, grid, scratch, HPA_NOALLOC_SCRATCH_BYTES, stream);
+                        softmax_scale, HPA_PLAN_DYNAMIC, grid, scratch,
+                        HPA_NOALLOC_SCRATCH_BYTES, stream);
 }

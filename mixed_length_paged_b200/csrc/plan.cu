@@ -11,7 +11,18 @@
 // One CTA of 1024 threads builds the whole plan on the device from the
 // device-side lengths, so a decode step needs no host round trip.  Units are
 // (sequence b, kv head g, tile t) in that order; segment s = b * Hkv + g.
+//
+// The dynamic plan is a contiguous partition of the unit list into ranges:
+// one primary range per persistent CTA over the first ~7/8 of the units, then
+// small tail chunks that CTAs take at run time, in order, as they finish
+// (bitbyai.com "vLLM x HPC-Ops", Attention Backend: the scheduler evaluates
+// progress dynamically).  SMs do not all get the same share of HBM
+// bandwidth, so equal static ranges would finish at different times; the
+// tail evens that out.  The partition itself is fixed by the plan, so the
+// split partials and their merge order -- and hence the result -- do not
+// depend on which CTA ends up running a chunk.
 #include <algorithm>
+#include <atomic>
 
 #include "hpa_common.cuh"
 
@@ -30,6 +41,7 @@ struct PlanParams {
 
 // Exclusive block-wide prefix sum of one int per thread; *total gets the sum.
 __device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+  constexpr int kWarps = kPlanThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -40,7 +52,7 @@ __device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
   if (lane == 31) s_warp[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < (kPlanThreads / 32) ? s_warp[lane] : 0;
+    int w = lane < kWarps ? s_warp[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -50,7 +62,7 @@ __device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
   }
   __syncthreads();
   const int before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
-  *total = s_warp[kPlanThreads / 32 - 1];
+  *total = s_warp[kWarps - 1];
   __syncthreads();
   return before;
 }
@@ -65,15 +77,52 @@ __device__ int seq_of_unit(const int32_t* tile_start, int B, int Hkv, long long 
   return lo;
 }
 
-// Dynamic plan: CTA holding unit u when U units are spread over P CTAs as
-// [floor(cU/P), floor((c+1)U/P)):  the largest c with floor(cU/P) <= u.
-__device__ __forceinline__ long long cta_of(long long u, long long U, long long P) {
-  return ((u + 1) * P - 1) / U;
-}
+// floor(a / b) for 0 <= a < 2^50 and a fixed divisor 0 < b < 2^31: the fp64
+// product with a precomputed reciprocal is within one of the quotient, and
+// one integer check each way makes it exact.  (Much cheaper than a 64-bit
+// integer division or an IEEE fp64 division per call.)
+struct FloorDiv {
+  long long b;
+  double inv;
+  __device__ void init(long long d, double reciprocal) {
+    b = d;
+    inv = reciprocal;
+  }
+  __device__ __forceinline__ long long operator()(long long a) const {
+    long long q = (long long)((double)a * inv);
+    if (q * b > a) --q;
+    else if ((q + 1) * b <= a) ++q;
+    return q;
+  }
+};
+
+// Dynamic plan geometry.  P persistent CTAs; U units.  If U <= P each active
+// CTA takes one unit.  Otherwise the first U1 = U - Ut units are spread over
+// the P primary ranges and the last Ut = min(floor(U/8), U - P) units over M =
+// min(4P, Ut) tail chunks, handed out at run time to whichever CTA is free.
+// For n units spread over m ranges as [floor(cn/m), floor((c+1)n/m)), the
+// range holding unit u is the largest c with floor(cn/m) <= u, i.e.
+// floor(((u+1)m - 1) / n).
+struct DynGeom {
+  long long U, P, Pd, U1, Ut, M;
+  FloorDiv by_Pd, by_M, by_U1, by_Ut;
+  // r[0..3]: reciprocals of Pd, M, U1, Ut (0 for a zero divisor)
+  __device__ void init_div(const double* r) {
+    by_Pd.init(Pd, r[0]);
+    by_M.init(M, r[1]);
+    by_U1.init(U1, r[2]);
+    by_Ut.init(Ut, r[3]);
+  }
+  __device__ long long range_of(long long u) const {
+    return u < U1 ? by_U1((u + 1) * Pd - 1) : P + by_Ut((u - U1 + 1) * M - 1);
+  }
+};
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
+  extern __shared__ int32_t ts[];  // tile_start[0..B], in shared memory
   __shared__ int s_warp[32];
   __shared__ int s_status;
+  __shared__ double s_recip[4];
   // The previous step's run kernel may still be reading this workspace.
   pdl_wait();
   const int tid = threadIdx.x;
@@ -94,51 +143,83 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     }
     int total;
     const int before = block_exclusive_scan(n, s_warp, &total);
-    if (b < p.B) p.ws.tile_start[b] = carry + before;
+    if (b < p.B) ts[b] = carry + before;
     carry += total;
   }
-  if (tid == 0) p.ws.tile_start[p.B] = carry;
-  __syncthreads();  // tile_start / lens visible block-wide
+  if (tid == 0) ts[p.B] = carry;
+  __syncthreads();
+  for (int i = tid; i <= p.B; i += kPlanThreads) p.ws.tile_start[i] = ts[i];
 
-  const int32_t* ts = p.ws.tile_start;
   const long long T = carry;
   const long long U = T * p.Hkv;
   const int S = p.B * p.Hkv;
-  const long long Pd = std::min<long long>(p.num_ctas, U);  // dynamic: active CTAs
   const int per = (p.kind == HPA_PLAN_DYNAMIC) ? 0 : p.grid / S;  // static: CTAs per segment
+  DynGeom dg;
+  dg.U = U;
+  dg.P = p.num_ctas;
+  if (U <= dg.P) {
+    dg.Pd = U; dg.U1 = U; dg.Ut = 0; dg.M = 0;
+  } else {
+    dg.Pd = dg.P;
+    dg.Ut = std::min<long long>(U / kTailFractionDiv, U - dg.P);
+    dg.U1 = U - dg.Ut;
+    dg.M = std::min<long long>((long long)kTailChunksPerCta * dg.P, dg.Ut);
+  }
+  // the four reciprocals, computed once for the whole CTA
+  if (tid < 4) {
+    const long long d = tid == 0 ? dg.Pd : tid == 1 ? dg.M : tid == 2 ? dg.U1 : dg.Ut;
+    s_recip[tid] = d > 0 ? 1.0 / (double)d : 0.0;
+  }
+  __syncthreads();
+  dg.init_div(s_recip);
+  const long long V = (p.kind == HPA_PLAN_DYNAMIC) ? dg.P + dg.M : p.grid;
 
-  // 2. per-CTA unit ranges and first-split indices
-  for (int c = tid; c < p.grid; c += kPlanThreads) {
+  // 2. per-range unit ranges, first-split indices and start states
+  for (int c = tid; c < V; c += kPlanThreads) {
     long long ub, ue;
-    int first = 0;
+    int first = 0, b0 = 0, g0 = 0, t0 = 0, n0 = 0;
     if (p.kind == HPA_PLAN_DYNAMIC) {
-      if (c < Pd) {
-        ub = (long long)c * U / Pd;
-        ue = (long long)(c + 1) * U / Pd;
-        const int b = seq_of_unit(ts, p.B, p.Hkv, ub);
-        const long long n = ts[b + 1] - ts[b];
-        const long long g = (ub - (long long)ts[b] * p.Hkv) / n;
-        const long long seg_start = (long long)ts[b] * p.Hkv + g * n;
-        first = (int)(c - cta_of(seg_start, U, Pd));
+      if (c < dg.P) {
+        if (c < dg.Pd) {
+          ub = dg.by_Pd((long long)c * dg.U1);
+          ue = dg.by_Pd((long long)(c + 1) * dg.U1);
+        } else {
+          ub = ue = U;
+        }
       } else {
-        ub = ue = U;
+        const long long j = c - dg.P;
+        ub = dg.U1 + dg.by_M(j * dg.Ut);
+        ue = dg.U1 + dg.by_M((j + 1) * dg.Ut);
+      }
+      if (ub < ue) {
+        b0 = seq_of_unit(ts, p.B, p.Hkv, ub);
+        n0 = ts[b0 + 1] - ts[b0];
+        const int rem = (int)(ub - (long long)ts[b0] * p.Hkv);  // < Hkv * n0 < 2^31
+        g0 = rem / n0;
+        t0 = rem - g0 * n0;
+        const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n0;
+        first = (int)(c - dg.range_of(seg_start));
       }
     } else {
       const int s = c / per, i = c % per;
-      const int b = s / p.Hkv, g = s % p.Hkv;
-      const long long n = ts[b + 1] - ts[b];
+      b0 = s / p.Hkv;
+      g0 = s % p.Hkv;
+      const long long n = ts[b0 + 1] - ts[b0];
       const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
-      const long long t0 = std::min<long long>((long long)i * C, n);
-      const long long t1 = std::min<long long>((long long)(i + 1) * C, n);
-      const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
-      ub = seg_start + t0;
-      ue = seg_start + t1;
-      first = t0 < t1 ? i : 0;
+      const long long c0 = std::min<long long>((long long)i * C, n);
+      const long long c1 = std::min<long long>((long long)(i + 1) * C, n);
+      const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n;
+      ub = seg_start + c0;
+      ue = seg_start + c1;
+      first = c0 < c1 ? i : 0;
+      t0 = (int)c0;
+      n0 = (int)n;
     }
-    p.ws.cta_desc[c] = make_int4((int)ub, (int)ue, first, 0);
+    p.ws.cta_desc[2 * c] = make_int4((int)ub, (int)ue, first, b0);
+    p.ws.cta_desc[2 * c + 1] = make_int4(g0, t0, n0, 0);
   }
 
-  // 3. split counts, partial slot bases, zeroed arrival counters
+  // 3. split counts and partial slot bases
   int pcarry = 0;
   for (int base = 0; base < S; base += kPlanThreads) {
     const int s = base + tid;
@@ -149,14 +230,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
       if (n > 0) {
         if (p.kind == HPA_PLAN_DYNAMIC) {
           const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
-          split = (int)(cta_of(seg_start + n - 1, U, Pd) - cta_of(seg_start, U, Pd) + 1);
+          split = (int)(dg.range_of(seg_start + n - 1) - dg.range_of(seg_start) + 1);
         } else {
           const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
           split = (int)((n + C - 1) / C);
         }
       }
       p.ws.split_count[s] = split;
-      p.ws.arrive[s] = 0;
     }
     int total;
     const int before = block_exclusive_scan(split > 1 ? split : 0, s_warp, &total);
@@ -164,7 +244,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     pcarry += total;
   }
 
-  __syncthreads();
   if (tid == 0) {
     int32_t* h = p.ws.header;
     h[kHdrStatus] = s_status;
@@ -176,6 +255,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrGroup] = p.G;
     h[kHdrHeadDim] = p.D;
     h[kHdrTiles] = (int32_t)T;
+    h[kHdrRanges] = (int32_t)V;
+    h[kHdrNext] = 0;
     __threadfence();
     h[kHdrMagic] = kPlanMagic;
   }
@@ -207,6 +288,9 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
   if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK)
     return HPA_ERR_INVALID_ARG;
   if ((long long)pt_stride * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
+  if (batch > kMaxPlanBatch) return HPA_ERR_UNSUPPORTED;
+  // the dynamic plan's range arithmetic keeps products below 2^50
+  if (kind == HPA_PLAN_DYNAMIC && num_ctas > 65536) return HPA_ERR_UNSUPPORTED;
   long long chunk = 0;
   const long long grid =
       plan_grid_ll(kind, batch, num_kv_heads, num_ctas, param, max_seq_len, &chunk);
@@ -214,7 +298,7 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
   // Units are indexed with int32 in the plan: bound the worst case.
   if ((long long)batch * pt_stride * num_kv_heads > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
   WsLayout L;
-  if (!ws_layout(batch, num_kv_heads, num_q_heads, head_dim, (int)grid, &L))
+  if (!ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, (int)grid, &L))
     return HPA_ERR_INVALID_ARG;
   if (ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return HPA_ERR_WORKSPACE;
 
@@ -231,10 +315,28 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
   p.chunk = chunk;
   p.ws = ws_view(workspace, L);
 
+  const size_t smem = (size_t(batch) + 1) * sizeof(int32_t);
+  if (smem > 48 * 1024) {
+    // tile offsets above 48 KiB of shared memory need the opt-in, once per device
+    static std::atomic<uint64_t> ready_mask{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    const uint64_t bit = (e == cudaSuccess && dev < 64) ? (1ull << dev) : 0;
+    if (!bit || !(ready_mask.load() & bit)) {
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)((size_t(kMaxPlanBatch) + 1) * sizeof(int32_t)));
+      if (e != cudaSuccess) {
+        set_cuda_error(e, "hpa_decode_plan smem attribute");
+        return HPA_ERR_CUDA;
+      }
+      ready_mask.fetch_or(bit);
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(kPlanThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -50,6 +50,9 @@ SHAPES = {
     "tiny": DecodeShape("tiny", 8, 2, 64),
     "uniform": DecodeShape("uniform", 64, 8, 128),
     "skewed": DecodeShape("skewed", 64, 8, 128),
+    # the skewed shape at a quarter of the lengths (264 MB of KV, above the
+    # 126 MB L2): the size used for detailed profiler captures
+    "skewed_quarter": DecodeShape("skewed_quarter", 64, 8, 128),
     "mix_prologue": DecodeShape("mix_prologue", 32, 8, 128, prologue=True),
     "fp8": DecodeShape("fp8", 64, 8, 128, kv_dtype="fp8_e4m3"),
 }
@@ -69,6 +72,8 @@ def cache_lengths(name: str, seed: int = 0) -> np.ndarray:
         return np.full(64, 512, dtype=np.int64)
     if name == "skewed":
         return np.array([131072] + [4096] * 31, dtype=np.int64)
+    if name == "skewed_quarter":
+        return np.array([32768] + [1024] * 31, dtype=np.int64)
     if name == "mix_prologue":
         u = rng.uniform(math.log(256.0), math.log(65536.0), size=128)
         return np.rint(np.exp(u)).astype(np.int64)

@@ -394,9 +394,15 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  * orders units by b, then g, then t.  A "segment" is the run of units of one
  * (b, g).  Three plans give every CTA a contiguous range of that list:
  *
- *   kind 0, dynamic: U units spread as evenly as possible over
- *     P' = min(P, U) CTAs, CTA c taking [floor(c U / P'), floor((c+1) U / P'));
- *     CTAs c >= P' take nothing.  Grid = P.
+ *   kind 0, dynamic: P persistent CTAs.  If U <= P, CTA c < U takes unit c
+ *     and the rest take nothing.  Otherwise the last Ut = min(floor(U/8),
+ *     U - P) units form M = min(4P, Ut) tail chunks and the first
+ *     U1 = U - Ut units P primary ranges, each spread as evenly as possible:
+ *     range c < P is [floor(c U1 / P), floor((c+1) U1 / P)), range P + j is
+ *     [U1 + floor(j Ut / M), U1 + floor((j+1) Ut / M)).  CTA c runs range c,
+ *     then whichever tail chunks it takes at run time (bitbyai.com "vLLM x
+ *     HPC-Ops", Attention Backend: progress is evaluated dynamically).
+ *     Grid = P; V = P + M ranges.
  *   kind 1, static fixed split count S (param, default ceil(P / (B Hkv))):
  *     one CTA per (segment, split i); each segment's n tiles cut into
  *     chunks of ceil(n / S) tiles, chunk i = [i C, min((i+1) C, n)).
@@ -407,11 +413,12 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  *     sequence were the longest; chunk i = [i C, min((i+1) C, n)), empty past
  *     the segment's end.  Grid = B * Hkv * NC.
  *
- * For each CTA the plan records (u_begin, u_end, first_split): first_split is
- * the index, among the CTAs holding units of the CTA's first segment, of this
- * CTA (0 if the segment starts in this CTA).  For each segment it records
- * split_count (CTAs holding its units) and partial_base (exclusive prefix sum
- * over segments of split_count, counting only segments with split_count > 1).
+ * For each range the plan records (u_begin, u_end, first_split): first_split
+ * is the index, among the ranges holding units of the range's first segment,
+ * of this range (0 if the segment starts in it).  For each segment it records
+ * split_count (ranges holding its units) and partial_base (exclusive prefix
+ * sum over segments of split_count, counting only segments with
+ * split_count > 1).  The static kinds have one range per CTA (V = grid).
  *
  * This implementation enumerates every unit explicitly and assigns it, then
  * counts; it does not use any closed form.
@@ -435,9 +442,9 @@ long oracle_plan_grid(int kind, int B, int Hkv, int num_ctas, int param, int max
 
 int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capacity_tokens,
                 int kind, int num_ctas, int param, int max_seq_len, int32_t* lens_out,
-                int32_t* tile_start, int32_t* cta_desc /* [grid][3] */,
+                int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][3] */,
                 int32_t* split_count /* [B*Hkv] */, int32_t* partial_base /* [B*Hkv] */,
-                int32_t* n_units_out) {
+                int32_t* n_units_out, int32_t* n_ranges_out) {
   if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 2)
     return ORC_BAD_ARG;
   long grid = oracle_plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len, page_size);
@@ -469,18 +476,30 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
         ++u;
       }
     }
-  /* 3. per-CTA ranges */
-  long* beg = malloc(sizeof(long) * grid);
-  long* end = malloc(sizeof(long) * grid);
+  /* 3. ranges */
+  long nranges = grid;
+  long* beg = malloc(sizeof(long) * grid * 5);
+  long* end = malloc(sizeof(long) * grid * 5);
   if (kind == 0) {
-    long P = num_ctas < U ? num_ctas : U;
-    for (long c = 0; c < grid; ++c) {
-      if (c < P) {
-        beg[c] = c * U / P;
-        end[c] = (c + 1) * U / P;
-      } else {
-        beg[c] = end[c] = U;
+    long P = num_ctas;
+    if (U <= P) {
+      for (long c = 0; c < P; ++c) {
+        beg[c] = c < U ? c : U;
+        end[c] = c < U ? c + 1 : U;
       }
+    } else {
+      long Ut = U / 8 < U - P ? U / 8 : U - P;
+      long U1 = U - Ut;
+      long M = 4 * P < Ut ? 4 * P : Ut;
+      for (long c = 0; c < P; ++c) {
+        beg[c] = c * U1 / P;
+        end[c] = (c + 1) * U1 / P;
+      }
+      for (long j = 0; j < M; ++j) {
+        beg[P + j] = U1 + j * Ut / M;
+        end[P + j] = U1 + (j + 1) * Ut / M;
+      }
+      nranges = P + M;
     }
   } else {
     long per = grid / S; /* chunks reserved per segment */
@@ -505,10 +524,10 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
       }
     }
   }
-  /* 4. walk each CTA's units: count the CTAs holding each segment, and the
-   *    split index of each CTA within its first segment */
+  /* 4. walk each range's units: count the ranges holding each segment, and
+   *    the split index of each range within its first segment */
   int32_t* holders = calloc(S, sizeof(int32_t));
-  for (long c = 0; c < grid; ++c) {
+  for (long c = 0; c < nranges; ++c) {
     int32_t first_split = 0;
     int last_seg = -1;
     for (long v = beg[c]; v < end[c]; ++v) {
@@ -523,6 +542,7 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
     cta_desc[c * 3 + 1] = (int32_t)end[c];
     cta_desc[c * 3 + 2] = first_split;
   }
+  *n_ranges_out = (int32_t)nranges;
   int32_t acc = 0;
   for (int s = 0; s < S; ++s) {
     split_count[s] = holders[s];

@@ -81,7 +81,8 @@ def gpu_decode(batch, *, kind=0, num_ctas=None, param=0, max_seq_len=None,
     if max_seq_len is None:
         max_seq_len = int(batch.seq_lens.max().item())
     grid = hpa.plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len)
-    ws = torch.zeros(hpa.decode_workspace_size(B, Hkv, Hq, D, grid), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(hpa.decode_workspace_size(kind, B, Hkv, Hq, D, grid), dtype=torch.uint8,
+                     device=dev)
     seq_lens = batch.seq_lens.to(dev)
     g = hpa.decode_plan(seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
                         pt_stride=batch.pt_stride, workspace=ws, kind=kind, num_ctas=num_ctas,
@@ -92,10 +93,11 @@ def gpu_decode(batch, *, kind=0, num_ctas=None, param=0, max_seq_len=None,
     pt = batch.page_table.to(dev)
     if fp8 is not None:
         kc, ks, vc, vs = (torch.from_numpy(x).to(dev) for x in fp8)
-        hpa.decode_run(q, kc, vc, pt, out, ws, grid, 1.0 / D ** 0.5, k_scale=ks, v_scale=vs)
+        hpa.decode_run(q, kc, vc, pt, out, ws, grid, 1.0 / D ** 0.5, kind=kind, k_scale=ks,
+                       v_scale=vs)
     else:
         hpa.decode_run(q, batch.k_cache.to(dev), batch.v_cache.to(dev), pt, out, ws, grid,
-                       1.0 / D ** 0.5)
+                       1.0 / D ** 0.5, kind=kind)
     torch.cuda.synchronize()
     if return_ws:
         return out, ws, grid

@@ -70,20 +70,24 @@ def test_plan_grid_matches_oracle(L, kind, B, Hkv, P, param, maxlen):
 
 
 def test_workspace_layout_is_aligned_and_ordered(L):
-    for args in [(32, 8, 64, 128, 148), (2, 2, 8, 64, 148), (256, 8, 64, 128, 4864)]:
-        lay = hpa.workspace_layout(*args)
+    for kind, args in [(0, (32, 8, 64, 128, 148)), (1, (2, 2, 8, 64, 148)),
+                       (2, (256, 8, 64, 128, 4864))]:
+        lay = hpa.workspace_layout(kind, *args)
         offs = [lay[k] for k in ["header", "lens", "tile_start", "cta_desc", "split_count",
-                                 "part_base", "arrive", "part_ml", "part_acc", "total"]]
+                                 "part_base", "part_ml", "part_acc", "total"]]
         assert all(o % 256 == 0 for o in offs)
         assert offs == sorted(offs)
         B, Hkv, Hq, D, grid = args
         G = Hq // Hkv
-        assert lay["part_acc"] - lay["part_ml"] >= 2 * grid * G * 8
-        assert lay["total"] - lay["part_acc"] >= 2 * grid * G * D * 4
+        V = 5 * grid if kind == 0 else grid  # dynamic: primary ranges + tail chunks
+        assert lay["part_acc"] - lay["part_ml"] >= 2 * V * G * 8
+        assert lay["total"] - lay["part_acc"] >= 2 * V * G * D * 4
         assert lay["cta_desc"] - lay["tile_start"] >= (B + 1) * 4
-        assert hpa.decode_workspace_size(*args) == lay["total"]
-    assert L.hpa_decode_workspace_size(0, 8, 64, 128, 148) == 0
-    assert L.hpa_decode_workspace_size(2, 3, 8, 64, 148) == 0  # Hq % Hkv != 0
+        assert lay["split_count"] - lay["cta_desc"] >= 32 * V
+        assert hpa.decode_workspace_size(kind, *args) == lay["total"]
+    assert L.hpa_decode_workspace_size(0, 0, 8, 64, 128, 148) == 0
+    assert L.hpa_decode_workspace_size(0, 2, 3, 8, 64, 148) == 0  # Hq % Hkv != 0
+    assert L.hpa_decode_workspace_size(7, 2, 2, 8, 64, 148) == 0  # unknown plan kind
 
 
 def _plan(L, **kw):
@@ -102,6 +106,8 @@ def _plan(L, **kw):
     (dict(num_kv_heads=0), 1), (dict(num_q_heads=7), 1), (dict(pt_stride=0), 1),
     (dict(num_ctas=0), 1), (dict(kind=3), 1), (dict(param=-1), 1), (dict(ws_bytes=16), 3),
     (dict(workspace=256 + 8), 3),
+    (dict(batch=32769), 2),  # more sequences than one plan holds
+    (dict(num_ctas=65537), 2),  # dynamic plans over at most 65536 CTAs
 ])
 def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
     rc, grid = _plan(L, **bad)
@@ -111,11 +117,11 @@ def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
 
 def _run(L, **kw):
     a = dict(q=256, k=256, v=256, ks=None, vs=None, kvd=0, pt=256, pts=4, pages=8, out=256,
-             outd=0, B=2, Hq=8, Hkv=2, D=64, scale=0.125, grid=148, ws=256, wsb=1 << 22)
+             outd=0, B=2, Hq=8, Hkv=2, D=64, scale=0.125, kind=0, grid=148, ws=256, wsb=1 << 24)
     a.update(kw)
     return L.hpa_decode_run(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["kvd"], a["pt"], a["pts"],
                             a["pages"], a["out"], a["outd"], a["B"], a["Hq"], a["Hkv"], a["D"],
-                            C.c_float(a["scale"]), a["grid"], a["ws"], a["wsb"], None)
+                            C.c_float(a["scale"]), a["kind"], a["grid"], a["ws"], a["wsb"], None)
 
 
 @pytest.mark.parametrize("bad,expect", [
@@ -126,8 +132,8 @@ def _run(L, **kw):
     (dict(Hq=64, Hkv=2), 2),   # G = 32
     (dict(D=96), 2), (dict(D=256), 2), (dict(kvd=1, ks=256, vs=256), 2),  # fp8 needs D = 128
     (dict(pages=1 << 26, Hkv=8, Hq=8), 2),  # rows overflow int32 TMA coordinates
-    (dict(k=256 + 8), 1), (dict(q=256 + 2), 1), (dict(out=256 + 2), 1),
-    (dict(wsb=64), 3), (dict(ws=256 + 16), 3),
+    (dict(k=256 + 8), 1), (dict(q=256 + 2), 1), (dict(q=256 + 8), 1), (dict(out=256 + 2), 1),
+    (dict(wsb=64), 3), (dict(ws=256 + 16), 3), (dict(kind=9), 1),
 ])
 def test_run_rejects_bad_arguments_without_launching(L, bad, expect):
     assert _run(L, **bad) == expect
@@ -158,7 +164,7 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     with pytest.raises(hpa.HpaLibraryMissing):
         hpa.lib()
     with pytest.raises(hpa.HpaLibraryMissing):
-        hpa.decode_workspace_size(2, 2, 8, 64, 148)
+        hpa.decode_workspace_size(0, 2, 2, 8, 64, 148)
 
 
 def test_product_path_does_not_reference_the_oracle():

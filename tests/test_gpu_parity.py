@@ -42,20 +42,21 @@ def _check(out, ref, max_abs=MAX_ABS, mean_abs=MEAN_ABS, rows=None):
 
 # ---------------------------------------------------------------- plan
 
-def _read_plan(ws, B, Hkv, Hq, D, grid):
-    lay = hpa.workspace_layout(B, Hkv, Hq, D, grid)
+def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
+    lay = hpa.workspace_layout(kind, B, Hkv, Hq, D, grid)
     w = ws.cpu().numpy()
 
     def i32(off, n):
         return w[off:off + 4 * n].view(np.int32)
 
     S = B * Hkv
+    header = i32(lay["header"], 16)
+    V = int(header[10])
     return {
-        "header": i32(lay["header"], 16), "lens": i32(lay["lens"], B),
+        "header": header, "lens": i32(lay["lens"], B),
         "tile_start": i32(lay["tile_start"], B + 1),
-        "cta": i32(lay["cta_desc"], 4 * grid).reshape(grid, 4),
+        "cta": i32(lay["cta_desc"], 8 * V).reshape(V, 8),
         "split_count": i32(lay["split_count"], S), "partial_base": i32(lay["part_base"], S),
-        "arrive": i32(lay["arrive"], S),
     }
 
 
@@ -63,6 +64,9 @@ def _read_plan(ws, B, Hkv, Hq, D, grid):
     ([131072] + [4096] * 31, 8, 148), ([512] * 64, 8, 148), ([37, 200], 2, 148),
     ([37, 200], 2, 3), ([0, 5, 0, 64, 65, 3000, 1], 4, 7), ([1], 1, 148), ([0, 0], 2, 5),
     (list(range(1, 3000, 7)), 2, 148),
+    # beyond 12K sequences the tile offsets need more than 48 KiB of shared memory
+    ([int(x) for x in np.random.default_rng(3).integers(0, 300, 20000)], 2, 148),
+    ([int(x) for x in np.random.default_rng(4).integers(1, 100, 32768)], 1, 148),  # the maximum
 ])
 @pytest.mark.parametrize("kind,param", [(0, 0), (1, 0), (1, 3), (2, 0), (2, 5)])
 def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
@@ -74,31 +78,42 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
     ref = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P, param=param,
                       max_seq_len=maxlen, capacity_tokens=pts * 64)
     assert grid == ref["grid"]
-    ws = torch.full((hpa.decode_workspace_size(B, Hkv, Hq, D, grid),), 0xAB, dtype=torch.uint8,
-                    device="cuda")
+    ws = torch.full((hpa.decode_workspace_size(kind, B, Hkv, Hq, D, grid),), 0xAB,
+                    dtype=torch.uint8, device="cuda")
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
     g = hpa.decode_plan(sl, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D, pt_stride=pts,
                         workspace=ws, kind=kind, num_ctas=P, param=param, max_seq_len=maxlen)
     torch.cuda.synchronize()
     assert g == grid
-    got = _read_plan(ws, B, Hkv, Hq, D, grid)
+    got = _read_plan(ws, kind, B, Hkv, Hq, D, grid)
+    assert got["header"][10] == ref["ranges"]
     np.testing.assert_array_equal(got["lens"], ref["lens"])
     np.testing.assert_array_equal(got["tile_start"], ref["tile_start"])
     np.testing.assert_array_equal(got["cta"][:, :3], ref["cta"])
+    # start state (b, g, t, tiles of b) of each CTA's first unit, from the oracle's offsets
+    ts = ref["tile_start"].astype(np.int64)
+    for c in range(ref["ranges"]):
+        ub, ue = int(ref["cta"][c, 0]), int(ref["cta"][c, 1])
+        if ub == ue:
+            continue
+        b0 = int(np.searchsorted(ts * Hkv, ub, side="right") - 1)
+        n0 = int(ts[b0 + 1] - ts[b0])
+        rem = ub - int(ts[b0]) * Hkv
+        assert tuple(got["cta"][c, [3, 4, 5, 6]]) == (b0, rem // n0, rem % n0, n0), c
     np.testing.assert_array_equal(got["split_count"], ref["split_count"])
     np.testing.assert_array_equal(got["partial_base"], ref["partial_base"])
-    assert np.all(got["arrive"] == 0)
     h = got["header"]
     assert h[2] == ref["n_units"] and h[3] == grid and h[1] == 0
 
 
 def test_plan_flags_clamped_lengths():
     sl = torch.tensor([-3, 100, 10_000], dtype=torch.int32, device="cuda")
-    ws = torch.zeros(hpa.decode_workspace_size(3, 2, 4, 64, 148), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(hpa.decode_workspace_size(0, 3, 2, 4, 64, 148), dtype=torch.uint8,
+                     device="cuda")
     hpa.decode_plan(sl, num_kv_heads=2, num_q_heads=4, head_dim=64, pt_stride=4, workspace=ws,
                     num_ctas=148)
     assert hpa.read_status(ws) & hpa.DEVICE_LEN_CLAMPED
-    got = _read_plan(ws, 3, 2, 4, 64, 148)
+    got = _read_plan(ws, 0, 3, 2, 4, 64, 148)
     np.testing.assert_array_equal(got["lens"], [0, 100, 256])
 
 
@@ -338,7 +353,8 @@ def test_run_without_plan_is_flagged():
     batch = W.make_batch(W.DecodeShape("np", 8, 2, 64), [100], seed=15)
     to_device(batch)
     grid = 148
-    ws = torch.zeros(hpa.decode_workspace_size(1, 2, 8, 64, grid), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(hpa.decode_workspace_size(0, 1, 2, 8, 64, grid), dtype=torch.uint8,
+                     device="cuda")
     out = torch.zeros(1, 8, 64, dtype=torch.bfloat16, device="cuda")
     hpa.decode_run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, ws, grid, 0.125)
     assert hpa.read_status(ws) & hpa.DEVICE_BAD_PLAN

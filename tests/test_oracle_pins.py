@@ -446,10 +446,11 @@ def _check_plan_invariants(p, lens, Hkv, kind):
     U = len(units)
     assert p["n_units"] == U
     cta = p["cta"]
+    R = p["ranges"]
     # ordered, contiguous, disjoint, covering [0, U) exactly once
     cover = np.zeros(U, dtype=int)
     prev_end = 0
-    for c in range(p["grid"]):
+    for c in range(R):
         a, e = int(cta[c, 0]), int(cta[c, 1])
         assert 0 <= a <= e <= U
         if a < e:
@@ -459,7 +460,7 @@ def _check_plan_invariants(p, lens, Hkv, kind):
     assert prev_end == U and np.all(cover == 1)
     # split counts and first-split indices, recounted with Python sets
     holders = {}
-    for c in range(p["grid"]):
+    for c in range(R):
         a, e = int(cta[c, 0]), int(cta[c, 1])
         segs = []
         for u in range(a, e):
@@ -481,11 +482,21 @@ def _check_plan_invariants(p, lens, Hkv, kind):
         if n > 1:
             base += n
     if kind == 0:
-        sizes = [int(cta[c, 1] - cta[c, 0]) for c in range(p["grid"])]
-        active = [s for s in sizes if s > 0]
-        assert len(active) == min(p["grid"], U)
-        if active:
-            assert max(active) - min(active) <= 1
+        P = p["grid"]
+        sizes = [int(cta[c, 1] - cta[c, 0]) for c in range(R)]
+        if U <= P:
+            # one unit per CTA, no tail
+            assert R == P and sorted(set(sizes)) in ([1], [0, 1], [0], [])
+        else:
+            # the tail holds min(U // 8, U - P) units in min(4P, tail) chunks;
+            # primary ranges and tail chunks are each even to within one unit
+            tail = min(U // 8, U - P)
+            assert R == P + min(4 * P, tail)
+            assert sum(sizes[P:]) == tail
+            prim, chunks = sizes[:P], sizes[P:]
+            assert min(prim) >= 1 and max(prim) - min(prim) <= 1
+            if chunks:
+                assert min(chunks) >= 1 and max(chunks) - min(chunks) <= 1
 
 
 @pytest.mark.parametrize("lens,Hkv,P", [

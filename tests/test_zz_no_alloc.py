@@ -39,7 +39,8 @@ def _reference(batch, out_dtype):
     B, Hq, D = batch.q.shape
     Hkv = batch.k_cache.shape[1]
     n = hpa.default_num_ctas(dev.index)
-    ws = torch.empty(hpa.decode_workspace_size(B, Hkv, Hq, D, n), dtype=torch.uint8, device=dev)
+    ws = torch.empty(hpa.decode_workspace_size(hpa.PLAN_DYNAMIC, B, Hkv, Hq, D, n),
+                     dtype=torch.uint8, device=dev)
     grid = hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
                            pt_stride=batch.pt_stride, workspace=ws, num_ctas=n)
     out = torch.empty(B, Hq, D, dtype=out_dtype, device=dev)
@@ -92,7 +93,7 @@ def test_noalloc_repeated_call_is_stable(L):
 def test_noalloc_refuses_oversized_request_on_host(L):
     # 2,000,000 sequences x 8 kv heads of per-segment plan data cannot fit in
     # the static array; refused before any CUDA call, so this runs without a GPU.
-    need = hpa.decode_workspace_size(2_000_000, 8, 64, 128, 148)
+    need = hpa.decode_workspace_size(hpa.PLAN_DYNAMIC, 2_000_000, 8, 64, 128, 148)
     assert need > hpa.NOALLOC_SCRATCH_BYTES
     rc = L.hpa_decode_noalloc(256, 256, 256, None, None, 0, 256, 4, 8, 256, 256, 0, 2_000_000, 64,
                               8, 128, C.c_float(0.088), 148, None)
