@@ -245,7 +245,7 @@ HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const v
  * Arguments are those of hpa_decode_plan + hpa_decode_run with the dynamic
  * plan; num_ctas = 0 means one CTA per SM.  Instead of a caller workspace the
  * step uses a library-owned static device array of HPA_NOALLOC_SCRATCH_BYTES
- * (8 MiB), which every GPU that loads the library holds until the process
+ * (16 MiB), which every GPU that loads the library holds until the process
  * exits.  A step whose workspace would exceed it (see
  * hpa_decode_workspace_size) returns HPA_ERR_WORKSPACE before any CUDA call.
  * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
@@ -259,7 +259,7 @@ HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const v
  * reach a result, but calls that overlap on the GPU (unordered streams) race
  * on the array.  The device status word of the array is not exposed.
  */
-#define HPA_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define HPA_NOALLOC_SCRATCH_BYTES (16u << 20)
 HPA_API hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                       const float* k_scale, const float* v_scale,
                                       hpa_kv_dtype kv_dtype, const int32_t* page_table,

@@ -35,7 +35,7 @@ OUT_BF16, OUT_F32 = 0, 1
 DEVICE_LEN_CLAMPED, DEVICE_BAD_PAGE, DEVICE_BAD_PLAN = 0x1, 0x2, 0x4
 DEVICE_BAD_POSITION, DEVICE_TIMEOUT = 0x8, 0x10
 PAGE_SIZE = 64
-NOALLOC_SCRATCH_BYTES = 8 << 20
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libhpa.so")
@@ -248,7 +248,7 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     """One decode step (dynamic plan + run) without a caller workspace.
 
     For callers that cannot allocate device memory where the step is issued:
-    the scratch is the library's static 8 MiB device array, shared by every
+    the scratch is the library's static 16 MiB device array, shared by every
     call on the device (calls that overlap on the GPU race on it).  The first
     call on a device looks the array up; make it before any stream capture."""
     _dev(q, "q", (torch.bfloat16,), 3)

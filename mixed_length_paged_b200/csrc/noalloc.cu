@@ -11,7 +11,7 @@
 // outputs; only the plan, the split partials and the arrival counters move
 // into this array.
 //
-// The array is HPA_NOALLOC_SCRATCH_BYTES (8 MiB) per GPU that loads the
+// The array is HPA_NOALLOC_SCRATCH_BYTES (16 MiB) per GPU that loads the
 // library and stays allocated until the process exits.  All calls on a
 // device share it and it keeps the previous call's contents: the plan kernel
 // rewrites every field the run reads and zeroes the arrival counters on each

@@ -4,7 +4,7 @@ Some callers cannot allocate device memory where they issue a decode step:
 code running inside a device memory pool that must not grow after start-up,
 code whose allocator belongs to another framework and is not reachable from
 there, or a C program that keeps cudaMalloc off its hot path.  For them the
-library keeps its scratch in a static 8 MiB device array.  These tests check
+library keeps its scratch in a static 16 MiB device array.  These tests check
 that this entry point gives the same result as the regular workspace-based
 plan + run on two calls in a row (the second call must not be disturbed by
 what the first left in the shared array), and that an oversized request is
