@@ -149,6 +149,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of every rank's x (device-timed durations are combined this
+    way: the job takes as long as its slowest rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank: int, world: int, seconds: float) -> float:
+    """Whole-job GB/s under weak scaling: every rank streams its own batch of
+    bytes_per_rank in `seconds` (the max over ranks)."""
+    return world * bytes_per_rank / seconds / 1e9
+
+
 def _smi_index(local_rank: int) -> str:
     """nvidia-smi id of this rank's GPU (honours CUDA_VISIBLE_DEVICES)."""
     vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
@@ -299,10 +317,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     total_ms = start.elapsed_time(end)
     run_ms = [ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(K)]
     plan_ms = [ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(K)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / K
     status = dec.status()
 
@@ -360,13 +375,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             e2e_step()
         b.record(stream)
         barrier()
-        e_ms = a.elapsed_time(b) / n
-        et = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e_ms = float(et.item())
+        e_ms = max_over_ranks(a.elapsed_time(b) / n, world, dev)
         h2d = q_h.numel() * 2 + sl_h.numel() * 4 + pt_h.numel() * 4
-        e2e = {"value": world * kv_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_throughput(kv_bytes, world, e_ms * 1e-3), "unit": "GB/s",
                "us_per_step": 1e3 * e_ms, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(out_h.numel() * 2)}
 
@@ -385,7 +396,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     run_avg_ms = statistics.mean(run_ms)
     achieved = run_bytes / (run_avg_ms * 1e-3) / 1e9
     traffic = _profiled_traffic()
-    value = world * kv_bytes / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(kv_bytes, world, ms_per_step * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,

@@ -1,0 +1,60 @@
+"""The benchmark's multi-rank plumbing on CPU: two gloo ranks, no GPU.
+
+Each rank of `bench.py --gpus N` runs its own decode batch (data-parallel
+replicas, weak scaling); the job's time is the slowest rank's and its
+throughput counts every rank's bytes.  These tests run that aggregation with
+world size 2 over gloo."""
+from __future__ import annotations
+
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        # rank r took (r + 1) * 10 ms for its batch; the job took 20 ms
+        job_ms = bench.max_over_ranks((rank + 1) * 10.0, world)
+        gbs = bench.job_throughput(1_000_000_000, world, job_ms * 1e-3)
+        dist.barrier()
+        q.put((rank, job_ms, gbs))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_rank_and_count_all_bytes():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [20.0, 20.0]
+    # 2 ranks x 1 GB in 20 ms
+    assert res[0][2] == pytest.approx(100.0) and res[1][2] == pytest.approx(100.0)
+
+
+def test_single_rank_is_the_identity():
+    import bench
+    assert bench.max_over_ranks(12.5, 1) == 12.5
+    assert bench.job_throughput(2_000_000_000, 1, 0.5) == pytest.approx(4.0)
