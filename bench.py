@@ -68,6 +68,35 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+WORKLOAD_DESC = {
+    "skewed": "skewed decode: 1 x 131072 + 31 x 4096 KV tokens, 64 q heads, 8 kv heads, "
+              "head_dim 128, bf16 KV, 64-token pages shuffled; dynamic plan",
+    "skewed_quarter": "skewed decode at a quarter of the lengths: 1 x 32768 + 31 x 1024",
+    "uniform": "uniform decode: 64 x 512 KV tokens, 64 q heads, 8 kv heads, head_dim 128, bf16",
+    "tiny": "tiny decode: 2 sequences {37, 200}, 8 q heads, 2 kv heads, head_dim 64, bf16",
+    "mix_prologue": "continuous-batching mix: 128 sequences, lengths log-uniform in [256, 65536], "
+                    "32 q heads, 8 kv heads, head_dim 128, bf16; fused RMSNorm+RoPE+KV-write "
+                    "prologue in every step",
+    "fp8": "FP8 KV: 256 sequences, lengths geometric (mean 2048, cap 16384), 64 q heads, "
+           "8 kv heads, head_dim 128, e4m3 K/V with fp32 per-(page, kv head) scales",
+}
+
+
+def _quantize_e4m3(values, live):
+    """Input preparation for the FP8 workload (not part of the timed step):
+    e4m3 codes + fp32 per-(page, kv head) scales = amax of the live tokens /
+    448, via torch's float8 cast.  Dead slots get the NaN code."""
+    import torch
+    P, Hkv, S, D = values.shape
+    slot = torch.arange(S, device=values.device).view(1, 1, S, 1)
+    alive = slot < live.view(P, 1, 1, 1).to(values.device)
+    amax = (values.abs() * alive).amax(dim=(2, 3))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).float()
+    codes = (values / scale.view(P, Hkv, 1, 1)).clamp(-448, 448).to(torch.float8_e4m3fn)
+    codes = codes.view(torch.uint8).masked_fill(~alive, 0x7F)
+    return codes.contiguous(), scale.contiguous()
+
+
 def _kernel_hash() -> str:
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
@@ -265,21 +294,43 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     batch = W.build(args.workload, device=dev, seed=0)
     shape = batch.shape
     B, Hq, Hkv, D = batch.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim
+    fp8 = shape.kv_dtype == "fp8_e4m3"
+    k_scale = v_scale = None
+    if fp8:
+        batch.k_cache, k_scale = _quantize_e4m3(batch.k_cache, batch.live)
+        batch.v_cache, v_scale = _quantize_e4m3(batch.v_cache, batch.live)
     lens = batch.seq_lens.cpu().numpy()
-    kv_bytes = W.live_kv_bytes(lens, Hkv, D, 2)
+    elt = 1 if fp8 else 2
+    kv_bytes = W.live_kv_bytes(lens, Hkv, D, elt)
     tiles = int(((lens + 63) // 64).sum())
-    # algorithmic bytes of one run launch: live KV + q + out + page-table entries read
-    run_bytes = kv_bytes + 2 * B * Hq * D * 2 + tiles * 4
+    # algorithmic bytes of one run launch: live KV + q + out + page-table entries
+    # read (+ the two fp32 scales of every (page, kv head) tile for FP8)
+    run_bytes = kv_bytes + 2 * B * Hq * D * 2 + tiles * 4 + (tiles * Hkv * 8 if fp8 else 0)
     scale = 1.0 / math.sqrt(D)
     num_ctas = args.num_ctas or hpa.default_num_ctas(local_rank)
     stream = torch.cuda.current_stream()
     dec = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, num_ctas=num_ctas, device=dev)
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
     seq_lens = batch.seq_lens
+    if shape.prologue:
+        # the step starts from the new token's raw projections: the fused
+        # prologue writes q and the K/V slot, then plan + run attend over L + 1
+        batch.q = torch.empty_like(batch.q_raw)
+
+    def prologue():
+        if shape.prologue:
+            hpa.kv_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
+                            batch.positions, batch.page_table, batch.k_cache, batch.v_cache,
+                            batch.q, eps=1e-6, rope_theta=10000.0)
+
+    def run():
+        dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale,
+                k_scale=k_scale, v_scale=v_scale)
 
     def step():
+        prologue()
         dec.plan(seq_lens)
-        dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale)
+        run()
 
     def barrier():
         if world > 1:
@@ -307,10 +358,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # steps with events around the plan and around the run call.
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * K)]
     for i in range(K):
+        prologue()
         ev[3 * i].record(stream)
         dec.plan(seq_lens)
         ev[3 * i + 1].record(stream)
-        dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale)
+        run()
         ev[3 * i + 2].record(stream)
     barrier()
     clocks = sampler.stop()
@@ -323,7 +375,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # static split-KV comparators: the same run kernel fed the static plans
     extras = {}
-    if not args.no_extras:
+    plain = not fp8 and not shape.prologue
+    if not args.no_extras and plain:
         for name, kind in (("static_nsplit", hpa.PLAN_STATIC_NSPLIT),
                            ("static_chunk", hpa.PLAN_STATIC_CHUNK)):
             sd = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, kind=kind, num_ctas=num_ctas,
@@ -348,7 +401,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # end to end through the public API: pinned host inputs -> device, step,
     # result -> pinned host, all inside the timed region
     e2e = None
-    if not args.no_extras:
+    if not args.no_extras and plain:
         q_h = batch.q.cpu().pin_memory()
         sl_h = batch.seq_lens.cpu().pin_memory()
         pt_h = batch.page_table.cpu().pin_memory()
@@ -382,7 +435,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                "d2h_bytes_per_step": int(out_h.numel() * 2)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         import oracle
         host = _host_sample(batch, CPU_SAMPLE_ROWS)
         _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))  # warm-up
@@ -397,15 +450,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     achieved = run_bytes / (run_avg_ms * 1e-3) / 1e9
     traffic = _profiled_traffic()
     value = job_throughput(kv_bytes, world, ms_per_step * 1e-3)
+    metric = METRIC if args.workload == WORKLOAD else \
+        f"KV-cache GB/s (% of HBM peak), µs/decode step, {args.workload}"
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "us_per_step": 1e3 * ms_per_step,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV / bf16" if fp8 else "bf16",
+        "data": "synthetic", "us_per_step": 1e3 * ms_per_step,
         "pct_of_hbm_peak": 100.0 * (kv_bytes / (ms_per_step * 1e-3) / 1e9) / peak,
         "config": {
-            "workload": "skewed decode: 1 x 131072 + 31 x 4096 KV tokens, 64 q heads, 8 kv heads, "
-                        "head_dim 128, bf16 KV, 64-token pages shuffled; dynamic plan",
+            "workload": WORKLOAD_DESC.get(args.workload, args.workload),
             "batch": B, "kv_bytes_per_step_per_gpu": kv_bytes, "num_ctas": num_ctas,
             "l2": "no flush: 1.06 GB of KV per step is larger than the 126 MB L2",
             "parallelism": f"data-parallel replicas x{world} (independent batches, no collective)",
@@ -419,7 +473,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "traffic": traffic, "algorithmic_bytes_per_launch": run_bytes},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 3 * K,
+        "gpu_launches": (4 if shape.prologue else 3) * K,
         "clocks": clocks,
         "static_splitkv": extras or None,
         "device_status": status,
