@@ -121,15 +121,18 @@ HPA_API size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_
                                          int num_q_heads, int head_dim, int grid);
 
 /* Byte offsets of the workspace regions, for inspection by tests and tools:
- * offsets[0..7] = header (int32[16]: magic, status, units, grid, kind, batch,
- * kv heads, group, head_dim, tiles, ranges V, ...), lens, tile_start,
- * range descriptors (int32 x8 per range: u_begin, u_end, first_split, and the
- * sequence, kv head, tile and tile count of its first unit), split_count,
- * partial_base, partial (m, l), partial acc; offsets[8] = total size.
+ * offsets[0..6] = header (int32[16]: magic, status, units, grid, kind, batch,
+ * kv heads, group, head_dim, tiles, ranges V, next tail chunk, ...), lens,
+ * tile_start, range descriptors (int32 x8 per range: u_begin, u_end, then
+ * the sequence, kv head, tile and tile count of its first unit, 0, 0),
+ * segment descriptors (int32 x2 per (sequence, kv head): slot of its first
+ * partial or -1, number of ranges holding it), partial (m, l), partial acc;
+ * offsets[7] = total size.  Range v keeps the partial of its first segment
+ * in slot 2v and that of its last segment in slot 2v + 1.
  * Returns HPA_OK or HPA_ERR_INVALID_ARG. */
 HPA_API hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_kv_heads,
                                         int num_q_heads, int head_dim, int grid,
-                                        size_t offsets[9]);
+                                        size_t offsets[8]);
 
 /*
  * hpa_decode_plan -- per-step tile plan (xiaodao.ai "HPC-Ops TPOT -48.8%",

@@ -154,11 +154,11 @@ def decode_workspace_size(kind: int, batch: int, num_kv_heads: int, num_q_heads:
 
 
 def workspace_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid) -> dict:
-    off = (_Z * 9)()
+    off = (_Z * 8)()
     _check(lib().hpa_workspace_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, off),
            "hpa_workspace_layout")
-    names = ["header", "lens", "tile_start", "cta_desc", "split_count", "part_base", "part_ml",
-             "part_acc", "total"]
+    names = ["header", "lens", "tile_start", "cta_desc", "seg_desc", "part_ml", "part_acc",
+             "total"]
     return {n: int(v) for n, v in zip(names, off)}
 
 

@@ -56,12 +56,12 @@ extern "C" size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int n
 
 extern "C" hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_kv_heads,
                                            int num_q_heads, int head_dim, int grid,
-                                           size_t offsets[9]) {
+                                           size_t offsets[8]) {
   WsLayout L;
   if (!offsets || !ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, &L))
     return HPA_ERR_INVALID_ARG;
-  const size_t v[9] = {L.header,    L.lens,    L.tile_start, L.cta_desc, L.split_count,
-                       L.part_base, L.part_ml, L.part_acc,   L.total};
+  const size_t v[8] = {L.header,   L.lens,    L.tile_start, L.cta_desc,
+                       L.seg_desc, L.part_ml, L.part_acc,   L.total};
   std::memcpy(offsets, v, sizeof v);
   return HPA_OK;
 }

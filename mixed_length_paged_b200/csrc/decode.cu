@@ -10,8 +10,8 @@
 // when the grid fits the SMs, two smaller co-resident CTAs per SM otherwise
 // (twice the warps to hide each other's latencies).
 //   producer: walks the CTA's unit range and resolves each unit's metadata
-//     (page id, live tokens, first/last tile of its segment, split slot, FP8
-//     scales) 32 units at a time, one per lane, so the global reads overlap.
+//     (page id, live tokens, first/last tile of its segment, partial slot,
+//     FP8 scales) 32 units at a time, one per lane, so the global reads overlap.
 //     For each unit it issues 2-D TMA loads of the K and V tiles of (page, kv
 //     head) -- each a contiguous 64 x D block -- into a ring of shared-memory
 //     stages with 128-byte swizzle (bank-conflict-free fragment loads) and an
@@ -114,13 +114,13 @@ constexpr int kLast = 2;    // last tile of its segment in this range
 constexpr int kEnd = 4;     // no unit: the producer has no more work
 struct alignas(16) StageInfo {
   int32_t b, g, valid, flags;   // sequence, kv head, live tokens in the tile, kFirst|kLast
-  int32_t nsplit, slot, pbase, pad;  // split count; partial slot and first slot (if split)
+  int32_t slot, pad0, pad1, pad;  // partial slot of the segment's piece (-1: whole segment)
   float k_scale, v_scale, pad2, pad3;
 };
 
 // Segment handed from the consumers to the epilogue warp.
 struct alignas(16) DepDesc {
-  int32_t b, g, nsplit, slot, pbase, stop, pad0, pad1;
+  int32_t b, g, slot, stop, pad0, pad1, pad2, pad3;
 };
 
 // 2^x on the SFU (ex2.approx, flush-to-zero): relative error ~2^-22, and
@@ -277,8 +277,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
         }
       }
       const int ub = max(0, d0.x), ue = min(d0.y, U);
-      Walk wk{d0.w, d1.x, d1.y, d1.z};
-      const int b_first = d0.w, g_first = d1.x, first_split = d0.z;
+      Walk wk{d0.z, d0.w, d1.x, d1.y};
       if (ub < ue && (wk.b < 0 || wk.b >= p.B || wk.n <= 0 || wk.n != ts[wk.b + 1] - ts[wk.b] ||
                       wk.g < 0 || wk.g >= p.Hkv || wk.t < 0 || wk.t >= wk.n)) {
         if (lane == 0) atomicOr(status, HPA_DEVICE_BAD_PLAN);
@@ -287,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
           Walk w2 = wk;
           for (int k = 0; k < lane && u0 + k + 1 < ue; ++k) w2.next(ts, p.Hkv);
           const int u = u0 + lane;
-          int row = 0, valid = 0, flags = 0, nsplit = 1, slot = -1, pbase = 0, bad = 0;
+          int row = 0, valid = 0, flags = 0, slot = -1, bad = 0;
           float ks = 1.f, vs = 1.f;
           if (u < ue) {
             const int page = __ldg(p.page_table + (long long)w2.b * p.pt_stride + w2.t);
@@ -295,17 +294,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
             valid = min(kPageSize, L - w2.t * kPageSize);
             flags = ((w2.t == 0 || u == ub) ? kFirst : 0) | ((w2.t == w2.n - 1 || u == ue - 1) ? kLast : 0);
             if (flags & kLast) {
-              const int sg = w2.b * p.Hkv + w2.g;
-              nsplit = p.ws.split_count[sg];
-              if (nsplit > 1) {
-                pbase = p.ws.part_base[sg];
-                const int sidx = (w2.b == b_first && w2.g == g_first) ? first_split : 0;
-                slot = pbase + sidx;
-                if (sidx >= nsplit || pbase < 0 || pbase + nsplit > p.slots) {
-                  atomicOr(status, HPA_DEVICE_BAD_PLAN);
-                  slot = -1;  // the output of this segment is void
-                }
-              }
+              // The piece of this segment in range v is whole if the segment
+              // starts inside the range and ends here.  Otherwise it is a
+              // partial: slot 2v if the segment is the range's first, else
+              // 2v + 1 (it is then the range's last).
+              const int useg = u - w2.t;  // unit of the segment's tile 0
+              if (useg < ub || w2.t != w2.n - 1) slot = 2 * v + (useg > ub ? 1 : 0);
             }
             if (page < 0 || page >= p.num_pages) {
               bad = 1;
@@ -329,15 +323,10 @@ __global__ void __launch_bounds__(kThreads, CPS)
             si.valid = pk & 127;
             si.flags = (pk >> 7) & 3;
             const int bk = (pk >> 9) & 1;
-            si.nsplit = 1;
             si.slot = -1;
-            si.pbase = 0;
-            if (si.flags & kLast) {  // warp-uniform: pk is the same in every lane
-              si.nsplit = __shfl_sync(0xffffffffu, nsplit, k);
+            if (si.flags & kLast)  // warp-uniform: pk is the same in every lane
               si.slot = __shfl_sync(0xffffffffu, slot, k);
-              si.pbase = __shfl_sync(0xffffffffu, pbase, k);
-            }
-            si.pad = 0;
+            si.pad0 = si.pad1 = si.pad = 0;
             si.k_scale = si.v_scale = 1.f;
             if constexpr (FP8) {
               si.k_scale = __shfl_sync(0xffffffffu, ks, k);
@@ -423,9 +412,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
       DepDesc dd = dep_desc[db];
       if (dd.stop) break;
       // Never trust a deposit as an index without checking it.
-      if (dd.b < 0 || dd.b >= p.B || dd.g < 0 || dd.g >= p.Hkv ||
-          (dd.nsplit > 1 && (dd.slot < 0 || dd.slot >= p.slots || dd.pbase < 0 ||
-                             dd.pbase + dd.nsplit > p.slots))) {
+      if (dd.b < 0 || dd.b >= p.B || dd.g < 0 || dd.g >= p.Hkv || dd.slot >= p.slots) {
         if (lane == 0) atomicOr(status, HPA_DEVICE_BAD_PLAN);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&dep_empty[db]));
@@ -460,12 +447,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
             o[0] += a.x * sc; o[1] += a.y * sc;
           }
         }
-        if (dd.nsplit <= 1) {
+        if (dd.slot < 0) {
           const float inv = 1.f / lam;
 #pragma unroll
           for (int v = 0; v < V; ++v) o[v] *= inv;
           store_out_vec<OUT_F32, V>(p.out, out_row0 + (long long)h * D + d, o);
-        } else if (dd.slot >= 0) {
+        } else {
           float* dst = p.ws.part_acc + ((long long)dd.slot * G + h) * D + d;
           if constexpr (V == 4) *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
           else *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
@@ -542,11 +529,9 @@ __global__ void __launch_bounds__(kThreads, CPS)
       DepDesc dd;
       dd.b = inf ? inf->b : -1;
       dd.g = inf ? inf->g : 0;
-      dd.nsplit = inf ? inf->nsplit : 0;
       dd.slot = inf ? inf->slot : -1;
-      dd.pbase = inf ? inf->pbase : 0;
       dd.stop = inf ? 0 : 1;
-      dd.pad0 = dd.pad1 = 0;
+      dd.pad0 = dd.pad1 = dd.pad2 = dd.pad3 = 0;
       dep_desc[db] = dd;
     }
     __syncwarp();
@@ -751,25 +736,32 @@ __global__ void __launch_bounds__(kThreads, CPS)
 
 
 // ---------------------------------------------------------------------------
-// Split merge: for every segment with more than one split, the log-sum-exp
-// combination of its partials in split order,
+// Split merge: for every segment with more than one piece, the log-sum-exp
+// combination of its partials in range order,
 //   M = max_i m_i,  Lambda = sum_i l_i 2^(m_i - M),  o = sum_i acc_i 2^(m_i - M) / Lambda
-// (m in log2 units).  One CTA per (segment, head) -- grid-stride -- and one
-// thread per output element: the CTA stages the head's (m, l) of all splits
-// in shared memory in one pass, forms the weights with warp reductions, and
-// every thread then loads its element of each split's partial in batches of
-// independent loads, so the merge costs a few L2 round trips.
+// (m in log2 units).  One warp per (segment, head), D / 32 output elements
+// per lane.  The slots follow from the segment descriptor, so after that one
+// read the warp issues the (m, l) of up to 32 pieces (one per lane) and its
+// share of their partial rows together: two L2 round trips in all for a
+// segment of at most kMergeBatch pieces.  Lane j forms piece j's weight; the
+// weights reach the other lanes by shuffle.
 // ---------------------------------------------------------------------------
-constexpr int kMergeBatch = 32;   // splits whose partial values are loaded together
+constexpr int kMergeWarps = 4;
 
-// L2-only load kept in program order (the batch below is issued before any
-// of its values is used).
-__device__ __forceinline__ float ld_cg(const float* p) {
-  float v;
-  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+// L2-only loads kept in program order (a batch is issued before any of its
+// values is used).
+__device__ __forceinline__ float2 ld_cg2(const float2* p) {
+  float2 v;
+  asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
   return v;
 }
-constexpr int kMergeStage = 1024; // (m, l) pairs staged per pass
+__device__ __forceinline__ float4 ld_cg4(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
 
 struct MergeParams {
   Ws ws;
@@ -778,66 +770,68 @@ struct MergeParams {
 };
 
 template <int D, bool OUT_F32>
-__global__ void __launch_bounds__(D) merge_kernel(const MergeParams p) {
-  __shared__ float s_w[kMergeStage];  // weights 2^(m_i - M) of the staged splits
-  __shared__ float s_red[2][D / 32];
-  pdl_wait();                         // the partials of the decode kernel
-  const int G = p.G;
-  const int d = threadIdx.x, warp = d >> 5, lane = d & 31;
-  for (int job = blockIdx.x; job < p.S * G; job += gridDim.x) {
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergeParams p) {
+  constexpr int kVec = D / 32;                 // output elements per lane
+  constexpr int kBatch = D == 128 ? 24 : 32;   // pieces loaded together (<= 32)
+  pdl_wait();                                  // the partials of the decode kernel
+  const int G = p.G, lane = threadIdx.x & 31;
+  const int jobs = p.S * G;
+  for (int job = blockIdx.x * kMergeWarps + (threadIdx.x >> 5); job < jobs;
+       job += gridDim.x * kMergeWarps) {
     const int s = job / G, h = job - s * G;
-    const int ns = p.ws.split_count[s];
+    const int2 sd = __ldcg(&p.ws.seg_desc[s]);
+    const int ns = sd.y;
     if (ns <= 1) continue;
-    const int base = p.ws.part_base[s];
-    if (base < 0 || base + ns > p.slots) {
-      if (d == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
+    const int r0 = sd.x >> 1;
+    if (sd.x < 0 || 2LL * (r0 + ns - 1) >= p.slots) {
+      if (lane == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
       continue;
     }
-    const float2* ml = p.ws.part_ml + (long long)base * G + h;
-    const float* acc = p.ws.part_acc + (long long)base * G * D + (long long)h * D + d;
-    // 1. the head's maximum over all splits
-    float M = -INFINITY;
-    for (int i = d; i < ns; i += D) M = fmaxf(M, __ldcg(&ml[(long long)i * G]).x);
+    // piece i sits in slot sd.x (i = 0), else 2 (r0 + i)
+    auto row = [&](int i) -> long long { return (i == 0 ? (long long)sd.x : 2LL * (r0 + i)) * G + h; };
+    float M = -INFINITY, lam = 0.f, o[kVec];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) s_red[0][warp] = M;
-    __syncthreads();
-    M = s_red[0][0];
+    for (int v = 0; v < kVec; ++v) o[v] = 0.f;
+    for (int i0 = 0; i0 < ns; i0 += kBatch) {
+      const int n = min(kBatch, ns - i0);
+      const float2 ml = lane < n ? ld_cg2(p.ws.part_ml + row(i0 + lane)) : make_float2(-INFINITY, 0.f);
+      float a[kBatch][kVec];
 #pragma unroll
-    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_red[0][w]);
-    // 2. weights (staged) and the weighted sum of the l's; 3. weighted partials
-    float lam = 0.f, o = 0.f;
-    for (int i0 = 0; i0 < ns; i0 += kMergeStage) {
-      const int n = min(kMergeStage, ns - i0);
-      __syncthreads();
-      for (int i = d; i < n; i += D) {
-        const float2 v = __ldcg(&ml[(long long)(i0 + i) * G]);
-        const float w = (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - M);
-        s_w[i] = w;
-        lam += v.y * w;
+      for (int j = 0; j < kBatch; ++j) {
+        const float* src = p.ws.part_acc + row(i0 + j) * D + lane * kVec;
+        if constexpr (kVec == 4) {
+          const float4 x = j < n ? ld_cg4(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          a[j][0] = x.x; a[j][1] = x.y; a[j][2] = x.z; a[j][3] = x.w;
+        } else {
+          const float2 x = j < n ? ld_cg2(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+          a[j][0] = x.x; a[j][1] = x.y;
+        }
       }
-      __syncthreads();
-      for (int j0 = 0; j0 < n; j0 += kMergeBatch) {
-        float a[kMergeBatch];
+      float Mn = ml.x;
 #pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j)
-          a[j] = (j0 + j < n) ? ld_cg(acc + (long long)(i0 + j0 + j) * G * D) : 0.f;
+      for (int off = 16; off > 0; off >>= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xffffffffu, Mn, off));
+      Mn = fmaxf(M, Mn);
+      const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - Mn);
+      const float sc = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
+      float lw = ml.y * w;
 #pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j)
-          if (j0 + j < n) o += a[j] * s_w[j0 + j];
+      for (int off = 16; off > 0; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+      lam = lam * sc + lw;
+#pragma unroll
+      for (int v = 0; v < kVec; ++v) o[v] *= sc;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
+#pragma unroll
+        for (int v = 0; v < kVec; ++v) o[v] += a[j][v] * wj;
       }
+      M = Mn;
     }
+    const float inv = 1.f / lam;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) lam += __shfl_xor_sync(0xffffffffu, lam, off);
-    __syncthreads();
-    if (lane == 0) s_red[1][warp] = lam;
-    __syncthreads();
-    lam = 0.f;
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) lam += s_red[1][w];
+    for (int v = 0; v < kVec; ++v) o[v] *= inv;
     const int b = s / p.Hkv, g = s - b * p.Hkv;
-    store_out<OUT_F32>(p.out, ((long long)b * p.Hq + (long long)g * G + h) * D + d, o / lam);
-    __syncthreads();  // s_red / s_w are reused by the next job
+    store_out_vec<OUT_F32, kVec>(p.out, ((long long)b * p.Hq + (long long)g * G + h) * D + lane * kVec, o);
   }
   pdl_trigger();
 }
@@ -1035,8 +1029,9 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
   mp.Hq = num_q_heads;
   mp.slots = (int)(2 * plan_ranges_ll(kind, grid));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::min<long long>((long long)mp.S * G, (long long)std::max(1, sms) * 16));
-  cfg.blockDim = dim3(head_dim);
+  const long long merge_ctas = ((long long)mp.S * G + kMergeWarps - 1) / kMergeWarps;
+  cfg.gridDim = dim3((unsigned)std::min<long long>(merge_ctas, (long long)std::max(1, sms) * 16));
+  cfg.blockDim = dim3(kMergeWarps * 32);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -17,22 +17,26 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
-//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T
+//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next
 //   lens        int32[B]     clamped lengths
 //   tile_start  int32[B+1]   exclusive prefix sum of tiles per sequence
-//   cta_desc    int4[2*V]    per virtual range v: (u_begin, u_end,
-//                            first_split, b0), (g0, t0, n0, 0): the unit
-//                            range, the split index of its first segment, and
-//                            the (sequence, kv head, tile, tiles of that
-//                            sequence) of its first unit.  V = grid for the
-//                            static plans; for the dynamic plan V <= 5 * grid
-//                            (grid primary ranges, then the tail chunks).
-//   split_count int32[B*Hkv]
-//   part_base   int32[B*Hkv]
-//   part_ml     float2[2*grid][G]     (m, l) of each partial, log2 units
-//   part_acc    float[2*grid][G][D]   un-normalised partial outputs
-// V contiguous ranges have at most 2*(V-1) partials (each range boundary
-// cuts at most one segment), so 2*V slots always suffice.
+//   cta_desc    int4[2*V]    per range v: (u_begin, u_end, b0, g0), (t0, n0,
+//                            0, 0): the unit range and the (sequence, kv
+//                            head, tile, tiles of that sequence) of its first
+//                            unit.  V = grid for the static plans; for the
+//                            dynamic plan V <= 5 * grid (grid primary ranges,
+//                            then the tail chunks).
+//   seg_desc    int2[B*Hkv]  per segment: (first partial slot, ranges holding
+//                            its units); a segment held by one range has no
+//                            partials.
+//   part_ml     float2[2V][G]     (m, l) of each partial, log2 units
+//   part_acc    float[2V][G][D]   un-normalised partial outputs
+// Partial slots follow from the ranges: range v stores the piece of its first
+// segment in slot 2v and the piece of its last segment in slot 2v + 1 (a
+// segment in the middle of a range is whole there).  The ranges holding a
+// segment are consecutive, r0 .. r0 + n - 1; the segment's piece in r0 is
+// in slot 2 r0 (if the segment starts where r0 does) or 2 r0 + 1, and its
+// piece in each later range r is in slot 2r.
 // ---------------------------------------------------------------------------
 enum HeaderField {
   kHdrMagic = 0, kHdrStatus = 1, kHdrUnits = 2, kHdrGrid = 3, kHdrKind = 4,
@@ -56,7 +60,7 @@ inline long long plan_ranges_ll(int kind, int grid) {
 }
 
 struct WsLayout {
-  size_t header, lens, tile_start, cta_desc, split_count, part_base, part_ml, part_acc, total;
+  size_t header, lens, tile_start, cta_desc, seg_desc, part_ml, part_acc, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -72,8 +76,7 @@ inline bool ws_layout(int kind, int B, int Hkv, int Hq, int D, int grid, WsLayou
   L->lens = off;        off = align256(off + size_t(B) * 4);
   L->tile_start = off;  off = align256(off + (size_t(B) + 1) * 4);
   L->cta_desc = off;    off = align256(off + V * 32);
-  L->split_count = off; off = align256(off + S * 4);
-  L->part_base = off;   off = align256(off + S * 4);
+  L->seg_desc = off;    off = align256(off + S * 8);
   L->part_ml = off;     off = align256(off + slots * G * 8);
   L->part_acc = off;    off = align256(off + slots * G * size_t(D) * 4);
   L->total = off;
@@ -86,8 +89,7 @@ struct Ws {
   int32_t* lens;
   int32_t* tile_start;
   int4* cta_desc;
-  int32_t* split_count;
-  int32_t* part_base;
+  int2* seg_desc;
   float2* part_ml;
   float* part_acc;
 };
@@ -96,8 +98,7 @@ inline Ws ws_view(void* base, const WsLayout& L) {
   char* p = static_cast<char*>(base);
   return Ws{reinterpret_cast<int32_t*>(p + L.header), reinterpret_cast<int32_t*>(p + L.lens),
             reinterpret_cast<int32_t*>(p + L.tile_start), reinterpret_cast<int4*>(p + L.cta_desc),
-            reinterpret_cast<int32_t*>(p + L.split_count),
-            reinterpret_cast<int32_t*>(p + L.part_base), reinterpret_cast<float2*>(p + L.part_ml),
+            reinterpret_cast<int2*>(p + L.seg_desc), reinterpret_cast<float2*>(p + L.part_ml),
             reinterpret_cast<float*>(p + L.part_acc)};
 }
 

@@ -8,9 +8,12 @@
 // (fixed split count; fixed split size with the grid sized by the longest
 // request) come out of the same kernel so that one run kernel serves all.
 //
-// One CTA of 1024 threads builds the whole plan on the device from the
-// device-side lengths, so a decode step needs no host round trip.  Units are
-// (sequence b, kv head g, tile t) in that order; segment s = b * Hkv + g.
+// The plan is built on the device from the device-side lengths, so a decode
+// step needs no host round trip.  Units are (sequence b, kv head g, tile t)
+// in that order; segment s = b * Hkv + g.  Every CTA of the plan grid scans
+// all lengths itself (a few hundred bytes for a typical batch) so that no CTA
+// waits for another; the range and segment descriptors are then spread over
+// the CTAs, each one a closed-form computation.
 //
 // The dynamic plan is a contiguous partition of the unit list into ranges:
 // one primary range per persistent CTA over the first ~7/8 of the units, then
@@ -29,7 +32,9 @@
 namespace hpa {
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;
+constexpr int kPlanWarps = kPlanThreads / 32;
+constexpr int kPlanMaxCtas = 64;  // each CTA repeats the length scan: keep the grid small
 
 struct PlanParams {
   const int32_t* seq_lens;
@@ -38,34 +43,6 @@ struct PlanParams {
   long long chunk;             // STATIC_CHUNK: tiles per split
   Ws ws;
 };
-
-// Exclusive block-wide prefix sum of one int per thread; *total gets the sum.
-__device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
-  constexpr int kWarps = kPlanThreads / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) s_warp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < kWarps ? s_warp[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    s_warp[lane] = w;  // inclusive prefix of warp sums
-  }
-  __syncthreads();
-  const int before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
-  *total = s_warp[kWarps - 1];
-  __syncthreads();
-  return before;
-}
 
 // Largest b in [0, B) with tile_start[b] * Hkv <= u (u < U).
 __device__ int seq_of_unit(const int32_t* tile_start, int B, int Hkv, long long u) {
@@ -106,102 +83,131 @@ struct FloorDiv {
 struct DynGeom {
   long long U, P, Pd, U1, Ut, M;
   FloorDiv by_Pd, by_M, by_U1, by_Ut;
-  // r[0..3]: reciprocals of Pd, M, U1, Ut (0 for a zero divisor)
+  __device__ void init(long long units, long long ctas) {
+    U = units;
+    P = ctas;
+    if (U <= P) {
+      Pd = U; U1 = U; Ut = 0; M = 0;
+    } else {
+      Pd = P;
+      Ut = std::min<long long>(U / kTailFractionDiv, U - P);
+      U1 = U - Ut;
+      M = std::min<long long>((long long)kTailChunksPerCta * P, Ut);
+    }
+  }
+  // the divisors whose reciprocals init_div takes, in order
+  __device__ long long divisor(int i) const { return i == 0 ? Pd : i == 1 ? M : i == 2 ? U1 : Ut; }
   __device__ void init_div(const double* r) {
     by_Pd.init(Pd, r[0]);
     by_M.init(M, r[1]);
     by_U1.init(U1, r[2]);
     by_Ut.init(Ut, r[3]);
   }
+  __device__ long long ranges() const { return P + M; }
   __device__ long long range_of(long long u) const {
     return u < U1 ? by_U1((u + 1) * Pd - 1) : P + by_Ut((u - U1 + 1) * M - 1);
+  }
+  __device__ void bounds(long long c, long long* ub, long long* ue) const {
+    if (c < P) {
+      if (c < Pd) {
+        *ub = by_Pd(c * U1);
+        *ue = by_Pd((c + 1) * U1);
+      } else {
+        *ub = *ue = U;
+      }
+    } else {
+      const long long j = c - P;
+      *ub = U1 + by_M(j * Ut);
+      *ue = U1 + by_M((j + 1) * Ut);
+    }
   }
 };
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
   extern __shared__ int32_t ts[];  // tile_start[0..B], in shared memory
-  __shared__ int s_warp[32];
+  __shared__ int s_warp[kPlanWarps];
   __shared__ int s_status;
   __shared__ double s_recip[4];
   // The previous step's run kernel may still be reading this workspace.
   pdl_wait();
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) s_status = 0;
   __syncthreads();
 
-  // 1. clamped lengths, tiles per sequence, exclusive tile prefix sum
+  // 1. clamped lengths -> tiles per sequence -> exclusive prefix sum, in
+  //    shared memory.  Warp w scans its own contiguous slice 32 entries at a
+  //    time (coalesced loads, shuffle scans); the slices' totals are added
+  //    after one barrier.
+  const int slice = (p.B + kPlanWarps - 1) / kPlanWarps;
+  const int lo = min(p.B, warp * slice), hi = min(p.B, lo + slice);
   int carry = 0;
-  for (int base = 0; base < p.B; base += kPlanThreads) {
-    const int b = base + tid;
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
     int n = 0;
-    if (b < p.B) {
-      const int L = p.seq_lens[b];
+    if (i < hi) {
+      const int L = p.seq_lens[i];
       const int Lc = min(max(L, 0), p.capacity);
       if (Lc != L) atomicOr(&s_status, HPA_DEVICE_LEN_CLAMPED);
-      p.ws.lens[b] = Lc;
       n = (Lc + kPageSize - 1) / kPageSize;
     }
-    int total;
-    const int before = block_exclusive_scan(n, s_warp, &total);
-    if (b < p.B) ts[b] = carry + before;
-    carry += total;
+    int x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (i < hi) ts[i] = carry + x - n;
+    carry += __shfl_sync(0xffffffffu, x, 31);
   }
-  if (tid == 0) ts[p.B] = carry;
+  if (lane == 0) s_warp[warp] = carry;
   __syncthreads();
-  for (int i = tid; i <= p.B; i += kPlanThreads) p.ws.tile_start[i] = ts[i];
-
-  const long long T = carry;
-  const long long U = T * p.Hkv;
-  const int S = p.B * p.Hkv;
-  const int per = (p.kind == HPA_PLAN_DYNAMIC) ? 0 : p.grid / S;  // static: CTAs per segment
-  DynGeom dg;
-  dg.U = U;
-  dg.P = p.num_ctas;
-  if (U <= dg.P) {
-    dg.Pd = U; dg.U1 = U; dg.Ut = 0; dg.M = 0;
-  } else {
-    dg.Pd = dg.P;
-    dg.Ut = std::min<long long>(U / kTailFractionDiv, U - dg.P);
-    dg.U1 = U - dg.Ut;
-    dg.M = std::min<long long>((long long)kTailChunksPerCta * dg.P, dg.Ut);
+  int off = 0, T = 0;
+#pragma unroll
+  for (int w = 0; w < kPlanWarps; ++w) {
+    off += w < warp ? s_warp[w] : 0;
+    T += s_warp[w];
   }
-  // the four reciprocals, computed once for the whole CTA
+  if (off)
+    for (int i = lo + lane; i < hi; i += 32) ts[i] += off;
+  if (tid == 0) ts[p.B] = T;
+
+  const long long U = (long long)T * p.Hkv;
+  const int S = p.B * p.Hkv;
+  const bool dyn = p.kind == HPA_PLAN_DYNAMIC;
+  const int per = dyn ? 0 : p.grid / S;  // static: CTAs per segment
+  DynGeom dg;
+  dg.init(U, p.num_ctas);
   if (tid < 4) {
-    const long long d = tid == 0 ? dg.Pd : tid == 1 ? dg.M : tid == 2 ? dg.U1 : dg.Ut;
+    const long long d = dg.divisor(tid);
     s_recip[tid] = d > 0 ? 1.0 / (double)d : 0.0;
   }
   __syncthreads();
   dg.init_div(s_recip);
-  const long long V = (p.kind == HPA_PLAN_DYNAMIC) ? dg.P + dg.M : p.grid;
+  const long long V = dyn ? dg.ranges() : p.grid;
+  const int stride = gridDim.x * kPlanThreads;
+  const int first = blockIdx.x * kPlanThreads + tid;
 
-  // 2. per-range unit ranges, first-split indices and start states
-  for (int c = tid; c < V; c += kPlanThreads) {
+  // lengths and tile offsets, written by all CTAs together
+  for (int i = first; i <= p.B; i += stride) {
+    p.ws.tile_start[i] = ts[i];
+    if (i < p.B) p.ws.lens[i] = min(max(p.seq_lens[i], 0), p.capacity);
+  }
+
+  // 2. per-range unit ranges and the state of each range's first unit
+  for (long long c = first; c < V; c += stride) {
     long long ub, ue;
-    int first = 0, b0 = 0, g0 = 0, t0 = 0, n0 = 0;
-    if (p.kind == HPA_PLAN_DYNAMIC) {
-      if (c < dg.P) {
-        if (c < dg.Pd) {
-          ub = dg.by_Pd((long long)c * dg.U1);
-          ue = dg.by_Pd((long long)(c + 1) * dg.U1);
-        } else {
-          ub = ue = U;
-        }
-      } else {
-        const long long j = c - dg.P;
-        ub = dg.U1 + dg.by_M(j * dg.Ut);
-        ue = dg.U1 + dg.by_M((j + 1) * dg.Ut);
-      }
+    int b0 = 0, g0 = 0, t0 = 0, n0 = 0;
+    if (dyn) {
+      dg.bounds(c, &ub, &ue);
       if (ub < ue) {
         b0 = seq_of_unit(ts, p.B, p.Hkv, ub);
         n0 = ts[b0 + 1] - ts[b0];
         const int rem = (int)(ub - (long long)ts[b0] * p.Hkv);  // < Hkv * n0 < 2^31
         g0 = rem / n0;
         t0 = rem - g0 * n0;
-        const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n0;
-        first = (int)(c - dg.range_of(seg_start));
       }
     } else {
-      const int s = c / per, i = c % per;
+      const int s = (int)c / per, i = (int)c % per;
       b0 = s / p.Hkv;
       g0 = s % p.Hkv;
       const long long n = ts[b0 + 1] - ts[b0];
@@ -211,40 +217,38 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
       const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n;
       ub = seg_start + c0;
       ue = seg_start + c1;
-      first = c0 < c1 ? i : 0;
       t0 = (int)c0;
       n0 = (int)n;
     }
-    p.ws.cta_desc[2 * c] = make_int4((int)ub, (int)ue, first, b0);
-    p.ws.cta_desc[2 * c + 1] = make_int4(g0, t0, n0, 0);
+    p.ws.cta_desc[2 * c] = make_int4((int)ub, (int)ue, b0, g0);
+    p.ws.cta_desc[2 * c + 1] = make_int4(t0, n0, 0, 0);
   }
 
-  // 3. split counts and partial slot bases
-  int pcarry = 0;
-  for (int base = 0; base < S; base += kPlanThreads) {
-    const int s = base + tid;
-    int split = 0;
-    if (s < S) {
-      const int b = s / p.Hkv, g = s % p.Hkv;
-      const long long n = ts[b + 1] - ts[b];
-      if (n > 0) {
-        if (p.kind == HPA_PLAN_DYNAMIC) {
-          const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
-          split = (int)(dg.range_of(seg_start + n - 1) - dg.range_of(seg_start) + 1);
-        } else {
-          const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
-          split = (int)((n + C - 1) / C);
+  // 3. per segment: the ranges holding it and the slot of its first partial
+  for (int s = first; s < S; s += stride) {
+    const int b = s / p.Hkv, g = s - b * p.Hkv;
+    const long long n = ts[b + 1] - ts[b];
+    int nsplit = 0, slot0 = -1;
+    if (n > 0) {
+      if (dyn) {
+        const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
+        const long long r0 = dg.range_of(seg_start);
+        nsplit = (int)(dg.range_of(seg_start + n - 1) - r0 + 1);
+        if (nsplit > 1) {
+          long long ub, ue;
+          dg.bounds(r0, &ub, &ue);
+          slot0 = (int)(2 * r0 + (ub == seg_start ? 0 : 1));
         }
+      } else {
+        const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
+        nsplit = (int)((n + C - 1) / C);
+        if (nsplit > 1) slot0 = 2 * s * per;  // chunk 0 starts its segment
       }
-      p.ws.split_count[s] = split;
     }
-    int total;
-    const int before = block_exclusive_scan(split > 1 ? split : 0, s_warp, &total);
-    if (s < S) p.ws.part_base[s] = pcarry + before;
-    pcarry += total;
+    p.ws.seg_desc[s] = make_int2(slot0, nsplit);
   }
 
-  if (tid == 0) {
+  if (blockIdx.x == 0 && tid == 0) {
     int32_t* h = p.ws.header;
     h[kHdrStatus] = s_status;
     h[kHdrUnits] = (int32_t)U;
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrKvHeads] = p.Hkv;
     h[kHdrGroup] = p.G;
     h[kHdrHeadDim] = p.D;
-    h[kHdrTiles] = (int32_t)T;
+    h[kHdrTiles] = T;
     h[kHdrRanges] = (int32_t)V;
     h[kHdrNext] = 0;
     __threadfence();
@@ -333,8 +337,11 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
       ready_mask.fetch_or(bit);
     }
   }
+  const long long V = plan_ranges_ll(kind, (int)grid);
+  const long long work = std::max<long long>(V, (long long)batch * num_kv_heads);
+  const int ctas = (int)std::min<long long>(kPlanMaxCtas, (work + kPlanThreads - 1) / kPlanThreads);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1);
+  cfg.gridDim = dim3(std::max(1, ctas));
   cfg.blockDim = dim3(kPlanThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);

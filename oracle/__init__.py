@@ -251,19 +251,19 @@ def plan(seq_lens, num_kv_heads: int, *, kind: int = 0, num_ctas: int, param: in
     S = B * num_kv_heads
     lens = np.zeros(B, dtype=np.int32)
     tile_start = np.zeros(B + 1, dtype=np.int32)
-    cta = np.zeros((5 * grid, 3), dtype=np.int32)
+    cta = np.zeros((5 * grid, 2), dtype=np.int32)
     split_count = np.zeros(S, dtype=np.int32)
-    partial_base = np.zeros(S, dtype=np.int32)
+    first_slot = np.zeros(S, dtype=np.int32)
     n_units = C.c_int32()
     n_ranges = C.c_int32()
     rc = lib().oracle_plan(_ptr(sl), B, num_kv_heads, page_size, capacity_tokens, kind,
                            num_ctas, param, max_seq_len, _ptr(lens), _ptr(tile_start),
-                           _ptr(cta), _ptr(split_count), _ptr(partial_base), C.byref(n_units),
+                           _ptr(cta), _ptr(split_count), _ptr(first_slot), C.byref(n_units),
                            C.byref(n_ranges))
     _check(rc, "plan")
     V = int(n_ranges.value)
     return {"grid": grid, "ranges": V, "lens": lens, "tile_start": tile_start, "cta": cta[:V],
-            "split_count": split_count, "partial_base": partial_base,
+            "split_count": split_count, "first_slot": first_slot,
             "n_units": int(n_units.value)}
 
 

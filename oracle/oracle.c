@@ -413,12 +413,15 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  *     sequence were the longest; chunk i = [i C, min((i+1) C, n)), empty past
  *     the segment's end.  Grid = B * Hkv * NC.
  *
- * For each range the plan records (u_begin, u_end, first_split): first_split
- * is the index, among the ranges holding units of the range's first segment,
- * of this range (0 if the segment starts in it).  For each segment it records
- * split_count (ranges holding its units) and partial_base (exclusive prefix
- * sum over segments of split_count, counting only segments with
- * split_count > 1).  The static kinds have one range per CTA (V = grid).
+ * For each range the plan records (u_begin, u_end).  A segment whose units
+ * lie in more than one range is computed in pieces, one per range, each
+ * leaving a partial (acc, m, l) that a log-sum-exp merge combines; the piece
+ * a range holds of its first segment goes to partial slot 2c, that of its
+ * last segment to slot 2c + 1 (a segment strictly inside a range is whole
+ * there).  For each segment the plan records split_count (ranges holding
+ * its units) and first_slot (the slot of its first piece, -1 if the
+ * segment is not split).  The static kinds have one range per CTA (V =
+ * grid).
  *
  * This implementation enumerates every unit explicitly and assigns it, then
  * counts; it does not use any closed form.
@@ -442,8 +445,8 @@ long oracle_plan_grid(int kind, int B, int Hkv, int num_ctas, int param, int max
 
 int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capacity_tokens,
                 int kind, int num_ctas, int param, int max_seq_len, int32_t* lens_out,
-                int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][3] */,
-                int32_t* split_count /* [B*Hkv] */, int32_t* partial_base /* [B*Hkv] */,
+                int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][2] */,
+                int32_t* split_count /* [B*Hkv] */, int32_t* first_slot /* [B*Hkv] */,
                 int32_t* n_units_out, int32_t* n_ranges_out) {
   if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 2)
     return ORC_BAD_ARG;
@@ -524,31 +527,37 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
       }
     }
   }
-  /* 4. walk each range's units: count the ranges holding each segment, and
-   *    the split index of each range within its first segment */
+  /* 4. walk each range's units: list its segments in order, count the
+   *    ranges holding each segment, and give every cut piece its slot */
   int32_t* holders = calloc(S, sizeof(int32_t));
+  long* seg_units = calloc(S, sizeof(long)); /* units of each segment */
+  for (long v = 0; v < U; ++v) seg_units[unit_seg[v]] += 1;
+  for (int s = 0; s < S; ++s) first_slot[s] = -1;
+  int32_t* segs = malloc(sizeof(int32_t) * (U > 0 ? U : 1));
+  long* held = malloc(sizeof(long) * (U > 0 ? U : 1));
   for (long c = 0; c < nranges; ++c) {
-    int32_t first_split = 0;
-    int last_seg = -1;
+    long nseg = 0;
     for (long v = beg[c]; v < end[c]; ++v) {
       int s = unit_seg[v];
-      if (s != last_seg) {
-        if (v == beg[c]) first_split = holders[s];
-        holders[s] += 1;
-        last_seg = s;
+      if (nseg == 0 || segs[nseg - 1] != s) {
+        segs[nseg] = s;
+        held[nseg] = 0;
+        ++nseg;
       }
+      held[nseg - 1] += 1;
     }
-    cta_desc[c * 3 + 0] = (int32_t)beg[c];
-    cta_desc[c * 3 + 1] = (int32_t)end[c];
-    cta_desc[c * 3 + 2] = first_split;
+    for (long i = 0; i < nseg; ++i) {
+      int s = segs[i];
+      if (holders[s] == 0 && held[i] < seg_units[s]) /* first piece of a cut segment */
+        first_slot[s] = (int32_t)(2 * c + (i == 0 ? 0 : 1));
+      holders[s] += 1;
+    }
+    cta_desc[c * 2 + 0] = (int32_t)beg[c];
+    cta_desc[c * 2 + 1] = (int32_t)end[c];
   }
   *n_ranges_out = (int32_t)nranges;
-  int32_t acc = 0;
-  for (int s = 0; s < S; ++s) {
-    split_count[s] = holders[s];
-    partial_base[s] = acc;
-    if (holders[s] > 1) acc += holders[s];
-  }
+  for (int s = 0; s < S; ++s) split_count[s] = holders[s];
+  free(seg_units); free(segs); free(held);
   free(ntile); free(unit_seg); free(unit_tile); free(seg_first_unit);
   free(beg); free(end); free(holders);
   return ORC_OK;

@@ -73,8 +73,8 @@ def test_workspace_layout_is_aligned_and_ordered(L):
     for kind, args in [(0, (32, 8, 64, 128, 148)), (1, (2, 2, 8, 64, 148)),
                        (2, (256, 8, 64, 128, 4864))]:
         lay = hpa.workspace_layout(kind, *args)
-        offs = [lay[k] for k in ["header", "lens", "tile_start", "cta_desc", "split_count",
-                                 "part_base", "part_ml", "part_acc", "total"]]
+        offs = [lay[k] for k in ["header", "lens", "tile_start", "cta_desc", "seg_desc",
+                                 "part_ml", "part_acc", "total"]]
         assert all(o % 256 == 0 for o in offs)
         assert offs == sorted(offs)
         B, Hkv, Hq, D, grid = args
@@ -83,7 +83,8 @@ def test_workspace_layout_is_aligned_and_ordered(L):
         assert lay["part_acc"] - lay["part_ml"] >= 2 * V * G * 8
         assert lay["total"] - lay["part_acc"] >= 2 * V * G * D * 4
         assert lay["cta_desc"] - lay["tile_start"] >= (B + 1) * 4
-        assert lay["split_count"] - lay["cta_desc"] >= 32 * V
+        assert lay["seg_desc"] - lay["cta_desc"] >= 32 * V
+        assert lay["part_ml"] - lay["seg_desc"] >= 8 * B * Hkv
         assert hpa.decode_workspace_size(kind, *args) == lay["total"]
     assert L.hpa_decode_workspace_size(0, 0, 8, 64, 128, 148) == 0
     assert L.hpa_decode_workspace_size(0, 2, 3, 8, 64, 148) == 0  # Hq % Hkv != 0

@@ -56,7 +56,7 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
         "header": header, "lens": i32(lay["lens"], B),
         "tile_start": i32(lay["tile_start"], B + 1),
         "cta": i32(lay["cta_desc"], 8 * V).reshape(V, 8),
-        "split_count": i32(lay["split_count"], S), "partial_base": i32(lay["part_base"], S),
+        "seg": i32(lay["seg_desc"], 2 * S).reshape(S, 2),
     }
 
 
@@ -89,7 +89,8 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
     assert got["header"][10] == ref["ranges"]
     np.testing.assert_array_equal(got["lens"], ref["lens"])
     np.testing.assert_array_equal(got["tile_start"], ref["tile_start"])
-    np.testing.assert_array_equal(got["cta"][:, :3], ref["cta"])
+    np.testing.assert_array_equal(got["cta"][:, :2], ref["cta"])
+    assert not got["cta"][:, 6:].any()
     # start state (b, g, t, tiles of b) of each CTA's first unit, from the oracle's offsets
     ts = ref["tile_start"].astype(np.int64)
     for c in range(ref["ranges"]):
@@ -99,9 +100,9 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
         b0 = int(np.searchsorted(ts * Hkv, ub, side="right") - 1)
         n0 = int(ts[b0 + 1] - ts[b0])
         rem = ub - int(ts[b0]) * Hkv
-        assert tuple(got["cta"][c, [3, 4, 5, 6]]) == (b0, rem // n0, rem % n0, n0), c
-    np.testing.assert_array_equal(got["split_count"], ref["split_count"])
-    np.testing.assert_array_equal(got["partial_base"], ref["partial_base"])
+        assert tuple(got["cta"][c, [2, 3, 4, 5]]) == (b0, rem // n0, rem % n0, n0), c
+    np.testing.assert_array_equal(got["seg"][:, 0], ref["first_slot"])
+    np.testing.assert_array_equal(got["seg"][:, 1], ref["split_count"])
     h = got["header"]
     assert h[2] == ref["n_units"] and h[3] == grid and h[1] == 0
 

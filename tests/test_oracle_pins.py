@@ -458,29 +458,41 @@ def _check_plan_invariants(p, lens, Hkv, kind):
             prev_end = e
         cover[a:e] += 1
     assert prev_end == U and np.all(cover == 1)
-    # split counts and first-split indices, recounted with Python sets
-    holders = {}
+    # split counts and partial slots, recounted with Python lists: range c
+    # keeps the piece of its first segment in slot 2c and that of its last in
+    # 2c + 1; the ranges holding a segment are consecutive
+    seg_units = {}
+    for (b, g, t) in units:
+        seg_units[b * Hkv + g] = seg_units.get(b * Hkv + g, 0) + 1
+    holders, pieces = {}, {}
     for c in range(R):
         a, e = int(cta[c, 0]), int(cta[c, 1])
         segs = []
         for u in range(a, e):
             s = units[u][0] * Hkv + units[u][1]
-            if not segs or segs[-1] != s:
-                segs.append(s)
-        for i, s in enumerate(segs):
-            if i == 0:
-                assert cta[c, 2] == len(holders.get(s, []))
+            if not segs or segs[-1][0] != s:
+                segs.append([s, 0])
+            segs[-1][1] += 1
+        for i, (s, n) in enumerate(segs):
             holders.setdefault(s, []).append(c)
-        if not segs:
-            assert cta[c, 2] == 0
+            if n < seg_units[s]:
+                # a cut piece is the range's first or last segment
+                assert i == 0 or i == len(segs) - 1
+                pieces.setdefault(s, []).append(2 * c + (0 if i == 0 else 1))
     S = len(lens) * Hkv
-    base = 0
     for s in range(S):
-        n = len(holders.get(s, []))
-        assert p["split_count"][s] == n
-        assert p["partial_base"][s] == base
-        if n > 1:
-            base += n
+        hs = holders.get(s, [])
+        assert p["split_count"][s] == len(hs)
+        assert hs == list(range(hs[0], hs[0] + len(hs))) if hs else True
+        if len(hs) > 1:
+            ps = pieces[s]
+            assert len(ps) == len(hs) and p["first_slot"][s] == ps[0]
+            assert ps[1:] == [2 * c for c in hs[1:]]
+        else:
+            assert p["first_slot"][s] == -1 and s not in pieces
+    # no slot is used twice
+    used = [x for ps in pieces.values() for x in ps]
+    assert len(used) == len(set(used)) and all(0 <= x < 2 * R for x in used)
     if kind == 0:
         P = p["grid"]
         sizes = [int(cta[c, 1] - cta[c, 0]) for c in range(R)]
