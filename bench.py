@@ -38,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "KV-cache GB/s (% of HBM peak), µs/decode step, skewed 1x128K+31x4K"
+L2_BYTES = 126 * 1000 * 1000  # B200 L2 capacity
 WORKLOAD = "skewed"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_run_skewed_ncu.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "mixed_length_paged_b200", "csrc", f)
@@ -54,6 +55,8 @@ def _args():
     ap.add_argument("--num-ctas", type=int, default=0,
                     help="persistent CTAs of the dynamic plan (0: the library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager launches instead of CUDA-graph replays of the step")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the static-plan comparison and the e2e leg")
     return ap.parse_args()
@@ -306,6 +309,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # algorithmic bytes of one run launch: live KV + q + out + page-table entries
     # read (+ the two fp32 scales of every (page, kv head) tile for FP8)
     run_bytes = kv_bytes + 2 * B * Hq * D * 2 + tiles * 4 + (tiles * Hkv * 8 if fp8 else 0)
+    if shape.prologue:
+        # the fused prologue also reads the new token's raw K and V rows and
+        # writes them (normalised, rotated) into their cache slots
+        run_bytes += 4 * B * Hkv * D * 2
     scale = 1.0 / math.sqrt(D)
     num_ctas = args.num_ctas or hpa.default_num_ctas(local_rank)
     stream = torch.cuda.current_stream()
@@ -313,22 +320,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
     seq_lens = batch.seq_lens
     if shape.prologue:
-        # the step starts from the new token's raw projections: the fused
-        # prologue writes q and the K/V slot, then plan + run attend over L + 1
+        # The step starts from the new token's raw projections: plan, then the
+        # run with the prologue (RMSNorm + RoPE of q and the new K row, the K/V
+        # slot write) fused into the decode kernel, attending over L + 1.
         batch.q = torch.empty_like(batch.q_raw)
 
-    def prologue():
-        if shape.prologue:
-            hpa.kv_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
-                            batch.positions, batch.page_table, batch.k_cache, batch.v_cache,
-                            batch.q, eps=1e-6, rope_theta=10000.0)
+    def prologue():  # the separate prologue kernel (comparator only)
+        hpa.kv_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
+                        batch.positions, batch.page_table, batch.k_cache, batch.v_cache,
+                        batch.q, eps=1e-6, rope_theta=10000.0)
 
     def run():
-        dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale,
-                k_scale=k_scale, v_scale=v_scale)
+        if shape.prologue:
+            dec.run_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
+                             batch.k_cache, batch.v_cache, batch.page_table, out, scale,
+                             eps=1e-6, rope_theta=10000.0)
+        else:
+            dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale,
+                    k_scale=k_scale, v_scale=v_scale)
 
     def step():
-        prologue()
         dec.plan(seq_lens)
         run()
 
@@ -339,6 +350,30 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     for _ in range(max(3, args.warmup)):
         step()
+    barrier()
+
+    def graphed(fn):
+        """One step captured as a CUDA graph (plan -> run -> merge keep their
+        programmatic-dependent-launch edges); replaying it costs one launch
+        call on the host.  A decode loop in a serving engine replays its step
+        this way; eagerly, ~35 us steps are bound by the host's launch rate."""
+        if args.eager:
+            return fn
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        graphs.append(g)
+        return g.replay
+
+    graphs = []
+    timed_step = graphed(step)
     barrier()
     K = args.steps
     sampler = ClockSampler(_smi_index(local_rank))
@@ -351,14 +386,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for _ in range(K):
-        step()
+        timed_step()
     end.record(stream)
     barrier()
     # Timed region 2 (per-kernel durations for the roofline): the same K
     # steps with events around the plan and around the run call.
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * K)]
     for i in range(K):
-        prologue()
         ev[3 * i].record(stream)
         dec.plan(seq_lens)
         ev[3 * i + 1].record(stream)
@@ -375,28 +409,75 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # static split-KV comparators: the same run kernel fed the static plans
     extras = {}
+    if not args.no_extras and shape.prologue:
+        # The same step with the prologue as its own kernel before plan + run,
+        # timed as an interleaved A/B against the fused step (blocks of 20
+        # steps each, alternating) so that clock and power drift over the run
+        # falls on both alike.
+        def separate():
+            prologue()
+            dec.plan(seq_lens)
+            dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale)
+
+        for _ in range(3):
+            separate()
+        torch.cuda.synchronize()
+        separate_step = graphed(separate)
+        blocks, per = 10, 20
+        ab = {"fused": 0.0, "separate": 0.0}
+        for _ in range(blocks):
+            for name, fn in (("fused", timed_step), ("separate", separate_step)):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(per):
+                    fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ab[name] += a.elapsed_time(b)
+        n = blocks * per
+        extras["separate_prologue_kernel"] = {
+            "us_per_step": 1e3 * ab["separate"] / n,
+            "fused_us_per_step_same_blocks": 1e3 * ab["fused"] / n,
+            "fused_speedup": ab["separate"] / ab["fused"],
+            "method": f"interleaved A/B, {blocks} x {per} steps each"}
+
     plain = not fp8 and not shape.prologue
     if not args.no_extras and plain:
+        # each static plan against the dynamic one as an interleaved A/B
+        # (alternating blocks of steps), so drift falls on both alike
+        blocks, per = 10, max(5, min(40, K // 10))
         for name, kind in (("static_nsplit", hpa.PLAN_STATIC_NSPLIT),
                            ("static_chunk", hpa.PLAN_STATIC_CHUNK)):
             sd = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, kind=kind, num_ctas=num_ctas,
                                   max_seq_len=int(lens.max()), device=dev)
+
+            def static_step():
+                sd(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale)
+
             for _ in range(3):
-                sd(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale)
+                static_step()
             torch.cuda.synchronize()
-            n = max(10, min(200, K))
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(n):
-                sd(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale)
-            b.record(stream)
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b) / n
+            static_timed = graphed(static_step)
+            ab = {"dynamic": 0.0, "static": 0.0}
+            for _ in range(blocks):
+                for which, fn in (("dynamic", timed_step), ("static", static_timed)):
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    for _ in range(per):
+                        fn()
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                    ab[which] += a.elapsed_time(b)
+            ms = ab["static"] / (blocks * per)
             extras[name] = {"us_per_step": 1e3 * ms, "GB_s": kv_bytes / (ms * 1e-3) / 1e9,
-                            "grid": sd.grid}
-        best_static = min(extras[k]["us_per_step"] for k in extras)
-        extras["dynamic_speedup_vs_best_static"] = best_static / (1e3 * ms_per_step)
+                            "grid": sd.grid,
+                            "dynamic_us_per_step_same_blocks": 1e3 * ab["dynamic"] / (blocks * per),
+                            "dynamic_speedup": ab["static"] / ab["dynamic"],
+                            "method": f"interleaved A/B, {blocks} x {per} steps each"}
+        extras["dynamic_speedup_vs_best_static"] = min(
+            extras[k]["dynamic_speedup"] for k in ("static_nsplit", "static_chunk"))
 
     # end to end through the public API: pinned host inputs -> device, step,
     # result -> pinned host, all inside the timed region
@@ -461,21 +542,30 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "config": {
             "workload": WORKLOAD_DESC.get(args.workload, args.workload),
             "batch": B, "kv_bytes_per_step_per_gpu": kv_bytes, "num_ctas": num_ctas,
-            "l2": "no flush: 1.06 GB of KV per step is larger than the 126 MB L2",
+            "l2": (f"no flush: {kv_bytes / 1e9:.3g} GB of KV per step is larger than the "
+                   "126 MB L2" if kv_bytes > L2_BYTES else
+                   f"L2-resident: {kv_bytes / 1e6:.3g} MB of KV per step fits the 126 MB L2 "
+                   "(a latency figure, not an HBM one)"),
+            "launch": "eager calls" if args.eager else
+                      "CUDA-graph replay of one captured step (plan + run)",
             "parallelism": f"data-parallel replicas x{world} (independent batches, no collective)",
         },
         "breakdown_us": {"plan": 1e3 * statistics.mean(plan_ms), "run": 1e3 * run_avg_ms,
                          "note": "events between the calls (timed region 2); the step time "
                                  "comes from timed region 1 without them"},
-        "roofline": {"bound": "hbm", "kernel": "hpa_decode_run (decode_kernel + merge_kernel)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("hpa_decode_run_prologue" if shape.prologue else "hpa_decode_run")
+                     + " (decode_kernel + merge_kernel)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy bandwidth",
                      "traffic": traffic, "algorithmic_bytes_per_launch": run_bytes},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (4 if shape.prologue else 3) * K,
+        "gpu_launches": 3 * K,  # plan, decode, merge
         "clocks": clocks,
-        "static_splitkv": extras or None,
+        "static_splitkv": {k: v for k, v in extras.items()
+                           if k.startswith(("static", "dynamic"))} or None,
+        "separate_prologue": extras.get("separate_prologue_kernel"),
         "device_status": status,
     }
     print(json.dumps(line), flush=True)

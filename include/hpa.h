@@ -205,6 +205,41 @@ HPA_API hpa_status hpa_decode_run(const void* q, const void* k_cache, const void
                           void* stream);
 
 /*
+ * hpa_decode_run_prologue -- hpa_decode_run with the decode prologue fused
+ * into the persistent kernel (bitbyai.com "vLLM x HPC-Ops", Attention
+ * Backend: RoPE, query-key normalisation and the KV write fused into one
+ * prologue to save launches and HBM round trips; here the prologue does not
+ * even get its own launch).
+ *
+ * Equivalent to hpa_kv_prologue(q_raw, k_raw, v_raw, q_gamma, k_gamma, eps,
+ * rope_theta, positions = seq_lens - 1, ...) followed by hpa_decode_run on
+ * its q_out, with the same bits in the output, in the written K/V slots and
+ * in q_out: every CTA that starts a piece of (sequence, kv head) normalises
+ * and rotates that head group's raw query rows in shared memory, and the CTA
+ * whose range holds a sequence's last tile computes the new token's K and V
+ * rows, stores them in their cache slot (position seq_len - 1) and only then
+ * loads that tile.
+ *
+ *   q_raw, k_raw, v_raw  device bf16 [batch][Hq][D] / [batch][Hkv][D], the
+ *                new token's pre-norm rows; 16-byte aligned.
+ *   q_gamma, k_gamma, eps, rope_theta  as for hpa_kv_prologue.
+ *   k_cache, v_cache  device bf16 caches (written at the new token's slot).
+ *   q_out        optional (NULL: not written) device bf16 [batch][Hq][D]:
+ *                the normalised, rotated queries.  Rows of sequences of
+ *                length 0 are not written.
+ *   the rest     as for hpa_decode_run; the plan's seq_lens are the
+ *                post-append lengths (the new token included).
+ * bf16 caches only (the call has no kv_dtype argument).  A length the plan
+ * clamped (HPA_DEVICE_LEN_CLAMPED) voids that step's output and K/V writes.
+ */
+HPA_API hpa_status hpa_decode_run_prologue(
+    const void* q_raw, const void* k_raw, const void* v_raw, const float* q_gamma,
+    const float* k_gamma, float eps, float rope_theta, void* k_cache, void* v_cache, void* q_out,
+    const int32_t* page_table, int pt_stride, int num_pages, void* out, hpa_out_dtype out_dtype,
+    int batch, int num_q_heads, int num_kv_heads, int head_dim, float softmax_scale,
+    hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * hpa_kv_prologue -- fused RMSNorm + RoPE + KV write for the new token of
  * each sequence (bitbyai.com "vLLM x HPC-Ops", Attention Backend: RoPE,
  * query-key normalisation and KV-write fused into one prologue).

@@ -9,7 +9,8 @@ it raises ``HpaLibraryMissing`` -- there is no fallback implementation.
 The functions mirror the C ABI in ``include/hpa.h``:
 
     decode_workspace_size, plan_grid, default_num_ctas, workspace_layout,
-    decode_plan, decode_run, kv_prologue, read_status
+    decode_plan, decode_run, decode_run_prologue, kv_prologue, read_status,
+    decode_noalloc
 
 and ``PagedDecoder`` bundles a workspace with plan + run for callers who do
 not want to manage it.
@@ -25,8 +26,8 @@ __all__ = [
     "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
     "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
-    "default_num_ctas", "workspace_layout", "decode_plan", "decode_run", "kv_prologue",
-    "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "default_num_ctas", "workspace_layout", "decode_plan", "decode_run", "decode_run_prologue",
+    "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
 PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2
@@ -84,6 +85,9 @@ def lib():
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
                                      _F, _I, _I, _V, _Z, _V]
+        L.hpa_decode_run_prologue.restype = _I
+        L.hpa_decode_run_prologue.argtypes = [_V, _V, _V, _V, _V, _F, _F, _V, _V, _V, _V, _I, _I,
+                                              _V, _I, _I, _I, _I, _I, _F, _I, _I, _V, _Z, _V]
         L.hpa_kv_prologue.restype = _I
         L.hpa_kv_prologue.argtypes = [_V, _V, _V, _V, _V, _F, _F, _V, _V, _I, _V, _V, _V, _I, _I,
                                       _I, _I, _I, _V, _V]
@@ -216,6 +220,45 @@ def decode_run(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     return out
 
 
+def decode_run_prologue(q_raw: torch.Tensor, k_raw: torch.Tensor, v_raw: torch.Tensor,
+                        q_gamma: torch.Tensor, k_gamma: torch.Tensor, k_cache: torch.Tensor,
+                        v_cache: torch.Tensor, page_table: torch.Tensor, out: torch.Tensor,
+                        workspace: torch.Tensor, grid: int, softmax_scale: float, *,
+                        q_out: torch.Tensor | None = None, eps: float = 1e-6,
+                        rope_theta: float = 10000.0, kind: int = PLAN_DYNAMIC,
+                        stream=None) -> torch.Tensor:
+    """decode_run with the prologue (RMSNorm + RoPE of q and of the new K row,
+    the K/V slot write) fused into the decode kernel; writes and returns
+    ``out``.  The plan in ``workspace`` must hold the post-append lengths; the
+    new token goes to position seq_len - 1.  bf16 caches only."""
+    for t, n, nd in ((q_raw, "q_raw", 3), (k_raw, "k_raw", 3), (v_raw, "v_raw", 3),
+                     (k_cache, "k_cache", 4), (v_cache, "v_cache", 4)):
+        _dev(t, n, (torch.bfloat16,), nd)
+    if q_out is not None:
+        _dev(q_out, "q_out", (torch.bfloat16,), 3)
+    _dev(q_gamma, "q_gamma", (torch.float32,), 1)
+    _dev(k_gamma, "k_gamma", (torch.float32,), 1)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    _dev(out, "out", (torch.bfloat16, torch.float32), 3)
+    _dev(workspace, "workspace", (torch.uint8,))
+    B, Hq, D = q_raw.shape
+    num_pages, Hkv, S, Dk = k_cache.shape
+    if S != PAGE_SIZE or Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or tuple(out.shape) != tuple(q_raw.shape) or page_table.shape[0] != B \
+            or tuple(k_raw.shape) != (B, Hkv, D) or tuple(v_raw.shape) != (B, Hkv, D) \
+            or q_gamma.numel() != D or k_gamma.numel() != D \
+            or (q_out is not None and tuple(q_out.shape) != tuple(q_raw.shape)):
+        raise HpaError("decode_run_prologue: inconsistent shapes")
+    rc = lib().hpa_decode_run_prologue(
+        _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(q_gamma), _ptr(k_gamma), float(eps),
+        float(rope_theta), _ptr(k_cache), _ptr(v_cache), _ptr(q_out), _ptr(page_table),
+        page_table.shape[1], num_pages, _ptr(out),
+        OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, Hq, Hkv, D,
+        float(softmax_scale), kind, grid, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "hpa_decode_run_prologue")
+    return out
+
+
 def kv_prologue(q_raw, k_raw, v_raw, q_gamma, k_gamma, positions, page_table, k_cache, v_cache,
                 q_out, *, eps: float = 1e-6, rope_theta: float = 10000.0, status=None,
                 stream=None) -> torch.Tensor:
@@ -307,6 +350,13 @@ class PagedDecoder:
         return decode_run(q, k_cache, v_cache, page_table, out, self.workspace, self.grid,
                           softmax_scale, kind=self.kind, k_scale=k_scale, v_scale=v_scale,
                           stream=stream)
+
+    def run_prologue(self, q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache, v_cache, page_table,
+                     out, softmax_scale, **kw):
+        """The planned step with the prologue fused in (decode_run_prologue)."""
+        return decode_run_prologue(q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache, v_cache,
+                                   page_table, out, self.workspace, self.grid, softmax_scale,
+                                   kind=self.kind, **kw)
 
     def __call__(self, q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, **kw):
         self.plan(seq_lens, stream=kw.get("stream"))

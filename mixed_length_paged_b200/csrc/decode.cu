@@ -51,6 +51,7 @@
 #include <cuda_bf16.h>
 
 #include "hpa_common.cuh"
+#include "prologue_math.cuh"
 
 namespace hpa {
 namespace {
@@ -64,7 +65,7 @@ constexpr int kSmemPerSm = 228 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any barrier wait
 constexpr int kDepBufs = 2;              // deposit slots between consumers and epilogue
 
-template <int D, int NT, bool FP8, int CPS>
+template <int D, int NT, bool FP8, int CPS, bool PRO>
 struct Cfg {
   static constexpr int kElt = FP8 ? 1 : 2;
   static constexpr int kRowBytes = D * kElt;           // one token row of one head
@@ -74,6 +75,9 @@ struct Cfg {
   static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
   static constexpr int kHeads = 8 * NT;                // MMA N (padded group)
   static constexpr int kQBytes = kHeads * D * 2;       // a segment's bf16 query rows
+  // fused prologue: the new token's raw K and V rows ride behind the q rows
+  static constexpr int kRawBytes = PRO ? 2 * D * 2 : 0;
+  static constexpr int kSlotBytes = kQBytes + kRawBytes; // per-stage q (+ raw rows) slot
   static constexpr int kAccStride = D + 4;             // floats; keeps deposits off one bank
   // one deposit: acc[warp][head][D + 4] floats, then (m, l)[warp][head]
   static constexpr int kDepAccFloats = kConsumerWarps * kHeads * kAccStride;
@@ -82,10 +86,10 @@ struct Cfg {
   // CPS CTAs share one SM's 228 KiB (1 KiB of it reserved per CTA)
   static constexpr int kBudget = CPS == 1 ? kSmemLimit : (kSmemPerSm / CPS - 1024);
   static constexpr int kStagesFit =
-      (kBudget - 1024 - kDepBufs * kDepBytes - kMisc) / (kStageBytes + kQBytes);
+      (kBudget - 1024 - kDepBufs * kDepBytes - kMisc) / (kStageBytes + kSlotBytes);
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
   static constexpr int kSmemBytes =
-      1024 + kStages * (kStageBytes + kQBytes) + kDepBufs * kDepBytes + kMisc;
+      1024 + kStages * (kStageBytes + kSlotBytes) + kDepBufs * kDepBytes + kMisc;
   static constexpr int kKSteps = D / 16;               // QK MMA k-steps
   static constexpr int kMTiles = D / 16;               // PV MMA m-tiles
   static constexpr int kVec = D / 32;                  // output floats per epilogue lane
@@ -95,7 +99,7 @@ struct Cfg {
 };
 
 struct RunParams {
-  const uint16_t* q;        // bf16 bits [B][Hq][D]
+  const uint16_t* q;        // bf16 bits [B][Hq][D] (raw, pre-norm rows under the fused prologue)
   const float* k_scale;     // [pages][Hkv] (FP8)
   const float* v_scale;
   const int32_t* page_table;
@@ -106,15 +110,29 @@ struct RunParams {
   Ws ws;
   int grid, kind;
   int slots;                // 2 * V partial slots in the workspace
+  // fused prologue only: raw new-token K/V rows, weights, caches to write
+  const __nv_bfloat16* k_raw;  // [B][Hkv][D]
+  const __nv_bfloat16* v_raw;
+  const float* q_gamma;        // [D]
+  const float* k_gamma;
+  float eps;
+  double log2_theta;
+  __nv_bfloat16* k_cache_w;    // the K/V caches the TMA maps read
+  __nv_bfloat16* v_cache_w;
+  __nv_bfloat16* q_out;        // optional copy of the normalised, rotated q
 };
 
 // What the producer resolved for the unit held in one stage.
 constexpr int kFirst = 1;   // first tile of its segment in this range
 constexpr int kLast = 2;    // last tile of its segment in this range
 constexpr int kEnd = 4;     // no unit: the producer has no more work
+constexpr int kNewTok = 8;  // fused prologue: the tile that receives the new token
+constexpr int kSegStart = 16;  // tile 0 of its segment
 struct alignas(16) StageInfo {
-  int32_t b, g, valid, flags;   // sequence, kv head, live tokens in the tile, kFirst|kLast
-  int32_t slot, pad0, pad1, pad;  // partial slot of the segment's piece (-1: whole segment)
+  int32_t b, g, valid, flags;   // sequence, kv head, live tokens in the tile, k* flags
+  int32_t slot, pos, row, pad;   // partial slot of the segment's piece (-1: whole
+                                 // segment); fused prologue: new token's position,
+                                 // first cache row of the tile
   float k_scale, v_scale, pad2, pad3;
 };
 
@@ -195,37 +213,51 @@ __device__ __forceinline__ void store_out_vec(void* out, long long i, const floa
   }
 }
 
-template <int D, int NT, bool FP8, bool OUT_F32, int CPS>
+template <int D, int NT, bool FP8, bool OUT_F32, int CPS, bool PRO>
 __global__ void __launch_bounds__(kThreads, CPS)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const RunParams p) {
-  using C = Cfg<D, NT, FP8, CPS>;
+  using C = Cfg<D, NT, FP8, CPS, PRO>;
+  static_assert(!(PRO && FP8), "the fused prologue writes bf16 caches");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   uint8_t* qslots = smem + C::kStages * C::kStageBytes;
-  uint8_t* deps = qslots + C::kStages * C::kQBytes;     // kDepBufs deposit slots
+  uint8_t* deps = qslots + C::kStages * C::kSlotBytes;  // kDepBufs deposit slots
   uint8_t* misc = deps + kDepBufs * C::kDepBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(misc);
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* dep_full = empty_bar + C::kStages;
   uint64_t* dep_empty = dep_full + kDepBufs;
-  StageInfo* info = reinterpret_cast<StageInfo*>(dep_empty + kDepBufs);
+  uint64_t* q_full = dep_empty + kDepBufs;  // a stage's small copies (q rows, raw rows) landed
+  // StageInfo / DepDesc are read and written as 16-byte vectors
+  StageInfo* info = reinterpret_cast<StageInfo*>(
+      (reinterpret_cast<uintptr_t>(q_full + C::kStages) + 15) & ~uintptr_t(15));
   DepDesc* dep_desc = reinterpret_cast<DepDesc*>(info + C::kStages);
   volatile int* s_flags = reinterpret_cast<volatile int*>(dep_desc + kDepBufs);
   volatile int* s_abort = s_flags;
   volatile int* s_plan_ok = s_flags + 1;
+  uint64_t* q_ready = reinterpret_cast<uint64_t*>(const_cast<int*>(s_flags) + 2);  // fused prologue: q rows done
+  // fused prologue: RMSNorm weights, in the upper half of the misc area
+  float* s_qgamma = reinterpret_cast<float*>(misc + C::kMisc / 2);
+  float* s_kgamma = s_qgamma + D;
+  static_assert(C::kMisc / 2 >= 2 * D * 4, "misc area too small for the weights");
+  static_assert(C::kStages * 24 + kDepBufs * 16 + 8 + C::kStages * sizeof(StageInfo) +
+                        kDepBufs * sizeof(DepDesc) + 16 <= C::kMisc / 2,
+                "misc area too small");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&q_full[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), kConsumerWarps);
     }
     for (int d = 0; d < kDepBufs; ++d) {
       mbar_init(smem_u32(&dep_full[d]), kConsumerWarps);
       mbar_init(smem_u32(&dep_empty[d]), 1);
     }
+    mbar_init(smem_u32(q_ready), kConsumerWarps * 32);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -244,6 +276,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
                     h[kHdrRanges] <= plan_ranges_ll(p.kind, p.grid);
     *s_plan_ok = ok;
     if (!ok) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
+  }
+  if constexpr (PRO) {
+    for (int i = threadIdx.x; i < D; i += kThreads) {
+      s_qgamma[i] = p.q_gamma[i];
+      s_kgamma[i] = p.k_gamma[i];
+    }
   }
   __syncthreads();
   if (!*s_plan_ok) return;
@@ -286,13 +324,15 @@ __global__ void __launch_bounds__(kThreads, CPS)
           Walk w2 = wk;
           for (int k = 0; k < lane && u0 + k + 1 < ue; ++k) w2.next(ts, p.Hkv);
           const int u = u0 + lane;
-          int row = 0, valid = 0, flags = 0, slot = -1, bad = 0;
+          int row = 0, valid = 0, flags = 0, slot = -1, bad = 0, pos = 0;
           float ks = 1.f, vs = 1.f;
           if (u < ue) {
             const int page = __ldg(p.page_table + (long long)w2.b * p.pt_stride + w2.t);
             const int L = p.ws.lens[w2.b];
             valid = min(kPageSize, L - w2.t * kPageSize);
-            flags = ((w2.t == 0 || u == ub) ? kFirst : 0) | ((w2.t == w2.n - 1 || u == ue - 1) ? kLast : 0);
+            flags = ((w2.t == 0 || u == ub) ? kFirst : 0) | ((w2.t == w2.n - 1 || u == ue - 1) ? kLast : 0) |
+                    (w2.t == 0 ? kSegStart : 0) | ((PRO && w2.t == w2.n - 1) ? kNewTok : 0);
+            pos = L - 1;  // the new token's position (post-append length - 1)
             if (flags & kLast) {
               // The piece of this segment in range v is whole if the segment
               // starts inside the range and ends here.  Otherwise it is a
@@ -311,39 +351,55 @@ __global__ void __launch_bounds__(kThreads, CPS)
               }
             }
           }
-          // small fields travel packed: valid (7 bits) | flags (2) | bad (1) | g (<< 10)
-          const int packed = valid | (flags << 7) | (bad << 9) | (w2.g << 10);
+          // small fields travel packed: valid (7 bits) | flags (5) | bad (1) | g (<< 13)
+          const int packed = valid | (flags << 7) | (bad << 12) | (w2.g << 13);
           const int cnt = min(32, ue - u0);
           for (int k = 0; k < cnt; ++k) {
             const int rk = __shfl_sync(0xffffffffu, row, k);
             const int pk = __shfl_sync(0xffffffffu, packed, k);
             StageInfo si;
             si.b = __shfl_sync(0xffffffffu, w2.b, k);
-            si.g = pk >> 10;
+            si.g = pk >> 13;
             si.valid = pk & 127;
-            si.flags = (pk >> 7) & 3;
-            const int bk = (pk >> 9) & 1;
+            si.flags = (pk >> 7) & 31;
+            const int bk = (pk >> 12) & 1;
             si.slot = -1;
             if (si.flags & kLast)  // warp-uniform: pk is the same in every lane
               si.slot = __shfl_sync(0xffffffffu, slot, k);
-            si.pad0 = si.pad1 = si.pad = 0;
+            si.pos = PRO ? __shfl_sync(0xffffffffu, pos, k) : 0;
+            si.pad = 0;
             si.k_scale = si.v_scale = 1.f;
             if constexpr (FP8) {
               si.k_scale = __shfl_sync(0xffffffffu, ks, k);
               si.v_scale = __shfl_sync(0xffffffffu, vs, k);
             }
             si.pad2 = si.pad3 = 0.f;
+            si.row = rk;
+            if (bk) si.flags &= ~kNewTok;  // no tile, no new row
             if (lane == 0) {
               const int s = it % C::kStages;
               const uint32_t par = ((it / C::kStages) & 1) ^ 1;
-              const uint32_t fb = smem_u32(&full_bar[s]);
+              const uint32_t fb = smem_u32(&full_bar[s]), qb = smem_u32(&q_full[s]);
               if (wait_bar(smem_u32(&empty_bar[s]), par, s_abort, status) && !bk) {
                 info[s] = si;
                 const bool first = si.flags & kFirst;
-                mbar_arrive_expect_tx(fb, C::kStageBytes + (first ? qbytes : 0));
+                const bool newtok = PRO && (si.flags & kNewTok);
+                // The small copies complete on q_full, so that the consumers
+                // can prepare the query (and the new K row) while the K/V
+                // tiles, which complete on full_bar, are still in flight.
+                mbar_arrive_expect_tx(qb, (first ? qbytes : 0) + (newtok ? 4 * D : 0));
                 if (first)
-                  bulk_load(smem_u32(qslots + s * C::kQBytes),
-                            p.q + ((long long)si.b * p.Hq + (long long)si.g * p.G) * D, qbytes, fb);
+                  bulk_load(smem_u32(qslots + s * C::kSlotBytes),
+                            p.q + ((long long)si.b * p.Hq + (long long)si.g * p.G) * D, qbytes, qb);
+                if (newtok) {
+                  // the new token's raw K and V rows, for the consumers to
+                  // patch into this tile
+                  const long long src = ((long long)si.b * p.Hkv + si.g) * D;
+                  const uint32_t raw = smem_u32(qslots + s * C::kSlotBytes + C::kQBytes);
+                  bulk_load(raw, p.k_raw + src, 2 * D, qb);
+                  bulk_load(raw + 2 * D, p.v_raw + src, 2 * D, qb);
+                }
+                mbar_arrive_expect_tx(fb, C::kStageBytes);
                 const uint32_t kdst = smem_u32(stages + s * C::kStageBytes);
                 const uint32_t vdst = kdst + C::kTileBytes;
     #pragma unroll
@@ -355,7 +411,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
               } else {
                 info[s] = si;
                 if (bk) atomicOr(status, HPA_DEVICE_BAD_PAGE);
-                mbar_arrive(fb);  // release the consumers without data (result void)
+                mbar_arrive(qb);  // release the consumers without data (result void)
+                mbar_arrive(fb);
               }
             }
             __syncwarp();
@@ -378,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
         StageInfo si = {};
         si.flags = kEnd;
         info[s] = si;
+        mbar_arrive(smem_u32(&q_full[s]));
         mbar_arrive(smem_u32(&full_bar[s]));
       }
     }
@@ -393,9 +451,10 @@ __global__ void __launch_bounds__(kThreads, CPS)
       const int first = max(0, it - C::kStages);
       for (int j = first; j < it; ++j) {
         const int s = j % C::kStages;
-        const uint32_t fb = smem_u32(&full_bar[s]);
+        const uint32_t fb = smem_u32(&full_bar[s]), qb = smem_u32(&q_full[s]);
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(fb, (j / C::kStages) & 1) && globaltimer() - t0 < kWaitNs) {
+        while (!(mbar_try_wait(fb, (j / C::kStages) & 1) && mbar_try_wait(qb, (j / C::kStages) & 1)) &&
+               globaltimer() - t0 < kWaitNs) {
         }
       }
     }
@@ -488,6 +547,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
   float acc[NT][C::kMTiles][4];
   float m_run[NT][2], l_run[NT][2];
   int nseg = 0;  // segments deposited so far
+  int nq = 0;    // fused prologue: q_ready phases completed
+  RopeLane<D> rope;  // fused prologue: cos/sin at the current piece's new-token position
 
   // Hand this warp's state of a finished segment to the epilogue warp.
   auto deposit = [&](const StageInfo* inf) {
@@ -541,15 +602,35 @@ __global__ void __launch_bounds__(kThreads, CPS)
 
   for (int it = 0;; ++it) {
     const int s = it % C::kStages;
-    if (!wait_bar(smem_u32(&full_bar[s]), (it / C::kStages) & 1, s_abort, status)) break;
+    const uint32_t par = (it / C::kStages) & 1;
+    if (!wait_bar(smem_u32(&q_full[s]), par, s_abort, status)) break;
     const StageInfo inf = info[s];
     if (inf.flags & kEnd) break;
     const uint32_t kt = smem_u32(stages + s * C::kStageBytes);
     const uint32_t vt = kt + C::kTileBytes;
 
     if (inf.flags & kFirst) {
+      if constexpr (PRO) {
+        // RMSNorm + RoPE of the G raw query rows, in place in the stage's q
+        // slot: consumer warp w takes rows w, w + 4, ...; the piece holding
+        // the segment's tile 0 also writes them out.  Every lane arrives on
+        // q_ready after its stores, and all wait for all.
+        __nv_bfloat16* qrows = reinterpret_cast<__nv_bfloat16*>(qslots + s * C::kSlotBytes);
+        rope.init(inf.pos, lane, p.log2_theta);  // kept for this piece's new K row
+        for (int h = warp; h < p.G; h += kConsumerWarps) {
+          __nv_bfloat16* qo = (p.q_out && (inf.flags & kSegStart))
+                                  ? p.q_out + ((long long)inf.b * p.Hq + (long long)inf.g * p.G + h) * D
+                                  : nullptr;
+          norm_rope_row<D>(qrows + h * D, qrows + h * D, qo, s_qgamma, p.eps, rope, lane);
+        }
+        // the slot is refilled by a bulk copy once the stage is released
+        fence_proxy_async_shared();
+        mbar_arrive(smem_u32(q_ready));
+        if (!wait_bar(smem_u32(q_ready), nq & 1, s_abort, status)) break;
+        ++nq;
+      }
       // query fragments (MMA B operand) of this kv head's G query heads
-      const uint16_t* qs = reinterpret_cast<const uint16_t*>(qslots + s * C::kQBytes);
+      const uint16_t* qs = reinterpret_cast<const uint16_t*>(qslots + s * C::kSlotBytes);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int hh = nt * 8 + r;
@@ -575,6 +656,52 @@ __global__ void __launch_bounds__(kThreads, CPS)
           for (int j = 0; j < 4; ++j) acc[nt][i][j] = 0.f;
         m_run[nt][0] = m_run[nt][1] = -INFINITY;
         l_run[nt][0] = l_run[nt][1] = 0.f;
+      }
+    }
+
+    // Fused prologue: if the new token's row lies in this warp's 16-token
+    // slice, form its K row (RMSNorm + RoPE of the raw row; the piece's
+    // cos/sin are already in `rope`) while the tiles are still in flight.
+    const bool patch = PRO && (inf.flags & kNewTok) && warp == ((inf.pos & (kPageSize - 1)) >> 4);
+    __nv_bfloat16 klo[D / 64], khi[D / 64];
+    if constexpr (PRO) {
+      if (patch)
+        norm_rope_vals<D>(reinterpret_cast<const __nv_bfloat16*>(qslots + s * C::kSlotBytes + C::kQBytes),
+                          s_kgamma, p.eps, rope, lane, klo, khi);
+    }
+
+    if (!wait_bar(smem_u32(&full_bar[s]), par, s_abort, status)) break;
+
+    if constexpr (PRO) {
+      if (patch) {
+        // patch the new K and V rows into the landed tiles (128-byte
+        // swizzle) and write them to their cache slot
+        const int tr = inf.pos & (kPageSize - 1);
+        const uint4* vraw = reinterpret_cast<const uint4*>(qslots + s * C::kSlotBytes + C::kQBytes + 2 * D);
+        uint8_t* ktile = stages + s * C::kStageBytes;
+        uint8_t* vtile = ktile + C::kTileBytes;
+        __nv_bfloat16* kdst = p.k_cache_w + ((long long)inf.row + tr) * D;
+        uint4* vdst = reinterpret_cast<uint4*>(p.v_cache_w + ((long long)inf.row + tr) * D);
+        // byte offset of 16-byte chunk j (of D * 2 / 16) of row tr inside a tile
+        auto chunk_off = [&](int j) {
+          return (j >> 3) * C::kBoxBytes + tr * 128 + (((j & 7) ^ (tr & 7)) << 4);
+        };
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j) {
+          const int i = lane + 32 * j, i2 = i + D / 2;
+          *reinterpret_cast<__nv_bfloat16*>(ktile + chunk_off(i >> 3) + (i & 7) * 2) = klo[j];
+          *reinterpret_cast<__nv_bfloat16*>(ktile + chunk_off(i2 >> 3) + (i2 & 7) * 2) = khi[j];
+          kdst[i] = klo[j];
+          kdst[i2] = khi[j];
+        }
+        if (lane < D / 8) {
+          const uint4 v = vraw[lane];
+          *reinterpret_cast<uint4*>(vtile + chunk_off(lane)) = v;
+          vdst[lane] = v;
+        }
+        // the stage is refilled by TMA once released
+        fence_proxy_async_shared();
+        __syncwarp();
       }
     }
 
@@ -860,7 +987,7 @@ EncodeTiledFn get_encode_fn() {
 
 // A cache viewed as a 2-D tensor [num_pages * Hkv * 64 rows][D]; one box is 64
 // rows x 128 bytes with 128-byte swizzle.
-bool make_cache_map(CUtensorMap* tm, const void* base, int num_pages, int Hkv, int D, bool fp8) {
+bool encode_cache_map(CUtensorMap* tm, const void* base, int num_pages, int Hkv, int D, bool fp8) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const int elt = fp8 ? 1 : 2;
@@ -875,11 +1002,37 @@ bool make_cache_map(CUtensorMap* tm, const void* base, int num_pages, int Hkv, i
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int NT, bool FP8, bool OUT_F32, int CPS>
+// The same caches come back every decode step: keep the last few maps per
+// host thread, keyed by everything the map encodes, instead of encoding two
+// maps per call.
+bool make_cache_map(CUtensorMap* tm, const void* base, int num_pages, int Hkv, int D, bool fp8) {
+  struct Entry {
+    const void* base;
+    int num_pages, Hkv, D;
+    bool fp8, used;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 8;
+  thread_local Entry cache[kEntries] = {};
+  thread_local int next = 0;
+  for (const Entry& e : cache)
+    if (e.used && e.base == base && e.num_pages == num_pages && e.Hkv == Hkv && e.D == D &&
+        e.fp8 == fp8) {
+      *tm = e.map;
+      return true;
+    }
+  if (!encode_cache_map(tm, base, num_pages, Hkv, D, fp8)) return false;
+  Entry& e = cache[next];
+  next = (next + 1) % kEntries;
+  e = Entry{base, num_pages, Hkv, D, fp8, true, *tm};
+  return true;
+}
+
+template <int D, int NT, bool FP8, bool OUT_F32, int CPS, bool PRO>
 hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams& p, int grid,
                   cudaStream_t stream) {
-  using C = Cfg<D, NT, FP8, CPS>;
-  auto kern = decode_kernel<D, NT, FP8, OUT_F32, CPS>;
+  using C = Cfg<D, NT, FP8, CPS, PRO>;
+  auto kern = decode_kernel<D, NT, FP8, OUT_F32, CPS, PRO>;
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<uint64_t> ready_mask{0};
   int dev = 0;
@@ -918,16 +1071,34 @@ hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams&
 // One persistent CTA per SM when the grid fits the SMs; two co-resident
 // (smaller) CTAs per SM when the grid is larger, so that twice as many
 // consumer warps hide each other's latencies.
-template <int D, bool FP8, bool OUT_F32>
+template <int D, bool FP8, bool OUT_F32, bool PRO>
 hpa_status launch_nt(int nt, int cps, const CUtensorMap& tk, const CUtensorMap& tv,
                      const RunParams& p, int grid, cudaStream_t s) {
   if (cps == 1)
-    return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1>(tk, tv, p, grid, s)
-                   : launch<D, 2, FP8, OUT_F32, 1>(tk, tv, p, grid, s);
+    return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s)
+                   : launch<D, 2, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s);
   // G = 16 (two n-tiles) does not fit two CTAs per SM: it always runs one
-  return nt == 1 ? launch<D, 1, FP8, OUT_F32, 2>(tk, tv, p, grid, s)
-                 : launch<D, 2, FP8, OUT_F32, 1>(tk, tv, p, grid, s);
+  return nt == 1 ? launch<D, 1, FP8, OUT_F32, 2, PRO>(tk, tv, p, grid, s)
+                 : launch<D, 2, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s);
 }
+
+template <bool OUT_F32, bool PRO>
+hpa_status launch_d(bool fp8, int head_dim, int nt, int cps, const CUtensorMap& tk,
+                    const CUtensorMap& tv, const RunParams& p, int grid, cudaStream_t s) {
+  if constexpr (!PRO) {
+    if (fp8) return launch_nt<128, true, OUT_F32, false>(nt, cps, tk, tv, p, grid, s);
+  }
+  return head_dim == 128 ? launch_nt<128, false, OUT_F32, PRO>(nt, cps, tk, tv, p, grid, s)
+                         : launch_nt<64, false, OUT_F32, PRO>(nt, cps, tk, tv, p, grid, s);
+}
+
+// Arguments of the fused prologue (hpa_decode_run_prologue).
+struct ProArgs {
+  const void *k_raw, *v_raw;
+  const float *q_gamma, *k_gamma;
+  float eps, rope_theta;
+  void* q_out;
+};
 
 // Cached SM count of the current device (0 if unknown).
 int sm_count() {
@@ -942,19 +1113,14 @@ int sm_count() {
   return n;
 }
 
-}  // namespace
-}  // namespace hpa
-
-using namespace hpa;
-
-extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const void* v_cache,
-                                     const float* k_scale, const float* v_scale,
-                                     hpa_kv_dtype kv_dtype, const int32_t* page_table,
-                                     int pt_stride, int num_pages, void* out,
-                                     hpa_out_dtype out_dtype, int batch, int num_q_heads,
-                                     int num_kv_heads, int head_dim, float softmax_scale,
-                                     hpa_plan_kind kind, int grid, void* workspace,
-                                     size_t ws_bytes, void* stream) {
+// Validation, parameters and launches shared by hpa_decode_run and
+// hpa_decode_run_prologue (pro != nullptr: q is the raw query).
+hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                    const float* v_scale, hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                    int pt_stride, int num_pages, void* out, hpa_out_dtype out_dtype, int batch,
+                    int num_q_heads, int num_kv_heads, int head_dim, float softmax_scale,
+                    hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream,
+                    const ProArgs* pro) {
   if (!q || !k_cache || !v_cache || !page_table || !out || !workspace) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || pt_stride <= 0 || num_pages <= 0 ||
       grid <= 0)
@@ -974,6 +1140,16 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
     return HPA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 3))
     return HPA_ERR_INVALID_ARG;
+  if (pro) {
+    if (!pro->k_raw || !pro->v_raw || !pro->q_gamma || !pro->k_gamma) return HPA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(pro->k_raw) | reinterpret_cast<uintptr_t>(pro->v_raw)) & 15)
+      return HPA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(pro->q_out) & 1) return HPA_ERR_INVALID_ARG;
+    if (!(pro->eps >= 0.f) || !std::isfinite(pro->eps) || !(pro->rope_theta > 0.f) ||
+        !std::isfinite(pro->rope_theta))
+      return HPA_ERR_INVALID_ARG;
+    if (fp8) return HPA_ERR_UNSUPPORTED;  // the new row would need a new page scale
+  }
   WsLayout L;
   if (!ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, &L))
     return HPA_ERR_INVALID_ARG;
@@ -1002,21 +1178,27 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
   p.grid = grid;
   p.kind = kind;
   p.slots = (int)(2 * plan_ranges_ll(kind, grid));
+  p.k_raw = pro ? static_cast<const __nv_bfloat16*>(pro->k_raw) : nullptr;
+  p.v_raw = pro ? static_cast<const __nv_bfloat16*>(pro->v_raw) : nullptr;
+  p.q_gamma = pro ? pro->q_gamma : nullptr;
+  p.k_gamma = pro ? pro->k_gamma : nullptr;
+  p.eps = pro ? pro->eps : 0.f;
+  p.log2_theta = pro ? std::log2((double)pro->rope_theta) : 0.0;
+  p.k_cache_w = pro ? static_cast<__nv_bfloat16*>(const_cast<void*>(k_cache)) : nullptr;
+  p.v_cache_w = pro ? static_cast<__nv_bfloat16*>(const_cast<void*>(v_cache)) : nullptr;
+  p.q_out = pro ? static_cast<__nv_bfloat16*>(pro->q_out) : nullptr;
   const int nt = G > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool f32 = out_dtype == HPA_OUT_F32;
   hpa_status st;
-  if (fp8)
-    st = f32 ? launch_nt<128, true, true>(nt, cps, tk, tv, p, grid, s)
-             : launch_nt<128, true, false>(nt, cps, tk, tv, p, grid, s);
-  else if (head_dim == 128)
-    st = f32 ? launch_nt<128, false, true>(nt, cps, tk, tv, p, grid, s)
-             : launch_nt<128, false, false>(nt, cps, tk, tv, p, grid, s);
+  if (pro)
+    st = f32 ? launch_d<true, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
+             : launch_d<false, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
   else
-    st = f32 ? launch_nt<64, false, true>(nt, cps, tk, tv, p, grid, s)
-             : launch_nt<64, false, false>(nt, cps, tk, tv, p, grid, s);
+    st = f32 ? launch_d<true, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
+             : launch_d<false, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
   if (st != HPA_OK) return st;
 
   // split merge, chained behind the decode kernel
@@ -1050,4 +1232,32 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
     return HPA_ERR_CUDA;
   }
   return HPA_OK;
+}
+
+}  // namespace
+}  // namespace hpa
+
+extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const void* v_cache,
+                                     const float* k_scale, const float* v_scale,
+                                     hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                                     int pt_stride, int num_pages, void* out,
+                                     hpa_out_dtype out_dtype, int batch, int num_q_heads,
+                                     int num_kv_heads, int head_dim, float softmax_scale,
+                                     hpa_plan_kind kind, int grid, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
+                       num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
+                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr);
+}
+
+extern "C" hpa_status hpa_decode_run_prologue(
+    const void* q_raw, const void* k_raw, const void* v_raw, const float* q_gamma,
+    const float* k_gamma, float eps, float rope_theta, void* k_cache, void* v_cache, void* q_out,
+    const int32_t* page_table, int pt_stride, int num_pages, void* out, hpa_out_dtype out_dtype,
+    int batch, int num_q_heads, int num_kv_heads, int head_dim, float softmax_scale,
+    hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream) {
+  const hpa::ProArgs pro{k_raw, v_raw, q_gamma, k_gamma, eps, rope_theta, q_out};
+  return hpa::run_impl(q_raw, k_cache, v_cache, nullptr, nullptr, HPA_KV_BF16, page_table,
+                       pt_stride, num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads,
+                       head_dim, softmax_scale, kind, grid, workspace, ws_bytes, stream, &pro);
 }

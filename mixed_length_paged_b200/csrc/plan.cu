@@ -193,59 +193,63 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     if (i < p.B) p.ws.lens[i] = min(max(p.seq_lens[i], 0), p.capacity);
   }
 
-  // 2. per-range unit ranges and the state of each range's first unit
-  for (long long c = first; c < V; c += stride) {
-    long long ub, ue;
-    int b0 = 0, g0 = 0, t0 = 0, n0 = 0;
-    if (dyn) {
-      dg.bounds(c, &ub, &ue);
-      if (ub < ue) {
-        b0 = seq_of_unit(ts, p.B, p.Hkv, ub);
-        n0 = ts[b0 + 1] - ts[b0];
-        const int rem = (int)(ub - (long long)ts[b0] * p.Hkv);  // < Hkv * n0 < 2^31
-        g0 = rem / n0;
-        t0 = rem - g0 * n0;
-      }
-    } else {
-      const int s = (int)c / per, i = (int)c % per;
-      b0 = s / p.Hkv;
-      g0 = s % p.Hkv;
-      const long long n = ts[b0 + 1] - ts[b0];
-      const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
-      const long long c0 = std::min<long long>((long long)i * C, n);
-      const long long c1 = std::min<long long>((long long)(i + 1) * C, n);
-      const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n;
-      ub = seg_start + c0;
-      ue = seg_start + c1;
-      t0 = (int)c0;
-      n0 = (int)n;
-    }
-    p.ws.cta_desc[2 * c] = make_int4((int)ub, (int)ue, b0, g0);
-    p.ws.cta_desc[2 * c + 1] = make_int4(t0, n0, 0, 0);
-  }
-
-  // 3. per segment: the ranges holding it and the slot of its first partial
-  for (int s = first; s < S; s += stride) {
-    const int b = s / p.Hkv, g = s - b * p.Hkv;
-    const long long n = ts[b + 1] - ts[b];
-    int nsplit = 0, slot0 = -1;
-    if (n > 0) {
+  // 2. per range: its unit range and the state of its first unit; per
+  //    segment: the ranges holding it and the slot of its first partial.
+  //    (One loop, so that the two independent latency chains overlap.)
+  const long long work = V > S ? V : S;
+  for (long long c = first; c < work; c += stride) {
+    if (c < V) {
+      long long ub, ue;
+      int b0 = 0, g0 = 0, t0 = 0, n0 = 0;
       if (dyn) {
-        const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
-        const long long r0 = dg.range_of(seg_start);
-        nsplit = (int)(dg.range_of(seg_start + n - 1) - r0 + 1);
-        if (nsplit > 1) {
-          long long ub, ue;
-          dg.bounds(r0, &ub, &ue);
-          slot0 = (int)(2 * r0 + (ub == seg_start ? 0 : 1));
+        dg.bounds(c, &ub, &ue);
+        if (ub < ue) {
+          b0 = seq_of_unit(ts, p.B, p.Hkv, ub);
+          n0 = ts[b0 + 1] - ts[b0];
+          const int rem = (int)(ub - (long long)ts[b0] * p.Hkv);  // < Hkv * n0 < 2^31
+          g0 = rem / n0;
+          t0 = rem - g0 * n0;
         }
       } else {
+        const int s = (int)c / per, i = (int)c % per;
+        b0 = s / p.Hkv;
+        g0 = s % p.Hkv;
+        const long long n = ts[b0 + 1] - ts[b0];
         const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
-        nsplit = (int)((n + C - 1) / C);
-        if (nsplit > 1) slot0 = 2 * s * per;  // chunk 0 starts its segment
+        const long long c0 = std::min<long long>((long long)i * C, n);
+        const long long c1 = std::min<long long>((long long)(i + 1) * C, n);
+        const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n;
+        ub = seg_start + c0;
+        ue = seg_start + c1;
+        t0 = (int)c0;
+        n0 = (int)n;
       }
+      p.ws.cta_desc[2 * c] = make_int4((int)ub, (int)ue, b0, g0);
+      p.ws.cta_desc[2 * c + 1] = make_int4(t0, n0, 0, 0);
     }
-    p.ws.seg_desc[s] = make_int2(slot0, nsplit);
+    if (c < S) {
+      const int s = (int)c;
+      const int b = s / p.Hkv, g = s - b * p.Hkv;
+      const long long n = ts[b + 1] - ts[b];
+      int nsplit = 0, slot0 = -1;
+      if (n > 0) {
+        if (dyn) {
+          const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
+          const long long r0 = dg.range_of(seg_start);
+          nsplit = (int)(dg.range_of(seg_start + n - 1) - r0 + 1);
+          if (nsplit > 1) {
+            long long ub, ue;
+            dg.bounds(r0, &ub, &ue);
+            slot0 = (int)(2 * r0 + (ub == seg_start ? 0 : 1));
+          }
+        } else {
+          const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
+          nsplit = (int)((n + C - 1) / C);
+          if (nsplit > 1) slot0 = 2 * s * per;  // chunk 0 starts its segment
+        }
+      }
+      p.ws.seg_desc[s] = make_int2(slot0, nsplit);
+    }
   }
 
   if (blockIdx.x == 0 && tid == 0) {
@@ -261,7 +265,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrTiles] = T;
     h[kHdrRanges] = (int32_t)V;
     h[kHdrNext] = 0;
-    __threadfence();
+    // (no fence before the magic word: the run kernel reads the plan only
+    // after griddepcontrol.wait, i.e. after this whole grid has completed)
     h[kHdrMagic] = kPlanMagic;
   }
   pdl_trigger();

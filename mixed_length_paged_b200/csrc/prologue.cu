@@ -4,19 +4,15 @@
 // The method (bitbyai.com "vLLM x HPC-Ops", Attention Backend): RoPE,
 // query-key normalisation and the KV-cache write are fused into one prologue,
 // saving launches and HBM round trips.  One CTA per sequence; one warp per
-// head row (q heads, then k heads, then v heads).  A lane owns the rotary
-// pairs (i, i + D/2) for i = lane and i = lane + 32, so RMSNorm's sum of
-// squares is one warp reduction and RoPE needs no data exchange.
-//
-// Precision: RMSNorm and the rotation run in fp32.  The rotation angle
-// pos * theta^(-2i/D) is formed and reduced modulo 2*pi in fp64 before the
-// fp32 sine/cosine: at pos ~ 65536 an fp32 angle would already be off by
-// ~4e-3 rad.
+// head row (q heads, then k heads, then v heads); the row arithmetic (and its
+// precision) is in prologue_math.cuh, shared with the decode kernel's fused
+// prologue.
 #include <cmath>
 
 #include <cuda_bf16.h>
 
 #include "hpa_common.cuh"
+#include "prologue_math.cuh"
 
 namespace hpa {
 namespace {
@@ -43,23 +39,13 @@ struct PrologueParams {
 
 template <int D>
 __global__ void __launch_bounds__(kPrologueWarps * 32) prologue_kernel(const PrologueParams p) {
-  constexpr int kPairs = D / 64;  // rotary pairs per lane
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
   const int pos = p.positions[b];
 
-  // cos/sin of this lane's rotary pairs
-  float cs[kPairs], sn[kPairs];
-#pragma unroll
-  for (int j = 0; j < kPairs; ++j) {
-    const int i = lane + 32 * j;
-    const double w = exp2(-(2.0 * i / D) * p.log2_theta);  // theta^(-2i/D)
-    double phi = (double)pos * w;
-    const double two_pi = 6.283185307179586476925;
-    phi -= two_pi * rint(phi / two_pi);
-    sincosf((float)phi, &sn[j], &cs[j]);
-  }
+  RopeLane<D> rope;
+  rope.init(pos, lane, p.log2_theta);
 
   // destination slot of the new K/V row
   long long slot_row = -1;
@@ -93,26 +79,7 @@ __global__ void __launch_bounds__(kPrologueWarps * 32) prologue_kernel(const Pro
         for (int i = lane; i < D; i += 32) dst[i] = src[i];
       continue;
     }
-    float x[2 * kPairs];  // x[j] = elem lane+32j (first half), x[kPairs+j] = its partner
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      x[j] = __bfloat162float(src[lane + 32 * j]);
-      x[kPairs + j] = __bfloat162float(src[lane + 32 * j + D / 2]);
-      ss += x[j] * x[j] + x[kPairs + j] * x[kPairs + j];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rinv = 1.0f / sqrtf(ss / D + p.eps);
-    if (!dst) continue;
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      const int i = lane + 32 * j;
-      const float a = x[j] * rinv * gamma[i];
-      const float c2 = x[kPairs + j] * rinv * gamma[i + D / 2];
-      dst[i] = __float2bfloat16_rn(a * cs[j] - c2 * sn[j]);
-      dst[i + D / 2] = __float2bfloat16_rn(c2 * cs[j] + a * sn[j]);
-    }
+    norm_rope_row<D>(src, dst, nullptr, gamma, p.eps, rope, lane);
   }
   pdl_trigger();
 }

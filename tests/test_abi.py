@@ -140,6 +140,30 @@ def test_run_rejects_bad_arguments_without_launching(L, bad, expect):
     assert _run(L, **bad) == expect
 
 
+def _run_pro(L, **kw):
+    a = dict(qr=256, kr=256, vr=256, gq=256, gk=256, eps=1e-6, theta=1e4, kc=256, vc=256, qo=None,
+             pt=256, pts=4, pages=8, out=256, outd=0, B=2, Hq=8, Hkv=2, D=64, scale=0.125,
+             kind=0, grid=148, ws=256, wsb=1 << 24)
+    a.update(kw)
+    return L.hpa_decode_run_prologue(
+        a["qr"], a["kr"], a["vr"], a["gq"], a["gk"], C.c_float(a["eps"]), C.c_float(a["theta"]),
+        a["kc"], a["vc"], a["qo"], a["pt"], a["pts"], a["pages"], a["out"], a["outd"], a["B"],
+        a["Hq"], a["Hkv"], a["D"], C.c_float(a["scale"]), a["kind"], a["grid"], a["ws"], a["wsb"],
+        None)
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(qr=None), 1), (dict(kr=None), 1), (dict(vr=None), 1), (dict(gq=None), 1),
+    (dict(gk=None), 1), (dict(kc=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
+    (dict(kr=256 + 8), 1), (dict(vr=256 + 4), 1), (dict(qr=256 + 8), 1), (dict(qo=256 + 1), 1),
+    (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1), (dict(theta=0.0), 1),
+    (dict(theta=float("nan")), 1), (dict(scale=0.0), 1), (dict(D=96), 2), (dict(Hq=24, Hkv=8), 2),
+    (dict(wsb=64), 3), (dict(kind=9), 1),
+])
+def test_run_prologue_rejects_bad_arguments_without_launching(L, bad, expect):
+    assert _run_pro(L, **bad) == expect
+
+
 def _prologue(L, **kw):
     a = dict(qr=256, kr=256, vr=256, gq=256, gk=256, eps=1e-6, theta=1e4, pos=256, pt=256, pts=4,
              kc=256, vc=256, qo=256, B=2, Hq=8, Hkv=2, D=64, pages=8, status=None)

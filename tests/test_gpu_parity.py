@@ -340,6 +340,88 @@ def test_mix_prologue_workload_sampled_rows():
     _check(out[rows], ref)
 
 
+# ---------------------------------------------------------------- fused prologue
+
+def _separate_and_fused(batch, *, kind=0, num_ctas=None, param=0, out_dtype=torch.bfloat16,
+                        with_q_out=True):
+    """The same step twice on copies of the caches: prologue kernel -> plan ->
+    run, and plan -> run with the prologue fused in."""
+    B, Hq, D = batch.q_raw.shape
+    Hkv = batch.k_raw.shape[1]
+    n = num_ctas or hpa.default_num_ctas()
+    maxlen = int(batch.seq_lens.max().item())
+    grid = hpa.plan_grid(kind, B, Hkv, n, param, maxlen)
+    res = []
+    for fused in (False, True):
+        kc, vc = batch.k_cache.clone(), batch.v_cache.clone()
+        q_out = torch.full_like(batch.q_raw, float("nan")) if (with_q_out or not fused) else None
+        ws = torch.zeros(hpa.decode_workspace_size(kind, B, Hkv, Hq, D, grid), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.full((B, Hq, D), float("nan"), dtype=out_dtype, device="cuda")
+        if not fused:
+            hpa.kv_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
+                            batch.positions, batch.page_table, kc, vc, q_out, eps=1e-6,
+                            rope_theta=10000.0)
+        hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
+                        pt_stride=batch.pt_stride, workspace=ws, kind=kind, num_ctas=n,
+                        param=param, max_seq_len=maxlen)
+        if fused:
+            hpa.decode_run_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma,
+                                    batch.k_gamma, kc, vc, batch.page_table, out, ws, grid,
+                                    1.0 / math.sqrt(D), q_out=q_out, eps=1e-6, rope_theta=1e4,
+                                    kind=kind)
+        else:
+            hpa.decode_run(q_out, kc, vc, batch.page_table, out, ws, grid, 1.0 / math.sqrt(D),
+                           kind=kind)
+        torch.cuda.synchronize()
+        assert hpa.read_status(ws) == 0
+        res.append((out, kc, vc, q_out))
+    return res
+
+
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 16, 4), (128, 16, 1), (128, 32, 2)])
+@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7)])
+def test_fused_prologue_bitwise_equals_separate(D, Hq, Hkv, kind, num_ctas):
+    # pre-append lengths: a first token, page edges, several pages, one long
+    lens = [0, 63, 64, 127, 1000, 4095, 1]
+    batch = _prologue_case(lens, Hq=Hq, Hkv=Hkv, D=D)
+    to_device(batch)
+    (oa, ka, va, qa), (ob, kb, vb, qb) = _separate_and_fused(batch, kind=kind, num_ctas=num_ctas)
+    # same bits: the caches (new slots and every other byte), q_out, and the output
+    assert torch.equal(bits_t(ka), bits_t(kb)) and torch.equal(bits_t(va), bits_t(vb))
+    assert torch.equal(bits_t(qa), bits_t(qb))
+    assert torch.equal(bits_t(oa), bits_t(ob))
+
+
+def test_fused_prologue_against_oracle_f32_out_no_q_out():
+    lens = [5, 200, 3000, 64]
+    batch = _prologue_case(lens, Hq=32, Hkv=8, D=128)
+    kc, vc = bits16(batch.k_cache).copy(), bits16(batch.v_cache).copy()
+    pt = batch.page_table.numpy()
+    q64 = oracle.prologue(bits16(batch.q_raw), bits16(batch.k_raw), bits16(batch.v_raw),
+                          batch.q_gamma.numpy(), batch.k_gamma.numpy(), 1e-6, 1e4,
+                          batch.positions.numpy(), pt, kc, vc)
+    ref = oracle.paged_decode(q64, kc, vc, pt, batch.seq_lens.numpy(), 8, 1 / math.sqrt(128))
+    to_device(batch)
+    (oa, *_), (ob, kb, vb, qb) = _separate_and_fused(batch, out_dtype=torch.float32,
+                                                     with_q_out=False)
+    assert qb is None
+    _check(ob, ref)
+    assert torch.equal(oa, ob)
+
+
+def test_fused_prologue_mix_workload_bitwise():
+    batch = W.build("mix_prologue", device="cuda")
+    (oa, ka, va, qa), (ob, kb, vb, qb) = _separate_and_fused(batch)
+    assert torch.equal(bits_t(oa), bits_t(ob)) and torch.equal(bits_t(qa), bits_t(qb))
+    assert torch.equal(bits_t(ka), bits_t(kb)) and torch.equal(bits_t(va), bits_t(vb))
+
+
+def bits_t(t: torch.Tensor) -> torch.Tensor:
+    """Bit pattern of a bf16/f32 tensor (NaN-safe equality)."""
+    return t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
+
+
 # ---------------------------------------------------------------- device-side checks
 
 def test_bad_page_id_is_flagged():
