@@ -40,6 +40,7 @@ class DecodeShape:
     head_dim: int
     kv_dtype: str = "bf16"  # "bf16" or "fp8_e4m3"
     prologue: bool = False
+    q_tokens: int = 1       # query tokens per sequence (multi-token decode if > 1)
 
     @property
     def group(self) -> int:
@@ -55,6 +56,9 @@ SHAPES = {
     "skewed_quarter": DecodeShape("skewed_quarter", 64, 8, 128),
     "mix_prologue": DecodeShape("mix_prologue", 32, 8, 128, prologue=True),
     "fp8": DecodeShape("fp8", 64, 8, 128, kv_dtype="fp8_e4m3"),
+    # the skewed batch with two query tokens per sequence (a draft token to
+    # verify, or a multi-token-prediction head): 8 heads x 2 tokens per kv head
+    "skewed_mtp2": DecodeShape("skewed_mtp2", 64, 8, 128, q_tokens=2),
 }
 
 
@@ -70,7 +74,7 @@ def cache_lengths(name: str, seed: int = 0) -> np.ndarray:
         return np.array([37, 200], dtype=np.int64)
     if name == "uniform":
         return np.full(64, 512, dtype=np.int64)
-    if name == "skewed":
+    if name in ("skewed", "skewed_mtp2"):
         return np.array([131072] + [4096] * 31, dtype=np.int64)
     if name == "skewed_quarter":
         return np.array([32768] + [1024] * 31, dtype=np.int64)
@@ -93,7 +97,7 @@ class DecodeBatch:
     num_pages: int
     k_cache: torch.Tensor           # [num_pages][Hkv][64][D] bf16 (or fp32 values for fp8, see below)
     v_cache: torch.Tensor
-    q: torch.Tensor | None = None   # [B][Hq][D] bf16 (no prologue)
+    q: torch.Tensor | None = None   # [B][Hq][D] bf16 (no prologue); [B][T][Hq][D] if q_tokens > 1
     # fp8 workloads: k_cache/v_cache hold fp32 N(0,1) values; a quantiser turns
     # them into e4m3 codes + per-(page, kv-head) scales.  live[p] counts the
     # live tokens in physical page p.
@@ -210,13 +214,17 @@ def make_batch(shape: DecodeShape, cache_lens, *, seed: int = 0, device="cpu",
         batch.q_gamma = _uniform((D,), 0.5, 1.5, gen, device)
         batch.k_gamma = _uniform((D,), 0.5, 1.5, gen, device)
         batch.positions = torch.from_numpy(cache_lens.astype(np.int32)).to(device)
+    elif shape.q_tokens > 1:
+        # the q_tokens new tokens are the last q_tokens of each sequence
+        batch.q = _normal((B, shape.q_tokens, Hq, D), gen, device, torch.bfloat16)
     else:
         batch.q = _normal((B, Hq, D), gen, device, torch.bfloat16)
     return batch
 
 
 def build(name: str, *, seed: int = 0, device="cpu", **kw) -> DecodeBatch:
-    """One of the five named workloads (tiny, uniform, skewed, mix_prologue, fp8)."""
+    """One of the named workloads (tiny, uniform, skewed, skewed_quarter, mix_prologue, fp8,
+    skewed_mtp2)."""
     return make_batch(SHAPES[name], cache_lengths(name, seed), seed=seed, device=device, **kw)
 
 

@@ -55,6 +55,9 @@ def _declare(L):
     L.oracle_prologue.restype = _I
     L.oracle_prologue.argtypes = [_P, _P, _P, _P, _P, _D, _D, _P, _P, _I, _P, _P, _P,
                                   _I, _I, _I, _I, _I, _I]
+    L.oracle_paged_decode_multi.restype = _I
+    L.oracle_paged_decode_multi.argtypes = [_P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _I, _I, _I,
+                                            _I, _I, _I, _I, _D, _P, _I, _P, _I]
     L.oracle_paged_decode.restype = _I
     L.oracle_paged_decode.argtypes = [_P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _I,
                                       _I, _I, _D, _P, _I, _P, _I]
@@ -197,6 +200,34 @@ def paged_decode(q, k_cache, v_cache, page_table, seq_lens, num_kv_heads: int, s
                                    _ptr(r), 0 if r is None else r.shape[0], _ptr(out),
                                    num_threads)
     _check(rc, "paged_decode")
+    return out
+
+
+def paged_decode_multi(q, k_cache, v_cache, page_table, seq_lens, num_kv_heads: int,
+                       scale: float, *, kv_fp8: bool = False, k_scale=None, v_scale=None,
+                       rows=None, page_size: int = 64, num_threads: int = 0) -> np.ndarray:
+    """Multi-token decode attention, fp64 [B][T][Hq][D]: q is [B][T][Hq][D]
+    (uint16 bf16 bits or float64); query token i of sequence b sees the
+    first seq_lens[b] - T + i + 1 tokens (the T new tokens are the last T of
+    the sequence, causal among themselves)."""
+    q = np.asarray(q)
+    q16 = _c(q, np.uint16) if q.dtype == np.uint16 else None
+    q64 = None if q16 is not None else _c(q, np.float64)
+    B, T, Hq, D = q.shape
+    kc = _c(k_cache, np.uint8 if kv_fp8 else np.uint16)
+    vc = _c(v_cache, np.uint8 if kv_fp8 else np.uint16)
+    ks = _c(k_scale, np.float32) if kv_fp8 else None
+    vs = _c(v_scale, np.float32) if kv_fp8 else None
+    pt = _c(page_table, np.int32)
+    sl = _c(seq_lens, np.int32)
+    r = None if rows is None else _c(rows, np.int32)
+    out = np.zeros((B, T, Hq, D), dtype=np.float64)
+    rc = lib().oracle_paged_decode_multi(_ptr(q16), _ptr(q64), _ptr(kc), _ptr(vc), int(kv_fp8),
+                                         _ptr(ks), _ptr(vs), _ptr(pt), pt.shape[1], _ptr(sl), B,
+                                         T, Hq, num_kv_heads, D, page_size, kc.shape[0],
+                                         float(scale), _ptr(r), 0 if r is None else r.shape[0],
+                                         _ptr(out), num_threads)
+    _check(rc, "paged_decode_multi")
     return out
 
 

@@ -291,22 +291,28 @@ static void load_q(const uint16_t* q16, const double* q64, long off, int D, doub
   for (int d = 0; d < D; ++d) q[d] = q64 ? q64[off + d] : oracle_bf16_to_f64(q16[off + d]);
 }
 
-/* Decode attention for the sequences listed in rows[0..n_rows) (all B if rows
- * is NULL).  q is given either as bf16 bits (q16) or fp64 (q64).  out is
- * [B][Hq][D] fp64; a sequence of length 0 gets a zero output (softmax over an
- * empty set is undefined; zero is this library's convention). */
-int oracle_paged_decode(const uint16_t* q16, const double* q64, const void* k_cache,
-                        const void* v_cache, int kv_fp8, const float* k_scale,
-                        const float* v_scale, const int32_t* page_table, int pt_stride,
-                        const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int page_size,
-                        int num_pages, double scale, const int32_t* rows, int n_rows,
-                        double* out, int num_threads) {
-  if (Hkv <= 0 || Hq % Hkv || D <= 0 || page_size <= 0) return ORC_BAD_ARG;
+/* Multi-token decode attention (speculative / multi-token-prediction decode:
+ * T new query tokens per sequence, already appended to the cache, causal
+ * among themselves).  Query token i of sequence b sits at position
+ * L_b - T + i and attends to positions [0, L_b - T + i], i.e. it is the
+ * single-token decode of that query over the first L_b - T + i + 1 tokens.
+ * For the sequences listed in rows[0..n_rows) (all B if rows is NULL); q is
+ * [B][T][Hq][D] as bf16 bits (q16) or fp64 (q64); out is [B][T][Hq][D] fp64.
+ * A query that sees no token (L_b - T + i + 1 <= 0, e.g. an empty sequence)
+ * gets a zero output (softmax over an empty set is undefined; zero is this
+ * library's convention). */
+int oracle_paged_decode_multi(const uint16_t* q16, const double* q64, const void* k_cache,
+                              const void* v_cache, int kv_fp8, const float* k_scale,
+                              const float* v_scale, const int32_t* page_table, int pt_stride,
+                              const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D,
+                              int page_size, int num_pages, double scale, const int32_t* rows,
+                              int n_rows, double* out, int num_threads) {
+  if (Hkv <= 0 || Hq % Hkv || D <= 0 || page_size <= 0 || T <= 0) return ORC_BAD_ARG;
   orc_cache c = {k_cache, v_cache, kv_fp8, k_scale, v_scale, page_table, pt_stride,
                  Hkv, D, page_size, num_pages};
   int G = Hq / Hkv;
   int nr = rows ? n_rows : B;
-  long total = (long)nr * Hq;
+  long total = (long)nr * T * Hq;
   int rc = ORC_OK;
 #ifdef _OPENMP
   if (num_threads > 0) omp_set_num_threads(num_threads);
@@ -322,23 +328,28 @@ int oracle_paged_decode(const uint16_t* q16, const double* q64, const void* k_ca
     double* q = malloc(sizeof(double) * D);
     double* acc = malloc(sizeof(double) * D);
 #pragma omp for schedule(dynamic, 1)
-    for (long i = 0; i < total; ++i) {
-      int b = rows ? rows[i / Hq] : (int)(i / Hq);
-      int h = (int)(i % Hq);
+    for (long it = 0; it < total; ++it) {
+      int b = rows ? rows[it / ((long)T * Hq)] : (int)(it / ((long)T * Hq));
+      int i = (int)(it / Hq % T);
+      int h = (int)(it % Hq);
       int g = h / G;
       long L = seq_lens[b];
-      double* o = out + ((long)b * Hq + h) * D;
-      if (L <= 0 || (L + page_size - 1) / page_size > pt_stride) {
+      long row = ((long)b * T + i) * Hq + h;
+      double* o = out + row * D;
+      long Li = L - T + i + 1; /* tokens this query sees */
+      if (L > 0 && (L + page_size - 1) / page_size > pt_stride) {
         for (int d = 0; d < D; ++d) o[d] = 0.0;
-        if (L > 0) {
 #pragma omp atomic write
-          rc = ORC_BAD_ARG;
-        }
+        rc = ORC_BAD_ARG;
         continue;
       }
-      load_q(q16, q64, ((long)b * Hq + h) * D, D, q);
+      if (Li <= 0) {
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        continue;
+      }
+      load_q(q16, q64, row * D, D, q);
       double m, l;
-      int e = partial_one(&c, q, b, g, 0, L, scale, s_buf, acc, &m, &l);
+      int e = partial_one(&c, q, b, g, 0, Li, scale, s_buf, acc, &m, &l);
       if (e != ORC_OK) {
 #pragma omp atomic write
         rc = e;
@@ -348,6 +359,19 @@ int oracle_paged_decode(const uint16_t* q16, const double* q64, const void* k_ca
     free(s_buf); free(q); free(acc);
   }
   return rc;
+}
+
+/* Decode attention of one query token per sequence: the T = 1 case above.
+ * q and out are [B][Hq][D]. */
+int oracle_paged_decode(const uint16_t* q16, const double* q64, const void* k_cache,
+                        const void* v_cache, int kv_fp8, const float* k_scale,
+                        const float* v_scale, const int32_t* page_table, int pt_stride,
+                        const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int page_size,
+                        int num_pages, double scale, const int32_t* rows, int n_rows,
+                        double* out, int num_threads) {
+  return oracle_paged_decode_multi(q16, q64, k_cache, v_cache, kv_fp8, k_scale, v_scale,
+                                   page_table, pt_stride, seq_lens, B, 1, Hq, Hkv, D, page_size,
+                                   num_pages, scale, rows, n_rows, out, num_threads);
 }
 
 /* Partial (acc[D], m, l) of one (b, h) over tokens [t0, t1). */

@@ -545,3 +545,58 @@ def test_planner_clamps_lengths_to_capacity():
                     capacity_tokens=128)
     np.testing.assert_array_equal(p["lens"], [0, 128, 64])
     np.testing.assert_array_equal(p["tile_start"], [0, 0, 2, 3])
+
+
+# ---------------------------------------------------------------- multi-token decode
+
+@pytest.mark.parametrize("seed,lens,T,Hq,Hkv,D", [
+    # tokens straddling a page edge (65 with T = 3), a sequence exactly T long,
+    # one shorter than T (its first query sees nothing), an empty one
+    (5, (65, 200, 3, 2, 0), 3, 8, 2, 32),
+    (6, (130, 64, 17), 2, 16, 2, 64),
+    (7, (300,), 4, 4, 1, 16),
+])
+def test_multi_token_decode_matches_causal_masked_dense(seed, lens, T, Hq, Hkv, D):
+    """Query token i of a sequence of L tokens sits at position L - T + i and
+    sees positions 0 .. L - T + i: written here as a dense [T x L] score
+    matrix with an explicit causal mask, one numpy softmax per head."""
+    shape = W.DecodeShape("mt", Hq, Hkv, D, q_tokens=T)
+    batch = W.make_batch(shape, list(lens), seed=seed)
+    kv = bf16_values(bits16(batch.k_cache))
+    vv = bf16_values(bits16(batch.v_cache))
+    qv = bf16_values(bits16(batch.q))          # [B][T][Hq][D]
+    pt = batch.page_table.numpy()
+    scale = 1.0 / math.sqrt(D)
+    out = oracle.paged_decode_multi(bits16(batch.q), bits16(batch.k_cache),
+                                    bits16(batch.v_cache), pt, batch.seq_lens.numpy(), Hkv,
+                                    scale)
+    G = Hq // Hkv
+    for b, L in enumerate(lens):
+        K = dense_kv(kv, pt, b, L)               # [L][Hkv][D]
+        V = dense_kv(vv, pt, b, L)
+        pos = L - T + np.arange(T)               # position of each query token
+        visible = np.arange(L)[None, :] <= pos[:, None]  # [T][L]
+        for h in range(Hq):
+            g = h // G
+            S = (qv[b, :, h, :] @ K[:, g, :].T) * scale  # [T][L]
+            for i in range(T):
+                if not visible[i].any():
+                    np.testing.assert_array_equal(out[b, i, h], 0.0)
+                    continue
+                s = np.where(visible[i], S[i], -np.inf)
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                np.testing.assert_allclose(out[b, i, h], p @ V[:, g, :], rtol=0, atol=1e-12)
+
+
+def test_multi_token_last_query_equals_single_token_decode():
+    """The last of T query tokens sees the whole sequence: it is the
+    single-token decode of that query (a different entry point of the oracle
+    computes it)."""
+    shape = W.DecodeShape("mt", 8, 2, 64, q_tokens=3)
+    batch = W.make_batch(shape, [100, 3, 70], seed=9)
+    args = (bits16(batch.k_cache), bits16(batch.v_cache), batch.page_table.numpy(),
+            batch.seq_lens.numpy(), 2, 0.125)
+    multi = oracle.paged_decode_multi(bits16(batch.q), *args)
+    single = oracle.paged_decode(np.ascontiguousarray(bits16(batch.q)[:, -1]), *args)
+    np.testing.assert_array_equal(multi[:, -1], single)
