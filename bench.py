@@ -82,6 +82,8 @@ WORKLOAD_DESC = {
                     "prologue in every step",
     "fp8": "FP8 KV: 256 sequences, lengths geometric (mean 2048, cap 16384), 64 q heads, "
            "8 kv heads, head_dim 128, e4m3 K/V with fp32 per-(page, kv head) scales",
+    "skewed_mtp2": "multi-token decode on the skewed batch: 2 query tokens per sequence "
+                   "(causal among themselves), 64 q heads, 8 kv heads, head_dim 128, bf16",
 }
 
 
@@ -308,16 +310,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     tiles = int(((lens + 63) // 64).sum())
     # algorithmic bytes of one run launch: live KV + q + out + page-table entries
     # read (+ the two fp32 scales of every (page, kv head) tile for FP8)
-    run_bytes = kv_bytes + 2 * B * Hq * D * 2 + tiles * 4 + (tiles * Hkv * 8 if fp8 else 0)
+    T = shape.q_tokens
+    run_bytes = kv_bytes + 2 * B * T * Hq * D * 2 + tiles * 4 + (tiles * Hkv * 8 if fp8 else 0)
     if shape.prologue:
         # the fused prologue also reads the new token's raw K and V rows and
         # writes them (normalised, rotated) into their cache slots
         run_bytes += 4 * B * Hkv * D * 2
     scale = 1.0 / math.sqrt(D)
-    num_ctas = args.num_ctas or hpa.default_num_ctas(local_rank)
+    num_ctas = args.num_ctas or hpa.decode_num_ctas(Hq, Hkv, shape.q_tokens, local_rank)
     stream = torch.cuda.current_stream()
-    dec = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, num_ctas=num_ctas, device=dev)
-    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    dec = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, num_ctas=num_ctas, q_tokens=T,
+                           device=dev)
+    out = torch.empty(batch.q.shape if T > 1 else (B, Hq, D), dtype=torch.bfloat16, device=dev)
     seq_lens = batch.seq_lens
     if shape.prologue:
         # The step starts from the new token's raw projections: plan, then the
@@ -442,7 +446,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "fused_speedup": ab["separate"] / ab["fused"],
             "method": f"interleaved A/B, {blocks} x {per} steps each"}
 
-    plain = not fp8 and not shape.prologue
+    plain = not fp8 and not shape.prologue and T == 1
     if not args.no_extras and plain:
         # each static plan against the dynamic one as an interleaved A/B
         # (alternating blocks of steps), so drift falls on both alike

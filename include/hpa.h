@@ -108,6 +108,14 @@ HPA_API int hpa_version(void);
  * device cannot be queried. */
 HPA_API int hpa_default_num_ctas(int device);
 
+/* Persistent CTA count (num_ctas of hpa_decode_plan) that matches how many
+ * run-kernel CTAs fit an SM for this head geometry: hpa_default_num_ctas
+ * when each kv head has at most 8 query rows (G * q_tokens <= 8), one per SM
+ * above that.  A dynamic plan for more CTAs than fit at once would leave
+ * part of its primary ranges to a second wave.  Returns -1 on invalid
+ * arguments or if the device cannot be queried. */
+HPA_API int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads, int q_tokens);
+
 /* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC,
  * B * Hkv * S for STATIC_NSPLIT, B * Hkv * ceil(T_max / C) for STATIC_CHUNK
  * (T_max = ceil(max_seq_len / 64), S and C the resolved params).  Host only;
@@ -203,6 +211,39 @@ HPA_API hpa_status hpa_decode_run(const void* q, const void* k_cache, const void
                           int num_kv_heads, int head_dim, float softmax_scale,
                           hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes,
                           void* stream);
+
+/*
+ * hpa_decode_run_multi -- hpa_decode_run for T = q_tokens new query tokens per
+ * sequence (a draft token to verify, or multi-token-prediction heads), causal
+ * among themselves.  The pages' attention API takes variable-length queries
+ * per sequence (openai-hub.com news/688: attention(q, k, v, cu_seqlens, ...,
+ * kv_cache_layout="paged")); this is its fixed-T decode form.
+ *
+ * The T tokens are the last T of each sequence and are already in the cache
+ * (seq_lens counts them).  Query token i (0 <= i < T) of sequence b sits at
+ * position seq_lens[b] - T + i and attends to positions 0 .. seq_lens[b] -
+ * T + i:
+ *     out[b][i][h] = sum_{j <= L_b - T + i} softmax_j(scale <q[b][i][h], K_b[j, g]>) V_b[j, g]
+ * A query that sees no token (seq_lens[b] < T - i) gets a zero row.
+ *
+ *   q, out       device [batch][q_tokens][num_q_heads][D] (bf16 q; bf16 or
+ *                fp32 out).
+ *   q_tokens     1 .. 16 with (num_q_heads / num_kv_heads) * q_tokens <= 16:
+ *                the G * T query rows of a kv head share one pass over its
+ *                tiles (HPA_ERR_UNSUPPORTED otherwise).
+ *   kind, grid, workspace  from hpa_decode_plan called with num_q_heads *
+ *                q_tokens in place of num_q_heads (the plan and the workspace
+ *                count G * T rows per kv head); size the workspace the same way.
+ *   the rest     as for hpa_decode_run; q_tokens = 1 is hpa_decode_run.
+ */
+HPA_API hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, const void* v_cache,
+                                        const float* k_scale, const float* v_scale,
+                                        hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                                        int pt_stride, int num_pages, void* out,
+                                        hpa_out_dtype out_dtype, int batch, int q_tokens,
+                                        int num_q_heads, int num_kv_heads, int head_dim,
+                                        float softmax_scale, hpa_plan_kind kind, int grid,
+                                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * hpa_decode_run_prologue -- hpa_decode_run with the decode prologue fused

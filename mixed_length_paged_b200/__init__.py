@@ -9,7 +9,7 @@ it raises ``HpaLibraryMissing`` -- there is no fallback implementation.
 The functions mirror the C ABI in ``include/hpa.h``:
 
     decode_workspace_size, plan_grid, default_num_ctas, workspace_layout,
-    decode_plan, decode_run, decode_run_prologue, kv_prologue, read_status,
+    decode_plan, decode_run, decode_run_multi, decode_run_prologue, kv_prologue, read_status,
     decode_noalloc
 
 and ``PagedDecoder`` bundles a workspace with plan + run for callers who do
@@ -26,7 +26,8 @@ __all__ = [
     "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
     "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
-    "default_num_ctas", "workspace_layout", "decode_plan", "decode_run", "decode_run_prologue",
+    "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run", "decode_run_multi",
+    "decode_run_prologue",
     "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -73,6 +74,8 @@ def lib():
         L.hpa_version.argtypes = []
         L.hpa_default_num_ctas.restype = _I
         L.hpa_default_num_ctas.argtypes = [_I]
+        L.hpa_decode_num_ctas.restype = _I
+        L.hpa_decode_num_ctas.argtypes = [_I, _I, _I, _I]
         L.hpa_plan_grid.restype = _I
         L.hpa_plan_grid.argtypes = [_I, _I, _I, _I, _I, _I]
         L.hpa_decode_workspace_size.restype = _Z
@@ -85,6 +88,9 @@ def lib():
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
                                      _F, _I, _I, _V, _Z, _V]
+        L.hpa_decode_run_multi.restype = _I
+        L.hpa_decode_run_multi.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I,
+                                           _I, _I, _I, _F, _I, _I, _V, _Z, _V]
         L.hpa_decode_run_prologue.restype = _I
         L.hpa_decode_run_prologue.argtypes = [_V, _V, _V, _V, _V, _F, _F, _V, _V, _V, _V, _I, _I,
                                               _V, _I, _I, _I, _I, _I, _F, _I, _I, _V, _Z, _V]
@@ -138,6 +144,17 @@ def default_num_ctas(device: int | None = None) -> int:
     n = lib().hpa_default_num_ctas(d)
     if n < 1:
         raise HpaError("hpa_default_num_ctas: " + lib().hpa_last_cuda_error().decode())
+    return n
+
+
+def decode_num_ctas(num_q_heads: int, num_kv_heads: int, q_tokens: int = 1,
+                    device: int | None = None) -> int:
+    """Persistent CTA count matching the run kernel's residency for this head
+    geometry (hpa_decode_num_ctas)."""
+    d = torch.cuda.current_device() if device is None else device
+    n = lib().hpa_decode_num_ctas(d, num_q_heads, num_kv_heads, q_tokens)
+    if n < 1:
+        raise HpaError("hpa_decode_num_ctas: invalid arguments or no device")
     return n
 
 
@@ -217,6 +234,42 @@ def decode_run(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                               float(softmax_scale), kind, grid, _ptr(workspace),
                               workspace.numel(), _stream(stream))
     _check(rc, "hpa_decode_run")
+    return out
+
+
+def decode_run_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     page_table: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                     grid: int, softmax_scale: float, *, kind: int = PLAN_DYNAMIC,
+                     k_scale: torch.Tensor | None = None, v_scale: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Multi-token decode: q and out are [B][T][Hq][D]; query token i of a
+    sequence of L tokens sees its first L - T + i + 1 tokens.  The plan in
+    ``workspace`` must have been made with num_q_heads = Hq * T."""
+    _dev(q, "q", (torch.bfloat16,), 4)
+    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
+    cache_types = (torch.uint8, torch.float8_e4m3fn) if fp8 else (torch.bfloat16,)
+    _dev(k_cache, "k_cache", cache_types, 4)
+    _dev(v_cache, "v_cache", cache_types, 4)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    _dev(out, "out", (torch.bfloat16, torch.float32), 4)
+    _dev(workspace, "workspace", (torch.uint8,))
+    if fp8:
+        if k_scale is None or v_scale is None:
+            raise HpaError("FP8 caches need k_scale and v_scale")
+        _dev(k_scale, "k_scale", (torch.float32,), 2)
+        _dev(v_scale, "v_scale", (torch.float32,), 2)
+    B, T, Hq, D = q.shape
+    num_pages, Hkv, S, Dk = k_cache.shape
+    if S != PAGE_SIZE or Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or tuple(out.shape) != tuple(q.shape) or page_table.shape[0] != B:
+        raise HpaError("decode_run_multi: inconsistent shapes")
+    rc = lib().hpa_decode_run_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                    _ptr(v_scale), KV_FP8_E4M3 if fp8 else KV_BF16,
+                                    _ptr(page_table), page_table.shape[1], num_pages, _ptr(out),
+                                    OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, T, Hq,
+                                    Hkv, D, float(softmax_scale), kind, grid, _ptr(workspace),
+                                    workspace.numel(), _stream(stream))
+    _check(rc, "hpa_decode_run_multi")
     return out
 
 
@@ -322,24 +375,29 @@ def read_status(workspace: torch.Tensor, stream=None) -> int:
 
 
 class PagedDecoder:
-    """A workspace sized for one batch shape, plus plan + run in one call."""
+    """A workspace sized for one batch shape, plus plan + run in one call.
+    ``q_tokens`` > 1: multi-token decode (q and out [B][T][Hq][D])."""
 
     def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  pt_stride: int, *, kind: int = PLAN_DYNAMIC, num_ctas: int | None = None,
-                 param: int = 0, max_seq_len: int = 0, device=None):
+                 param: int = 0, max_seq_len: int = 0, q_tokens: int = 1, device=None):
         self.device = torch.device("cuda" if device is None else device)
-        self.num_ctas = num_ctas or default_num_ctas(self.device.index or 0)
+        self.num_ctas = num_ctas or decode_num_ctas(num_q_heads, num_kv_heads, q_tokens,
+                                                    self.device.index or 0)
         self.kind, self.param, self.max_seq_len = kind, param, max_seq_len
+        self.q_tokens = q_tokens
         self.shape = (batch, num_q_heads, num_kv_heads, head_dim, pt_stride)
         grid = plan_grid(kind, batch, num_kv_heads, self.num_ctas, param, max_seq_len)
-        self.workspace = torch.empty(decode_workspace_size(kind, batch, num_kv_heads, num_q_heads,
-                                                           head_dim, grid),
+        # a multi-token plan counts G * T rows per kv head
+        self.workspace = torch.empty(decode_workspace_size(kind, batch, num_kv_heads,
+                                                           num_q_heads * q_tokens, head_dim, grid),
                                      dtype=torch.uint8, device=self.device)
         self.grid = grid
 
     def plan(self, seq_lens: torch.Tensor, stream=None) -> int:
         B, Hq, Hkv, D, pts = self.shape
-        self.grid = decode_plan(seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
+        self.grid = decode_plan(seq_lens, num_kv_heads=Hkv, num_q_heads=Hq * self.q_tokens,
+                                head_dim=D,
                                 pt_stride=pts, workspace=self.workspace, kind=self.kind,
                                 num_ctas=self.num_ctas, param=self.param,
                                 max_seq_len=self.max_seq_len, stream=stream)
@@ -347,6 +405,10 @@ class PagedDecoder:
 
     def run(self, q, k_cache, v_cache, page_table, out, softmax_scale, *, k_scale=None,
             v_scale=None, stream=None):
+        if q.dim() == 4:  # [B][T][Hq][D]: the multi-token entry (any T)
+            return decode_run_multi(q, k_cache, v_cache, page_table, out, self.workspace,
+                                    self.grid, softmax_scale, kind=self.kind, k_scale=k_scale,
+                                    v_scale=v_scale, stream=stream)
         return decode_run(q, k_cache, v_cache, page_table, out, self.workspace, self.grid,
                           softmax_scale, kind=self.kind, k_scale=k_scale, v_scale=v_scale,
                           stream=stream)

@@ -64,6 +64,7 @@ constexpr int kSmemLimit = 227 * 1024;   // per CTA
 constexpr int kSmemPerSm = 228 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any barrier wait
 constexpr int kDepBufs = 2;              // deposit slots between consumers and epilogue
+constexpr int kMaxQTokens = 16;          // query tokens per sequence (multi-token decode)
 
 template <int D, int NT, bool FP8, int CPS, bool PRO>
 struct Cfg {
@@ -106,6 +107,7 @@ struct RunParams {
   int pt_stride, num_pages;
   void* out;
   int B, Hq, Hkv, G;
+  int T, GT;                // query tokens per sequence; rows per kv head = G * T
   float scale_log2;         // softmax_scale * log2(e)
   Ws ws;
   int grid, kind;
@@ -271,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
     const int32_t* h = p.ws.header;
     const bool ok = h[kHdrMagic] == kPlanMagic && h[kHdrGrid] == p.grid &&
                     h[kHdrGrid] == (int)gridDim.x && h[kHdrBatch] == p.B &&
-                    h[kHdrKvHeads] == p.Hkv && h[kHdrGroup] == p.G && h[kHdrHeadDim] == D &&
+                    h[kHdrKvHeads] == p.Hkv && h[kHdrGroup] == p.GT && h[kHdrHeadDim] == D &&
                     h[kHdrKind] == p.kind && h[kHdrRanges] >= p.grid &&
                     h[kHdrRanges] <= plan_ranges_ll(p.kind, p.grid);
     *s_plan_ok = ok;
@@ -293,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     const uint64_t policy = l2_policy_evict_first();
-    const int qbytes = p.G * D * 2;
+    const int qrow_bytes = p.G * D * 2;  // one query token's rows of a kv head group
+    const int qbytes = p.T * qrow_bytes;
     const int U = p.ws.header[kHdrUnits];
     const int V = p.ws.header[kHdrRanges];
     const bool dyn = p.kind == HPA_PLAN_DYNAMIC;
@@ -329,7 +332,9 @@ __global__ void __launch_bounds__(kThreads, CPS)
           if (u < ue) {
             const int page = __ldg(p.page_table + (long long)w2.b * p.pt_stride + w2.t);
             const int L = p.ws.lens[w2.b];
-            valid = min(kPageSize, L - w2.t * kPageSize);
+            // tokens from the tile's start to the sequence end, capped where no
+            // query row's limit can reach (multi-token rows see up to T - 1 fewer)
+            valid = min(kPageSize + kMaxQTokens - 1, L - w2.t * kPageSize);
             flags = ((w2.t == 0 || u == ub) ? kFirst : 0) | ((w2.t == w2.n - 1 || u == ue - 1) ? kLast : 0) |
                     (w2.t == 0 ? kSegStart : 0) | ((PRO && w2.t == w2.n - 1) ? kNewTok : 0);
             pos = L - 1;  // the new token's position (post-append length - 1)
@@ -388,9 +393,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
                 // can prepare the query (and the new K row) while the K/V
                 // tiles, which complete on full_bar, are still in flight.
                 mbar_arrive_expect_tx(qb, (first ? qbytes : 0) + (newtok ? 4 * D : 0));
-                if (first)
-                  bulk_load(smem_u32(qslots + s * C::kSlotBytes),
-                            p.q + ((long long)si.b * p.Hq + (long long)si.g * p.G) * D, qbytes, qb);
+                if (first)  // rows n = i * G + h: query token i, head h of the group
+                  for (int i = 0; i < p.T; ++i)
+                    bulk_load(smem_u32(qslots + s * C::kSlotBytes) + i * qrow_bytes,
+                              p.q + (((long long)si.b * p.T + i) * p.Hq + (long long)si.g * p.G) * D,
+                              qrow_bytes, qb);
                 if (newtok) {
                   // the new token's raw K and V rows, for the consumers to
                   // patch into this tile
@@ -441,10 +448,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
     }
     __syncwarp();
     ++it;
-    // zero output rows of empty sequences (a softmax over no tokens)
+    // zero output rows of empty sequences (a softmax over no tokens), for
+    // every query token
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
       if (p.ws.lens[b] != 0) continue;
-      for (int i = lane; i < p.Hq * D; i += 32) store_out<OUT_F32>(p.out, (long long)b * p.Hq * D + i, 0.f);
+      const long long n = (long long)p.T * p.Hq * D;
+      for (long long i = lane; i < n; i += 32) store_out<OUT_F32>(p.out, (long long)b * n + i, 0.f);
     }
     // After an abort, make sure no copy is still landing in shared memory.
     if (lane == 0 && *s_abort) {
@@ -463,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
 
   if (warp == kEpilogueWarp) {
     // ------------------------------------------------------------ epilogue
-    const int G = p.G;
+    const int GT = p.GT;  // rows per kv head: query token i, head h at row i * G + h
     constexpr int V = C::kVec;
     for (int k = 0;; ++k) {
       const int db = k % kDepBufs;
@@ -479,10 +488,9 @@ __global__ void __launch_bounds__(kThreads, CPS)
       }
       const float* dacc = reinterpret_cast<const float*>(deps + db * C::kDepBytes);
       const float2* dml = reinterpret_cast<const float2*>(dacc + C::kDepAccFloats);
-      const long long out_row0 = ((long long)dd.b * p.Hq + (long long)dd.g * G) * D;
       const int d = lane * V;
-      // combine the four warps' states, head by head
-      for (int h = 0; h < G; ++h) {
+      // combine the four warps' states, row by row
+      for (int h = 0; h < GT; ++h) {
         float2 ml[kConsumerWarps];
         float M = -INFINITY;
 #pragma unroll
@@ -507,15 +515,18 @@ __global__ void __launch_bounds__(kThreads, CPS)
           }
         }
         if (dd.slot < 0) {
-          const float inv = 1.f / lam;
+          // a row that sees no token (a query ahead of the sequence) is 0
+          const float inv = lam > 0.f ? 1.f / lam : 0.f;
 #pragma unroll
           for (int v = 0; v < V; ++v) o[v] *= inv;
-          store_out_vec<OUT_F32, V>(p.out, out_row0 + (long long)h * D + d, o);
+          const int qi = h / p.G, hh = h - qi * p.G;
+          store_out_vec<OUT_F32, V>(
+              p.out, (((long long)dd.b * p.T + qi) * p.Hq + (long long)dd.g * p.G + hh) * D + d, o);
         } else {
-          float* dst = p.ws.part_acc + ((long long)dd.slot * G + h) * D + d;
+          float* dst = p.ws.part_acc + ((long long)dd.slot * GT + h) * D + d;
           if constexpr (V == 4) *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
           else *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
-          if (lane == 0) p.ws.part_ml[(long long)dd.slot * G + h] = make_float2(M, lam);
+          if (lane == 0) p.ws.part_ml[(long long)dd.slot * GT + h] = make_float2(M, lam);
         }
       }
       // the deposit slot is free again
@@ -547,6 +558,14 @@ __global__ void __launch_bounds__(kThreads, CPS)
   float acc[NT][C::kMTiles][4];
   float m_run[NT][2], l_run[NT][2];
   int nseg = 0;  // segments deposited so far
+  // Multi-token decode: column n of the MMA N dimension is query token n / G;
+  // it sees T - 1 - n / G tokens fewer than the last one (padding columns
+  // past G * T see what the last one sees).
+  int kshift[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) kshift[nt][e] = max(0, p.T - 1 - (nt * 8 + 2 * c + e) / p.G);
   int nq = 0;    // fused prologue: q_ready phases completed
   RopeLane<D> rope;  // fused prologue: cos/sin at the current piece's new-token position
 
@@ -634,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int hh = nt * 8 + r;
-        const bool hv = hh < p.G;
+        const bool hv = hh < p.GT;
         const uint16_t* qrow = qs + hh * D;
 #pragma unroll
         for (int ks = 0; ks < C::kKSteps; ++ks) {
@@ -777,8 +796,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
     if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
 
     // ---- online softmax (base 2)
-    const int valid = inf.valid - tok0;  // live tokens in this warp's slice
-    const bool tail = valid < 16;        // warp-uniform
+    // tokens from this warp's slice start to the sequence end; query row n
+    // (token n / G of the T new ones) sees kshift[n] of them fewer
+    const int valid = inf.valid - tok0;
+    const bool ktail = valid - (p.T - 1) < 16;  // warp-uniform: some logit is masked
+    const bool vtail = valid < 16;              // warp-uniform: some V row is past the end
     const float mul = p.scale_log2 * inf.k_scale;
     uint32_t pb[NT][2];
     float alpha[NT][2];
@@ -786,9 +808,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
     for (int nt = 0; nt < NT; ++nt) {
       float s0 = sacc[nt][0] * mul, s1 = sacc[nt][1] * mul;
       float s2 = sacc[nt][2] * mul, s3 = sacc[nt][3] * mul;
-      if (tail) {
-        if (r >= valid) { s0 = -INFINITY; s1 = -INFINITY; }
-        if (r + 8 >= valid) { s2 = -INFINITY; s3 = -INFINITY; }
+      if (ktail) {
+        const int lim0 = valid - kshift[nt][0], lim1 = valid - kshift[nt][1];
+        if (r >= lim0) s0 = -INFINITY;
+        if (r >= lim1) s1 = -INFINITY;
+        if (r + 8 >= lim0) s2 = -INFINITY;
+        if (r + 8 >= lim1) s3 = -INFINITY;
       }
       float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 4));
@@ -837,7 +862,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
 
     // ---- O^T += V_w^T . P^T   (V rows past the length are zeroed in registers:
     // their probabilities are 0 but the slot may hold NaN/Inf garbage)
-    if (tail) {
+    if (vtail) {
       const uint32_t m_lo = (2 * c < valid ? 0x0000ffffu : 0u) | (2 * c + 1 < valid ? 0xffff0000u : 0u);
       const uint32_t m_hi = (2 * c + 8 < valid ? 0x0000ffffu : 0u) | (2 * c + 9 < valid ? 0xffff0000u : 0u);
 #pragma unroll
@@ -894,6 +919,7 @@ struct MergeParams {
   Ws ws;
   void* out;
   int S, Hkv, G, Hq, slots;  // slots = 2 * V partial slots in the workspace
+  int T, GT;                 // query tokens per sequence; rows per segment = G * T
 };
 
 template <int D, bool OUT_F32>
@@ -901,7 +927,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   constexpr int kVec = D / 32;                 // output elements per lane
   constexpr int kBatch = D == 128 ? 24 : 32;   // pieces loaded together (<= 32)
   pdl_wait();                                  // the partials of the decode kernel
-  const int G = p.G, lane = threadIdx.x & 31;
+  const int G = p.GT, lane = threadIdx.x & 31;  // rows per segment
   const int jobs = p.S * G;
   for (int job = blockIdx.x * kMergeWarps + (threadIdx.x >> 5); job < jobs;
        job += gridDim.x * kMergeWarps) {
@@ -954,11 +980,13 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
       }
       M = Mn;
     }
-    const float inv = 1.f / lam;
+    const float inv = lam > 0.f ? 1.f / lam : 0.f;  // a row that sees no token is 0
 #pragma unroll
     for (int v = 0; v < kVec; ++v) o[v] *= inv;
     const int b = s / p.Hkv, g = s - b * p.Hkv;
-    store_out_vec<OUT_F32, kVec>(p.out, ((long long)b * p.Hq + (long long)g * G + h) * D + lane * kVec, o);
+    const int qi = h / p.G, hh = h - qi * p.G;  // row h = query token qi, head hh
+    store_out_vec<OUT_F32, kVec>(
+        p.out, (((long long)b * p.T + qi) * p.Hq + (long long)g * p.G + hh) * D + lane * kVec, o);
   }
   pdl_trigger();
 }
@@ -1120,7 +1148,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
                     int pt_stride, int num_pages, void* out, hpa_out_dtype out_dtype, int batch,
                     int num_q_heads, int num_kv_heads, int head_dim, float softmax_scale,
                     hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream,
-                    const ProArgs* pro) {
+                    const ProArgs* pro, int q_tokens) {
   if (!q || !k_cache || !v_cache || !page_table || !out || !workspace) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || pt_stride <= 0 || num_pages <= 0 ||
       grid <= 0)
@@ -1133,6 +1161,11 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   if (fp8 && (!k_scale || !v_scale)) return HPA_ERR_INVALID_ARG;
   const int G = num_q_heads / num_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return HPA_ERR_UNSUPPORTED;
+  if (q_tokens < 1) return HPA_ERR_INVALID_ARG;
+  // the G * T rows of a kv head ride on the MMA N dimension: at most 16
+  if (q_tokens > kMaxQTokens || G * q_tokens > 16) return HPA_ERR_UNSUPPORTED;
+  if (pro && q_tokens != 1) return HPA_ERR_UNSUPPORTED;
+  const int GT = G * q_tokens;
   if (head_dim != 64 && head_dim != 128) return HPA_ERR_UNSUPPORTED;
   if (fp8 && head_dim != 128) return HPA_ERR_UNSUPPORTED;
   if ((long long)num_pages * num_kv_heads * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
@@ -1151,7 +1184,8 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
     if (fp8) return HPA_ERR_UNSUPPORTED;  // the new row would need a new page scale
   }
   WsLayout L;
-  if (!ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid, &L))
+  // the plan and workspace of a multi-token step count G * T rows per kv head
+  if (!ws_layout(kind, batch, num_kv_heads, num_q_heads * q_tokens, head_dim, grid, &L))
     return HPA_ERR_INVALID_ARG;
   if (ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return HPA_ERR_WORKSPACE;
 
@@ -1173,6 +1207,8 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
   p.G = G;
+  p.T = q_tokens;
+  p.GT = GT;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.ws = ws_view(workspace, L);
   p.grid = grid;
@@ -1187,7 +1223,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.k_cache_w = pro ? static_cast<__nv_bfloat16*>(const_cast<void*>(k_cache)) : nullptr;
   p.v_cache_w = pro ? static_cast<__nv_bfloat16*>(const_cast<void*>(v_cache)) : nullptr;
   p.q_out = pro ? static_cast<__nv_bfloat16*>(pro->q_out) : nullptr;
-  const int nt = G > 8 ? 2 : 1;
+  const int nt = GT > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1208,10 +1244,12 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   mp.S = batch * num_kv_heads;
   mp.Hkv = num_kv_heads;
   mp.G = G;
+  mp.T = q_tokens;
+  mp.GT = GT;
   mp.Hq = num_q_heads;
   mp.slots = (int)(2 * plan_ranges_ll(kind, grid));
   cudaLaunchConfig_t cfg = {};
-  const long long merge_ctas = ((long long)mp.S * G + kMergeWarps - 1) / kMergeWarps;
+  const long long merge_ctas = ((long long)mp.S * GT + kMergeWarps - 1) / kMergeWarps;
   cfg.gridDim = dim3((unsigned)std::min<long long>(merge_ctas, (long long)std::max(1, sms) * 16));
   cfg.blockDim = dim3(kMergeWarps * 32);
   cfg.stream = s;
@@ -1247,7 +1285,20 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
                                      size_t ws_bytes, void* stream) {
   return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
                        num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
-                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr);
+                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr, 1);
+}
+
+extern "C" hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, const void* v_cache,
+                                           const float* k_scale, const float* v_scale,
+                                           hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                                           int pt_stride, int num_pages, void* out,
+                                           hpa_out_dtype out_dtype, int batch, int q_tokens,
+                                           int num_q_heads, int num_kv_heads, int head_dim,
+                                           float softmax_scale, hpa_plan_kind kind, int grid,
+                                           void* workspace, size_t ws_bytes, void* stream) {
+  return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
+                       num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
+                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr, q_tokens);
 }
 
 extern "C" hpa_status hpa_decode_run_prologue(
@@ -1259,5 +1310,5 @@ extern "C" hpa_status hpa_decode_run_prologue(
   const hpa::ProArgs pro{k_raw, v_raw, q_gamma, k_gamma, eps, rope_theta, q_out};
   return hpa::run_impl(q_raw, k_cache, v_cache, nullptr, nullptr, HPA_KV_BF16, page_table,
                        pt_stride, num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads,
-                       head_dim, softmax_scale, kind, grid, workspace, ws_bytes, stream, &pro);
+                       head_dim, softmax_scale, kind, grid, workspace, ws_bytes, stream, &pro, 1);
 }

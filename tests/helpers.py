@@ -57,6 +57,30 @@ def to_device(batch, device="cuda"):
     return batch
 
 
+def gpu_decode_multi(batch, *, kind=0, num_ctas=None, param=0, out_dtype=torch.bfloat16,
+                     fp8=None):
+    """Multi-token plan + run on the GPU through the C-ABI binding: q and the
+    returned output are [B][T][Hq][D]."""
+    import mixed_length_paged_b200 as hpa
+    dev = torch.device("cuda")
+    B, T, Hq, D = batch.q.shape
+    Hkv = batch.shape.num_kv_heads
+    dec = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, kind=kind, num_ctas=num_ctas,
+                           param=param, max_seq_len=int(batch.seq_lens.max().item()),
+                           q_tokens=T, device=dev)
+    out = torch.full((B, T, Hq, D), float("nan"), dtype=out_dtype, device=dev)
+    dec.plan(batch.seq_lens.to(dev))
+    kw = {}
+    kc, vc = batch.k_cache.to(dev), batch.v_cache.to(dev)
+    if fp8 is not None:
+        kc, ks, vc, vs = (torch.from_numpy(x).to(dev) for x in fp8)
+        kw = dict(k_scale=ks, v_scale=vs)
+    dec.run(batch.q.to(dev), kc, vc, batch.page_table.to(dev), out, 1.0 / D ** 0.5, **kw)
+    torch.cuda.synchronize()
+    assert hpa.read_status(dec.workspace) == 0
+    return out
+
+
 def quantize_fp8(batch):
     """e4m3 codes + scales of an fp8 workload, made by the oracle's quantiser on
     the host (the decode path only consumes them)."""

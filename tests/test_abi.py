@@ -140,6 +140,35 @@ def test_run_rejects_bad_arguments_without_launching(L, bad, expect):
     assert _run(L, **bad) == expect
 
 
+def _run_multi(L, **kw):
+    a = dict(q=256, k=256, v=256, ks=None, vs=None, kvd=0, pt=256, pts=4, pages=8, out=256,
+             outd=0, B=2, T=2, Hq=8, Hkv=2, D=64, scale=0.125, kind=0, grid=148, ws=256,
+             wsb=1 << 24)
+    a.update(kw)
+    return L.hpa_decode_run_multi(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["kvd"], a["pt"],
+                                  a["pts"], a["pages"], a["out"], a["outd"], a["B"], a["T"],
+                                  a["Hq"], a["Hkv"], a["D"], C.c_float(a["scale"]), a["kind"],
+                                  a["grid"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(T=0), 1), (dict(T=-3), 1), (dict(T=17, Hq=2, Hkv=2), 2),
+    (dict(T=3, Hq=64, Hkv=8), 2),    # G * T = 24 rows > 16
+    (dict(T=2, Hq=16, Hkv=1), 2),    # G = 16: no room for a second token
+    (dict(q=None), 1), (dict(q=256 + 8), 1), (dict(wsb=64), 3), (dict(kind=9), 1),
+])
+def test_run_multi_rejects_bad_arguments_without_launching(L, bad, expect):
+    assert _run_multi(L, **bad) == expect
+
+
+def test_multi_token_workspace_counts_rows_of_all_tokens(L):
+    # a 4-token step of G = 2 needs the workspace of G * T = 8 rows per kv head
+    assert hpa.decode_workspace_size(0, 32, 8, 16 * 4, 128, 296) == \
+        hpa.decode_workspace_size(0, 32, 8, 64, 128, 296)
+    assert _run_multi(L, T=4, Hq=4, Hkv=2,
+                      wsb=hpa.decode_workspace_size(0, 2, 2, 4, 64, 148)) == 3  # sized for T=1
+
+
 def _run_pro(L, **kw):
     a = dict(qr=256, kr=256, vr=256, gq=256, gk=256, eps=1e-6, theta=1e4, kc=256, vc=256, qo=None,
              pt=256, pts=4, pages=8, out=256, outd=0, B=2, Hq=8, Hkv=2, D=64, scale=0.125,
@@ -202,3 +231,10 @@ def test_product_path_does_not_reference_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "liboracle" not in text, f
+
+
+def test_decode_num_ctas_rejects_bad_geometry(L):
+    assert L.hpa_decode_num_ctas(0, 0, 8, 1) == -1
+    assert L.hpa_decode_num_ctas(0, 64, 0, 1) == -1
+    assert L.hpa_decode_num_ctas(0, 64, 8, 0) == -1
+    assert L.hpa_decode_num_ctas(0, 60, 8, 1) == -1  # Hq not a multiple of Hkv

@@ -16,7 +16,8 @@ import torch
 import oracle
 import mixed_length_paged_b200 as hpa
 from mixed_length_paged_b200 import workloads as W
-from tests.helpers import (bf16_values, bits16, compact_rows, errors, gpu_decode, oracle_decode,
+from tests.helpers import (bf16_values, bits16, compact_rows, errors, gpu_decode, gpu_decode_multi,
+                           oracle_decode,
                            quantize_fp8, to_device)
 
 pytestmark = pytest.mark.gpu
@@ -337,6 +338,68 @@ def test_mix_prologue_workload_sampled_rows():
     q_out, status = _run_prologue(batch)
     assert status == 0
     out = gpu_decode(batch, q=q_out)
+    _check(out[rows], ref)
+
+
+# ---------------------------------------------------------------- multi-token decode
+
+# pre-step lengths: new tokens straddling a page edge, a sequence exactly T
+# long, one shorter than T (its first queries see nothing), an empty one,
+# several pages, a long one
+MT_LENS = [65, 200, 2, 0, 1000, 64, 4097, 130]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,T", [(64, 8, 128, 2), (32, 8, 128, 4), (8, 4, 64, 8),
+                                        (4, 4, 128, 16), (16, 2, 64, 2)])
+@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7)])
+def test_multi_token_decode_matches_oracle(Hq, Hkv, D, T, kind, num_ctas):
+    batch = W.make_batch(W.DecodeShape("mt", Hq, Hkv, D, q_tokens=T), MT_LENS, seed=31)
+    ref = oracle.paged_decode_multi(bits16(batch.q), bits16(batch.k_cache),
+                                    bits16(batch.v_cache), batch.page_table.numpy(),
+                                    batch.seq_lens.numpy(), Hkv, 1 / math.sqrt(D))
+    out = gpu_decode_multi(batch, kind=kind, num_ctas=num_ctas, out_dtype=torch.float32)
+    _check(out, ref)
+
+
+def test_decode_num_ctas_matches_residency():
+    two = hpa.default_num_ctas()
+    assert hpa.decode_num_ctas(64, 8, 1) == two          # 8 rows per kv head: 2 CTAs / SM
+    assert hpa.decode_num_ctas(64, 8, 2) == two // 2     # 16 rows: one CTA / SM
+    assert hpa.decode_num_ctas(32, 2, 1) == two // 2     # G = 16
+    assert hpa.decode_num_ctas(8, 2, 2) == two           # G * T = 8
+
+
+def test_multi_token_fp8_and_bf16_out():
+    shape = W.DecodeShape("mt8", 32, 8, 128, kv_dtype="fp8_e4m3", q_tokens=2)
+    batch = W.make_batch(shape, [1, 63, 64, 65, 700, 3000], seed=32)
+    fp8 = quantize_fp8(batch)
+    kc, ks, vc, vs = fp8
+    ref = oracle.paged_decode_multi(bits16(batch.q), kc, vc, batch.page_table.numpy(),
+                                    batch.seq_lens.numpy(), 8, 1 / math.sqrt(128), kv_fp8=True,
+                                    k_scale=ks, v_scale=vs)
+    out = gpu_decode_multi(batch, fp8=fp8)
+    _check(out, ref, max_abs=FP8_MAX_ABS)
+
+
+def test_multi_token_one_token_equals_single_token_run():
+    # q_tokens = 1 through the multi-token entry is the regular run, bit for bit
+    batch = W.make_batch(W.DecodeShape("mt1", 64, 8, 128, q_tokens=1), [100, 5000, 3], seed=33)
+    to_device(batch)
+    single = gpu_decode(batch, out_dtype=torch.float32)
+    batch.q = batch.q.unsqueeze(1)
+    multi = gpu_decode_multi(batch, out_dtype=torch.float32)
+    assert torch.equal(single, multi[:, 0])
+
+
+def test_multi_token_workload_sampled_rows():
+    batch = W.build("skewed_mtp2", device="cuda")
+    out = gpu_decode_multi(batch)
+    rows = [0, 1, 31]
+    small = compact_rows(batch, rows)
+    small.q = batch.q[rows].cpu()
+    ref = oracle.paged_decode_multi(bits16(small.q), bits16(small.k_cache),
+                                    bits16(small.v_cache), small.page_table.numpy(),
+                                    small.seq_lens.numpy(), 8, 1 / math.sqrt(128))
     _check(out[rows], ref)
 
 
