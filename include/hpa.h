@@ -23,7 +23,7 @@
  *     which never trap: they skip the offending access and set a bit in a
  *     device status word (HPA_DEVICE_*), read back with hpa_read_status.
  *   - Shapes: head_dim D in {64, 128}; page (tile) size 64 tokens; GQA group
- *     G = num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
+ *     G = num_q_heads / num_kv_heads in 1 .. 16 (rows padded to whole MMA n-tiles of 8).
  *
  * Tensor layouts (row-major, innermost last):
  *   q, q_raw, out        [batch][num_q_heads][D]

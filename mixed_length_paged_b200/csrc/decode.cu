@@ -1160,7 +1160,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   const bool fp8 = kv_dtype == HPA_KV_FP8_E4M3;
   if (fp8 && (!k_scale || !v_scale)) return HPA_ERR_INVALID_ARG;
   const int G = num_q_heads / num_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return HPA_ERR_UNSUPPORTED;
+  if (G > 16) return HPA_ERR_UNSUPPORTED;  // a kv head's rows fill at most two MMA n-tiles
   if (q_tokens < 1) return HPA_ERR_INVALID_ARG;
   // the G * T rows of a kv head ride on the MMA N dimension: at most 16
   if (q_tokens > kMaxQTokens || G * q_tokens > 16) return HPA_ERR_UNSUPPORTED;

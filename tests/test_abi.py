@@ -129,7 +129,7 @@ def _run(L, **kw):
     (dict(q=None), 1), (dict(k=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
     (dict(B=0), 1), (dict(Hq=6, Hkv=4), 1), (dict(kvd=5), 1), (dict(outd=2), 1),
     (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(kvd=1), 1),  # fp8 w/o scales
-    (dict(Hq=24, Hkv=8), 2),   # G = 3
+    (dict(Hq=34, Hkv=2), 2),   # G = 17
     (dict(Hq=64, Hkv=2), 2),   # G = 32
     (dict(D=96), 2), (dict(D=256), 2), (dict(kvd=1, ks=256, vs=256), 2),  # fp8 needs D = 128
     (dict(pages=1 << 26, Hkv=8, Hq=8), 2),  # rows overflow int32 TMA coordinates
@@ -186,7 +186,7 @@ def _run_pro(L, **kw):
     (dict(gk=None), 1), (dict(kc=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
     (dict(kr=256 + 8), 1), (dict(vr=256 + 4), 1), (dict(qr=256 + 8), 1), (dict(qo=256 + 1), 1),
     (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1), (dict(theta=0.0), 1),
-    (dict(theta=float("nan")), 1), (dict(scale=0.0), 1), (dict(D=96), 2), (dict(Hq=24, Hkv=8), 2),
+    (dict(theta=float("nan")), 1), (dict(scale=0.0), 1), (dict(D=96), 2), (dict(Hq=34, Hkv=2), 2),
     (dict(wsb=64), 3), (dict(kind=9), 1),
 ])
 def test_run_prologue_rejects_bad_arguments_without_launching(L, bad, expect):

@@ -130,6 +130,11 @@ SMALL = [
     ("g2_d64", [33, 400, 1], 8, 4, 64),
     ("g16", [200, 1500], 32, 2, 128),
     ("b1", [3333], 8, 1, 128),
+    # group sizes that are not powers of two (rows padded to n-tiles of 8)
+    ("g7", [300, 64, 4100], 28, 4, 128),
+    ("g12", [129, 2000], 96, 8, 128),
+    ("g3_d64", [65, 1, 777], 6, 2, 64),
+    ("g5", [5000], 5, 1, 128),
 ]
 
 
@@ -350,7 +355,7 @@ MT_LENS = [65, 200, 2, 0, 1000, 64, 4097, 130]
 
 
 @pytest.mark.parametrize("Hq,Hkv,D,T", [(64, 8, 128, 2), (32, 8, 128, 4), (8, 4, 64, 8),
-                                        (4, 4, 128, 16), (16, 2, 64, 2)])
+                                        (4, 4, 128, 16), (16, 2, 64, 2), (12, 4, 128, 5)])
 @pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7)])
 def test_multi_token_decode_matches_oracle(Hq, Hkv, D, T, kind, num_ctas):
     batch = W.make_batch(W.DecodeShape("mt", Hq, Hkv, D, q_tokens=T), MT_LENS, seed=31)
