@@ -109,11 +109,11 @@ HPA_API int hpa_version(void);
 HPA_API int hpa_default_num_ctas(int device);
 
 /* Persistent CTA count (num_ctas of hpa_decode_plan) that matches how many
- * run-kernel CTAs fit an SM for this head geometry: hpa_default_num_ctas
- * when each kv head has at most 8 query rows (G * q_tokens <= 8), one per SM
- * above that.  A dynamic plan for more CTAs than fit at once would leave
- * part of its primary ranges to a second wave.  Returns -1 on invalid
- * arguments or if the device cannot be queried. */
+ * run-kernel CTAs fit at once for this head geometry; a dynamic plan for more
+ * CTAs than fit would leave part of its primary ranges to a second wave.
+ * Every supported geometry (G * q_tokens <= 16) fits two per SM, so this is
+ * hpa_default_num_ctas for valid arguments.  Returns -1 on invalid arguments
+ * or if the device cannot be queried. */
 HPA_API int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads, int q_tokens);
 
 /* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC,

@@ -51,12 +51,9 @@ extern "C" int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads
                                    int q_tokens) {
   if (num_q_heads <= 0 || num_kv_heads <= 0 || q_tokens <= 0 || num_q_heads % num_kv_heads)
     return -1;
-  const int n = hpa_default_num_ctas(device);
-  if (n < 0) return -1;
-  // more than 8 query rows per kv head (two MMA n-tiles) leave room for one
-  // run-kernel CTA per SM only
-  const long long rows = (long long)(num_q_heads / num_kv_heads) * q_tokens;
-  return rows > 8 ? n / HPA_CTAS_PER_SM : n;
+  // every supported geometry (up to 16 query rows per kv head) runs two
+  // run-kernel CTAs per SM: the two-n-tile kernel splits its warps by n-tile
+  return hpa_default_num_ctas(device);
 }
 
 extern "C" size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_kv_heads,

@@ -80,9 +80,19 @@ struct Cfg {
   static constexpr int kRawBytes = PRO ? 2 * D * 2 : 0;
   static constexpr int kSlotBytes = kQBytes + kRawBytes; // per-stage q (+ raw rows) slot
   static constexpr int kAccStride = D + 4;             // floats; keeps deposits off one bank
-  // one deposit: acc[warp][head][D + 4] floats, then (m, l)[warp][head]
-  static constexpr int kDepAccFloats = kConsumerWarps * kHeads * kAccStride;
-  static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kHeads * 8;
+  // Warp roles.  One n-tile (8 rows): warp w owns tokens [16w, 16w + 16) of
+  // every tile and all 8 rows.  Two n-tiles (9..16 rows): warp w owns n-tile
+  // w / 2 and tokens [32 (w % 2), + 32), as two 16-token blocks -- the same
+  // MMA work with the registers of the one-n-tile kernel, so two CTAs still
+  // fit an SM.
+  static constexpr bool kSplit = NT == 2;
+  static constexpr int kWarpTiles = kSplit ? 1 : NT;   // n-tiles per warp
+  static constexpr int kBlocks = kSplit ? 2 : 1;       // 16-token blocks per warp
+  static constexpr int kWarpRows = 8 * kWarpTiles;     // rows each warp deposits
+  static constexpr int kRowWarps = kSplit ? 2 : kConsumerWarps;  // warps holding a row
+  // one deposit: acc[warp][row of the warp][D + 4] floats, then (m, l)[warp][row]
+  static constexpr int kDepAccFloats = kConsumerWarps * kWarpRows * kAccStride;
+  static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kWarpRows * 8;
   static constexpr int kMisc = 2048;                   // barriers, stage info, flags
   // CPS CTAs share one SM's 228 KiB (1 KiB of it reserved per CTA)
   static constexpr int kBudget = CPS == 1 ? kSmemLimit : (kSmemPerSm / CPS - 1024);
@@ -489,23 +499,26 @@ __global__ void __launch_bounds__(kThreads, CPS)
       const float* dacc = reinterpret_cast<const float*>(deps + db * C::kDepBytes);
       const float2* dml = reinterpret_cast<const float2*>(dacc + C::kDepAccFloats);
       const int d = lane * V;
-      // combine the four warps' states, row by row
+      // combine the states of the warps that hold each row, row by row
       for (int h = 0; h < GT; ++h) {
-        float2 ml[kConsumerWarps];
+        const int w0 = C::kSplit ? 2 * (h >> 3) : 0;  // first warp holding row h
+        const int lr = C::kSplit ? (h & 7) : h;       // its row inside those warps
+        float2 ml[C::kRowWarps];
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          ml[w] = dml[w * C::kHeads + h];
-          M = fmaxf(M, ml[w].x);
+        for (int k = 0; k < C::kRowWarps; ++k) {
+          ml[k] = dml[(w0 + k) * C::kWarpRows + lr];
+          M = fmaxf(M, ml[k].x);
         }
         float lam = 0.f, o[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) o[v] = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float sc = (ml[w].x == -INFINITY) ? 0.f : fast_exp2(ml[w].x - M);
-          lam += ml[w].y * sc;
-          const float* src = dacc + (w * C::kHeads + h) * C::kAccStride + d;
+        for (int k = 0; k < C::kRowWarps; ++k) {
+          // a warp that saw no token of the piece holds m = -inf, acc = 0
+          const float sc = (ml[k].x == -INFINITY) ? 0.f : fast_exp2(ml[k].x - M);
+          lam += ml[k].y * sc;
+          const float* src = dacc + ((w0 + k) * C::kWarpRows + lr) * C::kAccStride + d;
           if constexpr (V == 4) {
             const float4 a = *reinterpret_cast<const float4*>(src);
             o[0] += a.x * sc; o[1] += a.y * sc; o[2] += a.z * sc; o[3] += a.w * sc;
@@ -537,16 +550,21 @@ __global__ void __launch_bounds__(kThreads, CPS)
   }
 
   // -------------------------------------------------------------- consumers
+  constexpr int W = C::kWarpTiles, MB = C::kBlocks;
   const int r = lane >> 2, c = lane & 3;          // MMA fragment coordinates
   const int lm = lane >> 3, lr = lane & 7;        // ldmatrix address lane roles
-  const int tok0 = warp * 16;                     // this warp's token slice
+  const int nt0 = C::kSplit ? (warp >> 1) : 0;    // this warp's first n-tile
+  const int tok0 = C::kSplit ? 32 * (warp & 1) : 16 * warp;  // its first token
   // ldmatrix row (token) for the QK A operand and the PV A operand
   const int k_tok = tok0 + (lm & 1) * 8 + lr;
   const int k_chk = lm >> 1;
   const int v_tok = FP8 ? tok0 + (lm & 1) * 8 + lr : tok0 + (lm >> 1) * 8 + lr;
   const int v_chk = FP8 ? (lm >> 1) : (lm & 1);
   // Byte offsets (inside a tile) of this lane's ldmatrix rows for chunk 2j +
-  // chk, j = 0..3, under the 128-byte swizzle; chunk 2j + 8 + chk adds one box.
+  // chk, j = 0..3, under the 128-byte swizzle; chunk 2j + 8 + chk adds one
+  // box, and the next 16-token block adds 16 rows of 128 bytes (the swizzle
+  // pattern repeats every 8 rows).
+  constexpr uint32_t kBlockBytes = 16 * 128;
   uint32_t koff[4], voff[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -554,18 +572,18 @@ __global__ void __launch_bounds__(kThreads, CPS)
     voff[j] = v_tok * 128 + ((((2 * j + v_chk) & 7) ^ (v_tok & 7)) << 4);
   }
 
-  uint32_t qf[NT][C::kKSteps][2];
-  float acc[NT][C::kMTiles][4];
-  float m_run[NT][2], l_run[NT][2];
+  uint32_t qf[W][C::kKSteps][2];
+  float acc[W][C::kMTiles][4];
+  float m_run[W][2], l_run[W][2];
   int nseg = 0;  // segments deposited so far
   // Multi-token decode: column n of the MMA N dimension is query token n / G;
   // it sees T - 1 - n / G tokens fewer than the last one (padding columns
   // past G * T see what the last one sees).
-  int kshift[NT][2];
+  int kshift[W][2];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int nt = 0; nt < W; ++nt)
 #pragma unroll
-    for (int e = 0; e < 2; ++e) kshift[nt][e] = max(0, p.T - 1 - (nt * 8 + 2 * c + e) / p.G);
+    for (int e = 0; e < 2; ++e) kshift[nt][e] = max(0, p.T - 1 - ((nt0 + nt) * 8 + 2 * c + e) / p.G);
   int nq = 0;    // fused prologue: q_ready phases completed
   RopeLane<D> rope;  // fused prologue: cos/sin at the current piece's new-token position
 
@@ -575,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
     wait_bar(smem_u32(&dep_empty[db]), ((nseg / kDepBufs) & 1) ^ 1, s_abort, status);
     if (inf) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < W; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           float v = l_run[nt][e];
@@ -586,10 +604,10 @@ __global__ void __launch_bounds__(kThreads, CPS)
         }
       float* dacc = reinterpret_cast<float*>(deps + db * C::kDepBytes);
       float2* dml = reinterpret_cast<float2*>(dacc + C::kDepAccFloats);
-      float* my_acc = dacc + warp * C::kHeads * C::kAccStride;
+      float* my_acc = dacc + warp * C::kWarpRows * C::kAccStride;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int h0 = nt * 8 + 2 * c;
+      for (int nt = 0; nt < W; ++nt) {
+        const int h0 = nt * 8 + 2 * c;  // row inside this warp's rows
 #pragma unroll
         for (int i = 0; i < C::kMTiles; ++i) {
           const int dr0 = FP8 ? 16 * i + 2 * r : 16 * i + r;
@@ -600,8 +618,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
           my_acc[(h0 + 1) * C::kAccStride + dr1] = acc[nt][i][3];
         }
         if (r == 0) {
-          dml[warp * C::kHeads + h0] = make_float2(m_run[nt][0], l_run[nt][0]);
-          dml[warp * C::kHeads + h0 + 1] = make_float2(m_run[nt][1], l_run[nt][1]);
+          dml[warp * C::kWarpRows + h0] = make_float2(m_run[nt][0], l_run[nt][0]);
+          dml[warp * C::kWarpRows + h0 + 1] = make_float2(m_run[nt][1], l_run[nt][1]);
         }
       }
     }
@@ -617,6 +635,32 @@ __global__ void __launch_bounds__(kThreads, CPS)
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&dep_full[db]));
     ++nseg;
+  };
+
+  // V fragments (MMA A operand of O^T += V^T P^T) of 16-token block mb.
+  auto load_v = [&](uint32_t vt, int mb, uint32_t (&va)[C::kMTiles][4]) {
+    const uint32_t vb = vt + mb * kBlockBytes;
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int i = 0; i < C::kMTiles; ++i)
+        ldsm_x4_t(vb + voff[i & 3] + (i >> 2) * C::kBoxBytes, va[i][0], va[i][1], va[i][2], va[i][3]);
+    } else {
+#pragma unroll
+      for (int ip = 0; ip < C::kMTiles / 2; ++ip) {
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_t(vb + voff[ip], r0, r1, r2, r3);
+        // r0/r1: tokens [0,8)/[8,16) of chunk 2ip; r2/r3: same for chunk 2ip+1.
+        // Each holds bytes {V(t,d), V(t,d+1), V(t+1,d), V(t+1,d+1)}.
+        va[2 * ip][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0020));
+        va[2 * ip][1] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0031));
+        va[2 * ip][2] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r1, 0, 0x0020));
+        va[2 * ip][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r1, 0, 0x0031));
+        va[2 * ip + 1][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r2, 0, 0x0020));
+        va[2 * ip + 1][1] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r2, 0, 0x0031));
+        va[2 * ip + 1][2] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0020));
+        va[2 * ip + 1][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0031));
+      }
+    }
   };
 
   for (int it = 0;; ++it) {
@@ -648,11 +692,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
         if (!wait_bar(smem_u32(q_ready), nq & 1, s_abort, status)) break;
         ++nq;
       }
-      // query fragments (MMA B operand) of this kv head's G query heads
+      // query fragments (MMA B operand) of this warp's rows
       const uint16_t* qs = reinterpret_cast<const uint16_t*>(qslots + s * C::kSlotBytes);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int hh = nt * 8 + r;
+      for (int nt = 0; nt < W; ++nt) {
+        const int hh = (nt0 + nt) * 8 + r;
         const bool hv = hh < p.GT;
         const uint16_t* qrow = qs + hh * D;
 #pragma unroll
@@ -678,10 +722,13 @@ __global__ void __launch_bounds__(kThreads, CPS)
       }
     }
 
-    // Fused prologue: if the new token's row lies in this warp's 16-token
-    // slice, form its K row (RMSNorm + RoPE of the raw row; the piece's
-    // cos/sin are already in `rope`) while the tiles are still in flight.
-    const bool patch = PRO && (inf.flags & kNewTok) && warp == ((inf.pos & (kPageSize - 1)) >> 4);
+    // Fused prologue: if the new token's row lies in this warp's tokens, form
+    // its K row (RMSNorm + RoPE of the raw row; the piece's cos/sin are
+    // already in `rope`) while the tiles are still in flight.  (With two
+    // n-tiles, the two warps on the slot's tokens both patch it, with the
+    // same bits.)
+    const int ptok = inf.pos & (kPageSize - 1);
+    const bool patch = PRO && (inf.flags & kNewTok) && ptok >= tok0 && ptok < tok0 + 16 * MB;
     __nv_bfloat16 klo[D / 64], khi[D / 64];
     if constexpr (PRO) {
       if (patch)
@@ -695,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
       if (patch) {
         // patch the new K and V rows into the landed tiles (128-byte
         // swizzle) and write them to their cache slot
-        const int tr = inf.pos & (kPageSize - 1);
+        const int tr = ptok;
         const uint4* vraw = reinterpret_cast<const uint4*>(qslots + s * C::kSlotBytes + C::kQBytes + 2 * D);
         uint8_t* ktile = stages + s * C::kStageBytes;
         uint8_t* vtile = ktile + C::kTileBytes;
@@ -724,98 +771,93 @@ __global__ void __launch_bounds__(kThreads, CPS)
       }
     }
 
-    // ---- S^T = K_w . Q^T, four independent accumulation chains (k-step mod 4)
+    // ---- S^T = K_w . Q^T per 16-token block, four independent accumulation
+    // chains (k-step mod 4)
     constexpr int kChains = 4;
-    float sch[kChains][NT][4];
+    float sacc[MB][W][4];
 #pragma unroll
-    for (int q = 0; q < kChains; ++q)
+    for (int mb = 0; mb < MB; ++mb) {
+      const uint32_t kb = kt + mb * kBlockBytes;
+      float sch[kChains][W][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int q = 0; q < kChains; ++q)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) sch[q][nt][j] = 0.f;
-    if constexpr (!FP8) {
+        for (int nt = 0; nt < W; ++nt)
 #pragma unroll
-      for (int ks = 0; ks < C::kKSteps; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(kt + koff[ks & 3] + (ks >> 2) * C::kBoxBytes, a0, a1, a2, a3);
+          for (int j = 0; j < 4; ++j) sch[q][nt][j] = 0.f;
+      if constexpr (!FP8) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          mma_bf16(sch[ks % kChains][nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
-      }
-    } else {
+        for (int ks = 0; ks < C::kKSteps; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kb + koff[ks & 3] + (ks >> 2) * C::kBoxBytes, a0, a1, a2, a3);
 #pragma unroll
-      for (int kp = 0; kp < C::kKSteps / 2; ++kp) {
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4(kt + koff[kp], r0, r1, r2, r3);
-        const uint32_t a[2][4] = {
-            {e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff), e4m3x2_to_f16x2(r0 >> 16),
-             e4m3x2_to_f16x2(r1 >> 16)},
-            {e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff), e4m3x2_to_f16x2(r2 >> 16),
-             e4m3x2_to_f16x2(r3 >> 16)}};
+          for (int nt = 0; nt < W; ++nt)
+            mma_bf16(sch[ks % kChains][nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+        }
+      } else {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_f16(sch[(2 * kp) % kChains][nt], a[0][0], a[0][1], a[0][2], a[0][3],
-                  qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-          mma_f16(sch[(2 * kp + 1) % kChains][nt], a[1][0], a[1][1], a[1][2], a[1][3],
-                  qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+        for (int kp = 0; kp < C::kKSteps / 2; ++kp) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(kb + koff[kp], r0, r1, r2, r3);
+          const uint32_t a[2][4] = {
+              {e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff), e4m3x2_to_f16x2(r0 >> 16),
+               e4m3x2_to_f16x2(r1 >> 16)},
+              {e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff), e4m3x2_to_f16x2(r2 >> 16),
+               e4m3x2_to_f16x2(r3 >> 16)}};
+#pragma unroll
+          for (int nt = 0; nt < W; ++nt) {
+            mma_f16(sch[(2 * kp) % kChains][nt], a[0][0], a[0][1], a[0][2], a[0][3],
+                    qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+            mma_f16(sch[(2 * kp + 1) % kChains][nt], a[1][0], a[1][1], a[1][2], a[1][3],
+                    qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+          }
         }
       }
+#pragma unroll
+      for (int nt = 0; nt < W; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          sacc[mb][nt][j] = (sch[0][nt][j] + sch[1][nt][j]) + (sch[2][nt][j] + sch[3][nt][j]);
     }
-    float sacc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        sacc[nt][j] = (sch[0][nt][j] + sch[1][nt][j]) + (sch[2][nt][j] + sch[3][nt][j]);
 
-    // V fragments now, so their shared-memory latency overlaps the softmax
+    // V fragments of the first block now, so their shared-memory latency
+    // overlaps the softmax
     uint32_t va[C::kMTiles][4];
-    if constexpr (!FP8) {
-#pragma unroll
-      for (int i = 0; i < C::kMTiles; ++i)
-        ldsm_x4_t(vt + voff[i & 3] + (i >> 2) * C::kBoxBytes, va[i][0], va[i][1], va[i][2], va[i][3]);
-    } else {
-#pragma unroll
-      for (int ip = 0; ip < C::kMTiles / 2; ++ip) {
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4_t(vt + voff[ip], r0, r1, r2, r3);
-        // r0/r1: tokens [0,8)/[8,16) of chunk 2ip; r2/r3: same for chunk 2ip+1.
-        // Each holds bytes {V(t,d), V(t,d+1), V(t+1,d), V(t+1,d+1)}.
-        va[2 * ip][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0020));
-        va[2 * ip][1] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0031));
-        va[2 * ip][2] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r1, 0, 0x0020));
-        va[2 * ip][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r1, 0, 0x0031));
-        va[2 * ip + 1][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r2, 0, 0x0020));
-        va[2 * ip + 1][1] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r2, 0, 0x0031));
-        va[2 * ip + 1][2] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0020));
-        va[2 * ip + 1][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0031));
-      }
+    load_v(vt, 0, va);
+    if constexpr (MB == 1) {
+      // all shared-memory reads of this stage are issued: hand it back
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
     }
-    // all shared-memory reads of this stage are issued: hand it back
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
 
-    // ---- online softmax (base 2)
-    // tokens from this warp's slice start to the sequence end; query row n
+    // ---- online softmax (base 2) over this warp's MB blocks
+    // tokens from this warp's first token to the sequence end; query row n
     // (token n / G of the T new ones) sees kshift[n] of them fewer
     const int valid = inf.valid - tok0;
-    const bool ktail = valid - (p.T - 1) < 16;  // warp-uniform: some logit is masked
-    const bool vtail = valid < 16;              // warp-uniform: some V row is past the end
     const float mul = p.scale_log2 * inf.k_scale;
-    uint32_t pb[NT][2];
-    float alpha[NT][2];
+    uint32_t pb[MB][W][2];
+    float alpha[W][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float s0 = sacc[nt][0] * mul, s1 = sacc[nt][1] * mul;
-      float s2 = sacc[nt][2] * mul, s3 = sacc[nt][3] * mul;
-      if (ktail) {
-        const int lim0 = valid - kshift[nt][0], lim1 = valid - kshift[nt][1];
-        if (r >= lim0) s0 = -INFINITY;
-        if (r >= lim1) s1 = -INFINITY;
-        if (r + 8 >= lim0) s2 = -INFINITY;
-        if (r + 8 >= lim1) s3 = -INFINITY;
+    for (int nt = 0; nt < W; ++nt) {
+      float sv[MB][4];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) {
+        sv[mb][0] = sacc[mb][nt][0] * mul;
+        sv[mb][1] = sacc[mb][nt][1] * mul;
+        sv[mb][2] = sacc[mb][nt][2] * mul;
+        sv[mb][3] = sacc[mb][nt][3] * mul;
+        const int vb = valid - 16 * mb;  // tokens from this block's start
+        if (vb - (p.T - 1) < 16) {       // warp-uniform: some logit of the block is masked
+          const int lim0 = vb - kshift[nt][0], lim1 = vb - kshift[nt][1];
+          if (r >= lim0) sv[mb][0] = -INFINITY;
+          if (r >= lim1) sv[mb][1] = -INFINITY;
+          if (r + 8 >= lim0) sv[mb][2] = -INFINITY;
+          if (r + 8 >= lim1) sv[mb][3] = -INFINITY;
+        }
+        mx0 = fmaxf(mx0, fmaxf(sv[mb][0], sv[mb][2]));
+        mx1 = fmaxf(mx1, fmaxf(sv[mb][1], sv[mb][3]));
       }
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 4));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 4));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 8));
@@ -826,31 +868,37 @@ __global__ void __launch_bounds__(kThreads, CPS)
       const float base0 = (mn0 == -INFINITY) ? 0.f : mn0;
       const float base1 = (mn1 == -INFINITY) ? 0.f : mn1;
       const float al0 = fast_exp2(m_run[nt][0] - base0), al1 = fast_exp2(m_run[nt][1] - base1);
-      const float p0 = fast_exp2(s0 - base0), p2 = fast_exp2(s2 - base0);
-      const float p1 = fast_exp2(s1 - base1), p3 = fast_exp2(s3 - base1);
-      l_run[nt][0] = l_run[nt][0] * al0 + p0 + p2;
-      l_run[nt][1] = l_run[nt][1] * al1 + p1 + p3;
+      float l0 = l_run[nt][0] * al0, l1 = l_run[nt][1] * al1;
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) {
+        const float p0 = fast_exp2(sv[mb][0] - base0), p2 = fast_exp2(sv[mb][2] - base0);
+        const float p1 = fast_exp2(sv[mb][1] - base1), p3 = fast_exp2(sv[mb][3] - base1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        if constexpr (!FP8) {
+          pb[mb][nt][0] = movm_t(pack_bf16(p0, p1));
+          pb[mb][nt][1] = movm_t(pack_bf16(p2, p3));
+        } else {
+          const float vsc = inf.v_scale;
+          pb[mb][nt][0] = movm_t(pack_f16(p0 * vsc, p1 * vsc));
+          pb[mb][nt][1] = movm_t(pack_f16(p2 * vsc, p3 * vsc));
+        }
+      }
+      l_run[nt][0] = l0;
+      l_run[nt][1] = l1;
       m_run[nt][0] = mn0;
       m_run[nt][1] = mn1;
       alpha[nt][0] = al0;
       alpha[nt][1] = al1;
-      if constexpr (!FP8) {
-        pb[nt][0] = movm_t(pack_bf16(p0, p1));
-        pb[nt][1] = movm_t(pack_bf16(p2, p3));
-      } else {
-        const float vsc = inf.v_scale;
-        pb[nt][0] = movm_t(pack_f16(p0 * vsc, p1 * vsc));
-        pb[nt][1] = movm_t(pack_f16(p2 * vsc, p3 * vsc));
-      }
     }
     // Rescale the accumulators only if some running max moved (once the
     // maxima settle, almost no tile needs it).
     bool moved = false;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) moved |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    for (int nt = 0; nt < W; ++nt) moved |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
     if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < W; ++nt)
 #pragma unroll
         for (int i = 0; i < C::kMTiles; ++i) {
           acc[nt][i][0] *= alpha[nt][0];
@@ -860,26 +908,39 @@ __global__ void __launch_bounds__(kThreads, CPS)
         }
     }
 
-    // ---- O^T += V_w^T . P^T   (V rows past the length are zeroed in registers:
-    // their probabilities are 0 but the slot may hold NaN/Inf garbage)
-    if (vtail) {
-      const uint32_t m_lo = (2 * c < valid ? 0x0000ffffu : 0u) | (2 * c + 1 < valid ? 0xffff0000u : 0u);
-      const uint32_t m_hi = (2 * c + 8 < valid ? 0x0000ffffu : 0u) | (2 * c + 9 < valid ? 0xffff0000u : 0u);
+    // ---- O^T += V_w^T . P^T per block   (V rows past the length are zeroed
+    // in registers: their probabilities are 0 but the slot may hold NaN/Inf
+    // garbage)
 #pragma unroll
-      for (int i = 0; i < C::kMTiles; ++i) {
-        va[i][0] &= m_lo;
-        va[i][1] &= m_lo;
-        va[i][2] &= m_hi;
-        va[i][3] &= m_hi;
+    for (int mb = 0; mb < MB; ++mb) {
+      if (mb > 0) {
+        load_v(vt, mb, va);
+        // all shared-memory reads of this stage are issued: hand it back
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
       }
+      const int vb = valid - 16 * mb;
+      if (vb < 16) {  // warp-uniform: some V row of the block is past the end
+        const uint32_t m_lo = (2 * c < vb ? 0x0000ffffu : 0u) | (2 * c + 1 < vb ? 0xffff0000u : 0u);
+        const uint32_t m_hi = (2 * c + 8 < vb ? 0x0000ffffu : 0u) | (2 * c + 9 < vb ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int i = 0; i < C::kMTiles; ++i) {
+          va[i][0] &= m_lo;
+          va[i][1] &= m_lo;
+          va[i][2] &= m_hi;
+          va[i][3] &= m_hi;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < C::kMTiles; ++i)
+#pragma unroll
+        for (int nt = 0; nt < W; ++nt) {
+          if constexpr (!FP8)
+            mma_bf16(acc[nt][i], va[i][0], va[i][1], va[i][2], va[i][3], pb[mb][nt][0], pb[mb][nt][1]);
+          else
+            mma_f16(acc[nt][i], va[i][0], va[i][1], va[i][2], va[i][3], pb[mb][nt][0], pb[mb][nt][1]);
+        }
     }
-#pragma unroll
-    for (int i = 0; i < C::kMTiles; ++i)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        if constexpr (!FP8) mma_bf16(acc[nt][i], va[i][0], va[i][1], va[i][2], va[i][3], pb[nt][0], pb[nt][1]);
-        else mma_f16(acc[nt][i], va[i][0], va[i][1], va[i][2], va[i][3], pb[nt][0], pb[nt][1]);
-      }
 
     if (inf.flags & kLast) deposit(&inf);
   }
@@ -1105,9 +1166,8 @@ hpa_status launch_nt(int nt, int cps, const CUtensorMap& tk, const CUtensorMap& 
   if (cps == 1)
     return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s)
                    : launch<D, 2, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s);
-  // G = 16 (two n-tiles) does not fit two CTAs per SM: it always runs one
   return nt == 1 ? launch<D, 1, FP8, OUT_F32, 2, PRO>(tk, tv, p, grid, s)
-                 : launch<D, 2, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s);
+                 : launch<D, 2, FP8, OUT_F32, 2, PRO>(tk, tv, p, grid, s);
 }
 
 template <bool OUT_F32, bool PRO>

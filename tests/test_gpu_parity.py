@@ -368,10 +368,9 @@ def test_multi_token_decode_matches_oracle(Hq, Hkv, D, T, kind, num_ctas):
 
 def test_decode_num_ctas_matches_residency():
     two = hpa.default_num_ctas()
-    assert hpa.decode_num_ctas(64, 8, 1) == two          # 8 rows per kv head: 2 CTAs / SM
-    assert hpa.decode_num_ctas(64, 8, 2) == two // 2     # 16 rows: one CTA / SM
-    assert hpa.decode_num_ctas(32, 2, 1) == two // 2     # G = 16
-    assert hpa.decode_num_ctas(8, 2, 2) == two           # G * T = 8
+    # 8 rows per kv head, and 16 (two n-tiles, warps split by n-tile): 2 CTAs / SM
+    for args in ((64, 8, 1), (64, 8, 2), (32, 2, 1), (8, 2, 2)):
+        assert hpa.decode_num_ctas(*args) == two, args
 
 
 def test_multi_token_fp8_and_bf16_out():
