@@ -28,6 +28,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -42,7 +43,7 @@ L2_BYTES = 126 * 1000 * 1000  # B200 L2 capacity
 WORKLOAD = "skewed"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_run_skewed_ncu.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "mixed_length_paged_b200", "csrc", f)
-                  for f in ("decode.cu", "hpa_common.cuh")]
+                  for f in ("decode.cu", "hpa_common.cuh", "prologue_math.cuh")]
 
 
 def _args():
@@ -102,11 +103,20 @@ def _quantize_e4m3(values, live):
     return codes.contiguous(), scale.contiguous()
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines (what the compiler sees;
+    the kernel sources hold no string literal with a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def _kernel_hash() -> str:
+    """Fingerprint of the run kernel's code (comments do not count)."""
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

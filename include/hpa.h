@@ -104,8 +104,9 @@ HPA_API const char* hpa_last_cuda_error(void);
 HPA_API int hpa_version(void);
 
 /* Number of persistent CTAs for `device`: two per SM (296 on B200), which
- * the run kernel executes as two co-resident CTAs per SM.  Returns -1 if the
- * device cannot be queried. */
+ * the run kernel executes as two co-resident CTAs per SM.  The environment
+ * variable HPA_NUM_CTAS (a decimal count 1 .. 65536) overrides it; other
+ * values of it are ignored.  Returns -1 if the device cannot be queried. */
 HPA_API int hpa_default_num_ctas(int device);
 
 /* Persistent CTA count (num_ctas of hpa_decode_plan) that matches how many

@@ -1,6 +1,7 @@
 // api.cu -- host-only entry points of libhpa.so: status strings, version,
 // workspace sizing and layout, default CTA count, status readback.
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "hpa_common.cuh"
@@ -38,6 +39,12 @@ extern "C" int hpa_version(void) { return 100; }
 #endif
 
 extern "C" int hpa_default_num_ctas(int device) {
+  // HPA_NUM_CTAS (a decimal count, 1 .. 65536) overrides the device default
+  if (const char* env = std::getenv("HPA_NUM_CTAS")) {
+    char* end = nullptr;
+    const long v = std::strtol(env, &end, 10);
+    if (end != env && *end == '\0' && v >= 1 && v <= 65536) return (int)v;
+  }
   int n = 0;
   cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
   if (e != cudaSuccess) {

@@ -18,23 +18,35 @@
 //     L2 evict-first hint; for the first tile of a segment it also bulk-copies
 //     the segment's query rows.  The metadata rides along in the stage.
 //   consumers: warp w owns tokens [16w, 16w+16) of every tile and keeps its own
-//     online-softmax state (m, l, acc) for the tile's G query heads:
-//       S^T[16 tok x 8 heads] = K_w[16 x D] . Q^T        (mma m16n8k16, fp32 acc)
+//     online-softmax state (m, l, acc) for the tile's query rows:
+//       S^T[16 tok x 8 rows] = K_w[16 x D] . Q^T        (mma m16n8k16, fp32 acc)
 //       online softmax in base 2 (logits pre-scaled by scale * log2 e)
-//       O^T[D x 8 heads]    += V_w^T[D x 16] . P^T      (P^T built in registers
-//                                                       with movmatrix)
-//     The GQA group sits on the MMA N dimension (8 heads per n-tile), so no
-//     padding is needed for G = 8.  At a segment end each warp deposits its
-//     state in a double-buffered shared-memory slot and carries on.
-//   epilogue: combines the four warps' states of each deposited segment; a
-//     segment held whole by the CTA is written directly, otherwise the CTA
-//     stores an (acc, m, l) partial.  This keeps the consumers streaming
-//     through segment boundaries.
+//       O^T[D x 8 rows]    += V_w^T[D x 16] . P^T      (P^T built in registers
+//                                                      with movmatrix)
+//     The query rows of a kv head (G heads, times T tokens for multi-token
+//     decode) sit on the MMA N dimension, 8 per n-tile, padded.  With 9..16
+//     rows (two n-tiles) warp w instead owns n-tile w / 2 and tokens
+//     [32 (w % 2), +32), which keeps the registers of the one-n-tile kernel.
+//     At a segment end each warp deposits its state in a double-buffered
+//     shared-memory slot and carries on.
+//   epilogue: combines the states of the warps holding each row of a
+//     deposited segment; a segment held whole by the CTA is written directly,
+//     otherwise the CTA stores an (acc, m, l) partial.  This keeps the
+//     consumers streaming through segment boundaries.
+// Each stage has two full barriers: one for its small copies (query rows;
+// the new token's raw K/V rows under the fused prologue) and one for the K/V
+// tiles, so work on the former overlaps the tiles' load.
 // A second, small kernel (chained by programmatic dependent launch) merges
-// the partials of every split segment in split order: one CTA per segment,
-// all partial rows loaded in parallel.  (Merging inside the persistent kernel
-// puts a single CTA's dependent L2 reads on the critical path: the splits of
-// a long sequence all finish together at the end of the step.)
+// the partials of every split segment in range order, one warp per (segment,
+// row), all partials loaded in parallel.  (Merging inside the persistent
+// kernel puts a single CTA's dependent L2 reads on the critical path: the
+// splits of a long sequence all finish together at the end of the step.)
+//
+// Fused prologue (hpa_decode_run_prologue): the consumers normalise and
+// rotate the raw query rows of each piece in shared memory; the warp whose
+// tokens hold the new token's slot patches its K/V rows into the landed tile
+// and stores them to the cache.  Multi-token decode (hpa_decode_run_multi):
+// row n = token n / G of T; each column masks the positions past its token.
 //
 // FP8 (e4m3) caches: K/V codes are converted in registers with
 // cvt.rn.f16x2.e4m3x2 (exact) and the products run as f16 MMAs; the

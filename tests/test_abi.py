@@ -238,3 +238,17 @@ def test_decode_num_ctas_rejects_bad_geometry(L):
     assert L.hpa_decode_num_ctas(0, 64, 0, 1) == -1
     assert L.hpa_decode_num_ctas(0, 64, 8, 0) == -1
     assert L.hpa_decode_num_ctas(0, 60, 8, 1) == -1  # Hq not a multiple of Hkv
+
+
+def test_num_ctas_environment_override():
+    # runs in a child process: the override is read from the environment at
+    # each call, and this needs no GPU
+    import subprocess
+    import sys
+    code = ("import mixed_length_paged_b200 as h; L = h.lib(); "
+            "print(L.hpa_default_num_ctas(0), L.hpa_decode_num_ctas(0, 64, 8, 2))")
+    for val, want in (("77", "77 77"), ("1", "1 1")):
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                           env={**os.environ, "HPA_NUM_CTAS": val},
+                           cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+        assert r.stdout.split() == want.split(), r.stderr

@@ -489,6 +489,60 @@ def bits_t(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
 
 
+# ---------------------------------------------------------------- canaries
+
+@pytest.mark.parametrize("kind,num_ctas,T", [(0, None, 1), (0, 5, 1), (1, None, 1),
+                                             (2, 7, 1), (0, None, 2)])
+def test_writes_stay_inside_out_and_workspace(kind, num_ctas, T):
+    """Guard bytes around the output and the workspace, and the whole KV
+    cache, are unchanged by plan + run (compute-sanitizer is not available,
+    so out-of-range writes are looked for this way)."""
+    Hq, Hkv, D = 32, 8, 128
+    batch = W.make_batch(W.DecodeShape("canary", Hq, Hkv, D, q_tokens=T),
+                         [0, 1, 64, 65, 4000, 300], seed=41)
+    to_device(batch)
+    B = batch.batch
+    n = num_ctas or hpa.default_num_ctas()
+    maxlen = int(batch.seq_lens.max().item())
+    grid = hpa.plan_grid(kind, B, Hkv, n, 0, maxlen)
+    ws_bytes = hpa.decode_workspace_size(kind, B, Hkv, Hq * T, D, grid)
+    guard = 4096
+    ws_all = torch.full((ws_bytes + 2 * guard,), 0x5A, dtype=torch.uint8, device="cuda")
+    ws = ws_all[guard:guard + ws_bytes]
+    out_shape = (B, T, Hq, D) if T > 1 else (B, Hq, D)
+    numel = B * T * Hq * D
+    out_all = torch.full((numel + 2 * guard,), 12345.0, dtype=torch.float32, device="cuda")
+    out = out_all[guard:guard + numel].view(out_shape)
+    kc, vc = bits16(batch.k_cache).copy(), bits16(batch.v_cache).copy()
+    hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq * T, head_dim=D,
+                    pt_stride=batch.pt_stride, workspace=ws, kind=kind, num_ctas=n,
+                    max_seq_len=maxlen)
+    run = hpa.decode_run_multi if T > 1 else hpa.decode_run
+    run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, ws, grid,
+        1 / math.sqrt(D), kind=kind)
+    torch.cuda.synchronize()
+    assert hpa.read_status(ws) == 0
+    assert torch.all(ws_all[:guard] == 0x5A) and torch.all(ws_all[guard + ws_bytes:] == 0x5A)
+    assert torch.all(out_all[:guard] == 12345.0) and torch.all(out_all[guard + numel:] == 12345.0)
+    assert torch.isfinite(out).all()
+    np.testing.assert_array_equal(bits16(batch.k_cache), kc)
+    np.testing.assert_array_equal(bits16(batch.v_cache), vc)
+
+
+def test_fused_prologue_writes_only_the_new_slots():
+    lens = [0, 63, 64, 1000]
+    batch = _prologue_case(lens, Hq=32, Hkv=8, D=128)
+    kc, vc = bits16(batch.k_cache).copy(), bits16(batch.v_cache).copy()
+    to_device(batch)
+    _, (_, ka, va, _) = _separate_and_fused(batch)  # the fused path's caches
+    pt = batch.page_table.cpu().numpy()
+    touched = np.zeros(kc.shape[:3], dtype=bool)
+    for b, pos in enumerate(lens):
+        touched[pt[b, pos // 64], :, pos % 64] = True
+    gk, gv = bits16(ka), bits16(va)
+    assert not (gk != kc)[~touched].any() and not (gv != vc)[~touched].any()
+
+
 # ---------------------------------------------------------------- device-side checks
 
 def test_bad_page_id_is_flagged():
