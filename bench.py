@@ -353,7 +353,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale,
                     k_scale=k_scale, v_scale=v_scale)
 
+    # The dynamic plan is made inside the decode kernel (hpa_decode_step)
+    # where that applies; the fused prologue still runs after a plan kernel.
+    use_step = not shape.prologue and B <= hpa.MAX_STEP_BATCH
+
     def step():
+        if use_step:
+            dec.step(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out,
+                     scale, k_scale=k_scale, v_scale=v_scale)
+        else:
+            dec.plan(seq_lens)
+            run()
+
+    def plan_then_run():  # the three-launch form (comparator)
         dec.plan(seq_lens)
         run()
 
@@ -404,13 +416,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     end.record(stream)
     barrier()
     # Timed region 2 (per-kernel durations for the roofline): the same K
-    # steps with events around the plan and around the run call.
+    # steps with events around the plan and around the run call (one call,
+    # decode + merge, when the plan is made in the kernel).
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * K)]
     for i in range(K):
         ev[3 * i].record(stream)
-        dec.plan(seq_lens)
+        if not use_step:
+            dec.plan(seq_lens)
         ev[3 * i + 1].record(stream)
-        run()
+        if use_step:
+            step()
+        else:
+            run()
         ev[3 * i + 2].record(stream)
     barrier()
     clocks = sampler.stop()
@@ -423,6 +440,27 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # static split-KV comparators: the same run kernel fed the static plans
     extras = {}
+    if not args.no_extras and use_step:
+        # the same step as plan kernel + run (three launches), interleaved A/B
+        sep = graphed(plan_then_run)
+        blocks, per = 10, max(5, min(40, K // 10))
+        ab = {"step": 0.0, "plan_run": 0.0}
+        for _ in range(blocks):
+            for name, fn in (("step", timed_step), ("plan_run", sep)):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(per):
+                    fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ab[name] += a.elapsed_time(b)
+        n = blocks * per
+        extras["plan_kernel_then_run"] = {
+            "us_per_step": 1e3 * ab["plan_run"] / n,
+            "in_kernel_plan_us_per_step_same_blocks": 1e3 * ab["step"] / n,
+            "in_kernel_plan_speedup": ab["plan_run"] / ab["step"],
+            "method": f"interleaved A/B, {blocks} x {per} steps each"}
     if not args.no_extras and shape.prologue:
         # The same step with the prologue as its own kernel before plan + run,
         # timed as an interleaved A/B against the fused step (blocks of 20
@@ -526,9 +564,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             s_comp.wait_event(ev["in"][k])
             if started[k]:
                 s_comp.wait_event(ev["out"][k])      # step i-2's output is on the host
-            dec.plan(sl_d[k], stream=s_comp)
-            dec.run(q_d[k], batch.k_cache, batch.v_cache, pt_d[k], out_d[k], scale,
-                    stream=s_comp)
+            dec.step(q_d[k], batch.k_cache, batch.v_cache, pt_d[k], sl_d[k], out_d[k], scale,
+                     stream=s_comp)
             ev["done"][k].record(s_comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev["done"][k])
@@ -591,22 +628,28 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    f"L2-resident: {kv_bytes / 1e6:.3g} MB of KV per step fits the 126 MB L2 "
                    "(a latency figure, not an HBM one)"),
             "launch": "eager calls" if args.eager else
-                      "CUDA-graph replay of one captured step (plan + run)",
+                      "CUDA-graph replay of one captured step",
+            "plan": "in the decode kernel (hpa_decode_step)" if use_step else
+                    "plan kernel (hpa_decode_plan) before the run",
             "parallelism": f"data-parallel replicas x{world} (independent batches, no collective)",
         },
         "breakdown_us": {"plan": 1e3 * statistics.mean(plan_ms), "run": 1e3 * run_avg_ms,
                          "note": "events between the calls (timed region 2); the step time "
                                  "comes from timed region 1 without them"},
         "roofline": {"bound": "hbm",
-                     "kernel": ("hpa_decode_run_prologue" if shape.prologue else "hpa_decode_run")
-                     + " (decode_kernel + merge_kernel)",
+                     "kernel": ("hpa_decode_run_prologue (decode_kernel + merge_kernel)"
+                                if shape.prologue else
+                                "hpa_decode_step (decode_kernel with the plan inside + "
+                                "merge_kernel)" if use_step else
+                                "hpa_decode_run (decode_kernel + merge_kernel)"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy bandwidth",
                      "traffic": traffic, "algorithmic_bytes_per_launch": run_bytes},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 3 * K,  # plan, decode, merge
+        "gpu_launches": (2 if use_step else 3) * K,  # (plan,) decode, merge
         "clocks": clocks,
+        "plan_kernel_then_run": extras.get("plan_kernel_then_run"),
         "static_splitkv": {k: v for k, v in extras.items()
                            if k.startswith(("static", "dynamic"))} or None,
         "separate_prologue": extras.get("separate_prologue_kernel"),

@@ -247,6 +247,41 @@ HPA_API hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, cons
                                         void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * hpa_decode_step -- one decode step with the dynamic plan made inside the
+ * decode kernel: hpa_decode_plan(kind = DYNAMIC, num_ctas) followed by
+ * hpa_decode_run_multi, in two launches instead of three (xiaodao.ai
+ * "HPC-Ops TPOT -48.8%", Attention section: the per-step load-balanced tile
+ * plan; here each persistent CTA scans the lengths itself and derives its own
+ * ranges from the same closed forms, so the step needs no plan kernel and no
+ * wait for one).  Same partition, same partial slots and merge order, hence
+ * the same bits as the two-call path.
+ *
+ *   seq_lens     device [batch] int32, as for hpa_decode_plan.
+ *   batch        1 .. 512 (the tile offsets live in shared memory;
+ *                HPA_ERR_UNSUPPORTED beyond: use hpa_decode_plan + run).
+ *   num_ctas     persistent CTAs (hpa_decode_num_ctas), 1 .. 65536; also the
+ *                grid the workspace is sized for.
+ *   workspace    >= hpa_decode_workspace_size(HPA_PLAN_DYNAMIC, batch,
+ *                num_kv_heads, num_q_heads * q_tokens, head_dim, num_ctas)
+ *                bytes, 256-byte aligned, zero-filled before its first use
+ *                (or last written by hpa_decode_plan); every dynamic run
+ *                leaves its run-time counters at zero for the next step.  The
+ *                plan fields of the header and the segment descriptors are
+ *                written as hpa_decode_plan writes them; the range
+ *                descriptors are not.  Status bits accumulate until a
+ *                hpa_decode_plan on the workspace clears them.
+ *   the rest     as for hpa_decode_run_multi (q_tokens = 1: single-token).
+ */
+HPA_API hpa_status hpa_decode_step(const int32_t* seq_lens, const void* q, const void* k_cache,
+                                   const void* v_cache, const float* k_scale,
+                                   const float* v_scale, hpa_kv_dtype kv_dtype,
+                                   const int32_t* page_table, int pt_stride, int num_pages,
+                                   void* out, hpa_out_dtype out_dtype, int batch, int q_tokens,
+                                   int num_q_heads, int num_kv_heads, int head_dim,
+                                   float softmax_scale, int num_ctas, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/*
  * hpa_decode_run_prologue -- hpa_decode_run with the decode prologue fused
  * into the persistent kernel (bitbyai.com "vLLM x HPC-Ops", Attention
  * Backend: RoPE, query-key normalisation and the KV write fused into one

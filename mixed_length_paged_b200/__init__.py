@@ -9,7 +9,8 @@ it raises ``HpaLibraryMissing`` -- there is no fallback implementation.
 The functions mirror the C ABI in ``include/hpa.h``:
 
     decode_workspace_size, plan_grid, default_num_ctas, workspace_layout,
-    decode_plan, decode_run, decode_run_multi, decode_run_prologue, kv_prologue, read_status,
+    decode_plan, decode_run, decode_step, decode_run_multi, decode_run_prologue, kv_prologue,
+    read_status,
     decode_noalloc
 
 and ``PagedDecoder`` bundles a workspace with plan + run for callers who do
@@ -26,7 +27,8 @@ __all__ = [
     "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
     "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
-    "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run", "decode_run_multi",
+    "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run",
+    "decode_step", "MAX_STEP_BATCH", "decode_run_multi",
     "decode_run_prologue",
     "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
@@ -88,6 +90,9 @@ def lib():
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
                                      _F, _I, _I, _V, _Z, _V]
+        L.hpa_decode_step.restype = _I
+        L.hpa_decode_step.argtypes = [_V, _V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I,
+                                      _I, _I, _F, _I, _V, _Z, _V]
         L.hpa_decode_run_multi.restype = _I
         L.hpa_decode_run_multi.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I,
                                            _I, _I, _I, _F, _I, _I, _V, _Z, _V]
@@ -234,6 +239,54 @@ def decode_run(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                               float(softmax_scale), kind, grid, _ptr(workspace),
                               workspace.numel(), _stream(stream))
     _check(rc, "hpa_decode_run")
+    return out
+
+
+MAX_STEP_BATCH = 512  # sequences hpa_decode_step plans in the kernel
+
+
+def decode_step(seq_lens: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, page_table: torch.Tensor, out: torch.Tensor,
+                workspace: torch.Tensor, num_ctas: int, softmax_scale: float, *,
+                k_scale: torch.Tensor | None = None, v_scale: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """One decode step with the dynamic plan made inside the decode kernel
+    (hpa_decode_step).  q/out are [B][Hq][D], or [B][T][Hq][D] for T query
+    tokens per sequence.  The workspace must be zero-filled before its first
+    use (or last written by decode_plan)."""
+    _dev(seq_lens, "seq_lens", (torch.int32,), 1)
+    if q.dim() not in (3, 4):
+        raise HpaError("q must be [B][Hq][D] or [B][T][Hq][D]")
+    _dev(q, "q", (torch.bfloat16,), q.dim())
+    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
+    cache_types = (torch.uint8, torch.float8_e4m3fn) if fp8 else (torch.bfloat16,)
+    _dev(k_cache, "k_cache", cache_types, 4)
+    _dev(v_cache, "v_cache", cache_types, 4)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    _dev(out, "out", (torch.bfloat16, torch.float32), q.dim())
+    _dev(workspace, "workspace", (torch.uint8,))
+    if fp8:
+        if k_scale is None or v_scale is None:
+            raise HpaError("FP8 caches need k_scale and v_scale")
+        _dev(k_scale, "k_scale", (torch.float32,), 2)
+        _dev(v_scale, "v_scale", (torch.float32,), 2)
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        T = 1
+    else:
+        B, T, Hq, D = q.shape
+    num_pages, Hkv, S, Dk = k_cache.shape
+    if S != PAGE_SIZE or Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or tuple(out.shape) != tuple(q.shape) or page_table.shape[0] != B \
+            or seq_lens.shape[0] != B:
+        raise HpaError("decode_step: inconsistent shapes")
+    rc = lib().hpa_decode_step(_ptr(seq_lens), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                               _ptr(k_scale), _ptr(v_scale), KV_FP8_E4M3 if fp8 else KV_BF16,
+                               _ptr(page_table), page_table.shape[1], num_pages, _ptr(out),
+                               OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, T, Hq, Hkv,
+                               D, float(softmax_scale), num_ctas, _ptr(workspace),
+                               workspace.numel(), _stream(stream))
+    _check(rc, "hpa_decode_step")
     return out
 
 
@@ -388,8 +441,9 @@ class PagedDecoder:
         self.q_tokens = q_tokens
         self.shape = (batch, num_q_heads, num_kv_heads, head_dim, pt_stride)
         grid = plan_grid(kind, batch, num_kv_heads, self.num_ctas, param, max_seq_len)
-        # a multi-token plan counts G * T rows per kv head
-        self.workspace = torch.empty(decode_workspace_size(kind, batch, num_kv_heads,
+        # a multi-token plan counts G * T rows per kv head; zero-filled so that
+        # step() can use it from the first call
+        self.workspace = torch.zeros(decode_workspace_size(kind, batch, num_kv_heads,
                                                            num_q_heads * q_tokens, head_dim, grid),
                                      dtype=torch.uint8, device=self.device)
         self.grid = grid
@@ -412,6 +466,19 @@ class PagedDecoder:
         return decode_run(q, k_cache, v_cache, page_table, out, self.workspace, self.grid,
                           softmax_scale, kind=self.kind, k_scale=k_scale, v_scale=v_scale,
                           stream=stream)
+
+    def step(self, q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, *,
+             k_scale=None, v_scale=None, stream=None):
+        """plan + run as one decode_step (the dynamic plan made inside the
+        decode kernel) when the plan is dynamic and the batch fits, else the
+        two calls."""
+        if self.kind == PLAN_DYNAMIC and self.shape[0] <= MAX_STEP_BATCH:
+            return decode_step(seq_lens, q, k_cache, v_cache, page_table, out, self.workspace,
+                               self.num_ctas, softmax_scale, k_scale=k_scale, v_scale=v_scale,
+                               stream=stream)
+        self.plan(seq_lens, stream=stream)
+        return self.run(q, k_cache, v_cache, page_table, out, softmax_scale, k_scale=k_scale,
+                        v_scale=v_scale, stream=stream)
 
     def run_prologue(self, q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache, v_cache, page_table,
                      out, softmax_scale, **kw):

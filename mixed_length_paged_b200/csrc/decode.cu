@@ -63,6 +63,7 @@
 #include <cuda_bf16.h>
 
 #include "hpa_common.cuh"
+#include "plan_geom.cuh"
 #include "prologue_math.cuh"
 
 namespace hpa {
@@ -77,8 +78,9 @@ constexpr int kSmemPerSm = 228 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any barrier wait
 constexpr int kDepBufs = 2;              // deposit slots between consumers and epilogue
 constexpr int kMaxQTokens = 16;          // query tokens per sequence (multi-token decode)
+constexpr int kMaxFusedBatch = 512;      // sequences an in-kernel plan keeps in shared memory
 
-template <int D, int NT, bool FP8, int CPS, bool PRO>
+template <int D, int NT, bool FP8, int CPS, bool PRO, bool FP>
 struct Cfg {
   static constexpr int kElt = FP8 ? 1 : 2;
   static constexpr int kRowBytes = D * kElt;           // one token row of one head
@@ -106,13 +108,15 @@ struct Cfg {
   static constexpr int kDepAccFloats = kConsumerWarps * kWarpRows * kAccStride;
   static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kWarpRows * 8;
   static constexpr int kMisc = 2048;                   // barriers, stage info, flags
+  // in-kernel plan: tile offsets of all sequences
+  static constexpr int kTsBytes = FP ? ((kMaxFusedBatch + 1) * 4 + 15) / 16 * 16 : 0;
   // CPS CTAs share one SM's 228 KiB (1 KiB of it reserved per CTA)
   static constexpr int kBudget = CPS == 1 ? kSmemLimit : (kSmemPerSm / CPS - 1024);
   static constexpr int kStagesFit =
-      (kBudget - 1024 - kDepBufs * kDepBytes - kMisc) / (kStageBytes + kSlotBytes);
+      (kBudget - 1024 - kDepBufs * kDepBytes - kMisc - kTsBytes) / (kStageBytes + kSlotBytes);
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
   static constexpr int kSmemBytes =
-      1024 + kStages * (kStageBytes + kSlotBytes) + kDepBufs * kDepBytes + kMisc;
+      1024 + kStages * (kStageBytes + kSlotBytes) + kDepBufs * kDepBytes + kMisc + kTsBytes;
   static constexpr int kKSteps = D / 16;               // QK MMA k-steps
   static constexpr int kMTiles = D / 16;               // PV MMA m-tiles
   static constexpr int kVec = D / 32;                  // output floats per epilogue lane
@@ -130,6 +134,8 @@ struct RunParams {
   void* out;
   int B, Hq, Hkv, G;
   int T, GT;                // query tokens per sequence; rows per kv head = G * T
+  const int32_t* seq_lens;  // in-kernel plan: the step's lengths (else the plan's)
+  int capacity;             // in-kernel plan: pt_stride * 64 tokens
   float scale_log2;         // softmax_scale * log2(e)
   Ws ws;
   int grid, kind;
@@ -237,12 +243,13 @@ __device__ __forceinline__ void store_out_vec(void* out, long long i, const floa
   }
 }
 
-template <int D, int NT, bool FP8, bool OUT_F32, int CPS, bool PRO>
+template <int D, int NT, bool FP8, bool OUT_F32, int CPS, bool PRO, bool FP>
 __global__ void __launch_bounds__(kThreads, CPS)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const RunParams p) {
-  using C = Cfg<D, NT, FP8, CPS, PRO>;
+  using C = Cfg<D, NT, FP8, CPS, PRO, FP>;
   static_assert(!(PRO && FP8), "the fused prologue writes bf16 caches");
+  static_assert(!(PRO && FP), "the in-kernel plan uses the weights' shared memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -269,6 +276,10 @@ __global__ void __launch_bounds__(kThreads, CPS)
   static_assert(C::kStages * 24 + kDepBufs * 16 + 8 + C::kStages * sizeof(StageInfo) +
                         kDepBufs * sizeof(DepDesc) + 16 <= C::kMisc / 2,
                 "misc area too small");
+  // in-kernel plan: tile offsets (after the misc area), and per-warp sums of
+  // the scan (in the weights' half of the misc area, unused without PRO)
+  int32_t* s_ts = reinterpret_cast<int32_t*>(misc + C::kMisc);
+  int* s_wsum = reinterpret_cast<int*>(misc + C::kMisc / 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -291,7 +302,51 @@ __global__ void __launch_bounds__(kThreads, CPS)
   }
   // Everything below reads what the plan (and possibly the prologue) wrote.
   pdl_wait();
-  if (threadIdx.x == 0) {
+  if constexpr (FP) {
+    // In-kernel plan (hpa_decode_step): every CTA turns the step's lengths
+    // into tile offsets in shared memory, as the plan kernel does -- warp w
+    // scans a contiguous slice 32 lengths at a time -- and then derives its
+    // own ranges from the same closed forms.
+    constexpr int kW = kThreads / 32;
+    const int slice = (p.B + kW - 1) / kW;
+    const int lo = min(p.B, warp * slice), hi = min(p.B, lo + slice);
+    int carry = 0;
+    bool clamped = false;
+    for (int i0 = lo; i0 < hi; i0 += 32) {
+      const int i = i0 + lane;
+      int n = 0;
+      if (i < hi) {
+        const int L = p.seq_lens[i];
+        const int Lc = min(max(L, 0), p.capacity);
+        clamped |= Lc != L;
+        n = (Lc + kPageSize - 1) / kPageSize;
+      }
+      int x = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (i < hi) s_ts[i] = carry + x - n;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) s_wsum[warp] = carry;
+    if (blockIdx.x == 0 && __any_sync(0xffffffffu, clamped) && lane == 0)
+      atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_LEN_CLAMPED);
+    __syncthreads();
+    int off = 0, T = 0;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+      off += w < warp ? s_wsum[w] : 0;
+      T += s_wsum[w];
+    }
+    if (off)
+      for (int i = lo + lane; i < hi; i += 32) s_ts[i] += off;
+    if (threadIdx.x == 0) {
+      s_ts[p.B] = T;
+      *s_plan_ok = 1;
+    }
+  } else if (threadIdx.x == 0) {
     const int32_t* h = p.ws.header;
     const bool ok = h[kHdrMagic] == kPlanMagic && h[kHdrGrid] == p.grid &&
                     h[kHdrGrid] == (int)gridDim.x && h[kHdrBatch] == p.B &&
@@ -312,22 +367,43 @@ __global__ void __launch_bounds__(kThreads, CPS)
   pdl_trigger();
 
   int32_t* status = &p.ws.header[kHdrStatus];
-  const int32_t* ts = p.ws.tile_start;
+  const int32_t* ts = FP ? s_ts : p.ws.tile_start;
+  // clamped length of sequence b
+  auto len_of = [&](int b) -> int {
+    if constexpr (FP) return min(max(p.seq_lens[b], 0), p.capacity);
+    else return p.ws.lens[b];
+  };
+  // the dynamic plan's geometry (in-kernel plan only)
+  DynGeom dg{};
+  if constexpr (FP) {
+    if (warp >= kConsumerWarps) {
+      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x);
+      double rc[4];
+      dyn_reciprocals(dg, rc);
+      dg.init_div(rc);
+    }
+  }
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     const uint64_t policy = l2_policy_evict_first();
     const int qrow_bytes = p.G * D * 2;  // one query token's rows of a kv head group
     const int qbytes = p.T * qrow_bytes;
-    const int U = p.ws.header[kHdrUnits];
-    const int V = p.ws.header[kHdrRanges];
+    const int U = FP ? (int)dg.U : p.ws.header[kHdrUnits];
+    const int V = FP ? (int)dg.ranges() : p.ws.header[kHdrRanges];
     const bool dyn = p.kind == HPA_PLAN_DYNAMIC;
     int it = 0;
     // This CTA's primary range first; under the dynamic plan it then takes
     // tail chunks, reserving the next one (and reading its descriptor) while
     // it streams the current one.
     int v = blockIdx.x;
-    int4 d0 = p.ws.cta_desc[2 * v], d1 = p.ws.cta_desc[2 * v + 1];
+    int4 d0, d1;
+    if constexpr (FP) {
+      dyn_range_desc(dg, ts, p.B, p.Hkv, v, &d0, &d1);
+    } else {
+      d0 = p.ws.cta_desc[2 * v];
+      d1 = p.ws.cta_desc[2 * v + 1];
+    }
     while (true) {
       int vn = V;
       int4 n0 = make_int4(0, 0, 0, 0), n1 = n0;
@@ -335,8 +411,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
         if (lane == 0) vn = p.grid + atomicAdd(&p.ws.header[kHdrNext], 1);
         vn = __shfl_sync(0xffffffffu, vn, 0);
         if (vn < V) {
-          n0 = p.ws.cta_desc[2 * vn];
-          n1 = p.ws.cta_desc[2 * vn + 1];
+          if constexpr (FP) {
+            dyn_range_desc(dg, ts, p.B, p.Hkv, vn, &n0, &n1);
+          } else {
+            n0 = p.ws.cta_desc[2 * vn];
+            n1 = p.ws.cta_desc[2 * vn + 1];
+          }
         }
       }
       const int ub = max(0, d0.x), ue = min(d0.y, U);
@@ -353,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
           float ks = 1.f, vs = 1.f;
           if (u < ue) {
             const int page = __ldg(p.page_table + (long long)w2.b * p.pt_stride + w2.t);
-            const int L = p.ws.lens[w2.b];
+            const int L = len_of(w2.b);
             // tokens from the tile's start to the sequence end, capped where no
             // query row's limit can reach (multi-token rows see up to T - 1 fewer)
             valid = min(kPageSize + kMaxQTokens - 1, L - w2.t * kPageSize);
@@ -473,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
     // zero output rows of empty sequences (a softmax over no tokens), for
     // every query token
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-      if (p.ws.lens[b] != 0) continue;
+      if (len_of(b) != 0) continue;
       const long long n = (long long)p.T * p.Hq * D;
       for (long long i = lane; i < n; i += 32) store_out<OUT_F32>(p.out, (long long)b * n + i, 0.f);
     }
@@ -489,6 +569,20 @@ __global__ void __launch_bounds__(kThreads, CPS)
         }
       }
     }
+    if (dyn) {
+      // The last CTA out resets the tail-chunk counter for the next step, so
+      // that a step whose plan is made in the kernel (hpa_decode_step) finds
+      // it at 0 whatever ran before on this workspace.  Every CTA gets here
+      // once (aborted ones too), after its last ticket, so the counter is no
+      // longer in use then.
+      if (lane == 0) {
+        __threadfence();
+        if (atomicAdd(&p.ws.header[kHdrDone], 1) == (int)gridDim.x - 1) {
+          atomicExch(&p.ws.header[kHdrNext], 0);
+          atomicExch(&p.ws.header[kHdrDone], 0);
+        }
+      }
+    }
     return;
   }
 
@@ -496,6 +590,26 @@ __global__ void __launch_bounds__(kThreads, CPS)
     // ------------------------------------------------------------ epilogue
     const int GT = p.GT;  // rows per kv head: query token i, head h at row i * G + h
     constexpr int V = C::kVec;
+    if constexpr (FP) {
+      // In-kernel plan: the segment descriptors the merge reads, shared out
+      // over the CTAs, and (CTA 0) the plan fields of the header.
+      const int S = p.B * p.Hkv;
+      for (int sg = blockIdx.x * 32 + lane; sg < S; sg += gridDim.x * 32)
+        p.ws.seg_desc[sg] = dyn_seg_desc(dg, ts, p.Hkv, sg);
+      if (blockIdx.x == 0 && lane == 0) {
+        int32_t* h = p.ws.header;
+        h[kHdrUnits] = (int32_t)dg.U;
+        h[kHdrGrid] = p.grid;
+        h[kHdrKind] = HPA_PLAN_DYNAMIC;
+        h[kHdrBatch] = p.B;
+        h[kHdrKvHeads] = p.Hkv;
+        h[kHdrGroup] = p.GT;
+        h[kHdrHeadDim] = D;
+        h[kHdrTiles] = ts[p.B];
+        h[kHdrRanges] = (int32_t)dg.ranges();
+        h[kHdrMagic] = kPlanMagic;
+      }
+    }
     for (int k = 0;; ++k) {
       const int db = k % kDepBufs;
       if (!wait_bar(smem_u32(&dep_full[db]), (k / kDepBufs) & 1, s_abort, status)) break;
@@ -1129,11 +1243,11 @@ bool make_cache_map(CUtensorMap* tm, const void* base, int num_pages, int Hkv, i
   return true;
 }
 
-template <int D, int NT, bool FP8, bool OUT_F32, int CPS, bool PRO>
+template <int D, int NT, bool FP8, bool OUT_F32, int CPS, bool PRO, bool FP>
 hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams& p, int grid,
                   cudaStream_t stream) {
-  using C = Cfg<D, NT, FP8, CPS, PRO>;
-  auto kern = decode_kernel<D, NT, FP8, OUT_F32, CPS, PRO>;
+  using C = Cfg<D, NT, FP8, CPS, PRO, FP>;
+  auto kern = decode_kernel<D, NT, FP8, OUT_F32, CPS, PRO, FP>;
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<uint64_t> ready_mask{0};
   int dev = 0;
@@ -1172,24 +1286,24 @@ hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams&
 // One persistent CTA per SM when the grid fits the SMs; two co-resident
 // (smaller) CTAs per SM when the grid is larger, so that twice as many
 // consumer warps hide each other's latencies.
-template <int D, bool FP8, bool OUT_F32, bool PRO>
+template <int D, bool FP8, bool OUT_F32, bool PRO, bool FP>
 hpa_status launch_nt(int nt, int cps, const CUtensorMap& tk, const CUtensorMap& tv,
                      const RunParams& p, int grid, cudaStream_t s) {
   if (cps == 1)
-    return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s)
-                   : launch<D, 2, FP8, OUT_F32, 1, PRO>(tk, tv, p, grid, s);
-  return nt == 1 ? launch<D, 1, FP8, OUT_F32, 2, PRO>(tk, tv, p, grid, s)
-                 : launch<D, 2, FP8, OUT_F32, 2, PRO>(tk, tv, p, grid, s);
+    return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s)
+                   : launch<D, 2, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s);
+  return nt == 1 ? launch<D, 1, FP8, OUT_F32, 2, PRO, FP>(tk, tv, p, grid, s)
+                 : launch<D, 2, FP8, OUT_F32, 2, PRO, FP>(tk, tv, p, grid, s);
 }
 
-template <bool OUT_F32, bool PRO>
+template <bool OUT_F32, bool PRO, bool FP>
 hpa_status launch_d(bool fp8, int head_dim, int nt, int cps, const CUtensorMap& tk,
                     const CUtensorMap& tv, const RunParams& p, int grid, cudaStream_t s) {
   if constexpr (!PRO) {
-    if (fp8) return launch_nt<128, true, OUT_F32, false>(nt, cps, tk, tv, p, grid, s);
+    if (fp8) return launch_nt<128, true, OUT_F32, false, FP>(nt, cps, tk, tv, p, grid, s);
   }
-  return head_dim == 128 ? launch_nt<128, false, OUT_F32, PRO>(nt, cps, tk, tv, p, grid, s)
-                         : launch_nt<64, false, OUT_F32, PRO>(nt, cps, tk, tv, p, grid, s);
+  return head_dim == 128 ? launch_nt<128, false, OUT_F32, PRO, FP>(nt, cps, tk, tv, p, grid, s)
+                         : launch_nt<64, false, OUT_F32, PRO, FP>(nt, cps, tk, tv, p, grid, s);
 }
 
 // Arguments of the fused prologue (hpa_decode_run_prologue).
@@ -1220,7 +1334,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
                     int pt_stride, int num_pages, void* out, hpa_out_dtype out_dtype, int batch,
                     int num_q_heads, int num_kv_heads, int head_dim, float softmax_scale,
                     hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream,
-                    const ProArgs* pro, int q_tokens) {
+                    const ProArgs* pro, int q_tokens, const int32_t* plan_lens) {
   if (!q || !k_cache || !v_cache || !page_table || !out || !workspace) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || pt_stride <= 0 || num_pages <= 0 ||
       grid <= 0)
@@ -1237,6 +1351,14 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   // the G * T rows of a kv head ride on the MMA N dimension: at most 16
   if (q_tokens > kMaxQTokens || G * q_tokens > 16) return HPA_ERR_UNSUPPORTED;
   if (pro && q_tokens != 1) return HPA_ERR_UNSUPPORTED;
+  if (plan_lens) {
+    // in-kernel plan: the dynamic plan for `grid` persistent CTAs, with the
+    // plan kernel's limits and the tile offsets in shared memory
+    if (pro || kind != HPA_PLAN_DYNAMIC) return HPA_ERR_INVALID_ARG;
+    if (batch > kMaxFusedBatch || grid > 65536) return HPA_ERR_UNSUPPORTED;
+    if ((long long)pt_stride * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
+    if ((long long)batch * pt_stride * num_kv_heads > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
+  }
   const int GT = G * q_tokens;
   if (head_dim != 64 && head_dim != 128) return HPA_ERR_UNSUPPORTED;
   if (fp8 && head_dim != 128) return HPA_ERR_UNSUPPORTED;
@@ -1295,6 +1417,8 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.k_cache_w = pro ? static_cast<__nv_bfloat16*>(const_cast<void*>(k_cache)) : nullptr;
   p.v_cache_w = pro ? static_cast<__nv_bfloat16*>(const_cast<void*>(v_cache)) : nullptr;
   p.q_out = pro ? static_cast<__nv_bfloat16*>(pro->q_out) : nullptr;
+  p.seq_lens = plan_lens;
+  p.capacity = pt_stride * kPageSize;
   const int nt = GT > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;
@@ -1302,11 +1426,14 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   const bool f32 = out_dtype == HPA_OUT_F32;
   hpa_status st;
   if (pro)
-    st = f32 ? launch_d<true, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
-             : launch_d<false, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
+    st = f32 ? launch_d<true, true, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
+             : launch_d<false, true, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
+  else if (plan_lens)
+    st = f32 ? launch_d<true, false, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
+             : launch_d<false, false, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
   else
-    st = f32 ? launch_d<true, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
-             : launch_d<false, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
+    st = f32 ? launch_d<true, false, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
+             : launch_d<false, false, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
   if (st != HPA_OK) return st;
 
   // split merge, chained behind the decode kernel
@@ -1357,7 +1484,7 @@ extern "C" hpa_status hpa_decode_run(const void* q, const void* k_cache, const v
                                      size_t ws_bytes, void* stream) {
   return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
                        num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
-                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr, 1);
+                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr, 1, nullptr);
 }
 
 extern "C" hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, const void* v_cache,
@@ -1370,7 +1497,23 @@ extern "C" hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, c
                                            void* workspace, size_t ws_bytes, void* stream) {
   return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
                        num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
-                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr, q_tokens);
+                       softmax_scale, kind, grid, workspace, ws_bytes, stream, nullptr, q_tokens,
+                       nullptr);
+}
+
+extern "C" hpa_status hpa_decode_step(const int32_t* seq_lens, const void* q, const void* k_cache,
+                                      const void* v_cache, const float* k_scale,
+                                      const float* v_scale, hpa_kv_dtype kv_dtype,
+                                      const int32_t* page_table, int pt_stride, int num_pages,
+                                      void* out, hpa_out_dtype out_dtype, int batch, int q_tokens,
+                                      int num_q_heads, int num_kv_heads, int head_dim,
+                                      float softmax_scale, int num_ctas, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  if (!seq_lens) return HPA_ERR_INVALID_ARG;
+  return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
+                       num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
+                       softmax_scale, HPA_PLAN_DYNAMIC, num_ctas, workspace, ws_bytes, stream,
+                       nullptr, q_tokens, seq_lens);
 }
 
 extern "C" hpa_status hpa_decode_run_prologue(
@@ -1382,5 +1525,6 @@ extern "C" hpa_status hpa_decode_run_prologue(
   const hpa::ProArgs pro{k_raw, v_raw, q_gamma, k_gamma, eps, rope_theta, q_out};
   return hpa::run_impl(q_raw, k_cache, v_cache, nullptr, nullptr, HPA_KV_BF16, page_table,
                        pt_stride, num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads,
-                       head_dim, softmax_scale, kind, grid, workspace, ws_bytes, stream, &pro, 1);
+                       head_dim, softmax_scale, kind, grid, workspace, ws_bytes, stream, &pro, 1,
+                       nullptr);
 }

@@ -17,7 +17,7 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
-//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next
+//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next, done
 //   lens        int32[B]     clamped lengths
 //   tile_start  int32[B+1]   exclusive prefix sum of tiles per sequence
 //   cta_desc    int4[2*V]    per range v: (u_begin, u_end, b0, g0), (t0, n0,
@@ -43,6 +43,7 @@ enum HeaderField {
   kHdrBatch = 5, kHdrKvHeads = 6, kHdrGroup = 7, kHdrHeadDim = 8, kHdrTiles = 9,
   kHdrRanges = 10,  // virtual ranges V (grid for static plans)
   kHdrNext = 11,    // dynamic plan: next tail chunk to hand out (run-time counter)
+  kHdrDone = 12,    // in-kernel plan: CTAs of the current step that finished
   kHdrWords = 16
 };
 

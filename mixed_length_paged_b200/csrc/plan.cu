@@ -28,6 +28,7 @@
 #include <atomic>
 
 #include "hpa_common.cuh"
+#include "plan_geom.cuh"
 
 namespace hpa {
 namespace {
@@ -42,85 +43,6 @@ struct PlanParams {
   int kind, num_ctas, grid;
   long long chunk;             // STATIC_CHUNK: tiles per split
   Ws ws;
-};
-
-// Largest b in [0, B) with tile_start[b] * Hkv <= u (u < U).
-__device__ int seq_of_unit(const int32_t* tile_start, int B, int Hkv, long long u) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if ((long long)tile_start[mid] * Hkv <= u) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// floor(a / b) for 0 <= a < 2^50 and a fixed divisor 0 < b < 2^31: the fp64
-// product with a precomputed reciprocal is within one of the quotient, and
-// one integer check each way makes it exact.  (Much cheaper than a 64-bit
-// integer division or an IEEE fp64 division per call.)
-struct FloorDiv {
-  long long b;
-  double inv;
-  __device__ void init(long long d, double reciprocal) {
-    b = d;
-    inv = reciprocal;
-  }
-  __device__ __forceinline__ long long operator()(long long a) const {
-    long long q = (long long)((double)a * inv);
-    if (q * b > a) --q;
-    else if ((q + 1) * b <= a) ++q;
-    return q;
-  }
-};
-
-// Dynamic plan geometry.  P persistent CTAs; U units.  If U <= P each active
-// CTA takes one unit.  Otherwise the first U1 = U - Ut units are spread over
-// the P primary ranges and the last Ut = min(floor(U/8), U - P) units over M =
-// min(4P, Ut) tail chunks, handed out at run time to whichever CTA is free.
-// For n units spread over m ranges as [floor(cn/m), floor((c+1)n/m)), the
-// range holding unit u is the largest c with floor(cn/m) <= u, i.e.
-// floor(((u+1)m - 1) / n).
-struct DynGeom {
-  long long U, P, Pd, U1, Ut, M;
-  FloorDiv by_Pd, by_M, by_U1, by_Ut;
-  __device__ void init(long long units, long long ctas) {
-    U = units;
-    P = ctas;
-    if (U <= P) {
-      Pd = U; U1 = U; Ut = 0; M = 0;
-    } else {
-      Pd = P;
-      Ut = std::min<long long>(U / kTailFractionDiv, U - P);
-      U1 = U - Ut;
-      M = std::min<long long>((long long)kTailChunksPerCta * P, Ut);
-    }
-  }
-  // the divisors whose reciprocals init_div takes, in order
-  __device__ long long divisor(int i) const { return i == 0 ? Pd : i == 1 ? M : i == 2 ? U1 : Ut; }
-  __device__ void init_div(const double* r) {
-    by_Pd.init(Pd, r[0]);
-    by_M.init(M, r[1]);
-    by_U1.init(U1, r[2]);
-    by_Ut.init(Ut, r[3]);
-  }
-  __device__ long long ranges() const { return P + M; }
-  __device__ long long range_of(long long u) const {
-    return u < U1 ? by_U1((u + 1) * Pd - 1) : P + by_Ut((u - U1 + 1) * M - 1);
-  }
-  __device__ void bounds(long long c, long long* ub, long long* ue) const {
-    if (c < P) {
-      if (c < Pd) {
-        *ub = by_Pd(c * U1);
-        *ue = by_Pd((c + 1) * U1);
-      } else {
-        *ub = *ue = U;
-      }
-    } else {
-      const long long j = c - P;
-      *ub = U1 + by_M(j * Ut);
-      *ue = U1 + by_M((j + 1) * Ut);
-    }
-  }
 };
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
@@ -199,56 +121,38 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
   const long long work = V > S ? V : S;
   for (long long c = first; c < work; c += stride) {
     if (c < V) {
-      long long ub, ue;
-      int b0 = 0, g0 = 0, t0 = 0, n0 = 0;
+      int4 d0, d1;
       if (dyn) {
-        dg.bounds(c, &ub, &ue);
-        if (ub < ue) {
-          b0 = seq_of_unit(ts, p.B, p.Hkv, ub);
-          n0 = ts[b0 + 1] - ts[b0];
-          const int rem = (int)(ub - (long long)ts[b0] * p.Hkv);  // < Hkv * n0 < 2^31
-          g0 = rem / n0;
-          t0 = rem - g0 * n0;
-        }
+        dyn_range_desc(dg, ts, p.B, p.Hkv, c, &d0, &d1);
       } else {
         const int s = (int)c / per, i = (int)c % per;
-        b0 = s / p.Hkv;
-        g0 = s % p.Hkv;
+        const int b0 = s / p.Hkv, g0 = s % p.Hkv;
         const long long n = ts[b0 + 1] - ts[b0];
         const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
         const long long c0 = std::min<long long>((long long)i * C, n);
         const long long c1 = std::min<long long>((long long)(i + 1) * C, n);
         const long long seg_start = (long long)ts[b0] * p.Hkv + (long long)g0 * n;
-        ub = seg_start + c0;
-        ue = seg_start + c1;
-        t0 = (int)c0;
-        n0 = (int)n;
+        d0 = make_int4((int)(seg_start + c0), (int)(seg_start + c1), b0, g0);
+        d1 = make_int4((int)c0, (int)n, 0, 0);
       }
-      p.ws.cta_desc[2 * c] = make_int4((int)ub, (int)ue, b0, g0);
-      p.ws.cta_desc[2 * c + 1] = make_int4(t0, n0, 0, 0);
+      p.ws.cta_desc[2 * c] = d0;
+      p.ws.cta_desc[2 * c + 1] = d1;
     }
     if (c < S) {
       const int s = (int)c;
-      const int b = s / p.Hkv, g = s - b * p.Hkv;
-      const long long n = ts[b + 1] - ts[b];
-      int nsplit = 0, slot0 = -1;
-      if (n > 0) {
-        if (dyn) {
-          const long long seg_start = (long long)ts[b] * p.Hkv + (long long)g * n;
-          const long long r0 = dg.range_of(seg_start);
-          nsplit = (int)(dg.range_of(seg_start + n - 1) - r0 + 1);
-          if (nsplit > 1) {
-            long long ub, ue;
-            dg.bounds(r0, &ub, &ue);
-            slot0 = (int)(2 * r0 + (ub == seg_start ? 0 : 1));
-          }
-        } else {
+      if (dyn) {
+        p.ws.seg_desc[s] = dyn_seg_desc(dg, ts, p.Hkv, s);
+      } else {
+        const int b = s / p.Hkv;
+        const long long n = ts[b + 1] - ts[b];
+        int nsplit = 0, slot0 = -1;
+        if (n > 0) {
           const long long C = (p.kind == HPA_PLAN_STATIC_NSPLIT) ? (n + per - 1) / per : p.chunk;
           nsplit = (int)((n + C - 1) / C);
           if (nsplit > 1) slot0 = 2 * s * per;  // chunk 0 starts its segment
         }
+        p.ws.seg_desc[s] = make_int2(slot0, nsplit);
       }
-      p.ws.seg_desc[s] = make_int2(slot0, nsplit);
     }
   }
 
@@ -265,6 +169,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrTiles] = T;
     h[kHdrRanges] = (int32_t)V;
     h[kHdrNext] = 0;
+    h[kHdrDone] = 0;
     // (no fence before the magic word: the run kernel reads the plan only
     // after griddepcontrol.wait, i.e. after this whole grid has completed)
     h[kHdrMagic] = kPlanMagic;

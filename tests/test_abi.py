@@ -252,3 +252,23 @@ def test_num_ctas_environment_override():
                            env={**os.environ, "HPA_NUM_CTAS": val},
                            cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
         assert r.stdout.split() == want.split(), r.stderr
+
+
+def _step_call(L, **kw):
+    a = dict(sl=256, q=256, k=256, v=256, ks=None, vs=None, kvd=0, pt=256, pts=4, pages=8,
+             out=256, outd=0, B=2, T=1, Hq=8, Hkv=2, D=64, scale=0.125, n=148, ws=256,
+             wsb=1 << 24)
+    a.update(kw)
+    return L.hpa_decode_step(a["sl"], a["q"], a["k"], a["v"], a["ks"], a["vs"], a["kvd"], a["pt"],
+                             a["pts"], a["pages"], a["out"], a["outd"], a["B"], a["T"], a["Hq"],
+                             a["Hkv"], a["D"], C.c_float(a["scale"]), a["n"], a["ws"], a["wsb"],
+                             None)
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(sl=None), 1), (dict(q=None), 1), (dict(B=0), 1), (dict(n=0), 1),
+    (dict(B=513), 2),                  # tile offsets of at most 512 sequences in shared memory
+    (dict(n=65537), 2), (dict(T=3, Hq=64, Hkv=8), 2), (dict(wsb=64), 3), (dict(D=96), 2),
+])
+def test_step_rejects_bad_arguments_without_launching(L, bad, expect):
+    assert _step_call(L, **bad) == expect

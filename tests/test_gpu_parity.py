@@ -489,6 +489,132 @@ def bits_t(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
 
 
+# ---------------------------------------------------------------- in-kernel plan (decode_step)
+
+def _plan_and_run(batch, num_ctas, out_dtype=torch.float32, fp8=None):
+    """Reference: hpa_decode_plan + hpa_decode_run(_multi) on a fresh workspace."""
+    q = batch.q
+    T = q.shape[1] if q.dim() == 4 else 1
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
+    Hkv = batch.k_cache.shape[1]
+    ws = torch.zeros(hpa.decode_workspace_size(0, B, Hkv, Hq * T, D, num_ctas), dtype=torch.uint8,
+                     device="cuda")
+    hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq * T, head_dim=D,
+                    pt_stride=batch.pt_stride, workspace=ws, num_ctas=num_ctas)
+    out = torch.full(q.shape, float("nan"), dtype=out_dtype, device="cuda")
+    kw = {}
+    kc, vc = batch.k_cache, batch.v_cache
+    if fp8 is not None:
+        kc, ks, vc, vs = (torch.from_numpy(x).cuda() for x in fp8)
+        kw = dict(k_scale=ks, v_scale=vs)
+    run = hpa.decode_run_multi if q.dim() == 4 else hpa.decode_run
+    run(q, kc, vc, batch.page_table, out, ws, num_ctas, 1 / math.sqrt(D), **kw)
+    return out, ws
+
+
+def _step(batch, num_ctas, ws=None, out_dtype=torch.float32, fp8=None):
+    q = batch.q
+    T = q.shape[1] if q.dim() == 4 else 1
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
+    Hkv = batch.k_cache.shape[1]
+    if ws is None:
+        ws = torch.zeros(hpa.decode_workspace_size(0, B, Hkv, Hq * T, D, num_ctas),
+                         dtype=torch.uint8, device="cuda")
+    out = torch.full(q.shape, float("nan"), dtype=out_dtype, device="cuda")
+    kw = {}
+    kc, vc = batch.k_cache, batch.v_cache
+    if fp8 is not None:
+        kc, ks, vc, vs = (torch.from_numpy(x).cuda() for x in fp8)
+        kw = dict(k_scale=ks, v_scale=vs)
+    hpa.decode_step(batch.seq_lens, q, kc, vc, batch.page_table, out, ws, num_ctas,
+                    1 / math.sqrt(D), **kw)
+    return out, ws
+
+
+STEP_CASES = [
+    # name, lens, Hq, Hkv, D, T, num_ctas
+    ("skewed_small", [8192] + [512] * 15, 64, 8, 128, 1, None),
+    ("few_units", [37, 200], 8, 2, 64, 1, None),          # U <= P: one unit per CTA
+    ("ragged", [0, 1, 63, 64, 65, 700, 3000, 2], 32, 8, 128, 1, 7),
+    ("g16", [129, 2000, 5], 32, 2, 128, 1, None),
+    ("mt2", [65, 300, 2, 4097], 64, 8, 128, 2, None),
+    ("mt4_d64", [130, 64, 1000], 16, 4, 64, 4, 5),
+    ("max_batch", [int(x) for x in np.random.default_rng(7).integers(0, 400, 512)], 8, 2, 64, 1,
+     None),
+]
+
+
+@pytest.mark.parametrize("name,lens,Hq,Hkv,D,T,num_ctas", STEP_CASES)
+def test_step_equals_plan_and_run_bitwise(name, lens, Hq, Hkv, D, T, num_ctas):
+    batch = W.make_batch(W.DecodeShape(name, Hq, Hkv, D, q_tokens=T), lens,
+                         seed=zlib.crc32(name.encode()) % 1000)
+    to_device(batch)
+    n = num_ctas or hpa.default_num_ctas()
+    ref, ws_ref = _plan_and_run(batch, n)
+    got, ws = _step(batch, n)
+    torch.cuda.synchronize()
+    assert hpa.read_status(ws) == 0
+    assert torch.equal(got, ref)
+    # the segment descriptors and the plan fields of the header, as the plan writes them
+    lay = hpa.workspace_layout(0, batch.batch, Hkv, Hq * T, D, n)
+    S = batch.batch * Hkv
+    a, b = ws.cpu().numpy(), ws_ref.cpu().numpy()
+    sd = slice(lay["seg_desc"], lay["seg_desc"] + 8 * S)
+    np.testing.assert_array_equal(a[sd], b[sd])
+    hdr_a = a[lay["header"]:lay["header"] + 64].view(np.int32)
+    hdr_b = b[lay["header"]:lay["header"] + 64].view(np.int32)
+    for f in (0, 2, 3, 4, 5, 6, 7, 8, 9, 10):  # magic, units, grid, kind, shapes, tiles, ranges
+        assert hdr_a[f] == hdr_b[f], f
+    assert hdr_a[11] == 0 and hdr_a[12] == 0  # run-time counters back at zero
+
+
+def test_step_fp8_equals_plan_and_run():
+    shape = W.DecodeShape("st8", 64, 8, 128, kv_dtype="fp8_e4m3")
+    batch = W.make_batch(shape, [1, 63, 64, 65, 700, 3000], seed=44)
+    fp8 = quantize_fp8(batch)
+    to_device(batch)
+    n = hpa.default_num_ctas()
+    ref, _ = _plan_and_run(batch, n, fp8=fp8)
+    got, _ = _step(batch, n, fp8=fp8)
+    assert torch.equal(got, ref)
+
+
+def test_step_repeated_with_changing_lengths_and_mixed_calls():
+    """One workspace through several steps whose lengths change, with plain
+    plan + run calls in between: every step must find the run-time counters
+    at zero."""
+    n = hpa.default_num_ctas()
+    steps = [[5000, 64, 1], [300] * 9, [1, 2, 3], [20000, 7, 4000, 640]]
+    # one buffer for all steps: each call lays the workspace out for its own
+    # batch size; the header (with the counters) sits at offset 0 for all
+    size = max(hpa.decode_workspace_size(0, len(l), 8, 32, 128, n) for l in steps)
+    ws = torch.zeros(size, dtype=torch.uint8, device="cuda")
+    for i, lens in enumerate(steps):
+        batch = W.make_batch(W.DecodeShape("rep", 32, 8, 128), lens, seed=50 + i)
+        to_device(batch)
+        ref, _ = _plan_and_run(batch, n)
+        got, _ = _step(batch, n, ws=ws)
+        assert torch.equal(got, ref), i
+        # a plain dynamic plan + run on the same workspace in between
+        hpa.decode_plan(batch.seq_lens, num_kv_heads=8, num_q_heads=32, head_dim=128,
+                        pt_stride=batch.pt_stride, workspace=ws, num_ctas=n)
+        out = torch.empty_like(ref)
+        hpa.decode_run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, ws, n,
+                       1 / math.sqrt(128))
+        assert torch.equal(out, ref), i
+    torch.cuda.synchronize()
+    assert hpa.read_status(ws) == 0
+
+
+def test_step_flags_clamped_lengths():
+    batch = W.make_batch(W.DecodeShape("clamp", 8, 2, 64), [100, 300], seed=45)
+    batch.seq_lens[1] = 100_000  # past the page table
+    to_device(batch)
+    _, ws = _step(batch, hpa.default_num_ctas())
+    torch.cuda.synchronize()
+    assert hpa.read_status(ws) & hpa.DEVICE_LEN_CLAMPED
+
+
 # ---------------------------------------------------------------- canaries
 
 @pytest.mark.parametrize("kind,num_ctas,T", [(0, None, 1), (0, 5, 1), (1, None, 1),
