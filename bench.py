@@ -43,7 +43,7 @@ L2_BYTES = 126 * 1000 * 1000  # B200 L2 capacity
 WORKLOAD = "skewed"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_run_skewed_ncu.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "mixed_length_paged_b200", "csrc", f)
-                  for f in ("decode.cu", "hpa_common.cuh", "prologue_math.cuh")]
+                  for f in ("decode.cu", "hpa_common.cuh", "plan_geom.cuh", "prologue_math.cuh")]
 
 
 def _args():
