@@ -353,12 +353,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             dec.run(batch.q, batch.k_cache, batch.v_cache, batch.page_table, out, scale,
                     k_scale=k_scale, v_scale=v_scale)
 
-    # The dynamic plan is made inside the decode kernel (hpa_decode_step)
-    # where that applies; the fused prologue still runs after a plan kernel.
-    use_step = not shape.prologue and B <= hpa.MAX_STEP_BATCH
+    # The dynamic plan is made inside the decode kernel (hpa_decode_step /
+    # hpa_decode_step_prologue) where the batch fits its shared memory.
+    use_step = B <= hpa.MAX_STEP_BATCH
 
     def step():
-        if use_step:
+        if use_step and shape.prologue:
+            dec.step_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma,
+                              batch.k_gamma, batch.k_cache, batch.v_cache, batch.page_table,
+                              seq_lens, out, scale, eps=1e-6, rope_theta=10000.0)
+        elif use_step:
             dec.step(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out,
                      scale, k_scale=k_scale, v_scale=v_scale)
         else:
@@ -637,7 +641,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                          "note": "events between the calls (timed region 2); the step time "
                                  "comes from timed region 1 without them"},
         "roofline": {"bound": "hbm",
-                     "kernel": ("hpa_decode_run_prologue (decode_kernel + merge_kernel)"
+                     "kernel": ("hpa_decode_step_prologue (decode_kernel with the prologue and "
+                                "the plan inside + merge_kernel)" if shape.prologue and use_step
+                                else "hpa_decode_run_prologue (decode_kernel + merge_kernel)"
                                 if shape.prologue else
                                 "hpa_decode_step (decode_kernel with the plan inside + "
                                 "merge_kernel)" if use_step else

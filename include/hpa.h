@@ -317,6 +317,27 @@ HPA_API hpa_status hpa_decode_run_prologue(
     hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * hpa_decode_step_prologue -- hpa_decode_step with the prologue of
+ * hpa_decode_run_prologue: a whole decode step -- RMSNorm + RoPE of q and of
+ * the new K row, the new token's K/V cache write, the dynamic tile plan,
+ * attention and the split merge -- in two launches (bitbyai.com "vLLM x
+ * HPC-Ops", Attention Backend: the fused prologue; xiaodao.ai "HPC-Ops TPOT
+ * -48.8%", Attention section: the per-step plan).  Same bits as
+ * hpa_kv_prologue + hpa_decode_plan + hpa_decode_run.
+ *
+ * Arguments as for hpa_decode_run_prologue, with seq_lens (post-append
+ * lengths), num_ctas and the workspace rules of hpa_decode_step (batch <= 512,
+ * workspace zero-filled before its first use).
+ */
+HPA_API hpa_status hpa_decode_step_prologue(
+    const int32_t* seq_lens, const void* q_raw, const void* k_raw, const void* v_raw,
+    const float* q_gamma, const float* k_gamma, float eps, float rope_theta, void* k_cache,
+    void* v_cache, void* q_out, const int32_t* page_table, int pt_stride, int num_pages,
+    void* out, hpa_out_dtype out_dtype, int batch, int num_q_heads, int num_kv_heads,
+    int head_dim, float softmax_scale, int num_ctas, void* workspace, size_t ws_bytes,
+    void* stream);
+
+/*
  * hpa_kv_prologue -- fused RMSNorm + RoPE + KV write for the new token of
  * each sequence (bitbyai.com "vLLM x HPC-Ops", Attention Backend: RoPE,
  * query-key normalisation and KV-write fused into one prologue).
@@ -369,10 +390,12 @@ HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const v
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) and the SM count with that device current; make that
  * first call before any stream capture.  All calls share the array and it
- * keeps the last call's contents; the plan rewrites everything the run reads
- * and zeroes the arrival counters on every call, so stale contents never
- * reach a result, but calls that overlap on the GPU (unordered streams) race
- * on the array.  The device status word of the array is not exposed.
+ * keeps the last call's contents; every call rewrites everything it reads
+ * (up to 512 sequences the plan is made inside the decode kernel, as
+ * hpa_decode_step does; beyond, hpa_decode_plan runs first) and leaves the
+ * run-time counters at zero, so stale contents never reach a result, but
+ * calls that overlap on the GPU (unordered streams) race on the array.  The
+ * device status word of the array is not exposed.
  */
 #define HPA_NOALLOC_SCRATCH_BYTES (16u << 20)
 HPA_API hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -28,7 +28,7 @@ __all__ = [
     "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
     "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run",
-    "decode_step", "MAX_STEP_BATCH", "decode_run_multi",
+    "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
     "decode_run_prologue",
     "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
@@ -90,6 +90,9 @@ def lib():
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
                                      _F, _I, _I, _V, _Z, _V]
+        L.hpa_decode_step_prologue.restype = _I
+        L.hpa_decode_step_prologue.argtypes = [_V, _V, _V, _V, _V, _V, _F, _F, _V, _V, _V, _V, _I,
+                                               _I, _V, _I, _I, _I, _I, _I, _F, _I, _V, _Z, _V]
         L.hpa_decode_step.restype = _I
         L.hpa_decode_step.argtypes = [_V, _V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I,
                                       _I, _I, _F, _I, _V, _Z, _V]
@@ -290,6 +293,44 @@ def decode_step(seq_lens: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     return out
 
 
+def decode_step_prologue(seq_lens: torch.Tensor, q_raw: torch.Tensor, k_raw: torch.Tensor,
+                         v_raw: torch.Tensor, q_gamma: torch.Tensor, k_gamma: torch.Tensor,
+                         k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                         out: torch.Tensor, workspace: torch.Tensor, num_ctas: int,
+                         softmax_scale: float, *, q_out: torch.Tensor | None = None,
+                         eps: float = 1e-6, rope_theta: float = 10000.0,
+                         stream=None) -> torch.Tensor:
+    """A whole decode step -- prologue, dynamic plan, attention, merge -- in two
+    launches (hpa_decode_step_prologue); seq_lens are post-append lengths."""
+    _dev(seq_lens, "seq_lens", (torch.int32,), 1)
+    for t, n, nd in ((q_raw, "q_raw", 3), (k_raw, "k_raw", 3), (v_raw, "v_raw", 3),
+                     (k_cache, "k_cache", 4), (v_cache, "v_cache", 4)):
+        _dev(t, n, (torch.bfloat16,), nd)
+    if q_out is not None:
+        _dev(q_out, "q_out", (torch.bfloat16,), 3)
+    _dev(q_gamma, "q_gamma", (torch.float32,), 1)
+    _dev(k_gamma, "k_gamma", (torch.float32,), 1)
+    _dev(page_table, "page_table", (torch.int32,), 2)
+    _dev(out, "out", (torch.bfloat16, torch.float32), 3)
+    _dev(workspace, "workspace", (torch.uint8,))
+    B, Hq, D = q_raw.shape
+    num_pages, Hkv, S, Dk = k_cache.shape
+    if S != PAGE_SIZE or Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or tuple(out.shape) != tuple(q_raw.shape) or page_table.shape[0] != B \
+            or tuple(k_raw.shape) != (B, Hkv, D) or tuple(v_raw.shape) != (B, Hkv, D) \
+            or seq_lens.shape[0] != B or q_gamma.numel() != D or k_gamma.numel() != D \
+            or (q_out is not None and tuple(q_out.shape) != tuple(q_raw.shape)):
+        raise HpaError("decode_step_prologue: inconsistent shapes")
+    rc = lib().hpa_decode_step_prologue(
+        _ptr(seq_lens), _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(q_gamma), _ptr(k_gamma),
+        float(eps), float(rope_theta), _ptr(k_cache), _ptr(v_cache), _ptr(q_out),
+        _ptr(page_table), page_table.shape[1], num_pages, _ptr(out),
+        OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, Hq, Hkv, D,
+        float(softmax_scale), num_ctas, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "hpa_decode_step_prologue")
+    return out
+
+
 def decode_run_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                      page_table: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
                      grid: int, softmax_scale: float, *, kind: int = PLAN_DYNAMIC,
@@ -479,6 +520,18 @@ class PagedDecoder:
         self.plan(seq_lens, stream=stream)
         return self.run(q, k_cache, v_cache, page_table, out, softmax_scale, k_scale=k_scale,
                         v_scale=v_scale, stream=stream)
+
+    def step_prologue(self, q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache, v_cache, page_table,
+                      seq_lens, out, softmax_scale, stream=None, **kw):
+        """A whole step with the prologue: decode_step_prologue when the plan is
+        dynamic and the batch fits, else plan + run_prologue."""
+        if self.kind == PLAN_DYNAMIC and self.shape[0] <= MAX_STEP_BATCH:
+            return decode_step_prologue(seq_lens, q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache,
+                                        v_cache, page_table, out, self.workspace, self.num_ctas,
+                                        softmax_scale, stream=stream, **kw)
+        self.plan(seq_lens, stream=stream)
+        return self.run_prologue(q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache, v_cache,
+                                 page_table, out, softmax_scale, stream=stream, **kw)
 
     def run_prologue(self, q_raw, k_raw, v_raw, q_gamma, k_gamma, k_cache, v_cache, page_table,
                      out, softmax_scale, **kw):

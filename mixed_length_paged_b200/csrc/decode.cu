@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(kThreads, CPS)
                   const RunParams p) {
   using C = Cfg<D, NT, FP8, CPS, PRO, FP>;
   static_assert(!(PRO && FP8), "the fused prologue writes bf16 caches");
-  static_assert(!(PRO && FP), "the in-kernel plan uses the weights' shared memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -274,12 +273,12 @@ __global__ void __launch_bounds__(kThreads, CPS)
   float* s_kgamma = s_qgamma + D;
   static_assert(C::kMisc / 2 >= 2 * D * 4, "misc area too small for the weights");
   static_assert(C::kStages * 24 + kDepBufs * 16 + 8 + C::kStages * sizeof(StageInfo) +
-                        kDepBufs * sizeof(DepDesc) + 16 <= C::kMisc / 2,
+                        kDepBufs * sizeof(DepDesc) + 16 + 32 <= C::kMisc / 2,
                 "misc area too small");
   // in-kernel plan: tile offsets (after the misc area), and per-warp sums of
-  // the scan (in the weights' half of the misc area, unused without PRO)
+  // the scan (behind q_ready)
   int32_t* s_ts = reinterpret_cast<int32_t*>(misc + C::kMisc);
-  int* s_wsum = reinterpret_cast<int*>(misc + C::kMisc / 2);
+  int* s_wsum = const_cast<int*>(s_flags) + 4;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -1354,7 +1353,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   if (plan_lens) {
     // in-kernel plan: the dynamic plan for `grid` persistent CTAs, with the
     // plan kernel's limits and the tile offsets in shared memory
-    if (pro || kind != HPA_PLAN_DYNAMIC) return HPA_ERR_INVALID_ARG;
+    if (kind != HPA_PLAN_DYNAMIC) return HPA_ERR_INVALID_ARG;
     if (batch > kMaxFusedBatch || grid > 65536) return HPA_ERR_UNSUPPORTED;
     if ((long long)pt_stride * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
     if ((long long)batch * pt_stride * num_kv_heads > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
@@ -1425,7 +1424,10 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool f32 = out_dtype == HPA_OUT_F32;
   hpa_status st;
-  if (pro)
+  if (pro && plan_lens)
+    st = f32 ? launch_d<true, true, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
+             : launch_d<false, true, true>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
+  else if (pro)
     st = f32 ? launch_d<true, true, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s)
              : launch_d<false, true, false>(fp8, head_dim, nt, cps, tk, tv, p, grid, s);
   else if (plan_lens)
@@ -1527,4 +1529,19 @@ extern "C" hpa_status hpa_decode_run_prologue(
                        pt_stride, num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads,
                        head_dim, softmax_scale, kind, grid, workspace, ws_bytes, stream, &pro, 1,
                        nullptr);
+}
+
+extern "C" hpa_status hpa_decode_step_prologue(
+    const int32_t* seq_lens, const void* q_raw, const void* k_raw, const void* v_raw,
+    const float* q_gamma, const float* k_gamma, float eps, float rope_theta, void* k_cache,
+    void* v_cache, void* q_out, const int32_t* page_table, int pt_stride, int num_pages,
+    void* out, hpa_out_dtype out_dtype, int batch, int num_q_heads, int num_kv_heads,
+    int head_dim, float softmax_scale, int num_ctas, void* workspace, size_t ws_bytes,
+    void* stream) {
+  if (!seq_lens) return HPA_ERR_INVALID_ARG;
+  const hpa::ProArgs pro{k_raw, v_raw, q_gamma, k_gamma, eps, rope_theta, q_out};
+  return hpa::run_impl(q_raw, k_cache, v_cache, nullptr, nullptr, HPA_KV_BF16, page_table,
+                       pt_stride, num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads,
+                       head_dim, softmax_scale, HPA_PLAN_DYNAMIC, num_ctas, workspace, ws_bytes,
+                       stream, &pro, 1, seq_lens);
 }

@@ -115,6 +115,14 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
                                                 head_dim, ctas);
   if (need == 0) return HPA_ERR_INVALID_ARG;
   if (need > HPA_NOALLOC_SCRATCH_BYTES) return HPA_ERR_WORKSPACE;
+  // Up to 512 sequences the plan is made inside the decode kernel (the
+  // static array starts zero-filled, and every dynamic run leaves its
+  // run-time counters at zero); larger batches take the plan kernel.
+  if (batch <= 512)
+    return hpa_decode_step(seq_lens, q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table,
+                           pt_stride, num_pages, out, out_dtype, batch, 1, num_q_heads,
+                           num_kv_heads, head_dim, softmax_scale, ctas, scratch,
+                           HPA_NOALLOC_SCRATCH_BYTES, stream);
   int grid = 0;
   st = hpa_decode_plan(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride,
                        HPA_PLAN_DYNAMIC, ctas, 0, 0, scratch, HPA_NOALLOC_SCRATCH_BYTES, &grid,

@@ -272,3 +272,22 @@ def _step_call(L, **kw):
 ])
 def test_step_rejects_bad_arguments_without_launching(L, bad, expect):
     assert _step_call(L, **bad) == expect
+
+
+def test_step_prologue_rejects_bad_arguments_without_launching(L):
+    def call(**kw):
+        a = dict(sl=256, qr=256, kr=256, vr=256, gq=256, gk=256, eps=1e-6, theta=1e4, kc=256,
+                 vc=256, qo=None, pt=256, pts=4, pages=8, out=256, outd=0, B=2, Hq=8, Hkv=2, D=64,
+                 scale=0.125, n=148, ws=256, wsb=1 << 24)
+        a.update(kw)
+        return L.hpa_decode_step_prologue(
+            a["sl"], a["qr"], a["kr"], a["vr"], a["gq"], a["gk"], C.c_float(a["eps"]),
+            C.c_float(a["theta"]), a["kc"], a["vc"], a["qo"], a["pt"], a["pts"], a["pages"],
+            a["out"], a["outd"], a["B"], a["Hq"], a["Hkv"], a["D"], C.c_float(a["scale"]), a["n"],
+            a["ws"], a["wsb"], None)
+    assert call(sl=None) == 1
+    assert call(kr=None) == 1
+    assert call(eps=-1.0) == 1
+    assert call(B=513) == 2
+    assert call(n=65537) == 2
+    assert call(wsb=64) == 3

@@ -460,6 +460,32 @@ def test_fused_prologue_bitwise_equals_separate(D, Hq, Hkv, kind, num_ctas):
     assert torch.equal(bits_t(oa), bits_t(ob))
 
 
+@pytest.mark.parametrize("D,Hq,Hkv,num_ctas", [(128, 32, 8, None), (64, 16, 4, 5),
+                                                (128, 16, 1, None), (128, 32, 2, 7)])
+def test_step_prologue_bitwise_equals_separate(D, Hq, Hkv, num_ctas):
+    """The whole step in two launches (prologue + plan inside the decode
+    kernel) against prologue kernel -> plan kernel -> run: same bits in the
+    output, q_out and both caches."""
+    lens = [0, 63, 64, 127, 1000, 4095, 1]
+    batch = _prologue_case(lens, Hq=Hq, Hkv=Hkv, D=D)
+    to_device(batch)
+    (oa, ka, va, qa), _ = _separate_and_fused(batch, num_ctas=num_ctas)
+    B = batch.batch
+    n = num_ctas or hpa.default_num_ctas()
+    kc, vc = batch.k_cache.clone(), batch.v_cache.clone()
+    q_out = torch.full_like(batch.q_raw, float("nan"))
+    ws = torch.zeros(hpa.decode_workspace_size(0, B, Hkv, Hq, D, n), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    hpa.decode_step_prologue(batch.seq_lens, batch.q_raw, batch.k_raw, batch.v_raw,
+                             batch.q_gamma, batch.k_gamma, kc, vc, batch.page_table, out, ws, n,
+                             1.0 / math.sqrt(D), q_out=q_out, eps=1e-6, rope_theta=1e4)
+    torch.cuda.synchronize()
+    assert hpa.read_status(ws) == 0
+    assert torch.equal(bits_t(out), bits_t(oa)) and torch.equal(bits_t(q_out), bits_t(qa))
+    assert torch.equal(bits_t(kc), bits_t(ka)) and torch.equal(bits_t(vc), bits_t(va))
+
+
 def test_fused_prologue_against_oracle_f32_out_no_q_out():
     lens = [5, 200, 3000, 64]
     batch = _prologue_case(lens, Hq=32, Hkv=8, D=128)
