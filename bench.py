@@ -535,6 +535,51 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         extras["dynamic_speedup_vs_best_static"] = min(
             extras[k]["dynamic_speedup"] for k in ("static_nsplit", "static_chunk"))
 
+    if not args.no_extras and plain and use_step:
+        # The batch spread by page range over R ranks (sharding.page_shard),
+        # the R shares run one after another on this GPU, each a decode step
+        # with log-sum-exps, then the merge of the R states.  The slowest
+        # share is what one of R GPUs would spend on its decode; the all-gather
+        # between the two is not measured (one GPU).  A sleep kernel first
+        # lets the host queue a whole round, so the events time the GPU only;
+        # consecutive shares read different pages, so L2 carries nothing over.
+        from mixed_length_paged_b200 import sharding as SH
+        extras["page_sharded"] = {}
+        for R in (2, 8):
+            parts = []
+            for r in range(R):
+                lr, ptr = SH.page_shard(batch.seq_lens, batch.page_table, R, r)
+                parts.append((hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, num_ctas=num_ctas,
+                                               device=dev),
+                              lr.to(dev), ptr.to(dev),
+                              torch.empty(B, Hq, D, dtype=torch.float32, device=dev),
+                              torch.empty(B, Hq, dtype=torch.float32, device=dev)))
+            o_parts, l_parts = [p[3] for p in parts], [p[4] for p in parts]
+            reps = 20
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(R + 2)]
+                   for _ in range(reps)]
+            for rep in range(reps + 3):
+                torch.cuda._sleep(5_000_000)
+                e = evs[rep - 3] if rep >= 3 else None
+                for r, (sd, lr, ptr, o, l) in enumerate(parts):
+                    if e:
+                        e[r].record(stream)
+                    sd.step(batch.q, batch.k_cache, batch.v_cache, ptr, lr, o, scale, lse=l)
+                if e:
+                    e[R].record(stream)
+                hpa.merge_states(o_parts, l_parts, out)
+                if e:
+                    e[R + 1].record(stream)
+                torch.cuda.synchronize()
+            share = np.array([[e[r].elapsed_time(e[r + 1]) for r in range(R)] for e in evs])
+            merge = np.array([e[R].elapsed_time(e[R + 1]) for e in evs])
+            extras["page_sharded"][str(R)] = {
+                "max_share_step_us": 1e3 * float(np.median(share, axis=0).max()),
+                "mean_share_step_us": 1e3 * float(np.median(share, axis=0).mean()),
+                "merge_states_us": 1e3 * float(np.median(merge)),
+                "all_shares_and_merge_on_one_gpu_us": 1e3 * float(np.median(share.sum(1) + merge)),
+                "method": f"median of {reps} rounds, events between launches"}
+
     # End to end through the public API (eager calls): every step copies its
     # inputs (q, seq_lens, page table) from pinned host memory to the device
     # and its output back, inside the timed region.  As a serving loop would,
@@ -659,6 +704,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "static_splitkv": {k: v for k, v in extras.items()
                            if k.startswith(("static", "dynamic"))} or None,
         "separate_prologue": extras.get("separate_prologue_kernel"),
+        "page_sharded": extras.get("page_sharded"),
         "device_status": status,
     }
     print(json.dumps(line), flush=True)

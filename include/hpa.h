@@ -338,6 +338,65 @@ HPA_API hpa_status hpa_decode_step_prologue(
     void* stream);
 
 /*
+ * hpa_decode_step_lse -- hpa_decode_step that also returns each output row's
+ * log-sum-exp, so that steps run over different parts of the same sequences
+ * (the GPUs of a tensor-parallel group holding different page ranges of every
+ * sequence, openai-hub.com news/688; a shared prefix and a private suffix)
+ * can be combined with hpa_merge_states.  This is the split-KV recombination
+ * of xiaodao.ai "HPC-Ops TPOT -48.8%" (Attention section) carried across
+ * calls.
+ *
+ *   lse          device fp32 [batch][q_tokens][num_q_heads], 4-byte aligned,
+ *                required: lse[b][i][h] = log sum_j exp(softmax_scale *
+ *                q[b][i][h] . k_j) over the keys row (b, i, h) attends, in
+ *                natural-log units; -inf (and a zero output row) where the row
+ *                attends no key (a sequence of length 0).
+ *   the rest     as for hpa_decode_step; `out` holds the normalised rows.
+ * Use HPA_OUT_F32 for `out` when the rows are merged afterwards.
+ */
+HPA_API hpa_status hpa_decode_step_lse(const int32_t* seq_lens, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const float* k_scale, const float* v_scale,
+                                       hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                                       int pt_stride, int num_pages, void* out,
+                                       hpa_out_dtype out_dtype, float* lse, int batch,
+                                       int q_tokens, int num_q_heads, int num_kv_heads,
+                                       int head_dim, float softmax_scale, int num_ctas,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hpa_merge_states -- log-sum-exp merge of attention states computed over
+ * disjoint key sets of the same rows (the recombination step of split-KV
+ * decode, xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section, across calls
+ * or GPUs).  For every row r, with M = max_i lse_i[r] and w_i = exp(lse_i[r]
+ * - M):
+ *
+ *     out[r]     = sum_i (w_i / sum_k w_k) o_i[r]     (folded in index order)
+ *     lse_out[r] = M + log sum_i w_i
+ *
+ * A state with lse = -inf contributes nothing and its o row is not read; a row
+ * whose states are all -inf gets out = 0 and lse_out = -inf.
+ *
+ *   o_parts      HOST array of num_states device pointers, each fp32
+ *                [rows][head_dim], 16-byte aligned (hpa_decode_step_lse with
+ *                HPA_OUT_F32).  A pointer may address a peer GPU's memory
+ *                mapped into the current context: the kernel reads it with
+ *                plain global loads.
+ *   lse_parts    HOST array of num_states device pointers, each fp32 [rows].
+ *   num_states   1 .. 16 (HPA_ERR_UNSUPPORTED beyond).
+ *   rows         >= 0; 0 enqueues nothing.
+ *   head_dim     64 or 128.
+ *   out          device [rows][head_dim], bf16 (8-byte aligned) or fp32
+ *                (16-byte aligned) per out_dtype; may not alias an o part.
+ *   lse_out      optional (NULL: not written) device fp32 [rows].
+ * Launched with programmatic dependent launch on `stream`, so it can start
+ * while the kernel before it drains.
+ */
+HPA_API hpa_status hpa_merge_states(const float* const* o_parts, const float* const* lse_parts,
+                                    int num_states, long long rows, int head_dim, void* out,
+                                    hpa_out_dtype out_dtype, float* lse_out, void* stream);
+
+/*
  * hpa_kv_prologue -- fused RMSNorm + RoPE + KV write for the new token of
  * each sequence (bitbyai.com "vLLM x HPC-Ops", Attention Backend: RoPE,
  * query-key normalisation and KV-write fused into one prologue).

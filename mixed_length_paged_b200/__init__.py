@@ -10,11 +10,13 @@ The functions mirror the C ABI in ``include/hpa.h``:
 
     decode_workspace_size, plan_grid, default_num_ctas, workspace_layout,
     decode_plan, decode_run, decode_step, decode_run_multi, decode_run_prologue, kv_prologue,
-    read_status,
+    merge_states, read_status,
     decode_noalloc
 
 and ``PagedDecoder`` bundles a workspace with plan + run for callers who do
-not want to manage it.
+not want to manage it.  ``mixed_length_paged_b200.sharding`` spreads a batch
+over the ranks of a process group (by kv head, or by page range with a
+log-sum-exp merge of the ranks' states).
 """
 from __future__ import annotations
 
@@ -31,6 +33,7 @@ __all__ = [
     "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
     "decode_run_prologue",
     "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "merge_states", "MAX_MERGE_STATES",
 ]
 
 PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2
@@ -96,6 +99,11 @@ def lib():
         L.hpa_decode_step.restype = _I
         L.hpa_decode_step.argtypes = [_V, _V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I,
                                       _I, _I, _F, _I, _V, _Z, _V]
+        L.hpa_decode_step_lse.restype = _I
+        L.hpa_decode_step_lse.argtypes = [_V, _V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _V, _I,
+                                          _I, _I, _I, _I, _F, _I, _V, _Z, _V]
+        L.hpa_merge_states.restype = _I
+        L.hpa_merge_states.argtypes = [_V, _V, _I, C.c_longlong, _I, _V, _I, _V, _V]
         L.hpa_decode_run_multi.restype = _I
         L.hpa_decode_run_multi.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I,
                                            _I, _I, _I, _F, _I, _I, _V, _Z, _V]
@@ -252,11 +260,13 @@ def decode_step(seq_lens: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                 v_cache: torch.Tensor, page_table: torch.Tensor, out: torch.Tensor,
                 workspace: torch.Tensor, num_ctas: int, softmax_scale: float, *,
                 k_scale: torch.Tensor | None = None, v_scale: torch.Tensor | None = None,
-                stream=None) -> torch.Tensor:
+                lse: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """One decode step with the dynamic plan made inside the decode kernel
     (hpa_decode_step).  q/out are [B][Hq][D], or [B][T][Hq][D] for T query
     tokens per sequence.  The workspace must be zero-filled before its first
-    use (or last written by decode_plan)."""
+    use (or last written by decode_plan).  With ``lse`` (fp32, q's shape
+    without D) each row's log-sum-exp is written too (hpa_decode_step_lse),
+    for merge_states."""
     _dev(seq_lens, "seq_lens", (torch.int32,), 1)
     if q.dim() not in (3, 4):
         raise HpaError("q must be [B][Hq][D] or [B][T][Hq][D]")
@@ -283,13 +293,61 @@ def decode_step(seq_lens: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
             or tuple(out.shape) != tuple(q.shape) or page_table.shape[0] != B \
             or seq_lens.shape[0] != B:
         raise HpaError("decode_step: inconsistent shapes")
+    out_kind = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    kv_kind = KV_FP8_E4M3 if fp8 else KV_BF16
+    if lse is not None:
+        _dev(lse, "lse", (torch.float32,), q.dim() - 1)
+        if tuple(lse.shape) != tuple(q.shape[:-1]):
+            raise HpaError("decode_step: lse must have q's shape without the head dim")
+        rc = lib().hpa_decode_step_lse(_ptr(seq_lens), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(k_scale), _ptr(v_scale), kv_kind, _ptr(page_table),
+                                       page_table.shape[1], num_pages, _ptr(out), out_kind,
+                                       _ptr(lse), B, T, Hq, Hkv, D, float(softmax_scale),
+                                       num_ctas, _ptr(workspace), workspace.numel(),
+                                       _stream(stream))
+        _check(rc, "hpa_decode_step_lse")
+        return out
     rc = lib().hpa_decode_step(_ptr(seq_lens), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                               _ptr(k_scale), _ptr(v_scale), KV_FP8_E4M3 if fp8 else KV_BF16,
-                               _ptr(page_table), page_table.shape[1], num_pages, _ptr(out),
-                               OUT_F32 if out.dtype == torch.float32 else OUT_BF16, B, T, Hq, Hkv,
+                               _ptr(k_scale), _ptr(v_scale), kv_kind, _ptr(page_table),
+                               page_table.shape[1], num_pages, _ptr(out), out_kind, B, T, Hq, Hkv,
                                D, float(softmax_scale), num_ctas, _ptr(workspace),
                                workspace.numel(), _stream(stream))
     _check(rc, "hpa_decode_step")
+    return out
+
+
+MAX_MERGE_STATES = 16  # states hpa_merge_states combines in one call
+
+
+def merge_states(o_parts, lse_parts, out: torch.Tensor, lse_out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """Log-sum-exp merge of attention states over disjoint key sets of the
+    same rows (hpa_merge_states): o_parts are fp32 tensors of out's shape
+    [..., D], lse_parts fp32 tensors of out's shape without D.  A part may
+    live on a peer GPU whose memory this context can address."""
+    o_parts, lse_parts = list(o_parts), list(lse_parts)
+    n = len(o_parts)
+    if n != len(lse_parts) or not 1 <= n <= MAX_MERGE_STATES:
+        raise HpaError(f"merge_states: 1..{MAX_MERGE_STATES} (o, lse) pairs, got {n} and "
+                       f"{len(lse_parts)}")
+    _dev(out, "out", (torch.bfloat16, torch.float32))
+    D = out.shape[-1]
+    rows = out.numel() // D if D else 0
+    for i, (o, l) in enumerate(zip(o_parts, lse_parts)):
+        _dev(o, f"o_parts[{i}]", (torch.float32,), out.dim())
+        _dev(l, f"lse_parts[{i}]", (torch.float32,), out.dim() - 1)
+        if tuple(o.shape) != tuple(out.shape) or tuple(l.shape) != tuple(out.shape[:-1]):
+            raise HpaError("merge_states: part shapes must match out")
+    if lse_out is not None:
+        _dev(lse_out, "lse_out", (torch.float32,), out.dim() - 1)
+        if tuple(lse_out.shape) != tuple(out.shape[:-1]):
+            raise HpaError("merge_states: lse_out must have out's shape without D")
+    o_ptrs = (C.c_void_p * n)(*[o.data_ptr() for o in o_parts])
+    l_ptrs = (C.c_void_p * n)(*[l.data_ptr() for l in lse_parts])
+    rc = lib().hpa_merge_states(o_ptrs, l_ptrs, n, rows, D, _ptr(out),
+                                OUT_F32 if out.dtype == torch.float32 else OUT_BF16,
+                                _ptr(lse_out), _stream(stream))
+    _check(rc, "hpa_merge_states")
     return out
 
 
@@ -509,14 +567,16 @@ class PagedDecoder:
                           stream=stream)
 
     def step(self, q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, *,
-             k_scale=None, v_scale=None, stream=None):
+             k_scale=None, v_scale=None, lse=None, stream=None):
         """plan + run as one decode_step (the dynamic plan made inside the
         decode kernel) when the plan is dynamic and the batch fits, else the
-        two calls."""
+        two calls.  ``lse`` (the rows' log-sum-exp) needs the first form."""
         if self.kind == PLAN_DYNAMIC and self.shape[0] <= MAX_STEP_BATCH:
             return decode_step(seq_lens, q, k_cache, v_cache, page_table, out, self.workspace,
                                self.num_ctas, softmax_scale, k_scale=k_scale, v_scale=v_scale,
-                               stream=stream)
+                               lse=lse, stream=stream)
+        if lse is not None:
+            raise HpaError(f"step: lse needs the dynamic plan and batch <= {MAX_STEP_BATCH}")
         self.plan(seq_lens, stream=stream)
         return self.run(q, k_cache, v_cache, page_table, out, softmax_scale, k_scale=k_scale,
                         v_scale=v_scale, stream=stream)

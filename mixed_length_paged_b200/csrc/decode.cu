@@ -132,6 +132,7 @@ struct RunParams {
   const int32_t* page_table;
   int pt_stride, num_pages;
   void* out;
+  float* lse;               // optional [B][T][Hq] log-sum-exp of each output row (natural log)
   int B, Hq, Hkv, G;
   int T, GT;                // query tokens per sequence; rows per kv head = G * T
   const int32_t* seq_lens;  // in-kernel plan: the step's lengths (else the plan's)
@@ -218,6 +219,14 @@ struct Walk {
     } while (n == 0);
   }
 };
+
+// Natural-log log-sum-exp of a row from its softmax state: M the running
+// max and lam = sum 2^(s_j - M) over the scaled logits s_j = scale * log2(e)
+// * q.k_j, so log sum_j e^(scale q.k_j) = (M + log2 lam) * ln 2.  A row that
+// saw no token (lam = 0) has -inf.
+__device__ __forceinline__ float lse_of(float M, float lam) {
+  return lam > 0.f ? (M + log2f(lam)) * 0.69314718055994531f : -INFINITY;
+}
 
 template <bool OUT_F32>
 __device__ __forceinline__ void store_out(void* out, long long i, float v) {
@@ -555,6 +564,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
       if (len_of(b) != 0) continue;
       const long long n = (long long)p.T * p.Hq * D;
       for (long long i = lane; i < n; i += 32) store_out<OUT_F32>(p.out, (long long)b * n + i, 0.f);
+      if (p.lse)
+        for (int i = lane; i < p.T * p.Hq; i += 32) p.lse[(long long)b * p.T * p.Hq + i] = -INFINITY;
     }
     // After an abort, make sure no copy is still landing in shared memory.
     if (lane == 0 && *s_abort) {
@@ -658,8 +669,9 @@ __global__ void __launch_bounds__(kThreads, CPS)
 #pragma unroll
           for (int v = 0; v < V; ++v) o[v] *= inv;
           const int qi = h / p.G, hh = h - qi * p.G;
-          store_out_vec<OUT_F32, V>(
-              p.out, (((long long)dd.b * p.T + qi) * p.Hq + (long long)dd.g * p.G + hh) * D + d, o);
+          const long long orow = ((long long)dd.b * p.T + qi) * p.Hq + (long long)dd.g * p.G + hh;
+          store_out_vec<OUT_F32, V>(p.out, orow * D + d, o);
+          if (p.lse && lane == 0) p.lse[orow] = lse_of(M, lam);
         } else {
           float* dst = p.ws.part_acc + ((long long)dd.slot * GT + h) * D + d;
           if constexpr (V == 4) *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
@@ -1104,6 +1116,7 @@ __device__ __forceinline__ float4 ld_cg4(const float4* p) {
 struct MergeParams {
   Ws ws;
   void* out;
+  float* lse;                // optional [B][T][Hq] log-sum-exp of each output row
   int S, Hkv, G, Hq, slots;  // slots = 2 * V partial slots in the workspace
   int T, GT;                 // query tokens per sequence; rows per segment = G * T
 };
@@ -1171,8 +1184,9 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
     for (int v = 0; v < kVec; ++v) o[v] *= inv;
     const int b = s / p.Hkv, g = s - b * p.Hkv;
     const int qi = h / p.G, hh = h - qi * p.G;  // row h = query token qi, head hh
-    store_out_vec<OUT_F32, kVec>(
-        p.out, (((long long)b * p.T + qi) * p.Hq + (long long)g * p.G + hh) * D + lane * kVec, o);
+    const long long orow = ((long long)b * p.T + qi) * p.Hq + (long long)g * p.G + hh;
+    store_out_vec<OUT_F32, kVec>(p.out, orow * D + lane * kVec, o);
+    if (p.lse && lane == 0) p.lse[orow] = lse_of(M, lam);
   }
   pdl_trigger();
 }
@@ -1333,7 +1347,8 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
                     int pt_stride, int num_pages, void* out, hpa_out_dtype out_dtype, int batch,
                     int num_q_heads, int num_kv_heads, int head_dim, float softmax_scale,
                     hpa_plan_kind kind, int grid, void* workspace, size_t ws_bytes, void* stream,
-                    const ProArgs* pro, int q_tokens, const int32_t* plan_lens) {
+                    const ProArgs* pro, int q_tokens, const int32_t* plan_lens,
+                    float* lse = nullptr) {
   if (!q || !k_cache || !v_cache || !page_table || !out || !workspace) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || pt_stride <= 0 || num_pages <= 0 ||
       grid <= 0)
@@ -1366,6 +1381,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
     return HPA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 3))
     return HPA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lse) & 3) return HPA_ERR_INVALID_ARG;
   if (pro) {
     if (!pro->k_raw || !pro->v_raw || !pro->q_gamma || !pro->k_gamma) return HPA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(pro->k_raw) | reinterpret_cast<uintptr_t>(pro->v_raw)) & 15)
@@ -1396,6 +1412,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.pt_stride = pt_stride;
   p.num_pages = num_pages;
   p.out = out;
+  p.lse = lse;
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
@@ -1442,6 +1459,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   MergeParams mp;
   mp.ws = p.ws;
   mp.out = out;
+  mp.lse = lse;
   mp.S = batch * num_kv_heads;
   mp.Hkv = num_kv_heads;
   mp.G = G;
@@ -1544,4 +1562,20 @@ extern "C" hpa_status hpa_decode_step_prologue(
                        pt_stride, num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads,
                        head_dim, softmax_scale, HPA_PLAN_DYNAMIC, num_ctas, workspace, ws_bytes,
                        stream, &pro, 1, seq_lens);
+}
+
+extern "C" hpa_status hpa_decode_step_lse(const int32_t* seq_lens, const void* q,
+                                          const void* k_cache, const void* v_cache,
+                                          const float* k_scale, const float* v_scale,
+                                          hpa_kv_dtype kv_dtype, const int32_t* page_table,
+                                          int pt_stride, int num_pages, void* out,
+                                          hpa_out_dtype out_dtype, float* lse, int batch,
+                                          int q_tokens, int num_q_heads, int num_kv_heads,
+                                          int head_dim, float softmax_scale, int num_ctas,
+                                          void* workspace, size_t ws_bytes, void* stream) {
+  if (!seq_lens || !lse) return HPA_ERR_INVALID_ARG;
+  return hpa::run_impl(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
+                       num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
+                       softmax_scale, HPA_PLAN_DYNAMIC, num_ctas, workspace, ws_bytes, stream,
+                       nullptr, q_tokens, seq_lens, lse);
 }

@@ -264,6 +264,45 @@ def lse_merge(acc, m, l) -> np.ndarray:
     return out
 
 
+def attention_state(q, k_cache, v_cache, page_table, num_kv_heads: int, scale: float, b: int,
+                    h: int, t0: int, t1: int, **kw):
+    """(o[D], lse) of row (b, h) over tokens [t0, t1): the normalised output
+    o = sum_j softmax_j v_j and its log-sum-exp lse = log sum_j exp(scale
+    q.k_j), the state a split-KV piece hands to the merge (xiaodao.ai
+    "HPC-Ops TPOT -48.8%", Attention section).  An empty range has the state
+    (0, -inf), which every merge ignores."""
+    D = np.asarray(q).shape[-1]
+    if t1 <= t0:
+        return np.zeros(D), -np.inf
+    acc, m, l = partial(q, k_cache, v_cache, page_table, num_kv_heads, scale, b, h, t0, t1, **kw)
+    return acc / l, m + np.log(l)
+
+
+def merge_states(o, lse):
+    """Log-sum-exp merge of n states (o_i[D], lse_i) of one row, computed over
+    disjoint key sets: with M = max_i lse_i and w_i = exp(lse_i - M), the
+    merged state is (sum_i w_i o_i / sum_i w_i, M + log sum_i w_i), folded in
+    index order; states with lse = -inf contribute nothing, and a row whose
+    states are all -inf merges to (0, -inf)."""
+    o = np.asarray(o, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    n, D = o.shape
+    M = -np.inf
+    for i in range(n):
+        M = max(M, lse[i])
+    if M == -np.inf:
+        return np.zeros(D), -np.inf
+    num = np.zeros(D)
+    den = 0.0
+    for i in range(n):
+        if lse[i] == -np.inf:
+            continue
+        w = np.exp(lse[i] - M)
+        num += w * o[i]
+        den += w
+    return num / den, M + np.log(den)
+
+
 # ---------------------------------------------------------------- planner
 
 PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2

@@ -291,3 +291,43 @@ def test_step_prologue_rejects_bad_arguments_without_launching(L):
     assert call(B=513) == 2
     assert call(n=65537) == 2
     assert call(wsb=64) == 3
+
+
+def test_step_lse_rejects_bad_arguments_without_launching(L):
+    def call(lse=256, **kw):
+        a = dict(sl=256, q=256, k=256, v=256, ks=None, vs=None, kvd=0, pt=256, pts=4, pages=8,
+                 out=256, outd=1, B=2, T=1, Hq=8, Hkv=2, D=64, scale=0.125, n=148, ws=256,
+                 wsb=1 << 24)
+        a.update(kw)
+        return L.hpa_decode_step_lse(a["sl"], a["q"], a["k"], a["v"], a["ks"], a["vs"], a["kvd"],
+                                     a["pt"], a["pts"], a["pages"], a["out"], a["outd"], lse,
+                                     a["B"], a["T"], a["Hq"], a["Hkv"], a["D"],
+                                     C.c_float(a["scale"]), a["n"], a["ws"], a["wsb"], None)
+    assert call(lse=None) == 1          # the log-sum-exps are the point of the call
+    assert call(lse=258) == 1           # fp32, 4-byte aligned
+    assert call(sl=None) == 1
+    assert call(B=513) == 2
+    assert call(D=96) == 2
+    assert call(wsb=64) == 3
+
+
+def test_merge_states_rejects_bad_arguments_without_launching(L):
+    def call(n=2, parts=None, lparts=None, rows=10, D=128, out=256, outd=1, lse_out=None):
+        o = (C.c_void_p * max(n, 1))(*([256] * max(n, 1))) if parts is None else parts
+        l = (C.c_void_p * max(n, 1))(*([512] * max(n, 1))) if lparts is None else lparts
+        return L.hpa_merge_states(o, l, n, rows, D, out, outd, lse_out, None)
+    assert call(n=0) == 1
+    assert call(n=17) == 2                          # at most 16 states per call
+    assert call(D=96) == 2
+    assert call(rows=-1) == 1
+    assert call(outd=7) == 1
+    assert call(out=None) == 1
+    assert call(parts=(C.c_void_p * 2)(256, None)) == 1
+    assert call(parts=(C.c_void_p * 2)(256, 264)) == 1      # o parts 16-byte aligned
+    assert call(lparts=(C.c_void_p * 2)(512, 514)) == 1     # lse parts 4-byte aligned
+    assert call(out=264, outd=1) == 1               # fp32 out: 16-byte aligned
+    assert call(out=260, outd=0) == 1               # bf16 out: 8-byte aligned
+    assert call(lse_out=258) == 1
+    assert L.hpa_merge_states(None, None, 1, 1, 128, 256, 1, None, None) == 1
+    # no rows: nothing to enqueue, so this succeeds without a GPU
+    assert call(rows=0) == 0
