@@ -535,6 +535,52 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         extras["dynamic_speedup_vs_best_static"] = min(
             extras[k]["dynamic_speedup"] for k in ("static_nsplit", "static_chunk"))
 
+    if not args.no_extras and not shape.prologue:
+        # The length-aware plan (cut points moved off segment ends, smallest
+        # end piece m tiles) against the dynamic plan, both as plan kernel +
+        # run, interleaved A/B.
+        blocks, per = 10, max(5, min(40, K // 10))
+        kw = dict(k_scale=k_scale, v_scale=v_scale)
+        dd = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, num_ctas=num_ctas, q_tokens=T,
+                              device=dev)
+
+        def dyn_pr():
+            dd(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale, **kw)
+
+        for _ in range(3):
+            dyn_pr()
+        dyn_timed = graphed(dyn_pr)
+        extras["length_aware"] = {}
+        for m in (2, 4, 8):
+            ld = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride, kind=hpa.PLAN_LENGTH_AWARE,
+                                  param=m, num_ctas=num_ctas, q_tokens=T, device=dev)
+
+            def la_step(ld=ld):
+                ld(batch.q, batch.k_cache, batch.v_cache, batch.page_table, seq_lens, out, scale,
+                   **kw)
+
+            for _ in range(3):
+                la_step()
+            torch.cuda.synchronize()
+            la_timed = graphed(la_step)
+            ab = {"dynamic": 0.0, "length_aware": 0.0}
+            for _ in range(blocks):
+                for which, fn in (("dynamic", dyn_timed), ("length_aware", la_timed)):
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    for _ in range(per):
+                        fn()
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                    ab[which] += a.elapsed_time(b)
+            n = blocks * per
+            extras["length_aware"][f"m{m}"] = {
+                "us_per_step": 1e3 * ab["length_aware"] / n,
+                "dynamic_plan_run_us_same_blocks": 1e3 * ab["dynamic"] / n,
+                "speedup_vs_dynamic": ab["dynamic"] / ab["length_aware"],
+                "method": f"plan kernel + run each, interleaved A/B, {blocks} x {per} steps"}
+
     if not args.no_extras and plain and use_step:
         # The batch spread by page range over R ranks (sharding.page_shard),
         # the R shares run one after another on this GPU, each a decode step
@@ -705,6 +751,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                            if k.startswith(("static", "dynamic"))} or None,
         "separate_prologue": extras.get("separate_prologue_kernel"),
         "page_sharded": extras.get("page_sharded"),
+        "length_aware": extras.get("length_aware"),
         "device_status": status,
     }
     print(json.dumps(line), flush=True)

@@ -80,11 +80,16 @@ typedef enum { HPA_OUT_BF16 = 0, HPA_OUT_F32 = 1 } hpa_out_dtype;
 
 /* Plan kinds.  DYNAMIC is the method; the two STATIC kinds are the static
  * split-KV schedules it is measured against, fed to the same run kernel
- * (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section). */
+ * (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section).  LENGTH_AWARE is
+ * DYNAMIC with the cut points moved so that short sequences stay whole and
+ * long ones are cut into pieces of at least `param` tiles (bitbyai.com "vLLM
+ * x HPC-Ops", Attention Backend: nearly-finished short requests first, long
+ * ones spread over the grid); see hpa_decode_plan. */
 typedef enum {
   HPA_PLAN_DYNAMIC = 0,        /* param unused */
   HPA_PLAN_STATIC_NSPLIT = 1,  /* param = splits per (seq, kv head); 0 = ceil(num_ctas / (B Hkv)) */
-  HPA_PLAN_STATIC_CHUNK = 2    /* param = tiles per split; 0 = ceil(T_max / ceil(num_ctas / Hkv)) */
+  HPA_PLAN_STATIC_CHUNK = 2,   /* param = tiles per split; 0 = ceil(T_max / ceil(num_ctas / Hkv)) */
+  HPA_PLAN_LENGTH_AWARE = 3    /* param = smallest end piece of a cut segment, tiles; 0 = 4 */
 } hpa_plan_kind;
 
 /* Bits of the device status word (hpa_read_status). */
@@ -117,8 +122,8 @@ HPA_API int hpa_default_num_ctas(int device);
  * or if the device cannot be queried. */
 HPA_API int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads, int q_tokens);
 
-/* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC,
- * B * Hkv * S for STATIC_NSPLIT, B * Hkv * ceil(T_max / C) for STATIC_CHUNK
+/* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC and
+ * LENGTH_AWARE, B * Hkv * S for STATIC_NSPLIT, B * Hkv * ceil(T_max / C) for STATIC_CHUNK
  * (T_max = ceil(max_seq_len / 64), S and C the resolved params).  Host only;
  * returns -1 on invalid arguments. */
 HPA_API int hpa_plan_grid(hpa_plan_kind kind, int batch, int num_kv_heads, int num_ctas, int param,
@@ -158,6 +163,17 @@ HPA_API hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_k
  * CTAs that got more HBM bandwidth do more of the tail.  A short sequence
  * lands whole in one range; a long one is spread over many.  The STATIC
  * kinds give one CTA per (segment, split) instead.
+ *
+ * LENGTH_AWARE (m = param, or 4 if 0): the DYNAMIC ranges with every cut point
+ * x moved as follows.  If x falls strictly inside a segment [s0, s1) (the
+ * units of one (sequence, kv head)) and would leave a piece of fewer than m
+ * tiles (x - s0 < m or s1 - x < m), it moves to the nearer end of the segment
+ * (s0 on a tie).  A segment of fewer than 2m tiles is never cut: it runs
+ * whole in one range and finishes without partials or a merge.  A longer one
+ * is spread as under DYNAMIC, but its first and last pieces have at least m
+ * tiles.  Ranges stay contiguous and in order; some may become empty.
+ * m = 1 gives DYNAMIC's ranges exactly.  Same workspace size and run-time
+ * tail as DYNAMIC; hpa_decode_run with kind = LENGTH_AWARE.
  *
  *   seq_lens     device [batch] int32; values are clamped to [0, pt_stride*64]
  *                (HPA_DEVICE_LEN_CLAMPED).  A sequence of length 0 gets a zero
@@ -374,8 +390,9 @@ HPA_API hpa_status hpa_decode_step_lse(const int32_t* seq_lens, const void* q,
  *     out[r]     = sum_i (w_i / sum_k w_k) o_i[r]     (folded in index order)
  *     lse_out[r] = M + log sum_i w_i
  *
- * A state with lse = -inf contributes nothing and its o row is not read; a row
- * whose states are all -inf gets out = 0 and lse_out = -inf.
+ * A state with lse = -inf contributes nothing (its o row is loaded but not
+ * used, so it may hold anything, NaN included); a row whose states are all
+ * -inf gets out = 0 and lse_out = -inf.
  *
  *   o_parts      HOST array of num_states device pointers, each fp32
  *                [rows][head_dim], 16-byte aligned (hpa_decode_step_lse with

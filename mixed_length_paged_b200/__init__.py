@@ -27,7 +27,7 @@ import torch
 
 __all__ = [
     "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
-    "PLAN_STATIC_CHUNK", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
+    "PLAN_STATIC_CHUNK", "PLAN_LENGTH_AWARE", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
     "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run",
     "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
@@ -36,7 +36,7 @@ __all__ = [
     "merge_states", "MAX_MERGE_STATES",
 ]
 
-PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2
+PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK, PLAN_LENGTH_AWARE = 0, 1, 2, 3
 KV_BF16, KV_FP8_E4M3 = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 DEVICE_LEN_CLAMPED, DEVICE_BAD_PAGE, DEVICE_BAD_PLAN = 0x1, 0x2, 0x4

@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
     const int qbytes = p.T * qrow_bytes;
     const int U = FP ? (int)dg.U : p.ws.header[kHdrUnits];
     const int V = FP ? (int)dg.ranges() : p.ws.header[kHdrRanges];
-    const bool dyn = p.kind == HPA_PLAN_DYNAMIC;
+    const bool dyn = plan_is_dynamic(p.kind);  // tail chunks taken at run time
     int it = 0;
     // This CTA's primary range first; under the dynamic plan it then takes
     // tail chunks, reserving the next one (and reading its descriptor) while

@@ -51,13 +51,22 @@ enum HeaderField {
 // hands out up to kTailChunksPerCta * P tail chunks at run time.
 constexpr int kTailChunksPerCta = 4;
 constexpr int kTailFractionDiv = 8;  // the tail holds floor(U / 8) units (fewer if U is small)
+constexpr int kLaDefaultMinPiece = 4;  // LENGTH_AWARE: smallest piece of a cut segment, tiles
+
+#if defined(__CUDACC__)
+#define HPA_HD __host__ __device__
+#else
+#define HPA_HD
+#endif
+
+// DYNAMIC and LENGTH_AWARE: P primary ranges + up to 4P run-time tail chunks
+HPA_HD inline bool plan_is_dynamic(int kind) {
+  return kind == HPA_PLAN_DYNAMIC || kind == HPA_PLAN_LENGTH_AWARE;
+}
 
 // Virtual ranges a plan of this kind and grid can describe.
-#if defined(__CUDACC__)
-__host__ __device__
-#endif
-inline long long plan_ranges_ll(int kind, int grid) {
-  return kind == HPA_PLAN_DYNAMIC ? (long long)grid * (1 + kTailChunksPerCta) : grid;
+HPA_HD inline long long plan_ranges_ll(int kind, int grid) {
+  return plan_is_dynamic(kind) ? (long long)grid * (1 + kTailChunksPerCta) : grid;
 }
 
 struct WsLayout {
@@ -68,7 +77,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline bool ws_layout(int kind, int B, int Hkv, int Hq, int D, int grid, WsLayout* L) {
   if (B <= 0 || Hkv <= 0 || Hq <= 0 || D <= 0 || grid <= 0 || Hq % Hkv) return false;
-  if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK)
+  if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK &&
+      kind != HPA_PLAN_LENGTH_AWARE)
     return false;
   const size_t V = size_t(plan_ranges_ll(kind, grid));
   const size_t G = size_t(Hq / Hkv), S = size_t(B) * Hkv, slots = 2 * V;
@@ -108,7 +118,7 @@ inline long long plan_grid_ll(int kind, int B, int Hkv, int num_ctas, int param,
                               int max_seq_len, long long* chunk_out) {
   if (B <= 0 || Hkv <= 0 || num_ctas <= 0 || param < 0 || max_seq_len < 0) return -1;
   if (chunk_out) *chunk_out = 0;
-  if (kind == HPA_PLAN_DYNAMIC) return num_ctas;
+  if (plan_is_dynamic(kind)) return num_ctas;
   const long long S = (long long)B * Hkv;
   if (kind == HPA_PLAN_STATIC_NSPLIT) {
     long long s = param > 0 ? param : (num_ctas + S - 1) / S;

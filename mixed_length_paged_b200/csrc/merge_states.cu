@@ -17,11 +17,12 @@
 // evaluated as M = max_i lse_i, w_i = exp(lse_i - M), lam = sum_i w_i,
 // o = sum_i (w_i / lam) o_i (folded in index order), L = M + log lam.
 //
-// One warp per row: lane i fetches lse_i, the weights come from two warp
-// reductions, then every lane loads its D/32 elements of all live states at
-// once (a state with lse = -inf is not read) and accumulates them.  The loads
-// are plain (coherent) global loads, neither TMA nor the read-only path, so a
-// state may live in a peer GPU's memory mapped into this context.
+// One warp per row: lane i fetches lse_i while every lane loads its D/32
+// elements of all the states' rows (one round trip to memory); the weights
+// come from two warp reductions, and a state with lse = -inf is left out of
+// the sum (its row may hold anything).  The loads are plain (coherent) global
+// loads, neither TMA nor the read-only path, so a state may live in a peer
+// GPU's memory mapped into this context.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -53,7 +54,21 @@ __global__ void __launch_bounds__(kStateWarps * 32) merge_states_kernel(const St
   const long long stride = (long long)gridDim.x * kStateWarps;
   for (long long r = (long long)blockIdx.x * kStateWarps + (threadIdx.x >> 5); r < p.rows;
        r += stride) {
+    // the states' rows and log-sum-exps are loaded together (one round trip)
     const float li = lane < p.n ? p.lse[lane][r] : -INFINITY;
+    float x[kMaxStates][kVec];
+#pragma unroll
+    for (int i = 0; i < kMaxStates; ++i) {
+      const float* src = p.o[i < p.n ? i : 0] + r * D + lane * kVec;
+      if constexpr (kVec == 4) {
+        const float4 a = i < p.n ? *reinterpret_cast<const float4*>(src)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[i][0] = a.x; x[i][1] = a.y; x[i][2] = a.z; x[i][3] = a.w;
+      } else {
+        const float2 a = i < p.n ? *reinterpret_cast<const float2*>(src) : make_float2(0.f, 0.f);
+        x[i][0] = a.x; x[i][1] = a.y;
+      }
+    }
     float M = li;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
@@ -66,25 +81,10 @@ __global__ void __launch_bounds__(kStateWarps * 32) merge_states_kernel(const St
     for (int v = 0; v < kVec; ++v) o[v] = 0.f;
     if (lam > 0.f) {  // warp-uniform
       const float inv = 1.f / lam;
-      float x[kMaxStates][kVec];
-#pragma unroll
-      for (int i = 0; i < kMaxStates; ++i) {
-        const float wi = __shfl_sync(0xffffffffu, w, i);
-        const float* src = p.o[i < p.n ? i : 0] + r * D + lane * kVec;
-        if constexpr (kVec == 4) {
-          const float4 a = (i < p.n && wi != 0.f) ? *reinterpret_cast<const float4*>(src)
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-          x[i][0] = a.x; x[i][1] = a.y; x[i][2] = a.z; x[i][3] = a.w;
-        } else {
-          const float2 a = (i < p.n && wi != 0.f) ? *reinterpret_cast<const float2*>(src)
-                                                   : make_float2(0.f, 0.f);
-          x[i][0] = a.x; x[i][1] = a.y;
-        }
-      }
 #pragma unroll
       for (int i = 0; i < kMaxStates; ++i) {
         const float wi = __shfl_sync(0xffffffffu, w, i) * inv;
-        if (i < p.n && wi != 0.f) {
+        if (i < p.n && wi != 0.f) {  // an empty state's row is never used
 #pragma unroll
           for (int v = 0; v < kVec; ++v) o[v] = fmaf(wi, x[i][v], o[v]);
         }

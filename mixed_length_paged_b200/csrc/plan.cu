@@ -24,6 +24,11 @@
 // tail evens that out.  The partition itself is fixed by the plan, so the
 // split partials and their merge order -- and hence the result -- do not
 // depend on which CTA ends up running a chunk.
+//
+// The length-aware plan (HPA_PLAN_LENGTH_AWARE) is the same partition with
+// its cut points moved to segment ends wherever they would leave a piece of
+// fewer than m tiles (plan_geom.cuh, LaGeom): short sequences run whole in
+// one range, long ones are spread in pieces of at least m tiles.
 #include <algorithm>
 #include <atomic>
 
@@ -41,7 +46,7 @@ struct PlanParams {
   const int32_t* seq_lens;
   int B, Hkv, G, D, capacity;  // capacity = pt_stride * 64 tokens
   int kind, num_ctas, grid;
-  long long chunk;             // STATIC_CHUNK: tiles per split
+  long long chunk;             // STATIC_CHUNK: tiles per split; LENGTH_AWARE: smallest piece
   Ws ws;
 };
 
@@ -95,10 +100,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
 
   const long long U = (long long)T * p.Hkv;
   const int S = p.B * p.Hkv;
-  const bool dyn = p.kind == HPA_PLAN_DYNAMIC;
+  const bool dyn = plan_is_dynamic(p.kind);
+  const bool la = p.kind == HPA_PLAN_LENGTH_AWARE;
   const int per = dyn ? 0 : p.grid / S;  // static: CTAs per segment
   DynGeom dg;
   dg.init(U, p.num_ctas);
+  const LaGeom lg{&dg, ts, p.B, p.Hkv, la ? p.chunk : 1};
   if (tid < 4) {
     const long long d = dg.divisor(tid);
     s_recip[tid] = d > 0 ? 1.0 / (double)d : 0.0;
@@ -122,7 +129,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
   for (long long c = first; c < work; c += stride) {
     if (c < V) {
       int4 d0, d1;
-      if (dyn) {
+      if (la) {
+        la_range_desc(lg, c, &d0, &d1);
+      } else if (dyn) {
         dyn_range_desc(dg, ts, p.B, p.Hkv, c, &d0, &d1);
       } else {
         const int s = (int)c / per, i = (int)c % per;
@@ -140,7 +149,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     }
     if (c < S) {
       const int s = (int)c;
-      if (dyn) {
+      if (la) {
+        p.ws.seg_desc[s] = la_seg_desc(lg, s);
+      } else if (dyn) {
         p.ws.seg_desc[s] = dyn_seg_desc(dg, ts, p.Hkv, s);
       } else {
         const int b = s / p.Hkv;
@@ -199,15 +210,18 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
       param < 0 || max_seq_len < 0)
     return HPA_ERR_INVALID_ARG;
   if (num_q_heads % num_kv_heads) return HPA_ERR_INVALID_ARG;
-  if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK)
+  if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK &&
+      kind != HPA_PLAN_LENGTH_AWARE)
     return HPA_ERR_INVALID_ARG;
   if ((long long)pt_stride * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
   if (batch > kMaxPlanBatch) return HPA_ERR_UNSUPPORTED;
   // the dynamic plan's range arithmetic keeps products below 2^50
-  if (kind == HPA_PLAN_DYNAMIC && num_ctas > 65536) return HPA_ERR_UNSUPPORTED;
+  if (plan_is_dynamic(kind) && num_ctas > 65536) return HPA_ERR_UNSUPPORTED;
+  if (kind == HPA_PLAN_LENGTH_AWARE && param > (1 << 20)) return HPA_ERR_UNSUPPORTED;
   long long chunk = 0;
   const long long grid =
       plan_grid_ll(kind, batch, num_kv_heads, num_ctas, param, max_seq_len, &chunk);
+  if (kind == HPA_PLAN_LENGTH_AWARE) chunk = param > 0 ? param : kLaDefaultMinPiece;
   if (grid < 1 || grid > (1LL << 30)) return HPA_ERR_UNSUPPORTED;
   // Units are indexed with int32 in the plan: bound the worst case.
   if ((long long)batch * pt_stride * num_kv_heads > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;

@@ -135,4 +135,93 @@ __device__ __forceinline__ int2 dyn_seg_desc(const DynGeom& dg, const int32_t* t
   return make_int2(slot0, nsplit);
 }
 
+// LENGTH_AWARE plan geometry (bitbyai.com "vLLM x HPC-Ops", Attention
+// Backend: short requests are finished first, long ones spread over the
+// grid): the dynamic partition with every cut point x moved by snap().  If x
+// lies strictly inside a segment [s0, s0 + n), a = x - s0: when a < m or
+// n - a < m it moves to the nearer end of the segment (s0 on a tie), else it
+// stays.  A segment of fewer than 2m tiles stays whole, and the first and
+// last pieces of a cut segment have at least m tiles.  snap() is
+// non-decreasing in x and moves a cut by less than m, so the ranges stay
+// contiguous and in order, and the range holding unit u is found among the
+// dynamic ranges within m - 1 units of u.
+struct LaGeom {
+  const DynGeom* dg;
+  const int32_t* ts;
+  int B, Hkv;
+  long long m;
+
+  __device__ long long snap(long long x) const {
+    if (m <= 1 || x <= 0 || x >= dg->U) return x;
+    const int b = seq_of_unit(ts, B, Hkv, x);
+    const long long n = ts[b + 1] - ts[b];
+    const long long base = (long long)ts[b] * Hkv;
+    const long long a = (x - base) % n;  // tiles of x's segment before x
+    if (a == 0) return x;
+    const long long r = n - a;
+    if (a < m || r < m) return a <= r ? x - a : x + r;
+    return x;
+  }
+  // first unit of range c (c = V: U), before and after the move
+  __device__ long long raw_start(long long c) const {
+    if (c >= dg->ranges()) return dg->U;
+    long long ub, ue;
+    dg->bounds(c, &ub, &ue);
+    return ub;
+  }
+  __device__ void bounds(long long c, long long* ub, long long* ue) const {
+    long long a, e;
+    dg->bounds(c, &a, &e);
+    *ub = snap(a);
+    *ue = snap(e);
+  }
+  // the last range whose moved start is <= u (for u < U: the range holding u)
+  __device__ long long range_of(long long u) const {
+    long long lo = dg->range_of(u - (m - 1) > 0 ? u - (m - 1) : 0);
+    long long hi = dg->range_of(u + (m - 1) < dg->U - 1 ? u + (m - 1) : dg->U - 1);
+    while (lo < hi) {
+      const long long mid = (lo + hi + 1) >> 1;
+      if (snap(raw_start(mid)) <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+};
+
+// Range descriptor (as dyn_range_desc) of range c of the length-aware plan.
+__device__ __forceinline__ void la_range_desc(const LaGeom& lg, long long c, int4* d0, int4* d1) {
+  long long ub, ue;
+  int b0 = 0, g0 = 0, t0 = 0, n0 = 0;
+  lg.bounds(c, &ub, &ue);
+  if (ub < ue) {
+    b0 = seq_of_unit(lg.ts, lg.B, lg.Hkv, ub);
+    n0 = lg.ts[b0 + 1] - lg.ts[b0];
+    const int rem = (int)(ub - (long long)lg.ts[b0] * lg.Hkv);
+    g0 = rem / n0;
+    t0 = rem - g0 * n0;
+  }
+  *d0 = make_int4((int)ub, (int)ue, b0, g0);
+  *d1 = make_int4(t0, n0, 0, 0);
+}
+
+// Segment descriptor (as dyn_seg_desc) of segment s of the length-aware plan.
+// The ranges holding a segment are consecutive, as the merge's slot order
+// needs: the cuts inside a segment did not move, so they are distinct, and
+// only a segment's ends can collect several cuts (empty ranges).
+__device__ __forceinline__ int2 la_seg_desc(const LaGeom& lg, int s) {
+  const int b = s / lg.Hkv, g = s - b * lg.Hkv;
+  const long long n = lg.ts[b + 1] - lg.ts[b];
+  int nsplit = 0, slot0 = -1;
+  if (n > 0) {
+    const long long seg_start = (long long)lg.ts[b] * lg.Hkv + (long long)g * n;
+    const long long r0 = lg.range_of(seg_start);
+    nsplit = (int)(lg.range_of(seg_start + n - 1) - r0 + 1);
+    if (nsplit > 1) {
+      long long ub, ue;
+      lg.bounds(r0, &ub, &ue);
+      slot0 = (int)(2 * r0 + (ub == seg_start ? 0 : 1));
+    }
+  }
+  return make_int2(slot0, nsplit);
+}
+
 }  // namespace hpa

@@ -305,7 +305,7 @@ def merge_states(o, lse):
 
 # ---------------------------------------------------------------- planner
 
-PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK = 0, 1, 2
+PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK, PLAN_LENGTH_AWARE = 0, 1, 2, 3
 
 
 def plan_grid(kind, batch, num_kv_heads, num_ctas, param=0, max_seq_len=0, page_size=64) -> int:

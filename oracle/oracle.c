@@ -436,6 +436,11 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  *     NC = ceil(T_max / C) chunks reserved for every segment, as if every
  *     sequence were the longest; chunk i = [i C, min((i+1) C, n)), empty past
  *     the segment's end.  Grid = B * Hkv * NC.
+ *   kind 3, length-aware with smallest piece m tiles (param, default 4): the
+ *     ranges of kind 0 with every range end moved by snap_cut, so that a
+ *     segment of fewer than 2m tiles is never cut and the first and last
+ *     pieces of a cut segment have at least m tiles (cuts further inside
+ *     stay, so the ranges holding a segment remain consecutive).  Grid = P.
  *
  * For each range the plan records (u_begin, u_end).  A segment whose units
  * lie in more than one range is computed in pieces, one per range, each
@@ -452,7 +457,7 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  */
 long oracle_plan_grid(int kind, int B, int Hkv, int num_ctas, int param, int max_seq_len,
                       int page_size) {
-  if (kind == 0) return num_ctas;
+  if (kind == 0 || kind == 3) return num_ctas;
   if (kind == 1) {
     long S = param > 0 ? param : (num_ctas + (long)B * Hkv - 1) / ((long)B * Hkv);
     if (S < 1) S = 1;
@@ -467,12 +472,29 @@ long oracle_plan_grid(int kind, int B, int Hkv, int num_ctas, int param, int max
   return (long)B * Hkv * NC;
 }
 
+/* Length-aware plan (bitbyai.com "vLLM x HPC-Ops", Attention Backend: short
+ * requests finish first, long ones are spread over the grid): the cut point
+ * x between units x-1 and x.  If x lies strictly inside a segment of n tiles,
+ * a = tiles of the segment before x, r = n - a after it.  When a < m or
+ * r < m the cut moves to the segment's start (a <= r) or end (a > r);
+ * otherwise it stays. */
+static long snap_cut(long x, long U, long m, const int32_t* unit_seg, const int32_t* unit_tile,
+                     const long* ntile, int Hkv) {
+  if (x <= 0 || x >= U) return x;
+  long a = unit_tile[x];
+  if (a == 0) return x; /* already between two segments */
+  long n = ntile[unit_seg[x] / Hkv];
+  long r = n - a;
+  if (a < m || r < m) return a <= r ? x - a : x + r;
+  return x;
+}
+
 int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capacity_tokens,
                 int kind, int num_ctas, int param, int max_seq_len, int32_t* lens_out,
                 int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][2] */,
                 int32_t* split_count /* [B*Hkv] */, int32_t* first_slot /* [B*Hkv] */,
                 int32_t* n_units_out, int32_t* n_ranges_out) {
-  if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 2)
+  if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 3)
     return ORC_BAD_ARG;
   long grid = oracle_plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len, page_size);
   int S = B * Hkv;
@@ -507,7 +529,7 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
   long nranges = grid;
   long* beg = malloc(sizeof(long) * grid * 5);
   long* end = malloc(sizeof(long) * grid * 5);
-  if (kind == 0) {
+  if (kind == 0 || kind == 3) {
     long P = num_ctas;
     if (U <= P) {
       for (long c = 0; c < P; ++c) {
@@ -549,6 +571,17 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
         beg[c] = seg_first_unit[s] + t0;
         end[c] = seg_first_unit[s] + t1;
       }
+    }
+  }
+  /* 3b. length-aware kind: move every cut point that would leave a piece of
+   *     fewer than m tiles to the nearer end of its segment (the start on a
+   *     tie).  Every range end is the next range's start, so moving both ends
+   *     of every range by the same rule keeps the ranges contiguous. */
+  if (kind == 3) {
+    long m = param > 0 ? param : 4;
+    for (long c = 0; c < nranges; ++c) {
+      beg[c] = snap_cut(beg[c], U, m, unit_seg, unit_tile, ntile, Hkv);
+      end[c] = snap_cut(end[c], U, m, unit_seg, unit_tile, ntile, Hkv);
     }
   }
   /* 4. walk each range's units: list its segments in order, count the

@@ -105,10 +105,12 @@ def _plan(L, **kw):
 @pytest.mark.parametrize("bad,expect", [
     (dict(seq_lens=None), 1), (dict(workspace=None), 1), (dict(batch=0), 1),
     (dict(num_kv_heads=0), 1), (dict(num_q_heads=7), 1), (dict(pt_stride=0), 1),
-    (dict(num_ctas=0), 1), (dict(kind=3), 1), (dict(param=-1), 1), (dict(ws_bytes=16), 3),
+    (dict(num_ctas=0), 1), (dict(kind=4), 1), (dict(param=-1), 1), (dict(ws_bytes=16), 3),
     (dict(workspace=256 + 8), 3),
     (dict(batch=32769), 2),  # more sequences than one plan holds
     (dict(num_ctas=65537), 2),  # dynamic plans over at most 65536 CTAs
+    (dict(kind=3, num_ctas=65537), 2),
+    (dict(kind=3, param=(1 << 20) + 1), 2),  # smallest end piece at most 2^20 tiles
 ])
 def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
     rc, grid = _plan(L, **bad)

@@ -69,7 +69,8 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
     ([int(x) for x in np.random.default_rng(3).integers(0, 300, 20000)], 2, 148),
     ([int(x) for x in np.random.default_rng(4).integers(1, 100, 32768)], 1, 148),  # the maximum
 ])
-@pytest.mark.parametrize("kind,param", [(0, 0), (1, 0), (1, 3), (2, 0), (2, 5)])
+@pytest.mark.parametrize("kind,param", [(0, 0), (1, 0), (1, 3), (2, 0), (2, 5), (3, 0), (3, 2),
+                                        (3, 9)])
 def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
     B, Hq, D = len(lens), Hkv * 2, 64
     cap = max(64, max(lens))
@@ -209,7 +210,8 @@ def test_split_schedules_agree(lens):
     to_device(batch)
     U = sum((L + 63) // 64 for L in lens) * 8
     plans = [(0, None, 0), (0, 1, 0), (0, U, 0), (0, 37, 0), (1, None, 0), (1, None, 3),
-             (2, None, 0), (2, None, 1), (2, None, 7)]
+             (2, None, 0), (2, None, 1), (2, None, 7), (3, None, 0), (3, 37, 2), (3, None, 16),
+             (3, U, 3)]
     outs = []
     for kind, nc, param in plans:
         o = gpu_decode(batch, kind=kind, num_ctas=nc, param=param, out_dtype=torch.float32)
@@ -218,6 +220,30 @@ def test_split_schedules_agree(lens):
         outs.append(o)
     for o in outs[1:]:
         assert (o - outs[0]).abs().max().item() <= SCHED_TOL
+
+
+def test_length_aware_plan_with_unit_pieces_is_the_dynamic_plan():
+    # smallest piece 1 tile: no cut moves, so the same ranges, partials and bits
+    batch = W.make_batch(W.DecodeShape("la1", 64, 8, 128), [9000, 64, 1, 700, 2047, 0], seed=11)
+    to_device(batch)
+    a = gpu_decode(batch, kind=hpa.PLAN_DYNAMIC, out_dtype=torch.float32)
+    b = gpu_decode(batch, kind=hpa.PLAN_LENGTH_AWARE, param=1, out_dtype=torch.float32)
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name,lens", [
+    ("uniform_small", [512] * 64),
+    ("mixed", [1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7]),
+])
+@pytest.mark.parametrize("param", [0, 3])
+def test_length_aware_plan_matches_oracle(name, lens, param):
+    batch = W.make_batch(W.DecodeShape(name, 64, 8, 128), lens, seed=12)
+    ref = oracle_decode(batch)
+    to_device(batch)
+    out = gpu_decode(batch, kind=hpa.PLAN_LENGTH_AWARE, param=param)
+    _check(out, ref)
+    ws = gpu_decode(batch, kind=hpa.PLAN_LENGTH_AWARE, param=param, return_ws=True)[1]
+    assert hpa.read_status(ws) == 0
 
 
 # ---------------------------------------------------------------- named workloads

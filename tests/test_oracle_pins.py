@@ -527,6 +527,82 @@ def test_planner_invariants(lens, Hkv, P, kind):
     _check_plan_invariants(p, lens, Hkv, kind)
 
 
+@pytest.mark.parametrize("lens,Hkv,P", [
+    ([131072] + [4096] * 31, 8, 148),
+    ([512] * 64, 8, 148),
+    ([37, 200], 2, 148),
+    ([37, 200], 2, 3),
+    ([0, 5, 0, 64, 65], 4, 7),
+    ([1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7], 8, 296),
+    ([0, 0], 2, 5),
+])
+@pytest.mark.parametrize("m", [1, 2, 4, 9])
+def test_length_aware_planner(lens, Hkv, P, m):
+    """The length-aware plan: every cut point of the dynamic plan that would
+    leave a piece of fewer than m tiles at a segment's end moves to that end."""
+    sl = np.array(lens, dtype=np.int32)
+    cap = max(64, max(lens))
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap)
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap)
+    _check_plan_invariants(la, lens, Hkv, 3)
+    assert la["grid"] == P and la["ranges"] == dyn["ranges"]
+    units = _units(lens, Hkv)
+    seg_n = {}
+    for (b, g, t) in units:
+        seg_n[(b, g)] = seg_n.get((b, g), 0) + 1
+    # pieces of every segment, from the ranges
+    pieces = {}
+    for c in range(la["ranges"]):
+        a, e = int(la["cta"][c, 0]), int(la["cta"][c, 1])
+        for u in range(a, e):
+            key = units[u][:2]
+            if u == a or units[u - 1][:2] != key:
+                pieces.setdefault(key, []).append(0)
+            pieces[key][-1] += 1
+    for key, ps in pieces.items():
+        assert sum(ps) == seg_n[key]
+        if len(ps) > 1:
+            assert ps[0] >= m and ps[-1] >= m, (key, ps)   # no end piece below m tiles
+        if seg_n[key] < 2 * m:
+            assert len(ps) == 1, (key, ps)            # short segments stay whole
+    # every cut moved by less than m, and only where a piece would be short
+    for c in range(la["ranges"]):
+        for j in (0, 1):
+            x, xd = int(la["cta"][c, j]), int(dyn["cta"][c, j])
+            assert abs(x - xd) < m
+            if 0 < xd < len(units) and units[xd][2] > 0:
+                t, n = units[xd][2], seg_n[units[xd][:2]]
+                if t >= m and n - t >= m:
+                    assert x == xd
+                else:
+                    assert x in (xd - t, xd + n - t)   # an end of the segment
+    if m == 1:
+        for k in ("cta", "split_count", "first_slot"):
+            np.testing.assert_array_equal(la[k], dyn[k])
+
+
+def test_length_aware_planner_hand_cases():
+    # 2 tiles, 1 kv head, 2 CTAs: the dynamic plan gives each CTA one tile;
+    # with m = 2 the cut after tile 1 leaves 1 tile on each side (a tie) and
+    # moves to the segment's start, so the second range holds the whole segment
+    p = oracle.plan(np.array([128], dtype=np.int32), 1, kind=3, num_ctas=2, param=2,
+                    capacity_tokens=128)
+    np.testing.assert_array_equal(p["cta"], [[0, 0], [0, 2]])
+    assert p["split_count"][0] == 1 and p["first_slot"][0] == -1
+    # 3 tiles, 3 CTAs, m = 2: the cut after tile 1 (a=1, r=2) moves to the
+    # start, the cut after tile 2 (a=2, r=1) to the end: one whole range
+    p = oracle.plan(np.array([192], dtype=np.int32), 1, kind=3, num_ctas=3, param=2,
+                    capacity_tokens=192)
+    np.testing.assert_array_equal(p["cta"], [[0, 0], [0, 3], [3, 3]])
+    # 8 tiles, 2 CTAs: the dynamic plan has primary ranges [0, 3), [3, 7) and
+    # one tail chunk [7, 8).  m = 2 keeps the cut at 3 (a=3, r=5) and moves
+    # the one at 7 (r=1) to the end; m = 4 also moves the cut at 3 (a=3 < 4)
+    for m, want in ((2, [[0, 3], [3, 8], [8, 8]]), (4, [[0, 0], [0, 8], [8, 8]])):
+        p = oracle.plan(np.array([512], dtype=np.int32), 1, kind=3, num_ctas=2, param=m,
+                        capacity_tokens=512)
+        np.testing.assert_array_equal(p["cta"], want)
+
+
 def test_planner_static_shapes():
     lens = [131072] + [4096] * 31
     pA = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=1, num_ctas=148, max_seq_len=131072,
