@@ -244,3 +244,31 @@ def test_page_sharded_decoder_single_rank_is_the_plain_step():
              D ** -0.5)
     torch.cuda.synchronize()
     assert torch.equal(out, plain)
+
+
+def test_page_sharded_skewed_workload_full_size():
+    # the benchmark's skewed batch (1 x 131072 + 31 x 4096 tokens) over 8 page
+    # shares: every row against the unsharded step, sampled rows against the
+    # oracle (the 128K-token sequence among them)
+    from tests.helpers import compact_rows
+    batch = W.build("skewed", device="cuda")
+    whole, whole_lse = _step(batch)
+    R = 8
+    o_parts, l_parts = [], []
+    for r in range(R):
+        lr, ptr = SH.page_shard(batch.seq_lens, batch.page_table, R, r)
+        o, l = _step(batch, seq_lens=lr.cuda(), page_table=ptr.cuda())
+        o_parts.append(o)
+        l_parts.append(l)
+    out = torch.empty(whole.shape, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.empty_like(whole)
+    lse = torch.empty_like(whole_lse)
+    hpa.merge_states(o_parts, l_parts, out32, lse)
+    hpa.merge_states(o_parts, l_parts, out)
+    torch.cuda.synchronize()
+    assert (out32 - whole).abs().max().item() <= SCHED_TOL
+    assert (lse - whole_lse).abs().max().item() <= LSE_TOL
+    rows = [0, 1, 17, 31]
+    ref = oracle_decode(compact_rows(batch, rows))
+    mx, mn = errors(out[rows], ref)
+    assert mx <= MAX_ABS and mn <= MEAN_ABS, (mx, mn)
