@@ -382,7 +382,8 @@ MT_LENS = [65, 200, 2, 0, 1000, 64, 4097, 130]
 
 @pytest.mark.parametrize("Hq,Hkv,D,T", [(64, 8, 128, 2), (32, 8, 128, 4), (8, 4, 64, 8),
                                         (4, 4, 128, 16), (16, 2, 64, 2), (12, 4, 128, 5)])
-@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7)])
+@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7), (3, None),
+                                            (3, 5)])
 def test_multi_token_decode_matches_oracle(Hq, Hkv, D, T, kind, num_ctas):
     batch = W.make_batch(W.DecodeShape("mt", Hq, Hkv, D, q_tokens=T), MT_LENS, seed=31)
     ref = oracle.paged_decode_multi(bits16(batch.q), bits16(batch.k_cache),
@@ -409,6 +410,17 @@ def test_multi_token_fp8_and_bf16_out():
                                     k_scale=ks, v_scale=vs)
     out = gpu_decode_multi(batch, fp8=fp8)
     _check(out, ref, max_abs=FP8_MAX_ABS)
+
+
+def test_length_aware_plan_fp8():
+    shape = W.DecodeShape("la8", 64, 8, 128, kv_dtype="fp8_e4m3")
+    batch = W.make_batch(shape, [1, 63, 64, 65, 700, 3000, 511, 512, 513], seed=34)
+    fp8 = quantize_fp8(batch)
+    ref = oracle_decode(batch, fp8=fp8)
+    to_device(batch)
+    for param, nc in ((0, None), (3, 7)):
+        out = gpu_decode(batch, kind=hpa.PLAN_LENGTH_AWARE, param=param, num_ctas=nc, fp8=fp8)
+        _check(out, ref, max_abs=FP8_MAX_ABS, mean_abs=MEAN_ABS)
 
 
 def test_multi_token_one_token_equals_single_token_run():
@@ -473,7 +485,7 @@ def _separate_and_fused(batch, *, kind=0, num_ctas=None, param=0, out_dtype=torc
 
 
 @pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 16, 4), (128, 16, 1), (128, 32, 2)])
-@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7)])
+@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 5), (1, None), (2, 7), (3, 7)])
 def test_fused_prologue_bitwise_equals_separate(D, Hq, Hkv, kind, num_ctas):
     # pre-append lengths: a first token, page edges, several pages, one long
     lens = [0, 63, 64, 127, 1000, 4095, 1]
