@@ -83,6 +83,7 @@ WORKLOAD_DESC = {
                     "prologue in every step",
     "fp8": "FP8 KV: 256 sequences, lengths geometric (mean 2048, cap 16384), 64 q heads, "
            "8 kv heads, head_dim 128, e4m3 K/V with fp32 per-(page, kv head) scales",
+    "fp8_quarter": "the first 64 sequences of the FP8 batch (profiler captures)",
     "skewed_mtp2": "multi-token decode on the skewed batch: 2 query tokens per sequence "
                    "(causal among themselves), 64 q heads, 8 kv heads, head_dim 128, bf16",
 }
