@@ -635,33 +635,40 @@ __global__ void __launch_bounds__(kThreads, CPS)
       const float* dacc = reinterpret_cast<const float*>(deps + db * C::kDepBytes);
       const float2* dml = reinterpret_cast<const float2*>(dacc + C::kDepAccFloats);
       const int d = lane * V;
-      // combine the states of the warps that hold each row, row by row
-      for (int h = 0; h < GT; ++h) {
+      // combine the states of the warps that hold each row, two rows at a
+      // time: both rows' deposits are read before either is combined, so
+      // their shared-memory latencies overlap
+      constexpr int R = C::kRowWarps;
+      auto load_row = [&](int h, float2 (&ml)[R], float (&a)[R][V]) {
         const int w0 = C::kSplit ? 2 * (h >> 3) : 0;  // first warp holding row h
         const int lr = C::kSplit ? (h & 7) : h;       // its row inside those warps
-        float2 ml[C::kRowWarps];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+          ml[k] = dml[(w0 + k) * C::kWarpRows + lr];
+          const float* src = dacc + ((w0 + k) * C::kWarpRows + lr) * C::kAccStride + d;
+          if constexpr (V == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src);
+            a[k][0] = x.x; a[k][1] = x.y; a[k][2] = x.z; a[k][3] = x.w;
+          } else {
+            const float2 x = *reinterpret_cast<const float2*>(src);
+            a[k][0] = x.x; a[k][1] = x.y;
+          }
+        }
+      };
+      auto finish_row = [&](int h, const float2 (&ml)[R], const float (&a)[R][V]) {
         float M = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < C::kRowWarps; ++k) {
-          ml[k] = dml[(w0 + k) * C::kWarpRows + lr];
-          M = fmaxf(M, ml[k].x);
-        }
+        for (int k = 0; k < R; ++k) M = fmaxf(M, ml[k].x);
         float lam = 0.f, o[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) o[v] = 0.f;
 #pragma unroll
-        for (int k = 0; k < C::kRowWarps; ++k) {
+        for (int k = 0; k < R; ++k) {
           // a warp that saw no token of the piece holds m = -inf, acc = 0
           const float sc = (ml[k].x == -INFINITY) ? 0.f : fast_exp2(ml[k].x - M);
           lam += ml[k].y * sc;
-          const float* src = dacc + ((w0 + k) * C::kWarpRows + lr) * C::kAccStride + d;
-          if constexpr (V == 4) {
-            const float4 a = *reinterpret_cast<const float4*>(src);
-            o[0] += a.x * sc; o[1] += a.y * sc; o[2] += a.z * sc; o[3] += a.w * sc;
-          } else {
-            const float2 a = *reinterpret_cast<const float2*>(src);
-            o[0] += a.x * sc; o[1] += a.y * sc;
-          }
+#pragma unroll
+          for (int v = 0; v < V; ++v) o[v] += a[k][v] * sc;
         }
         if (dd.slot < 0) {
           // a row that sees no token (a query ahead of the sequence) is 0
@@ -678,6 +685,21 @@ __global__ void __launch_bounds__(kThreads, CPS)
           else *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
           if (lane == 0) p.ws.part_ml[(long long)dd.slot * GT + h] = make_float2(M, lam);
         }
+      };
+      int h = 0;
+      for (; h + 1 < GT; h += 2) {
+        float2 ml0[R], ml1[R];
+        float a0[R][V], a1[R][V];
+        load_row(h, ml0, a0);
+        load_row(h + 1, ml1, a1);
+        finish_row(h, ml0, a0);
+        finish_row(h + 1, ml1, a1);
+      }
+      if (h < GT) {
+        float2 ml0[R];
+        float a0[R][V];
+        load_row(h, ml0, a0);
+        finish_row(h, ml0, a0);
       }
       // the deposit slot is free again
       __syncwarp();
