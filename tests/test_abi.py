@@ -59,7 +59,7 @@ def test_status_strings(L):
     assert L.hpa_version() == 100
 
 
-@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("kind", [0, 1, 2, 3])
 @pytest.mark.parametrize("B,Hkv,P,param,maxlen", [
     (32, 8, 148, 0, 131072), (64, 8, 148, 0, 512), (2, 2, 148, 0, 200), (2, 2, 148, 3, 200),
     (5, 4, 7, 5, 65), (1, 1, 1, 0, 1), (256, 8, 148, 0, 16384), (3, 2, 5, 0, 0),
@@ -71,7 +71,7 @@ def test_plan_grid_matches_oracle(L, kind, B, Hkv, P, param, maxlen):
 
 def test_workspace_layout_is_aligned_and_ordered(L):
     for kind, args in [(0, (32, 8, 64, 128, 148)), (1, (2, 2, 8, 64, 148)),
-                       (2, (256, 8, 64, 128, 4864))]:
+                       (2, (256, 8, 64, 128, 4864)), (3, (32, 8, 64, 128, 148))]:
         lay = hpa.workspace_layout(kind, *args)
         offs = [lay[k] for k in ["header", "lens", "tile_start", "cta_desc", "seg_desc",
                                  "part_ml", "part_acc", "total"]]
@@ -333,3 +333,11 @@ def test_merge_states_rejects_bad_arguments_without_launching(L):
     assert L.hpa_merge_states(None, None, 1, 1, 128, 256, 1, None, None) == 1
     # no rows: nothing to enqueue, so this succeeds without a GPU
     assert call(rows=0) == 0
+
+
+def test_length_aware_workspace_equals_dynamic(L):
+    # the length-aware plan has the dynamic plan's ranges, grid and tail, so
+    # its workspace is laid out the same way
+    for args in [(32, 8, 64, 128, 296), (1, 1, 8, 64, 7), (512, 8, 64, 128, 296)]:
+        assert hpa.decode_workspace_size(3, *args) == hpa.decode_workspace_size(0, *args)
+        assert hpa.workspace_layout(3, *args) == hpa.workspace_layout(0, *args)
