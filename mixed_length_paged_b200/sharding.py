@@ -74,18 +74,32 @@ def page_shard(seq_lens, page_table, num_shards: int, shard: int):
     return torch.from_numpy(lens.astype(np.int32)), torch.from_numpy(out)
 
 
-def gather_states(o_local: torch.Tensor, lse_local: torch.Tensor, group=None):
+def _world(group) -> int:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return 1
+    return dist.get_world_size(group)
+
+
+def gather_states(o_local: torch.Tensor, lse_local: torch.Tensor, group=None, *,
+                  o_all=None, lse_all=None):
     """Every rank's (o, lse) state, in rank order, on every rank: an
     all-gather over ``group`` (one collective per tensor), or the local pair
-    alone outside a process group of several ranks."""
+    alone outside a process group of several ranks.  ``o_all`` / ``lse_all``:
+    optional lists of receive tensors (one per rank, shaped like the local
+    ones), so that a step allocates nothing."""
     import torch.distributed as dist
-    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+    n = _world(group)
+    if n == 1:
         return [o_local], [lse_local]
-    n = dist.get_world_size(group)
     if n > MAX_MERGE_STATES:
         raise HpaError(f"gather_states: at most {MAX_MERGE_STATES} ranks merge in one call")
-    o_all = [torch.empty_like(o_local) for _ in range(n)]
-    lse_all = [torch.empty_like(lse_local) for _ in range(n)]
+    if o_all is None:
+        o_all = [torch.empty_like(o_local) for _ in range(n)]
+    if lse_all is None:
+        lse_all = [torch.empty_like(lse_local) for _ in range(n)]
+    if len(o_all) != n or len(lse_all) != n:
+        raise HpaError("gather_states: one receive tensor per rank")
     dist.all_gather(o_all, o_local, group=group)
     dist.all_gather(lse_all, lse_local, group=group)
     return o_all, lse_all
@@ -102,16 +116,23 @@ class PageShardedDecoder:
                  pt_stride: int, *, group=None, num_ctas: int | None = None, device=None):
         if batch > MAX_STEP_BATCH:
             raise HpaError(f"PageShardedDecoder: batch <= {MAX_STEP_BATCH}")
+        world = _world(group)
+        if world > MAX_MERGE_STATES:
+            raise HpaError(f"PageShardedDecoder: at most {MAX_MERGE_STATES} ranks")
         self.group = group
         self.dec = PagedDecoder(batch, num_q_heads, num_kv_heads, head_dim, pt_stride,
                                 num_ctas=num_ctas, device=device)
         dev = self.dec.device
         self.o_local = torch.empty(batch, num_q_heads, head_dim, dtype=torch.float32, device=dev)
         self.lse_local = torch.empty(batch, num_q_heads, dtype=torch.float32, device=dev)
+        # receive buffers of the all-gather, allocated once
+        self.o_all = [torch.empty_like(self.o_local) for _ in range(world)] if world > 1 else None
+        self.lse_all = [torch.empty_like(self.lse_local) for _ in range(world)] if world > 1 else None
 
     def step(self, q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, *,
              k_scale=None, v_scale=None, lse_out=None):
         self.dec.step(q, k_cache, v_cache, page_table, seq_lens, self.o_local, softmax_scale,
                       k_scale=k_scale, v_scale=v_scale, lse=self.lse_local)
-        o_all, lse_all = gather_states(self.o_local, self.lse_local, self.group)
+        o_all, lse_all = gather_states(self.o_local, self.lse_local, self.group,
+                                       o_all=self.o_all, lse_all=self.lse_all)
         return merge_states(o_all, lse_all, out, lse_out)

@@ -220,6 +220,13 @@ def _gloo_worker(rank: int, world: int, port: int, q):
                 err = max(err, float(np.abs(m - whole[b, h]).max()))
         # the local state arrived unchanged at its own slot
         assert torch.equal(o_all[rank], o) and torch.equal(lse_all[rank], lse)
+        # the same exchange into receive buffers allocated beforehand
+        ob = [torch.full_like(o, float("nan")) for _ in range(world)]
+        lb = [torch.full_like(lse, float("nan")) for _ in range(world)]
+        o2, l2 = S.gather_states(o, lse, o_all=ob, lse_all=lb)
+        assert o2 is ob and l2 is lb
+        assert all(torch.equal(x, y) for x, y in zip(ob, o_all))
+        assert all(torch.equal(x, y) for x, y in zip(lb, lse_all))
         dist.barrier()
         q.put((rank, err))
     finally:
