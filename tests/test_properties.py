@@ -1,0 +1,66 @@
+"""Property-based checks (hypothesis) of the oracle planner and the host-side
+page split, on random batches: the invariants the plan kinds promise, which
+the parametrised pins check on fixed cases."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+from hypothesis import given, settings, strategies as st
+
+import oracle
+from mixed_length_paged_b200 import sharding as SH
+from tests.test_oracle_pins import _check_plan_invariants, _units
+
+lens_st = st.lists(st.integers(min_value=0, max_value=3000), min_size=1, max_size=24)
+
+
+@settings(max_examples=60, deadline=None)
+@given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
+       m=st.integers(1, 12))
+def test_length_aware_plan_properties(lens, Hkv, P, m):
+    sl = np.array(lens, dtype=np.int32)
+    cap = max(64, max(lens))
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap)
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap)
+    # coverage, contiguity, consecutive holders and partial slots
+    _check_plan_invariants(la, lens, Hkv, 3)
+    assert la["ranges"] == dyn["ranges"]
+    units = _units(lens, Hkv)
+    seg_n = {}
+    for (b, g, t) in units:
+        seg_n[(b, g)] = seg_n.get((b, g), 0) + 1
+    pieces = {}
+    for c in range(la["ranges"]):
+        a, e = int(la["cta"][c, 0]), int(la["cta"][c, 1])
+        assert abs(a - int(dyn["cta"][c, 0])) < m and abs(e - int(dyn["cta"][c, 1])) < m
+        for u in range(a, e):
+            key = units[u][:2]
+            if u == a or units[u - 1][:2] != key:
+                pieces.setdefault(key, []).append(0)
+            pieces[key][-1] += 1
+    for key, ps in pieces.items():
+        if seg_n[key] < 2 * m:
+            assert len(ps) == 1
+        if len(ps) > 1:
+            assert ps[0] >= m and ps[-1] >= m
+    # never more pieces than the dynamic plan cuts the segment into
+    for s in range(len(lens) * Hkv):
+        assert la["split_count"][s] <= dyn["split_count"][s]
+
+
+@settings(max_examples=60, deadline=None)
+@given(lens=lens_st, N=st.integers(1, 9), extra=st.integers(0, 3))
+def test_page_shard_properties(lens, N, extra):
+    L = np.array(lens, dtype=np.int32)
+    pts = int((L.max() + 63) // 64) + extra + 1
+    pt = np.arange(len(lens) * pts, dtype=np.int32).reshape(len(lens), pts)
+    shares = [SH.page_shard(torch.from_numpy(L), torch.from_numpy(pt), N, r) for r in range(N)]
+    np.testing.assert_array_equal(sum(s[0].numpy().astype(np.int64) for s in shares), L)
+    for b in range(len(lens)):
+        got = []
+        for lr, ptr in shares:
+            k = (int(lr[b]) + 63) // 64
+            got.extend(ptr.numpy()[b, :k].tolist())
+        assert got == pt[b, :(int(L[b]) + 63) // 64].tolist()
+        sizes = [(int(lr[b]) + 63) // 64 for lr, _ in shares]
+        assert max(sizes) - min(sizes) <= 1        # shares even to within a tile
