@@ -9,7 +9,11 @@
  *     hpa_decode_run    (persistent paged GQA decode + log-sum-exp merge)
  *
  * all asynchronous on one CUDA stream, with no host synchronisation in
- * between, so a step can be captured in a CUDA graph.
+ * between, so a step can be captured in a CUDA graph.  hpa_decode_step and
+ * hpa_decode_step_prologue make the plan inside the decode kernel (two
+ * launches per step).  A batch whose sequences' pages are spread over
+ * several GPUs is decoded per GPU with hpa_decode_step_lse and the GPUs'
+ * states combined with hpa_merge_states.
  *
  * Conventions for every call:
  *   - Pointers marked "device" are CUDA device (or managed) pointers owned by
