@@ -253,3 +253,84 @@ def test_gather_states_outside_a_process_group_is_the_local_state():
     o, l = torch.ones(2, 3, 4), torch.zeros(2, 3)
     oa, la = SH.gather_states(o, l)
     assert len(oa) == 1 and oa[0] is o and la[0] is l
+
+
+def _decoder_worker(rank: int, world: int, port: int, q):
+    """PageShardedDecoder's host logic on gloo: its GPU step and merge are
+    replaced by the oracle (the decoder's own code still allocates the
+    receive buffers, gathers the states in rank order and hands them on)."""
+    import sys
+    from datetime import timedelta
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import oracle as O
+    from mixed_length_paged_b200 import sharding as S
+    from mixed_length_paged_b200 import workloads as WL
+    from tests.helpers import bits16 as b16
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        lens = (0, 1, 37, 200, 129, 700)
+        B, Hq, Hkv, D = len(lens), 8, 2, 64
+        batch = WL.make_batch(WL.DecodeShape("s", Hq, Hkv, D), list(lens), seed=41)
+        qb, kc, vc = b16(batch.q), b16(batch.k_cache), b16(batch.v_cache)
+        calls = []
+
+        class FakeDecoder:  # the local decode step, computed by the oracle
+            def __init__(self, *a, **kw):
+                self.device = torch.device("cpu")
+
+            def step(self, q, k, v, pt, sl, out, scale, *, k_scale=None, v_scale=None, lse=None):
+                calls.append("step")
+                for b in range(B):
+                    for h in range(Hq):
+                        o, l = O.attention_state(qb, kc, vc, pt.numpy(), Hkv, scale, b, h, 0,
+                                                 int(sl[b]))
+                        out[b, h] = torch.from_numpy(o)
+                        lse[b, h] = l
+                return out
+
+        def fake_merge(o_parts, l_parts, out, lse_out=None):
+            calls.append(("merge", len(o_parts)))
+            for b in range(B):
+                for h in range(Hq):
+                    m, _ = O.merge_states([x[b, h].double().numpy() for x in o_parts],
+                                          [float(x[b, h]) for x in l_parts])
+                    out[b, h] = torch.from_numpy(m)
+            return out
+
+        S.PagedDecoder = FakeDecoder
+        S.merge_states = fake_merge
+        dec = S.PageShardedDecoder(B, Hq, Hkv, D, batch.pt_stride)
+        assert len(dec.o_all) == world and len(dec.lse_all) == world
+        lr, ptr = S.page_shard(batch.seq_lens, batch.page_table, world, rank)
+        out = torch.full((B, Hq, D), float("nan"), dtype=torch.float32)
+        for _ in range(2):  # a second step reuses the same receive buffers
+            bufs = [id(x) for x in dec.o_all]
+            dec.step(batch.q, batch.k_cache, batch.v_cache, ptr, lr, out, 1 / 8)
+            assert [id(x) for x in dec.o_all] == bufs
+        whole = O.paged_decode(qb, kc, vc, batch.page_table.numpy(), batch.seq_lens.numpy(),
+                               Hkv, 1 / 8)
+        err = float(np.abs(out.double().numpy() - whole).max())
+        assert calls == ["step", ("merge", world)] * 2, calls
+        dist.barrier()
+        q.put((rank, err))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_page_sharded_decoder_host_logic():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decoder_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # fp32 states merged: within fp32 rounding of the fp64 whole-batch result
+    assert max(r[1] for r in res) <= 1e-5, res
