@@ -257,10 +257,29 @@ def _host_sample(batch, rows):
             "D": batch.shape.head_dim}
 
 
-# sample for the CPU legs: the 31 short sequences (126,976 tokens x 8 kv heads)
+# the reference arm's sample: the 31 short sequences of the skewed batch
 CPU_SAMPLE_ROWS = list(range(1, 32))
-CPU_SAMPLE_DESC = ("oracle (fp64, OpenMP over (sequence, head)) on the 31 x 4096-token "
-                   "sequences of the skewed batch (126,976 KV tokens, 12% of a step's KV)")
+CPU_BASELINE_SECONDS = 10.0   # the CPU baseline repeats the whole step for at least this long
+REF_BUDGET_SECONDS = 150.0    # the whole --impl reference run (all of its steps)
+
+
+def _oracle_for(host, rows, min_seconds: float):
+    """The oracle on sequences `rows`, repeated until at least `min_seconds`
+    have passed: (GB/s over all repetitions, seconds, repetitions)."""
+    reps, secs, nbytes = 0, 0.0, 0
+    while reps == 0 or secs < min_seconds:
+        _, dt, toks = _cpu_baseline_sample(host, rows)
+        secs += dt
+        nbytes += toks * 2 * host["Hkv"] * host["D"] * 2
+        reps += 1
+    return nbytes / secs / 1e9, secs, reps
+
+
+def _reference_rows(t_one: float, calls: int, available: int) -> int:
+    """Sequences per reference step so that `calls` steps of the oracle fit
+    the run's time budget (one sequence takes `t_one` seconds)."""
+    per_call = REF_BUDGET_SECONDS / max(1, calls)
+    return max(1, min(available, int(per_call / max(t_one, 1e-6))))
 
 
 def run_reference(args, rank: int):
@@ -274,22 +293,31 @@ def run_reference(args, rank: int):
     batch = W.build(args.workload, device="cpu")
     host = _host_sample(batch, CPU_SAMPLE_ROWS)
     cores = oracle.num_threads()
-    for _ in range(max(0, min(args.warmup, 1))):
-        _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))
+    # size each step so that all of them fit the run's budget: one sequence
+    # timed after a warm-up call, then as many sequences per step as fit
+    _cpu_baseline_sample(host, [0])
+    _, t_one, _ = _cpu_baseline_sample(host, [0])
+    calls = args.steps + min(args.warmup, 1)
+    rows = list(range(_reference_rows(t_one, calls, len(CPU_SAMPLE_ROWS))))
+    for _ in range(min(args.warmup, 1)):
+        _cpu_baseline_sample(host, rows)
     times, gbs = [], []
     for _ in range(args.steps):
-        g, dt, toks = _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))
+        g, dt, toks = _cpu_baseline_sample(host, rows)
         times.append(dt)
         gbs.append(g)
     value = statistics.median(gbs)
+    sample = (f"oracle (fp64, OpenMP over (sequence, head)) per step on {len(rows)} of the "
+              f"skewed batch's 4096-token sequences ({toks:,} KV tokens), sized so that all "
+              f"{args.steps} steps fit about {REF_BUDGET_SECONDS:.0f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "skewed 1x131072+31x4096 sample", "sample": CPU_SAMPLE_DESC},
+        "config": {"workload": "skewed 1x131072+31x4096 sample", "sample": sample},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": CPU_SAMPLE_DESC},
+                         "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     del torch
@@ -695,11 +723,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         import oracle
-        host = _host_sample(batch, CPU_SAMPLE_ROWS)
-        _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))  # warm-up
-        g, dt, toks = _cpu_baseline_sample(host, list(range(len(CPU_SAMPLE_ROWS))))
+        # the whole step (every sequence of the batch), repeated for at least
+        # CPU_BASELINE_SECONDS
+        rows = list(range(B))
+        host = _host_sample(batch, rows)
+        _cpu_baseline_sample(host, [1])  # warm-up
+        g, dt, reps = _oracle_for(host, rows, CPU_BASELINE_SECONDS)
         cpu = {"value": g, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
-               "sample": CPU_SAMPLE_DESC, "seconds": dt}
+               "sample": (f"oracle (fp64, OpenMP over (sequence, head)) on the whole skewed "
+                          f"step (1 x 131072 + 31 x 4096 tokens), {reps} times in {dt:.1f} s"),
+               "seconds": dt}
 
     if rank != 0:
         return

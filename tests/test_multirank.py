@@ -58,3 +58,19 @@ def test_single_rank_is_the_identity():
     import bench
     assert bench.max_over_ranks(12.5, 1) == 12.5
     assert bench.job_throughput(2_000_000_000, 1, 0.5) == pytest.approx(4.0)
+
+
+def test_oracle_legs_are_time_bounded():
+    """The CPU legs of the benchmark: the baseline repeats its sample until a
+    time floor is met; the reference arm sizes each step to a run budget."""
+    import bench
+    from mixed_length_paged_b200 import workloads as W
+    batch = W.build("tiny")
+    host = bench._host_sample(batch, [0, 1])
+    gbs, secs, reps = bench._oracle_for(host, [0, 1], 0.05)
+    assert gbs > 0 and secs >= 0.05 and reps >= 1
+    # one sequence per step when steps are many, all of them when few
+    assert bench._reference_rows(10.0, 2000, 31) == 1
+    assert bench._reference_rows(0.5, 4, 31) == 31
+    n = bench._reference_rows(0.01, 2001, 31)
+    assert n == 7 and n * 0.01 * 2001 <= bench.REF_BUDGET_SECONDS
