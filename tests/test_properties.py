@@ -64,3 +64,18 @@ def test_page_shard_properties(lens, N, extra):
         assert got == pt[b, :(int(L[b]) + 63) // 64].tolist()
         sizes = [(int(lr[b]) + 63) // 64 for lr, _ in shares]
         assert max(sizes) - min(sizes) <= 1        # shares even to within a tile
+
+
+@settings(max_examples=60, deadline=None)
+@given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
+       kind=st.sampled_from([0, 1, 2]), param=st.integers(0, 9))
+def test_plan_kinds_properties(lens, Hkv, P, kind, param):
+    """Every plan kind covers each unit exactly once with contiguous ranges,
+    consecutive holders per segment and distinct partial slots; the dynamic
+    plan's primary ranges and tail chunks are even to within one unit."""
+    sl = np.array(lens, dtype=np.int32)
+    cap = max(64, max(lens))
+    p = oracle.plan(sl, Hkv, kind=kind, num_ctas=P, param=param if kind else 0,
+                    max_seq_len=max(lens), capacity_tokens=cap)
+    _check_plan_invariants(p, lens, Hkv, kind)
+    assert p["n_units"] == len(_units(lens, Hkv))
