@@ -2,20 +2,25 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = hpa_decode_plan + hpa_decode_run (the whole decode path for a batch
-without a prologue) over the skewed workload: 1 x 131072 + 31 x 4096 KV
-tokens, 64 query heads, 8 KV heads, head_dim 128, bf16 cache, 64-token pages
-shuffled over HBM (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention section, the
-1 x 128K + 31 x 4K case).  Inputs are synthetic (seeded N(0,1)) and resident
-in HBM; 1.06 GB of live KV per step is far above the 126 MB L2, so no flush
-is needed between steps.
+One step = the whole decode path for a batch without a prologue: the
+dynamic tile plan, attention and the split merge (hpa_decode_step: the plan
+made inside the decode kernel, two launches; hpa_decode_plan +
+hpa_decode_run above 512 sequences) over the skewed workload: 1 x 131072 +
+31 x 4096 KV tokens, 64 query heads, 8 KV heads, head_dim 128, bf16 cache,
+64-token pages shuffled over HBM (xiaodao.ai "HPC-Ops TPOT -48.8%",
+Attention section, the 1 x 128K + 31 x 4K case).  Inputs are synthetic
+(seeded N(0,1)) and resident in HBM; 1.06 GB of live KV per step is far
+above the 126 MB L2, so no flush is needed between steps.
 
 Printed (rank 0, one JSON line): value = live KV bytes per step / step time
 (whole job over N GPUs: each rank runs its own batch, weak scaling), the run
 kernel's roofline against the measured HBM copy bandwidth, an end-to-end
-figure through the public API with host buffers, the fp64 oracle timed on a
-bounded sample on the host cores, the static split-KV plans fed to the same
-kernel, and SM clocks sampled during the timed region.
+figure through the public API with host buffers, the fp64 oracle timed on
+the host cores, SM clocks sampled during the timed region, and comparisons
+timed as interleaved A/B runs: the static split-KV plans and the
+length-aware plan fed to the same kernel, the three-launch form, and the
+batch split by page range over 2 and 8 shares (run one after another on
+this GPU, then merged).
 
 --impl reference times the oracle (the plain fp64 CPU implementation) on the
 host cores on a bounded sample of the same workload and prints the same line
