@@ -64,7 +64,8 @@ def _args():
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of CUDA-graph replays of the step")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the static-plan comparison and the e2e leg")
+                    help="skip the comparisons (static, length-aware and three-launch plans, "
+                         "page-sharded shares, separate prologue) and the e2e leg")
     return ap.parse_args()
 
 
