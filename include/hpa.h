@@ -90,11 +90,25 @@ typedef enum { HPA_OUT_BF16 = 0, HPA_OUT_F32 = 1 } hpa_out_dtype;
  * x HPC-Ops", Attention Backend: nearly-finished short requests first, long
  * ones spread over the grid); see hpa_decode_plan. */
 typedef enum {
-  HPA_PLAN_DYNAMIC = 0,        /* param unused */
+  HPA_PLAN_DYNAMIC = 0,        /* param unused; tail shape: hpa_decode_plan_tail */
   HPA_PLAN_STATIC_NSPLIT = 1,  /* param = splits per (seq, kv head); 0 = ceil(num_ctas / (B Hkv)) */
   HPA_PLAN_STATIC_CHUNK = 2,   /* param = tiles per split; 0 = ceil(T_max / ceil(num_ctas / Hkv)) */
   HPA_PLAN_LENGTH_AWARE = 3    /* param = smallest end piece of a cut segment, tiles; 0 = 4 */
 } hpa_plan_kind;
+
+/* Shape of the run-time tail of the DYNAMIC and LENGTH_AWARE plans (see
+ * hpa_decode_plan): the last Ut = min(floor(U / tail_den), U - P) units
+ * (none if tail_den = 0) are cut into M = min(tail_chunks * P, Ut) chunks.
+ * These are this library's tuning choices, not part of the method: the pages
+ * fix only that the global tile list is spread as evenly as possible over the
+ * persistent CTAs, which every (tail_den, tail_chunks) does, and tail_den = 0
+ * is that even spread with nothing left to run time.  hpa_decode_plan, the
+ * in-kernel plans (hpa_decode_step*) and hpa_decode_noalloc use the defaults;
+ * hpa_decode_plan_tail takes both as arguments.  HPA_TAIL_CHUNKS_MAX bounds
+ * tail_chunks (the workspace has room for that many chunks per CTA). */
+#define HPA_TAIL_DEN_DEFAULT 8
+#define HPA_TAIL_CHUNKS_DEFAULT 4
+#define HPA_TAIL_CHUNKS_MAX 4
 
 /* Bits of the device status word (hpa_read_status). */
 #define HPA_DEVICE_LEN_CLAMPED 0x1  /* a seq_len < 0 or > pt_stride * 64 was clamped */
@@ -140,7 +154,8 @@ HPA_API size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_
 
 /* Byte offsets of the workspace regions, for inspection by tests and tools:
  * offsets[0..6] = header (int32[16]: magic, status, units, grid, kind, batch,
- * kv heads, group, head_dim, tiles, ranges V, next tail chunk, ...), lens,
+ * kv heads, group, head_dim, tiles, ranges V, next tail chunk, finished CTAs,
+ * tail_den, tail_chunks (0, 0 for the static kinds), 0), lens,
  * tile_start, range descriptors (int32 x8 per range: u_begin, u_end, then
  * the sequence, kv head, tile and tile count of its first unit, 0, 0),
  * segment descriptors (int32 x2 per (sequence, kv head): slot of its first
@@ -160,7 +175,8 @@ HPA_API hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_k
  * (sequence b, kv head g, tile t); the global list orders units by b, g, t,
  * and the plan cuts it into contiguous ranges.  DYNAMIC (P = num_ctas
  * persistent CTAs, U units): if U <= P, CTA c < U takes unit c; otherwise the
- * last Ut = min(floor(U/8), U - P) units form M = min(4P, Ut) tail chunks
+ * last Ut units (Ut from the tail shape above: min(floor(U/8), U - P) by
+ * default) form M tail chunks (min(4P, Ut) by default)
  * [U1 + floor(jUt/M), U1 + floor((j+1)Ut/M)) and the first U1 = U - Ut units
  * the P primary ranges [floor(cU1/P), floor((c+1)U1/P)).  CTA c runs primary
  * range c, then takes tail chunks in order from a counter as it finishes, so
@@ -198,6 +214,29 @@ HPA_API hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int num_k
                            int num_q_heads, int head_dim, int pt_stride, hpa_plan_kind kind,
                            int num_ctas, int param, int max_seq_len, void* workspace,
                            size_t ws_bytes, int* grid_out, void* stream);
+
+/*
+ * hpa_decode_plan_tail -- hpa_decode_plan for the DYNAMIC or LENGTH_AWARE kind
+ * with the run-time tail's shape given explicitly (xiaodao.ai "HPC-Ops TPOT
+ * -48.8%", Attention section: the even spread of the tile list; bitbyai.com
+ * "vLLM x HPC-Ops", Attention Backend: progress evaluated at run time).
+ *
+ *   tail_den     0 .. 2^20: the tail holds min(floor(U / tail_den), U - P)
+ *                units; 0 = no tail (the primary ranges are the even
+ *                partition of all U units).
+ *   tail_chunks  1 .. HPA_TAIL_CHUNKS_MAX: the tail is cut into
+ *                min(tail_chunks * P, Ut) chunks (ignored if the tail is empty).
+ *   the rest     as for hpa_decode_plan (max_seq_len is not needed).
+ * Any other kind, or a parameter out of range, returns HPA_ERR_INVALID_ARG.
+ * The workspace size and hpa_decode_run's arguments do not depend on the
+ * tail shape.  hpa_decode_plan(kind, ...) equals hpa_decode_plan_tail(kind,
+ * ..., HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT, ...).
+ */
+HPA_API hpa_status hpa_decode_plan_tail(const int32_t* seq_lens, int batch, int num_kv_heads,
+                                        int num_q_heads, int head_dim, int pt_stride,
+                                        hpa_plan_kind kind, int num_ctas, int param,
+                                        int tail_den, int tail_chunks, void* workspace,
+                                        size_t ws_bytes, int* grid_out, void* stream);
 
 /*
  * hpa_decode_run -- persistent paged GQA decode attention with split-KV

@@ -78,7 +78,6 @@ constexpr int kSmemPerSm = 228 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any barrier wait
 constexpr int kDepBufs = 2;              // deposit slots between consumers and epilogue
 constexpr int kMaxQTokens = 16;          // query tokens per sequence (multi-token decode)
-constexpr int kMaxFusedBatch = 512;      // sequences an in-kernel plan keeps in shared memory
 
 template <int D, int NT, bool FP8, int CPS, bool PRO, bool FP>
 struct Cfg {
@@ -137,6 +136,7 @@ struct RunParams {
   int T, GT;                // query tokens per sequence; rows per kv head = G * T
   const int32_t* seq_lens;  // in-kernel plan: the step's lengths (else the plan's)
   int capacity;             // in-kernel plan: pt_stride * 64 tokens
+  int tail_den, tail_chunks;  // in-kernel plan: the run-time tail's shape
   float scale_log2;         // softmax_scale * log2(e)
   Ws ws;
   int grid, kind;
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
   DynGeom dg{};
   if constexpr (FP) {
     if (warp >= kConsumerWarps) {
-      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x);
+      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x, p.tail_den, p.tail_chunks);
       double rc[4];
       dyn_reciprocals(dg, rc);
       dg.init_div(rc);
@@ -617,6 +617,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
         h[kHdrHeadDim] = D;
         h[kHdrTiles] = ts[p.B];
         h[kHdrRanges] = (int32_t)dg.ranges();
+        h[kHdrTailDen] = p.tail_den;
+        h[kHdrTailChunks] = p.tail_chunks;
         h[kHdrMagic] = kPlanMagic;
       }
     }
@@ -1457,6 +1459,8 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.q_out = pro ? static_cast<__nv_bfloat16*>(pro->q_out) : nullptr;
   p.seq_lens = plan_lens;
   p.capacity = pt_stride * kPageSize;
+  p.tail_den = HPA_TAIL_DEN_DEFAULT;
+  p.tail_chunks = HPA_TAIL_CHUNKS_DEFAULT;
   const int nt = GT > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;

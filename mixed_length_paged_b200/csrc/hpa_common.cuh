@@ -13,11 +13,13 @@ namespace hpa {
 
 constexpr int kPageSize = 64;            // tokens per page == tokens per tile
 constexpr int kMaxPlanBatch = 32768;     // sequences per plan (tile offsets live in shared memory)
+constexpr int kMaxFusedBatch = 512;      // sequences an in-kernel plan keeps in shared memory
 constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
-//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next, done
+//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next, done,
+//                          tail_den, tail_chunks
 //   lens        int32[B]     clamped lengths
 //   tile_start  int32[B+1]   exclusive prefix sum of tiles per sequence
 //   cta_desc    int4[2*V]    per range v: (u_begin, u_end, b0, g0), (t0, n0,
@@ -44,13 +46,15 @@ enum HeaderField {
   kHdrRanges = 10,  // virtual ranges V (grid for static plans)
   kHdrNext = 11,    // dynamic plan: next tail chunk to hand out (run-time counter)
   kHdrDone = 12,    // in-kernel plan: CTAs of the current step that finished
+  kHdrTailDen = 13,     // dynamic plans: the tail parameters the plan was made with
+  kHdrTailChunks = 14,
   kHdrWords = 16
 };
 
 // The dynamic plan gives each of its P persistent CTAs one primary range and
-// hands out up to kTailChunksPerCta * P tail chunks at run time.
-constexpr int kTailChunksPerCta = 4;
-constexpr int kTailFractionDiv = 8;  // the tail holds floor(U / 8) units (fewer if U is small)
+// hands out up to tail_chunks * P tail chunks at run time (tail_chunks <=
+// HPA_TAIL_CHUNKS_MAX, which sizes the workspace).
+constexpr int kMaxTailChunksPerCta = HPA_TAIL_CHUNKS_MAX;
 constexpr int kLaDefaultMinPiece = 4;  // LENGTH_AWARE: smallest piece of a cut segment, tiles
 
 #if defined(__CUDACC__)
@@ -60,13 +64,14 @@ constexpr int kLaDefaultMinPiece = 4;  // LENGTH_AWARE: smallest piece of a cut 
 #endif
 
 // DYNAMIC and LENGTH_AWARE: P primary ranges + up to 4P run-time tail chunks
+// (HPA_TAIL_CHUNKS_MAX per CTA)
 HPA_HD inline bool plan_is_dynamic(int kind) {
   return kind == HPA_PLAN_DYNAMIC || kind == HPA_PLAN_LENGTH_AWARE;
 }
 
 // Virtual ranges a plan of this kind and grid can describe.
 HPA_HD inline long long plan_ranges_ll(int kind, int grid) {
-  return plan_is_dynamic(kind) ? (long long)grid * (1 + kTailChunksPerCta) : grid;
+  return plan_is_dynamic(kind) ? (long long)grid * (1 + kMaxTailChunksPerCta) : grid;
 }
 
 struct WsLayout {

@@ -419,14 +419,19 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  * (b, g).  Three plans give every CTA a contiguous range of that list:
  *
  *   kind 0, dynamic: P persistent CTAs.  If U <= P, CTA c < U takes unit c
- *     and the rest take nothing.  Otherwise the last Ut = min(floor(U/8),
- *     U - P) units form M = min(4P, Ut) tail chunks and the first
- *     U1 = U - Ut units P primary ranges, each spread as evenly as possible:
- *     range c < P is [floor(c U1 / P), floor((c+1) U1 / P)), range P + j is
- *     [U1 + floor(j Ut / M), U1 + floor((j+1) Ut / M)).  CTA c runs range c,
- *     then whichever tail chunks it takes at run time (bitbyai.com "vLLM x
- *     HPC-Ops", Attention Backend: progress is evaluated dynamically).
- *     Grid = P; V = P + M ranges.
+ *     and the rest take nothing.  Otherwise the unit list is spread as evenly
+ *     as possible over P primary ranges, except for a tail of Ut units that
+ *     is spread as evenly as possible over M smaller chunks which CTAs take
+ *     at run time as they finish (bitbyai.com "vLLM x HPC-Ops", Attention
+ *     Backend: progress is evaluated dynamically).  The pages fix the even
+ *     spread but not the size of the tail, so this is a FAMILY of plans with
+ *     two parameters given by the caller: the tail divisor den and the chunks
+ *     per CTA k.  Ut = min(floor(U / den), U - P) (every primary range keeps
+ *     at least one unit; den = 0 means no tail, Ut = 0), M = min(k P, Ut).
+ *     With U1 = U - Ut, range c < P is [floor(c U1 / P), floor((c+1) U1 / P))
+ *     and range P + j is [U1 + floor(j Ut / M), U1 + floor((j+1) Ut / M)).
+ *     With den = 0 the ranges are the plain even partition
+ *     [floor(c U / P), floor((c+1) U / P)).  Grid = P; V = P + M ranges.
  *   kind 1, static fixed split count S (param, default ceil(P / (B Hkv))):
  *     one CTA per (segment, split i); each segment's n tiles cut into
  *     chunks of ceil(n / S) tiles, chunk i = [i C, min((i+1) C, n)).
@@ -490,12 +495,14 @@ static long snap_cut(long x, long U, long m, const int32_t* unit_seg, const int3
 }
 
 int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capacity_tokens,
-                int kind, int num_ctas, int param, int max_seq_len, int32_t* lens_out,
+                int kind, int num_ctas, int param, int max_seq_len, int tail_den,
+                int tail_chunks, int32_t* lens_out,
                 int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][2] */,
                 int32_t* split_count /* [B*Hkv] */, int32_t* first_slot /* [B*Hkv] */,
                 int32_t* n_units_out, int32_t* n_ranges_out) {
   if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 3)
     return ORC_BAD_ARG;
+  if (tail_den < 0 || tail_chunks < 1) return ORC_BAD_ARG;
   long grid = oracle_plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len, page_size);
   int S = B * Hkv;
   /* 1. lengths clamped to [0, capacity], tiles per sequence, tile offsets */
@@ -537,9 +544,10 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
         end[c] = c < U ? c + 1 : U;
       }
     } else {
-      long Ut = U / 8 < U - P ? U / 8 : U - P;
+      long Ut = 0; /* tail units: none when den = 0 */
+      if (tail_den > 0) Ut = U / tail_den < U - P ? U / tail_den : U - P;
       long U1 = U - Ut;
-      long M = 4 * P < Ut ? 4 * P : Ut;
+      long M = (long)tail_chunks * P < Ut ? (long)tail_chunks * P : Ut;
       for (long c = 0; c < P; ++c) {
         beg[c] = c * U1 / P;
         end[c] = (c + 1) * U1 / P;

@@ -118,6 +118,40 @@ def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
     assert grid == -7  # nothing reported, nothing enqueued
 
 
+def _plan_tail(L, **kw):
+    a = dict(seq_lens=1, batch=2, num_kv_heads=2, num_q_heads=8, head_dim=64, pt_stride=4,
+             kind=0, num_ctas=148, param=0, tail_den=8, tail_chunks=4, workspace=256,
+             ws_bytes=1 << 20)
+    a.update(kw)
+    g = C.c_int(-7)
+    rc = L.hpa_decode_plan_tail(a["seq_lens"], a["batch"], a["num_kv_heads"], a["num_q_heads"],
+                                a["head_dim"], a["pt_stride"], a["kind"], a["num_ctas"],
+                                a["param"], a["tail_den"], a["tail_chunks"], a["workspace"],
+                                a["ws_bytes"], C.byref(g), None)
+    return rc, g.value
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(kind=1), 1), (dict(kind=2), 1),           # the static kinds have no tail
+    (dict(tail_den=-1), 1), (dict(tail_den=(1 << 20) + 1), 1),
+    (dict(tail_chunks=0), 1), (dict(tail_chunks=hpa.TAIL_CHUNKS_MAX + 1), 1),
+    (dict(tail_den=0, tail_chunks=0), 1),
+    (dict(seq_lens=None), 1), (dict(ws_bytes=16), 3), (dict(num_ctas=65537), 2),
+])
+def test_plan_tail_rejects_bad_arguments_without_launching(L, bad, expect):
+    rc, grid = _plan_tail(L, **bad)
+    assert rc == expect
+    assert grid == -7
+
+
+def test_tail_defaults_match_the_header():
+    src = open(HEADER).read()
+    for name, val in [("HPA_TAIL_DEN_DEFAULT", hpa.TAIL_DEN_DEFAULT),
+                      ("HPA_TAIL_CHUNKS_DEFAULT", hpa.TAIL_CHUNKS_DEFAULT),
+                      ("HPA_TAIL_CHUNKS_MAX", hpa.TAIL_CHUNKS_MAX)]:
+        assert re.search(rf"#define {name} {val}\b", src), name
+
+
 def _run(L, **kw):
     a = dict(q=256, k=256, v=256, ks=None, vs=None, kvd=0, pt=256, pts=4, pages=8, out=256,
              outd=0, B=2, Hq=8, Hkv=2, D=64, scale=0.125, kind=0, grid=148, ws=256, wsb=1 << 24)

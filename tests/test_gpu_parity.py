@@ -6,6 +6,7 @@ fp32 output; plans and slot writes are compared bit for bit.
 """
 from __future__ import annotations
 
+import copy
 import math
 import zlib
 
@@ -16,9 +17,8 @@ import torch
 import oracle
 import mixed_length_paged_b200 as hpa
 from mixed_length_paged_b200 import workloads as W
-from tests.helpers import (bf16_values, bits16, compact_rows, errors, gpu_decode, gpu_decode_multi,
-                           oracle_decode,
-                           quantize_fp8, to_device)
+from tests.helpers import (bf16_values, bits16, check_rows_relative, compact_rows, errors,
+                           gpu_decode, gpu_decode_multi, oracle_decode, quantize_fp8, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,6 +61,11 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
     }
 
 
+# The library's member of the dynamic plan family (hpa.h: HPA_TAIL_DEN_DEFAULT,
+# HPA_TAIL_CHUNKS_DEFAULT), and other members called with hpa_decode_plan_tail.
+LIB_TAIL = (8, 4)
+
+
 @pytest.mark.parametrize("lens,Hkv,P", [
     ([131072] + [4096] * 31, 8, 148), ([512] * 64, 8, 148), ([37, 200], 2, 148),
     ([37, 200], 2, 3), ([0, 5, 0, 64, 65, 3000, 1], 4, 7), ([1], 1, 148), ([0, 0], 2, 5),
@@ -69,22 +74,29 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
     ([int(x) for x in np.random.default_rng(3).integers(0, 300, 20000)], 2, 148),
     ([int(x) for x in np.random.default_rng(4).integers(1, 100, 32768)], 1, 148),  # the maximum
 ])
-@pytest.mark.parametrize("kind,param", [(0, 0), (1, 0), (1, 3), (2, 0), (2, 5), (3, 0), (3, 2),
-                                        (3, 9)])
-def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
+@pytest.mark.parametrize("kind,param,tail", [
+    (0, 0, None), (1, 0, None), (1, 3, None), (2, 0, None), (2, 5, None), (3, 0, None),
+    (3, 2, None), (3, 9, None),
+    (0, 0, (0, 1)), (0, 0, (3, 1)), (0, 0, (16, 2)), (0, 0, (1, 4)), (3, 4, (0, 1)),
+    (3, 2, (5, 3))])
+def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail):
+    """tail None: hpa_decode_plan (the library's default tail, LIB_TAIL);
+    else hpa_decode_plan_tail with that tail shape (0, 1 = no tail)."""
     B, Hq, D = len(lens), Hkv * 2, 64
     cap = max(64, max(lens))
     pts = (cap + 63) // 64
     maxlen = max(lens)
     grid = hpa.plan_grid(kind, B, Hkv, P, param, maxlen)
     ref = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P, param=param,
-                      max_seq_len=maxlen, capacity_tokens=pts * 64)
+                      max_seq_len=maxlen, capacity_tokens=pts * 64,
+                      tail=LIB_TAIL if tail is None else tail)
     assert grid == ref["grid"]
     ws = torch.full((hpa.decode_workspace_size(kind, B, Hkv, Hq, D, grid),), 0xAB,
                     dtype=torch.uint8, device="cuda")
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
     g = hpa.decode_plan(sl, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D, pt_stride=pts,
-                        workspace=ws, kind=kind, num_ctas=P, param=param, max_seq_len=maxlen)
+                        workspace=ws, kind=kind, num_ctas=P, param=param, max_seq_len=maxlen,
+                        tail=tail)
     torch.cuda.synchronize()
     assert g == grid
     got = _read_plan(ws, kind, B, Hkv, Hq, D, grid)
@@ -107,6 +119,9 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param):
     np.testing.assert_array_equal(got["seg"][:, 1], ref["split_count"])
     h = got["header"]
     assert h[2] == ref["n_units"] and h[3] == grid and h[1] == 0
+    # the tail shape the plan was made with, recorded in the header
+    want = (LIB_TAIL if tail is None else tail) if kind in (0, 3) else (0, 0)
+    assert (int(h[13]), int(h[14])) == want
 
 
 def test_plan_flags_clamped_lengths():
@@ -255,16 +270,62 @@ def test_uniform_workload():
     _check(out, ref)
 
 
-def test_skewed_workload_sampled_rows():
+def _bench_step(batch, out_dtype=torch.bfloat16):
+    """The benchmark's launch: hpa_decode_step (plan inside the decode kernel)
+    over the persistent CTA count hpa_decode_num_ctas gives."""
+    B, Hq, D = batch.batch, batch.shape.num_q_heads, batch.shape.head_dim
+    Hkv = batch.shape.num_kv_heads
+    dec = hpa.PagedDecoder(B, Hq, Hkv, D, batch.pt_stride)
+    out = torch.full((B, Hq, D), float("nan"), dtype=out_dtype, device="cuda")
+    dec.step(batch.q, batch.k_cache, batch.v_cache, batch.page_table, batch.seq_lens, out,
+             1.0 / math.sqrt(D))
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    return out
+
+
+def test_skewed_workload_all_rows():
+    """The whole skewed batch (1 x 131072 + 31 x 4096) against the oracle, every
+    row, in the benchmark's launch and through plan + run; each row also
+    within 5 % of its own magnitude, so a wrong 128K row cannot hide under the
+    absolute tolerance."""
     batch = W.build("skewed", device="cuda")
-    out = gpu_decode(batch)  # dynamic plan, one CTA per SM: the benchmark's launch
-    rows = [0, 1, 17, 31]
-    small = compact_rows(batch, rows)
-    ref = oracle_decode(small)
-    _check(out[rows], ref)
+    ref = oracle_decode(batch)
+    for out in (_bench_step(batch), gpu_decode(batch)):
+        _check(out, ref)
+        check_rows_relative(out, ref)
     outA = gpu_decode(batch, kind=1, out_dtype=torch.float32)
     outD = gpu_decode(batch, out_dtype=torch.float32)
     assert (outA - outD).abs().max().item() <= SCHED_TOL
+
+
+def test_needle_in_the_128k_sequence_full_batch():
+    """Needle pin of the page mapping at scale, on the full skewed batch in the
+    benchmark's launch: for one query head h of every kv group g, the key at a
+    random position j_g of the 131072-token sequence is set to
+    40 q_h / |q_h| (a logit of ~40 against N(0, 1) logits), so head h's output
+    is V[j_g] to within bf16 rounding while the other heads of the group stay
+    far from it.  The sequence is spread over ~74 CTAs per kv head, so this
+    checks the tile-to-page mapping, the split and the merge together."""
+    batch = W.build("skewed", device="cuda")
+    G, D = batch.shape.group, batch.shape.head_dim
+    rng = np.random.default_rng(2024)
+    planted = []
+    for g in range(batch.shape.num_kv_heads):
+        h = g * G + int(rng.integers(0, G))
+        j = int(rng.integers(0, 131072))
+        qh = batch.q[0, h].float()
+        batch.k_cache[int(batch.page_table[0, j // 64]), g, j % 64] = \
+            (40.0 * qh / qh.norm()).to(torch.bfloat16)
+        planted.append((g, h, j))
+    for out in (_bench_step(batch), gpu_decode(batch, num_ctas=37)):
+        o = out[0].float()
+        for g, h, j in planted:
+            v = batch.v_cache[int(batch.page_table[0, j // 64]), g, j % 64].float()
+            assert (o[h] - v).abs().max().item() <= MAX_ABS, (g, h, j)
+            for h2 in range(g * G, (g + 1) * G):
+                if h2 != h:
+                    assert (o[h2] - v).abs().max().item() > 0.5, (g, h2, j)
 
 
 def test_fp8_small():
@@ -350,26 +411,43 @@ def test_prologue_bad_position_is_flagged_not_written():
     assert len(changed) == 2  # sequence 0's K row for its two kv heads only
 
 
-def test_mix_prologue_workload_sampled_rows():
+def test_mix_prologue_workload_all_rows():
+    """The whole 128-sequence continuous-batching mix with the prologue, every
+    row against the oracle's prologue + attention, in the benchmark's launch
+    (hpa_decode_step_prologue) and as prologue kernel + plan + run; each row
+    also within 5 % of its own magnitude."""
     batch = W.build("mix_prologue", device="cuda")
-    rows = [0, 1, 50, 127]
-    L = batch.positions.cpu().numpy()
-    rows.append(int(np.argmax(L)))
-    small = compact_rows(batch, rows)
-    small.q_raw = batch.q_raw[rows].cpu()
-    small.k_raw = batch.k_raw[rows].cpu()
-    small.v_raw = batch.v_raw[rows].cpu()
-    small.positions = batch.positions[rows].cpu()
-    kc, vc = bits16(small.k_cache).copy(), bits16(small.v_cache).copy()
-    q64 = oracle.prologue(bits16(small.q_raw), bits16(small.k_raw), bits16(small.v_raw),
+    host = copy.copy(batch)
+    for name in ("q_raw", "k_raw", "v_raw", "positions", "page_table", "seq_lens"):
+        setattr(host, name, getattr(batch, name).cpu())
+    kc, vc = bits16(batch.k_cache).copy(), bits16(batch.v_cache).copy()
+    q64 = oracle.prologue(bits16(host.q_raw), bits16(host.k_raw), bits16(host.v_raw),
                           batch.q_gamma.cpu().numpy(), batch.k_gamma.cpu().numpy(), 1e-6, 1e4,
-                          small.positions.numpy(), small.page_table.numpy(), kc, vc)
-    ref = oracle.paged_decode(q64, kc, vc, small.page_table.numpy(), small.seq_lens.numpy(), 8,
+                          host.positions.numpy(), host.page_table.numpy(), kc, vc)
+    ref = oracle.paged_decode(q64, kc, vc, host.page_table.numpy(), host.seq_lens.numpy(), 8,
                               1 / math.sqrt(128))
+    del kc, vc
+    B, Hq, D = batch.q_raw.shape
+    kc0, vc0 = batch.k_cache.clone(), batch.v_cache.clone()
+    # 1. the benchmark's launch: the whole step in two launches
+    dec = hpa.PagedDecoder(B, Hq, 8, D, batch.pt_stride)
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dec.step_prologue(batch.q_raw, batch.k_raw, batch.v_raw, batch.q_gamma, batch.k_gamma,
+                      batch.k_cache, batch.v_cache, batch.page_table, batch.seq_lens, out,
+                      1 / math.sqrt(D), eps=1e-6, rope_theta=1e4)
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    _check(out, ref)
+    check_rows_relative(out, ref)
+    # 2. prologue kernel, then plan + run, on fresh copies of the caches
+    batch.k_cache.copy_(kc0)
+    batch.v_cache.copy_(vc0)
+    del kc0, vc0
     q_out, status = _run_prologue(batch)
     assert status == 0
-    out = gpu_decode(batch, q=q_out)
-    _check(out[rows], ref)
+    out2 = gpu_decode(batch, q=q_out)
+    _check(out2, ref)
+    check_rows_relative(out2, ref)
 
 
 # ---------------------------------------------------------------- multi-token decode

@@ -10,6 +10,7 @@ from __future__ import annotations
 import json
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -441,7 +442,7 @@ def _units(lens, Hkv):
     return out
 
 
-def _check_plan_invariants(p, lens, Hkv, kind):
+def _check_plan_invariants(p, lens, Hkv, kind, tail=None):
     units = _units(lens, Hkv)
     U = len(units)
     assert p["n_units"] == U
@@ -494,21 +495,55 @@ def _check_plan_invariants(p, lens, Hkv, kind):
     used = [x for ps in pieces.values() for x in ps]
     assert len(used) == len(set(used)) and all(0 <= x < 2 * R for x in used)
     if kind == 0:
-        P = p["grid"]
-        sizes = [int(cta[c, 1] - cta[c, 0]) for c in range(R)]
-        if U <= P:
-            # one unit per CTA, no tail
-            assert R == P and sorted(set(sizes)) in ([1], [0, 1], [0], [])
+        _check_dynamic_family(p, U, tail)
+
+
+def _even_ranges(n, m):
+    """Unit list [0, n) cut into m contiguous ranges as evenly as possible,
+    enumerated from scratch: scale the list onto m equal ranges and give unit
+    u the range in which its right end (u + 1) * m / n falls, with each range
+    closed on the right.  Exact rational arithmetic; returns [(begin, end)]."""
+    owner = [math.ceil(Fraction((u + 1) * m, n)) - 1 for u in range(n)]
+    out = []
+    for c in range(m):
+        us = [u for u in range(n) if owner[u] == c]
+        if us:
+            assert us == list(range(us[0], us[-1] + 1))
+            out.append((us[0], us[-1] + 1))
         else:
-            # the tail holds min(U // 8, U - P) units in min(4P, tail) chunks;
-            # primary ranges and tail chunks are each even to within one unit
-            tail = min(U // 8, U - P)
-            assert R == P + min(4 * P, tail)
-            assert sum(sizes[P:]) == tail
-            prim, chunks = sizes[:P], sizes[P:]
-            assert min(prim) >= 1 and max(prim) - min(prim) <= 1
-            if chunks:
-                assert min(chunks) >= 1 and max(chunks) - min(chunks) <= 1
+            b = out[-1][1] if out else 0
+            out.append((b, b))
+    return out
+
+
+def _check_dynamic_family(p, U, tail):
+    """A dynamic plan of the family (den, k): the primary ranges are the even
+    partition of the first U1 units over P CTAs and the tail chunks the even
+    partition of the last Ut units over M chunks, where Ut is the largest tail
+    with Ut <= U / den that still leaves every primary range a unit (no tail
+    for den = 0) and M the largest chunk count with M <= k P and M <= Ut."""
+    den, k = tail
+    P = p["grid"]
+    R = p["ranges"]
+    cta = [(int(a), int(e)) for a, e in p["cta"]]
+    if U <= P:
+        # one unit per CTA, no tail
+        assert R == P and cta == [(min(c, U), min(c + 1, U)) for c in range(P)]
+        return
+    M = R - P
+    Ut = U - cta[P - 1][1] if M else 0
+    if den == 0:
+        assert Ut == 0 and M == 0
+    else:
+        assert Ut * den <= U and U - Ut >= P
+        assert (Ut + 1) * den > U or U - Ut == P      # no larger tail would do
+        if Ut:
+            assert 1 <= M <= k * P and M <= Ut
+            assert M == k * P or M == Ut
+        else:
+            assert M == 0
+    assert cta[:P] == _even_ranges(U - Ut, P)
+    assert [(a - (U - Ut), e - (U - Ut)) for a, e in cta[P:]] == (_even_ranges(Ut, M) if M else [])
 
 
 @pytest.mark.parametrize("lens,Hkv,P", [
@@ -520,11 +555,35 @@ def _check_plan_invariants(p, lens, Hkv, kind):
     ([1], 1, 148),
     ([0, 0], 2, 5),
 ])
-@pytest.mark.parametrize("kind", [0, 1, 2])
-def test_planner_invariants(lens, Hkv, P, kind):
+@pytest.mark.parametrize("kind,tail", [(0, (8, 4)), (0, (0, 1)), (0, (3, 1)), (0, (16, 2)),
+                                       (0, (1, 4)), (1, (8, 4)), (2, (8, 4))])
+def test_planner_invariants(lens, Hkv, P, kind, tail):
     p = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P,
-                    max_seq_len=max(lens), capacity_tokens=max(64, max(lens)))
-    _check_plan_invariants(p, lens, Hkv, kind)
+                    max_seq_len=max(lens), capacity_tokens=max(64, max(lens)), tail=tail)
+    _check_plan_invariants(p, lens, Hkv, kind, tail)
+
+
+def test_even_ranges_enumerator_hand_cases():
+    # the enumerator the dynamic-plan pins compare with, on cases worked by hand
+    assert _even_ranges(7, 3) == [(0, 2), (2, 4), (4, 7)]
+    assert _even_ranges(3, 5) == [(0, 0), (0, 1), (1, 1), (1, 2), (2, 3)]
+    assert _even_ranges(6, 3) == [(0, 2), (2, 4), (4, 6)]
+    assert _even_ranges(10, 4) == [(0, 2), (2, 5), (5, 7), (7, 10)]
+
+
+@pytest.mark.parametrize("U,P", [(5, 5), (6, 5), (7, 3), (100, 7), (32256, 148), (4096, 296),
+                                 (301, 300), (1000, 1)])
+def test_dynamic_plan_without_tail_is_the_even_partition(U, P):
+    """With no run-time tail (den = 0) the dynamic plan is the plain even
+    partition of the unit list over the CTAs: range c holds units
+    [floor(cU/P), floor((c+1)U/P))."""
+    # U units as one sequence of U tiles with one kv head
+    p = oracle.plan(np.array([64 * U], dtype=np.int32), 1, kind=0, num_ctas=P,
+                    capacity_tokens=64 * U, tail=(0, 1))
+    assert p["ranges"] == P
+    assert [(int(a), int(e)) for a, e in p["cta"]] == _even_ranges(U, P)
+    # one split count and consecutive slots, recounted
+    _check_plan_invariants(p, [64 * U], 1, 0, (0, 1))
 
 
 @pytest.mark.parametrize("lens,Hkv,P", [
@@ -542,8 +601,8 @@ def test_length_aware_planner(lens, Hkv, P, m):
     leave a piece of fewer than m tiles at a segment's end moves to that end."""
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
-    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap)
-    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap)
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4))
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4))
     _check_plan_invariants(la, lens, Hkv, 3)
     assert la["grid"] == P and la["ranges"] == dyn["ranges"]
     units = _units(lens, Hkv)
@@ -586,30 +645,30 @@ def test_length_aware_planner_hand_cases():
     # with m = 2 the cut after tile 1 leaves 1 tile on each side (a tie) and
     # moves to the segment's start, so the second range holds the whole segment
     p = oracle.plan(np.array([128], dtype=np.int32), 1, kind=3, num_ctas=2, param=2,
-                    capacity_tokens=128)
+                    capacity_tokens=128, tail=(8, 4))
     np.testing.assert_array_equal(p["cta"], [[0, 0], [0, 2]])
     assert p["split_count"][0] == 1 and p["first_slot"][0] == -1
     # 3 tiles, 3 CTAs, m = 2: the cut after tile 1 (a=1, r=2) moves to the
     # start, the cut after tile 2 (a=2, r=1) to the end: one whole range
     p = oracle.plan(np.array([192], dtype=np.int32), 1, kind=3, num_ctas=3, param=2,
-                    capacity_tokens=192)
+                    capacity_tokens=192, tail=(8, 4))
     np.testing.assert_array_equal(p["cta"], [[0, 0], [0, 3], [3, 3]])
-    # 8 tiles, 2 CTAs: the dynamic plan has primary ranges [0, 3), [3, 7) and
-    # one tail chunk [7, 8).  m = 2 keeps the cut at 3 (a=3, r=5) and moves
+    # 8 tiles, 2 CTAs, tail (8, 4): the dynamic plan has primary ranges
+    # [0, 3), [3, 7) and one tail chunk [7, 8).  m = 2 keeps the cut at 3 (a=3, r=5) and moves
     # the one at 7 (r=1) to the end; m = 4 also moves the cut at 3 (a=3 < 4)
     for m, want in ((2, [[0, 3], [3, 8], [8, 8]]), (4, [[0, 0], [0, 8], [8, 8]])):
         p = oracle.plan(np.array([512], dtype=np.int32), 1, kind=3, num_ctas=2, param=m,
-                        capacity_tokens=512)
+                        capacity_tokens=512, tail=(8, 4))
         np.testing.assert_array_equal(p["cta"], want)
 
 
 def test_planner_static_shapes():
     lens = [131072] + [4096] * 31
     pA = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=1, num_ctas=148, max_seq_len=131072,
-                     capacity_tokens=131072)
+                     capacity_tokens=131072, tail=(8, 4))
     assert pA["grid"] == 32 * 8  # ceil(148 / 256) = 1 split per (seq, kv head)
     pB = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=2, num_ctas=148, max_seq_len=131072,
-                     capacity_tokens=131072)
+                     capacity_tokens=131072, tail=(8, 4))
     # chunk = ceil(2048 / ceil(148 / 8)) = 108 tiles; 19 chunks per segment
     assert pB["grid"] == 32 * 8 * 19
     sizes = pB["cta"][:, 1] - pB["cta"][:, 0]
@@ -618,7 +677,7 @@ def test_planner_static_shapes():
 
 def test_planner_clamps_lengths_to_capacity():
     p = oracle.plan(np.array([-5, 1000, 64], dtype=np.int32), 2, kind=0, num_ctas=4,
-                    capacity_tokens=128)
+                    capacity_tokens=128, tail=(8, 4))
     np.testing.assert_array_equal(p["lens"], [0, 128, 64])
     np.testing.assert_array_equal(p["tile_start"], [0, 0, 2, 3])
 

@@ -20,8 +20,8 @@ lens_st = st.lists(st.integers(min_value=0, max_value=3000), min_size=1, max_siz
 def test_length_aware_plan_properties(lens, Hkv, P, m):
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
-    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap)
-    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap)
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4))
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4))
     # coverage, contiguity, consecutive holders and partial slots
     _check_plan_invariants(la, lens, Hkv, 3)
     assert la["ranges"] == dyn["ranges"]
@@ -68,14 +68,38 @@ def test_page_shard_properties(lens, N, extra):
 
 @settings(max_examples=60, deadline=None)
 @given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
-       kind=st.sampled_from([0, 1, 2]), param=st.integers(0, 9))
-def test_plan_kinds_properties(lens, Hkv, P, kind, param):
+       kind=st.sampled_from([0, 1, 2]), param=st.integers(0, 9),
+       den=st.integers(0, 40), k=st.integers(1, 4))
+def test_plan_kinds_properties(lens, Hkv, P, kind, param, den, k):
     """Every plan kind covers each unit exactly once with contiguous ranges,
-    consecutive holders per segment and distinct partial slots; the dynamic
-    plan's primary ranges and tail chunks are even to within one unit."""
+    consecutive holders per segment and distinct partial slots; a dynamic plan
+    of any tail shape (den, k) has the even primary ranges and the even tail
+    chunks of that shape."""
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
     p = oracle.plan(sl, Hkv, kind=kind, num_ctas=P, param=param if kind else 0,
-                    max_seq_len=max(lens), capacity_tokens=cap)
-    _check_plan_invariants(p, lens, Hkv, kind)
+                    max_seq_len=max(lens), capacity_tokens=cap, tail=(den, k))
+    _check_plan_invariants(p, lens, Hkv, kind, (den, k))
     assert p["n_units"] == len(_units(lens, Hkv))
+
+
+@settings(max_examples=60, deadline=None)
+@given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
+       den=st.integers(1, 40), k=st.integers(1, 4))
+def test_dynamic_tail_covers_the_last_units_evenly(lens, Hkv, P, den, k):
+    """Whatever the tail shape, the tail chunks are the last units of the list,
+    in order, each within one unit of the others, and the primary ranges the
+    units before them, also within one unit of each other."""
+    sl = np.array(lens, dtype=np.int32)
+    p = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=max(64, max(lens)),
+                    tail=(den, k))
+    U, R = p["n_units"], p["ranges"]
+    if U <= P:
+        return
+    sizes = [int(e - a) for a, e in p["cta"]]
+    prim, chunks = sizes[:P], sizes[P:]
+    assert min(prim) >= 1 and max(prim) - min(prim) <= 1
+    assert sum(prim) + sum(chunks) == U
+    if chunks:
+        assert min(chunks) >= 1 and max(chunks) - min(chunks) <= 1
+        assert int(p["cta"][P][0]) == sum(prim) and int(p["cta"][R - 1][1]) == U
