@@ -529,6 +529,27 @@ HPA_API hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, const 
  * after the work queued on `stream` so far; synchronises the stream. */
 HPA_API hpa_status hpa_read_status(const void* workspace, int32_t* status_out, void* stream);
 
+/*
+ * hpa_read_cta_times -- per-CTA timeline of the last run on a workspace, for
+ * measuring how evenly the plan loaded the persistent CTAs (the tail idle time
+ * the dynamic scheduler exists to remove: bitbyai.com "vLLM x HPC-Ops",
+ * Attention Backend, static splits leave GPU compute units idle).
+ *
+ * Every run-kernel launch (hpa_decode_run*, hpa_decode_step*) writes, for each
+ * of its `grid` CTAs c, four uint64 values to the workspace:
+ *   times_out[4c + 0]  %globaltimer (ns) when CTA c started its work (after
+ *                      waiting for the kernel before it)
+ *   times_out[4c + 1]  when its producer warp had issued its last tile
+ *   times_out[4c + 2]  when its epilogue warp had written its last result
+ *   times_out[4c + 3]  units (tiles of one kv head) it streamed
+ * The shape arguments are those the workspace was sized with
+ * (hpa_decode_workspace_size); times_out is a HOST array of 4 * grid values.
+ * Synchronises the stream.  Values of CTAs of an aborted run are undefined.
+ */
+HPA_API hpa_status hpa_read_cta_times(const void* workspace, hpa_plan_kind kind, int batch,
+                                      int num_kv_heads, int num_q_heads, int head_dim, int grid,
+                                      uint64_t* times_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,7 +34,7 @@ __all__ = [
     "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
     "decode_run_prologue",
     "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
-    "merge_states", "MAX_MERGE_STATES",
+    "merge_states", "MAX_MERGE_STATES", "read_cta_times", "tail_idle",
 ]
 
 PLAN_DYNAMIC, PLAN_STATIC_NSPLIT, PLAN_STATIC_CHUNK, PLAN_LENGTH_AWARE = 0, 1, 2, 3
@@ -122,6 +122,8 @@ def lib():
         L.hpa_decode_noalloc.restype = _I
         L.hpa_decode_noalloc.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _V, _I, _I, _I,
                                          _I, _I, _F, _I, _V]
+        L.hpa_read_cta_times.restype = _I
+        L.hpa_read_cta_times.argtypes = [_V, _I, _I, _I, _I, _I, _I, _V, _V]
         L.hpa_read_status.restype = _I
         L.hpa_read_status.argtypes = [_V, C.POINTER(C.c_int32), _V]
         _lib = L
@@ -543,6 +545,37 @@ def read_status(workspace: torch.Tensor, stream=None) -> int:
     return int(v.value)
 
 
+def read_cta_times(workspace: torch.Tensor, kind: int, batch: int, num_kv_heads: int,
+                   num_q_heads: int, head_dim: int, grid: int, stream=None):
+    """Per-CTA timeline of the last run on ``workspace`` (hpa_read_cta_times):
+    an int64 tensor [grid][4] of (start ns, producer done ns, epilogue done ns,
+    units streamed).  The shape arguments are those the workspace was sized
+    with; synchronises the stream."""
+    t = torch.zeros((grid, 4), dtype=torch.int64)
+    _check(lib().hpa_read_cta_times(_ptr(workspace), kind, batch, num_kv_heads, num_q_heads,
+                                    head_dim, grid, t.data_ptr(), _stream(stream)),
+           "hpa_read_cta_times")
+    return t
+
+
+def tail_idle(times: torch.Tensor) -> dict:
+    """Load balance of one run from its CTA timeline: the span from the first
+    CTA start to the last epilogue, the spread of the CTAs' finishing times and
+    the idle fraction sum_c (last end - end_c) / (CTAs x span) -- the share of
+    the CTAs' time spent waiting for the slowest one."""
+    t = times.to(torch.float64)
+    t0, end = t[:, 0].min(), t[:, 2]
+    span = float(end.max() - t0)
+    ends = (end - t0).sort().values
+    n = ends.numel()
+    return {"span_us": span / 1e3,
+            "end_min_us": float(ends[0]) / 1e3,
+            "end_median_us": float(ends[n // 2]) / 1e3,
+            "end_max_us": float(ends[-1]) / 1e3,
+            "idle_fraction": float((ends[-1] - ends).sum()) / (n * span) if span > 0 else 0.0,
+            "units_min": int(times[:, 3].min()), "units_max": int(times[:, 3].max())}
+
+
 class PagedDecoder:
     """A workspace sized for one batch shape, plus plan + run in one call.
     ``q_tokens`` > 1: multi-token decode (q and out [B][T][Hq][D])."""
@@ -623,3 +656,9 @@ class PagedDecoder:
 
     def status(self, stream=None) -> int:
         return read_status(self.workspace, stream)
+
+    def cta_times(self, stream=None) -> torch.Tensor:
+        """Per-CTA timeline of the last run (read_cta_times)."""
+        B, Hq, Hkv, D, _ = self.shape
+        return read_cta_times(self.workspace, self.kind, B, Hkv, Hq * self.q_tokens, D,
+                              self.grid, stream)

@@ -94,3 +94,22 @@ extern "C" hpa_status hpa_read_status(const void* workspace, int32_t* status_out
   }
   return HPA_OK;
 }
+
+extern "C" hpa_status hpa_read_cta_times(const void* workspace, hpa_plan_kind kind, int batch,
+                                         int num_kv_heads, int num_q_heads, int head_dim,
+                                         int grid, uint64_t* times_out, void* stream) {
+  WsLayout L;
+  if (!workspace || !times_out || !ws_layout(kind, batch, num_kv_heads, num_q_heads, head_dim,
+                                             grid, &L))
+    return HPA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const char* src = static_cast<const char*>(workspace) + L.trace;
+  cudaError_t e = cudaMemcpyAsync(times_out, src, size_t(grid) * 4 * sizeof(uint64_t),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    set_cuda_error(e, "hpa_read_cta_times");
+    return HPA_ERR_CUDA;
+  }
+  return HPA_OK;
+}

@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
   }
   // Everything below reads what the plan (and possibly the prologue) wrote.
   pdl_wait();
+  const uint64_t t_cta0 = globaltimer();  // this CTA's start, for the trace region
   if constexpr (FP) {
     // In-kernel plan (hpa_decode_step): every CTA turns the step's lengths
     // into tile offsets in shared memory, as the plan kernel does -- warp w
@@ -558,6 +559,13 @@ __global__ void __launch_bounds__(kThreads, CPS)
     }
     __syncwarp();
     ++it;
+    if (lane == 0) {
+      // trace: start, end of the producer's work, units streamed
+      unsigned long long* tr = p.ws.trace + 4ull * blockIdx.x;
+      tr[0] = t_cta0;
+      tr[1] = globaltimer();
+      tr[3] = (unsigned long long)(it - 1);
+    }
     // zero output rows of empty sequences (a softmax over no tokens), for
     // every query token
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
@@ -707,6 +715,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dep_empty[db]));
     }
+    if (lane == 0) p.ws.trace[4ull * blockIdx.x + 2] = globaltimer();  // trace: epilogue done
     return;
   }
 

@@ -33,6 +33,9 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 //                            partials.
 //   part_ml     float2[2V][G]     (m, l) of each partial, log2 units
 //   part_acc    float[2V][G][D]   un-normalised partial outputs
+//   trace       uint64[grid][4]   per run-kernel CTA: %globaltimer (ns) at its
+//                                 start, when its producer ran out of work and
+//                                 when its epilogue finished; units it streamed
 // Partial slots follow from the ranges: range v stores the piece of its first
 // segment in slot 2v and the piece of its last segment in slot 2v + 1 (a
 // segment in the middle of a range is whole there).  The ranges holding a
@@ -75,7 +78,7 @@ HPA_HD inline long long plan_ranges_ll(int kind, int grid) {
 }
 
 struct WsLayout {
-  size_t header, lens, tile_start, cta_desc, seg_desc, part_ml, part_acc, total;
+  size_t header, lens, tile_start, cta_desc, seg_desc, part_ml, part_acc, trace, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -95,6 +98,7 @@ inline bool ws_layout(int kind, int B, int Hkv, int Hq, int D, int grid, WsLayou
   L->seg_desc = off;    off = align256(off + S * 8);
   L->part_ml = off;     off = align256(off + slots * G * 8);
   L->part_acc = off;    off = align256(off + slots * G * size_t(D) * 4);
+  L->trace = off;       off = align256(off + size_t(grid) * 32);
   L->total = off;
   return true;
 }
@@ -108,6 +112,7 @@ struct Ws {
   int2* seg_desc;
   float2* part_ml;
   float* part_acc;
+  unsigned long long* trace;
 };
 
 inline Ws ws_view(void* base, const WsLayout& L) {
@@ -115,7 +120,8 @@ inline Ws ws_view(void* base, const WsLayout& L) {
   return Ws{reinterpret_cast<int32_t*>(p + L.header), reinterpret_cast<int32_t*>(p + L.lens),
             reinterpret_cast<int32_t*>(p + L.tile_start), reinterpret_cast<int4*>(p + L.cta_desc),
             reinterpret_cast<int2*>(p + L.seg_desc), reinterpret_cast<float2*>(p + L.part_ml),
-            reinterpret_cast<float*>(p + L.part_acc)};
+            reinterpret_cast<float*>(p + L.part_acc),
+            reinterpret_cast<unsigned long long*>(p + L.trace)};
 }
 
 // Host-side grid of a plan (must equal the oracle's definition; see hpa.h).

@@ -9,17 +9,29 @@ in two ways that need no exchange inside the attention itself:
   and the q heads of their groups.  Its decode is the plain decode of that
   head slice; the ranks' outputs are disjoint head ranges of the full output
   (what a tensor-parallel layer's output projection consumes as it is).
-* by page range: rank r holds tiles [floor(r n_b / N), floor((r+1) n_b / N))
-  of every sequence b, n_b = ceil(L_b / 64).  A single-token query attends
-  every earlier token, so a rank's share of a sequence is an ordinary shorter
-  sequence.  Each rank computes its rows' normalised outputs and
-  log-sum-exps (hpa_decode_step_lse); the ranks all-gather them (B Hq (D + 1)
-  fp32 per rank) and every rank combines them with the log-sum-exp merge
-  (hpa_merge_states) -- the split-KV recombination of xiaodao.ai "HPC-Ops
-  TPOT -48.8%" (Attention section) carried across GPUs.
+* by page: tile t of sequence b (tokens [64 t, 64 t + 64)) is held by rank
+  (s_b + t) mod N, where s_b is the sequence's start rank.  A single-token
+  query attends every earlier token, so a rank's share of a sequence -- its
+  tiles in order, only the sequence's last tile possibly partial -- is an
+  ordinary shorter sequence.  Each rank computes its rows' normalised outputs
+  and log-sum-exps (hpa_decode_step_lse); the ranks all-gather them
+  (B Hq (D + 1) fp32 per rank) and every rank combines them with the
+  log-sum-exp merge (hpa_merge_states) -- the split-KV recombination of
+  xiaodao.ai "HPC-Ops TPOT -48.8%" (Attention section) carried across GPUs.
 
-The split of pages and heads is host logic run when a cache is laid out;
-the per-step work runs in the library's kernels plus one collective.
+The page rule is stable under decode: a tile's rank depends only on its index
+and the sequence's start rank, so as a sequence grows no page that has been
+written ever changes rank, and each rank's page list only grows at its end.
+A new page goes to the rank after the one holding the previous tile, so
+every sequence stays spread within one tile of even, and start ranks that
+differ between sequences (by default s_b = b mod N) spread the batch's odd
+tiles over the ranks.  (Cutting each sequence into N contiguous runs would
+keep a rank's tokens contiguous, but every new page would shift the run
+boundaries and move written pages between ranks.)
+
+The split of pages and heads is host logic run when a cache is laid out and
+when a sequence gets a new page; the per-step work runs in the library's
+kernels plus one collective.
 """
 from __future__ import annotations
 
@@ -29,7 +41,7 @@ import torch
 from . import (HpaError, MAX_MERGE_STATES, MAX_STEP_BATCH, PAGE_SIZE, PagedDecoder,
                merge_states)
 
-__all__ = ["head_shard", "page_shard", "gather_states", "PageShardedDecoder"]
+__all__ = ["head_shard", "page_owner", "page_shard", "gather_states", "PageShardedDecoder"]
 
 
 def head_shard(num_q_heads: int, num_kv_heads: int, num_shards: int, shard: int):
@@ -47,13 +59,22 @@ def head_shard(num_q_heads: int, num_kv_heads: int, num_shards: int, shard: int)
     return (g0, g1), (g0 * G, g1 * G)
 
 
-def page_shard(seq_lens, page_table, num_shards: int, shard: int):
+def page_owner(tile, start, num_shards: int):
+    """Rank holding tile ``tile`` of a sequence whose start rank is ``start``
+    (scalars or arrays): (start + tile) mod num_shards."""
+    return (np.asarray(start, dtype=np.int64) + np.asarray(tile, dtype=np.int64)) % num_shards
+
+
+def page_shard(seq_lens, page_table, num_shards: int, shard: int, start=None):
     """(lens_r, page_table_r), int32 CPU tensors: rank ``shard``'s share of
-    every sequence when each sequence's n_b = ceil(L_b / 64) tiles are cut
-    into ``num_shards`` contiguous runs, run r = tiles [floor(r n_b / N),
-    floor((r+1) n_b / N)).  lens_r[b] counts the tokens of b in that run (the
-    last run ends at L_b); page_table_r[b] lists its pages first and keeps the
-    input's width (unused entries are 0 and never read)."""
+    every sequence when tile t of sequence b is held by rank
+    page_owner(t, start[b], N) = (start[b] + t) mod N.  ``start`` [B] gives
+    each sequence's start rank (default b mod N; keep it with the sequence
+    for as long as it lives).  page_table_r[b] lists the rank's pages in tile
+    order and keeps the input's width (unused entries are 0 and never read);
+    lens_r[b] counts the tokens in them: 64 per tile, less the unfilled part
+    of the sequence's last tile if the rank holds it (that tile is then last
+    in its list, so only a list's last page is ever partial)."""
     if num_shards < 1 or not 0 <= shard < num_shards:
         raise HpaError(f"page_shard: shard {shard} of {num_shards}")
     L = np.asarray(torch.as_tensor(seq_lens).cpu(), dtype=np.int64)
@@ -62,15 +83,21 @@ def page_shard(seq_lens, page_table, num_shards: int, shard: int):
         raise HpaError("page_shard: seq_lens [B] and page_table [B][pt_stride] expected")
     if (L < 0).any():
         raise HpaError("page_shard: negative length")
+    B = L.shape[0]
+    st = np.arange(B, dtype=np.int64) % num_shards if start is None else \
+        np.asarray(torch.as_tensor(start).cpu(), dtype=np.int64)
+    if st.shape != (B,) or (st < 0).any() or (st >= num_shards).any():
+        raise HpaError("page_shard: start ranks [B] in [0, num_shards) expected")
     n = (L + PAGE_SIZE - 1) // PAGE_SIZE
     if (n > pt.shape[1]).any():
         raise HpaError("page_shard: a sequence needs more pages than page_table holds")
-    t0 = (shard * n) // num_shards
-    t1 = ((shard + 1) * n) // num_shards
-    lens = np.clip(np.minimum(L, t1 * PAGE_SIZE) - t0 * PAGE_SIZE, 0, None)
+    first = (shard - st) % num_shards                      # this rank's first tile of b
+    count = np.where(n > first, (n - first + num_shards - 1) // num_shards, 0)
+    holds_last = (n > 0) & (page_owner(n - 1, st, num_shards) == shard)
+    lens = count * PAGE_SIZE - np.where(holds_last, n * PAGE_SIZE - L, 0)
     out = np.zeros_like(pt)
-    for b in range(L.shape[0]):
-        out[b, : t1[b] - t0[b]] = pt[b, t0[b]:t1[b]]
+    for b in range(B):
+        out[b, :count[b]] = pt[b, first[b]:n[b]:num_shards]
     return torch.from_numpy(lens.astype(np.int32)), torch.from_numpy(out)
 
 

@@ -375,3 +375,18 @@ def test_length_aware_workspace_equals_dynamic(L):
     for args in [(32, 8, 64, 128, 296), (1, 1, 8, 64, 7), (512, 8, 64, 128, 296)]:
         assert hpa.decode_workspace_size(3, *args) == hpa.decode_workspace_size(0, *args)
         assert hpa.workspace_layout(3, *args) == hpa.workspace_layout(0, *args)
+
+
+def test_read_cta_times_rejects_bad_arguments(L):
+    buf = (C.c_uint64 * 8)()
+    assert L.hpa_read_cta_times(None, 0, 2, 2, 8, 64, 2, buf, None) == 1
+    assert L.hpa_read_cta_times(256, 0, 2, 2, 8, 64, 2, None, None) == 1
+    assert L.hpa_read_cta_times(256, 0, 0, 2, 8, 64, 2, buf, None) == 1   # batch 0
+    assert L.hpa_read_cta_times(256, 9, 2, 2, 8, 64, 2, buf, None) == 1   # unknown kind
+
+
+def test_workspace_has_room_for_the_cta_trace(L):
+    # the trace region (grid x 4 uint64) sits after the partials
+    for grid in (1, 148, 296, 4864):
+        lay = hpa.workspace_layout(0, 32, 8, 64, 128, grid)
+        assert lay["total"] - lay["part_acc"] >= 2 * 5 * grid * 8 * 128 * 4 + grid * 32

@@ -837,3 +837,32 @@ def test_status_clean_on_normal_run():
     to_device(batch)
     _, ws, _ = gpu_decode(batch, return_ws=True)
     assert hpa.read_status(ws) == 0
+
+
+# ---------------------------------------------------------------- per-CTA trace
+
+@pytest.mark.parametrize("name,lens,kind", [
+    ("skewed_small", [8192] + [512] * 31, 0), ("uniform_small", [512] * 64, 0),
+    ("mixed", [1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7], 0),
+    ("mixed_static", [1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7], 1)])
+def test_cta_times_account_for_every_unit(name, lens, kind):
+    """hpa_read_cta_times: every CTA's stamps are ordered (start <= producer
+    done <= epilogue done, within one launch) and the units the CTAs report
+    streaming add up to the plan's units, each streamed once."""
+    batch = W.make_batch(W.DecodeShape(name, 64, 8, 128), lens, seed=5)
+    to_device(batch)
+    B, Hkv = batch.batch, 8
+    dec = hpa.PagedDecoder(B, 64, Hkv, 128, batch.pt_stride, kind=kind,
+                           max_seq_len=max(lens))
+    out = torch.empty(B, 64, 128, dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        dec.step(batch.q, batch.k_cache, batch.v_cache, batch.page_table, batch.seq_lens, out,
+                 1 / math.sqrt(128))
+    t = dec.cta_times()
+    assert t.shape == (dec.grid, 4)
+    assert torch.all(t[:, 0] <= t[:, 1]) and torch.all(t[:, 1] <= t[:, 2])
+    assert int(t[:, 2].max() - t[:, 0].min()) < 1_000_000_000  # one launch, not stale values
+    U = sum((L + 63) // 64 for L in lens) * Hkv
+    assert int(t[:, 3].sum()) == U
+    ti = hpa.tail_idle(t)
+    assert 0.0 <= ti["idle_fraction"] < 1.0 and ti["span_us"] > 0

@@ -60,17 +60,38 @@ def test_single_rank_is_the_identity():
     assert bench.job_throughput(2_000_000_000, 1, 0.5) == pytest.approx(4.0)
 
 
+def _host_case(batch, fp8=False):
+    from types import SimpleNamespace
+    s = batch.shape
+    return SimpleNamespace(batch=batch, fp8=fp8, prologue=s.prologue, Hkv=s.num_kv_heads,
+                           D=s.head_dim, k_scale=None, v_scale=None)
+
+
 def test_oracle_legs_are_time_bounded():
     """The CPU legs of the benchmark: the baseline repeats its sample until a
-    time floor is met; the reference arm sizes each step to a run budget."""
+    time floor is met (plain and prologue workloads); the reference arm sizes
+    each step to a run budget."""
     import bench
     from mixed_length_paged_b200 import workloads as W
-    batch = W.build("tiny")
-    host = bench._host_sample(batch, [0, 1])
-    gbs, secs, reps = bench._oracle_for(host, [0, 1], 0.05)
-    assert gbs > 0 and secs >= 0.05 and reps >= 1
+    leg = bench._cpu_leg(_host_case(W.build("tiny")), [0, 1], 0.05, "tiny")
+    assert leg["value"] > 0 and leg["seconds"] >= 0.05 and leg["cores"] >= 1
+    pro = W.make_batch(W.DecodeShape("p", 8, 2, 64, prologue=True), [10, 300, 64], seed=3)
+    leg = bench._cpu_leg(_host_case(pro), [0, 2], 0.05, "prologue sample")
+    assert leg["value"] > 0 and leg["kind"] == "oracle"
+    host = bench._host_sample(W.build("tiny"), [0, 1])
+    g, dt, toks = bench._cpu_baseline_sample(host, [0, 1])
+    assert g > 0 and toks == 237
     # one sequence per step when steps are many, all of them when few
     assert bench._reference_rows(10.0, 2000, 31) == 1
     assert bench._reference_rows(0.5, 4, 31) == 31
     n = bench._reference_rows(0.01, 2001, 31)
     assert n == 7 and n * 0.01 * 2001 <= bench.REF_BUDGET_SECONDS
+
+
+def test_percentile_and_config_samples():
+    import bench
+    assert bench._pct(list(range(1, 51)), 0.9) == 45
+    assert bench._pct([3.0], 0.9) == 3.0
+    assert bench._cpu_rows("fp8", 256)[0] == list(range(0, 256, 4))
+    assert bench._cpu_rows("uniform", 64)[0] == list(range(64))
+    assert bench.ClockSampler.summarize([None])["sm_mhz"] is None

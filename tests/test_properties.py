@@ -49,19 +49,26 @@ def test_length_aware_plan_properties(lens, Hkv, P, m):
 
 
 @settings(max_examples=60, deadline=None)
-@given(lens=lens_st, N=st.integers(1, 9), extra=st.integers(0, 3))
-def test_page_shard_properties(lens, N, extra):
+@given(lens=lens_st, N=st.integers(1, 9), extra=st.integers(0, 3), seed=st.integers(0, 99))
+def test_page_shard_properties(lens, N, extra, seed):
     L = np.array(lens, dtype=np.int32)
     pts = int((L.max() + 63) // 64) + extra + 1
     pt = np.arange(len(lens) * pts, dtype=np.int32).reshape(len(lens), pts)
-    shares = [SH.page_shard(torch.from_numpy(L), torch.from_numpy(pt), N, r) for r in range(N)]
+    start = np.random.default_rng(seed).integers(0, N, len(lens))
+    shares = [SH.page_shard(torch.from_numpy(L), torch.from_numpy(pt), N, r,
+                            start=torch.from_numpy(start)) for r in range(N)]
     np.testing.assert_array_equal(sum(s[0].numpy().astype(np.int64) for s in shares), L)
     for b in range(len(lens)):
-        got = []
-        for lr, ptr in shares:
+        n = (int(L[b]) + 63) // 64
+        got = {}
+        for r, (lr, ptr) in enumerate(shares):
             k = (int(lr[b]) + 63) // 64
-            got.extend(ptr.numpy()[b, :k].tolist())
-        assert got == pt[b, :(int(L[b]) + 63) // 64].tolist()
+            for p in ptr.numpy()[b, :k].tolist():
+                got[p] = r
+        # every page once, on the rank the rule names
+        assert sorted(got) == pt[b, :n].tolist()
+        for t in range(n):
+            assert got[int(pt[b, t])] == (int(start[b]) + t) % N
         sizes = [(int(lr[b]) + 63) // 64 for lr, _ in shares]
         assert max(sizes) - min(sizes) <= 1        # shares even to within a tile
 

@@ -107,30 +107,83 @@ def test_merge_states_special_cases():
 
 # ---------------------------------------------------------------- host logic
 
+def _tiles_by_rule(n, start, N):
+    """Tile t of a sequence of n tiles goes to rank (start + t) mod N: the
+    tiles of each rank, listed by walking the tiles once."""
+    held = [[] for _ in range(N)]
+    for t in range(n):
+        held[(start + t) % N].append(t)
+    return held
+
+
 @pytest.mark.parametrize("N", [1, 2, 3, 4, 8])
 def test_page_shard_covers_every_token_once(N):
     rng = np.random.default_rng(20 + N)
     lens = np.concatenate([[0, 1, 63, 64, 65, 128, 4096], rng.integers(0, 3000, 40)]).astype(np.int32)
     pts = int((lens.max() + 63) // 64) + 1
     pt = rng.permutation(len(lens) * pts).reshape(len(lens), pts).astype(np.int32)
-    shards = [SH.page_shard(torch.from_numpy(lens), torch.from_numpy(pt), N, r) for r in range(N)]
-    total = sum(s[0].numpy().astype(np.int64) for s in shards)
-    np.testing.assert_array_equal(total, lens)
-    for b, L in enumerate(lens):
-        n = (int(L) + 63) // 64
-        pages = []
-        for r, (lr, ptr) in enumerate(shards):
-            lr, ptr = int(lr[b]), ptr.numpy()
-            k = (lr + 63) // 64
-            assert ptr.shape == pt.shape
-            pages.extend(ptr[b, :k].tolist())
-            assert not ptr[b, k:].any()
-            # each rank holds floor((r+1) n / N) - floor(r n / N) tiles; all
-            # but the last tile of the sequence are full
-            assert k == ((r + 1) * n) // N - (r * n) // N
-            if ((r + 1) * n) // N < n:
-                assert lr == 64 * k
-        assert pages == pt[b, :n].tolist()
+    start = rng.integers(0, N, len(lens))
+    for st in (None, start):
+        shards = [SH.page_shard(torch.from_numpy(lens), torch.from_numpy(pt), N, r,
+                                start=None if st is None else torch.from_numpy(st))
+                  for r in range(N)]
+        total = sum(s[0].numpy().astype(np.int64) for s in shards)
+        np.testing.assert_array_equal(total, lens)
+        for b, L in enumerate(lens):
+            n = (int(L) + 63) // 64
+            held = _tiles_by_rule(n, b % N if st is None else int(st[b]), N)
+            for r, (lr, ptr) in enumerate(shards):
+                lr, ptr = int(lr[b]), ptr.numpy()
+                k = (lr + 63) // 64
+                assert ptr.shape == pt.shape
+                assert k == len(held[r])
+                assert ptr[b, :k].tolist() == [int(pt[b, t]) for t in held[r]]
+                assert not ptr[b, k:].any()
+                # every tile but the sequence's last is full
+                if n - 1 not in held[r]:
+                    assert lr == 64 * k
+                else:
+                    assert lr == 64 * (k - 1) + (int(L) - 64 * (n - 1))
+            # within one tile of even
+            sizes = [len(h) for h in held]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_page_shard_is_stable_as_sequences_grow():
+    """200 decode steps, every sequence growing by one token a step (crossing
+    page boundaries): no page that was written ever changes rank, and each
+    rank's page list at a step is a prefix of its list at the next step (so
+    its cache layout only grows at the end)."""
+    N = 3
+    rng = np.random.default_rng(5)
+    base = np.array([0, 1, 63, 64, 127, 300, 1000], dtype=np.int64)
+    steps = 200
+    final = base + steps
+    pts = int((final.max() + 63) // 64)
+    pt = rng.permutation(len(base) * pts).reshape(len(base), pts).astype(np.int32)
+    start = torch.from_numpy(rng.integers(0, N, len(base)))
+    owner, lists = {}, None
+    for s in range(steps + 1):
+        L = torch.from_numpy((base + s).astype(np.int32))
+        shares = [SH.page_shard(L, torch.from_numpy(pt), N, r, start=start) for r in range(N)]
+        now = []
+        for r, (lr, ptr) in enumerate(shares):
+            per_seq = []
+            for b in range(len(base)):
+                k = (int(lr[b]) + 63) // 64
+                pages = ptr.numpy()[b, :k].tolist()
+                per_seq.append(pages)
+                for p in pages:
+                    assert owner.setdefault(p, r) == r, (s, b, p)
+            now.append(per_seq)
+        if lists is not None:
+            for r in range(N):
+                for b in range(len(base)):
+                    prev = lists[r][b]
+                    assert now[r][b][:len(prev)] == prev, (s, r, b)
+        lists = now
+    # every page of the final lengths was handed out, each to one rank
+    assert len(owner) == int(((final + 63) // 64).sum())
 
 
 def test_page_shard_rejects_bad_input():
@@ -141,6 +194,10 @@ def test_page_shard_rejects_bad_input():
         SH.page_shard(torch.tensor([5]), pt, 2, 2)
     with pytest.raises(HpaError):
         SH.page_shard(torch.tensor([-1]), pt, 1, 0)
+    with pytest.raises(HpaError):
+        SH.page_shard(torch.tensor([5]), pt, 2, 0, start=torch.tensor([2]))  # start >= N
+    with pytest.raises(HpaError):
+        SH.page_shard(torch.tensor([5]), pt, 2, 0, start=torch.tensor([0, 1]))
 
 
 @pytest.mark.parametrize("N", [1, 2, 3, 5])
@@ -239,6 +296,76 @@ def test_two_gloo_ranks_page_sharded_decode_equals_whole():
     q = ctx.Queue()
     port = _free_port()
     procs = [ctx.Process(target=_gloo_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[0] for r in res] == [0, 1]
+    assert max(r[1] for r in res) <= 1e-12, res
+
+
+def _growing_worker(rank: int, world: int, port: int, q):
+    """Several decode steps on gloo ranks while the sequences grow across page
+    boundaries: each step, every rank takes its share by the stable page rule,
+    computes its states with the oracle, all-gathers them and merges; the
+    result must equal the whole-sequence oracle, and a rank's page list may
+    only grow at its end."""
+    import sys
+    from datetime import timedelta
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import oracle as O
+    from mixed_length_paged_b200 import sharding as S
+    from mixed_length_paged_b200 import workloads as WL
+    from tests.helpers import bits16 as b16
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        base = np.array([62, 127, 1, 190, 0, 63])
+        steps = 6
+        # the cache already holds every token the steps will reach
+        batch = WL.make_batch(WL.DecodeShape("g", 8, 2, 64), list(base + steps), seed=42)
+        qb, kc, vc = b16(batch.q), b16(batch.k_cache), b16(batch.v_cache)
+        pt = batch.page_table.numpy()
+        start = torch.tensor([1, 0, 1, 1, 0, 0])
+        err, prev = 0.0, None
+        for s in range(steps + 1):
+            L = torch.from_numpy((base + s).astype(np.int32))
+            lr, ptr = S.page_shard(L, batch.page_table, world, rank, start=start)
+            pages = [ptr.numpy()[b, :(int(lr[b]) + 63) // 64].tolist() for b in range(len(base))]
+            if prev is not None:
+                assert all(pages[b][:len(prev[b])] == prev[b] for b in range(len(base)))
+            prev = pages
+            o = torch.zeros(len(base), 8, 64, dtype=torch.float64)
+            lse = torch.full((len(base), 8), -math.inf, dtype=torch.float64)
+            for b in range(len(base)):
+                for h in range(8):
+                    ob, lb = O.attention_state(qb, kc, vc, ptr.numpy(), 2, 1 / 8, b, h, 0,
+                                               int(lr[b]))
+                    o[b, h] = torch.from_numpy(ob)
+                    lse[b, h] = lb
+            o_all, lse_all = S.gather_states(o, lse)
+            whole = O.paged_decode(qb, kc, vc, pt, L.numpy(), 2, 1 / 8)
+            for b in range(len(base)):
+                for h in range(8):
+                    m, _ = O.merge_states([x[b, h].numpy() for x in o_all],
+                                          [float(x[b, h]) for x in lse_all])
+                    err = max(err, float(np.abs(m - whole[b, h]).max()))
+        dist.barrier()
+        q.put((rank, err))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_page_sharded_decode_while_sequences_grow():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_growing_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=180) for _ in range(2))
