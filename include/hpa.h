@@ -153,9 +153,11 @@ HPA_API size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_
                                          int num_q_heads, int head_dim, int grid);
 
 /* Byte offsets of the workspace regions, for inspection by tests and tools:
- * offsets[0..6] = header (int32[16]: magic, status, units, grid, kind, batch,
+ * offsets[0..6] = header (int32[32]: magic, status, units, grid, kind, batch,
  * kv heads, group, head_dim, tiles, ranges V, next tail chunk, finished CTAs,
- * tail_den, tail_chunks (0, 0 for the static kinds), 0), lens,
+ * tail_den, tail_chunks (0, 0 for the static kinds), 0, split segments
+ * listed for the merge (two counts, by step parity), the step parity, then
+ * zeros), lens,
  * tile_start, range descriptors (int32 x8 per range: u_begin, u_end, then
  * the sequence, kv head, tile and tile count of its first unit, 0, 0),
  * segment descriptors (int32 x2 per (sequence, kv head): slot of its first
@@ -324,7 +326,10 @@ HPA_API hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, cons
  *                num_kv_heads, num_q_heads * q_tokens, head_dim, num_ctas)
  *                bytes, 256-byte aligned, zero-filled before its first use
  *                (or last written by hpa_decode_plan); every dynamic run
- *                leaves its run-time counters at zero for the next step.  The
+ *                leaves its run-time counters at zero for the next step, and
+ *                the merge empties the list of split segments the decode
+ *                kernel makes for it.  (After a call that returned
+ *                HPA_ERR_CUDA, zero the workspace or plan on it again.)  The
  *                plan fields of the header and the segment descriptors are
  *                written as hpa_decode_plan writes them; the range
  *                descriptors are not.  Status bits accumulate until a
@@ -498,7 +503,9 @@ HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const v
  * have no counterpart of this call; it exists for such integrations.
  *
  * Arguments are those of hpa_decode_plan + hpa_decode_run with the dynamic
- * plan; num_ctas = 0 means one CTA per SM.  Instead of a caller workspace the
+ * plan; num_ctas = 0 means one CTA per SM (the device's SM count: unlike
+ * hpa_default_num_ctas, the HPA_NUM_CTAS variable does not change it, since
+ * the CTA count sizes the scratch).  Instead of a caller workspace the
  * step uses a library-owned static device array of HPA_NOALLOC_SCRATCH_BYTES
  * (16 MiB), which every GPU that loads the library holds until the process
  * exits.  A step whose workspace would exceed it (see
@@ -514,7 +521,11 @@ HPA_API hpa_status hpa_kv_prologue(const void* q_raw, const void* k_raw, const v
  * hpa_decode_step does; beyond, hpa_decode_plan runs first) and leaves the
  * run-time counters at zero, so stale contents never reach a result, but
  * calls that overlap on the GPU (unordered streams) race on the array.  The
- * device status word of the array is not exposed.
+ * array's address is cached per device for the life of the process: calls
+ * must not cross a cudaDeviceReset (or any other end of the device's primary
+ * context).  Device-side problems (a page id out of range, a clamped length,
+ * a timed-out wait) set bits in the array's status word, read with
+ * hpa_noalloc_read_status.
  */
 #define HPA_NOALLOC_SCRATCH_BYTES (16u << 20)
 HPA_API hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
@@ -524,6 +535,15 @@ HPA_API hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, const 
                                       void* out, hpa_out_dtype out_dtype, int batch,
                                       int num_q_heads, int num_kv_heads, int head_dim,
                                       float softmax_scale, int num_ctas, void* stream);
+
+/* The status word (HPA_DEVICE_* bits) of hpa_decode_noalloc's static array on
+ * the current device, copied to *status_out (host) after the work queued on
+ * `stream` so far; with clear != 0 the word is then reset to 0 (in stream
+ * order).  The bits of every call accumulate until cleared, except that a
+ * call of more than 512 sequences starts by rewriting the word with its own
+ * plan's bits.  Synchronises the stream; allocates nothing.  The first call
+ * on a device does the array set-up described at hpa_decode_noalloc. */
+HPA_API hpa_status hpa_noalloc_read_status(int32_t* status_out, int clear, void* stream);
 
 /* Copies the device status word of a plan's workspace to *status_out (host)
  * after the work queued on `stream` so far; synchronises the stream. */

@@ -33,7 +33,7 @@ __all__ = [
     "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run",
     "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
     "decode_run_prologue",
-    "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "kv_prologue", "read_status", "PagedDecoder", "version", "decode_noalloc", "noalloc_read_status", "NOALLOC_SCRATCH_BYTES",
     "merge_states", "MAX_MERGE_STATES", "read_cta_times", "tail_idle",
 ]
 
@@ -122,6 +122,8 @@ def lib():
         L.hpa_decode_noalloc.restype = _I
         L.hpa_decode_noalloc.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _V, _I, _I, _I,
                                          _I, _I, _F, _I, _V]
+        L.hpa_noalloc_read_status.restype = _I
+        L.hpa_noalloc_read_status.argtypes = [C.POINTER(C.c_int32), _I, _V]
         L.hpa_read_cta_times.restype = _I
         L.hpa_read_cta_times.argtypes = [_V, _I, _I, _I, _I, _I, _I, _V, _V]
         L.hpa_read_status.restype = _I
@@ -526,6 +528,20 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     _dev(page_table, "page_table", (torch.int32,), 2)
     _dev(seq_lens, "seq_lens", (torch.int32,), 1)
     _dev(out, "out", (torch.bfloat16, torch.float32), 3)
+    if fp8:
+        if k_scale is None or v_scale is None:
+            raise HpaError("FP8 caches need k_scale and v_scale")
+        _dev(k_scale, "k_scale", (torch.float32,), 2)
+        _dev(v_scale, "v_scale", (torch.float32,), 2)
+    # the call uses the current device's scratch array and stream: every
+    # tensor must live on that device
+    cur = torch.cuda.current_device()
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("page_table", page_table), ("seq_lens", seq_lens), ("out", out),
+                    ("k_scale", k_scale), ("v_scale", v_scale)):
+        if t is not None and t.device.index != cur:
+            raise HpaError(f"decode_noalloc: {name} is on {t.device}, the current device is "
+                           f"cuda:{cur}")
     B, Hq, D = q.shape
     num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
     rc = lib().hpa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
@@ -536,6 +552,16 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
                                   Hkv, D, float(softmax_scale), num_ctas, _stream(stream))
     _check(rc, "hpa_decode_noalloc")
     return out
+
+
+def noalloc_read_status(clear: bool = False, stream=None) -> int:
+    """Status word (DEVICE_* bits) of decode_noalloc's static array on the
+    current device (hpa_noalloc_read_status); ``clear`` resets it to 0
+    afterwards.  Synchronises the stream."""
+    v = C.c_int32(0)
+    _check(lib().hpa_noalloc_read_status(C.byref(v), int(bool(clear)), _stream(stream)),
+           "hpa_noalloc_read_status")
+    return int(v.value)
 
 
 def read_status(workspace: torch.Tensor, stream=None) -> int:

@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
   // the scan (behind q_ready)
   int32_t* s_ts = reinterpret_cast<int32_t*>(misc + C::kMisc);
   int* s_wsum = const_cast<int*>(s_flags) + 4;
+  volatile int* s_parity = s_flags + 10;  // in-kernel plan: step parity (after the warp sums)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -354,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
     if (threadIdx.x == 0) {
       s_ts[p.B] = T;
       *s_plan_ok = 1;
+      *s_parity = __ldcg(&p.ws.header[kHdrParity]) & 1;  // this step's merge-list count
     }
   } else if (threadIdx.x == 0) {
     const int32_t* h = p.ws.header;
@@ -598,6 +600,15 @@ __global__ void __launch_bounds__(kThreads, CPS)
         if (atomicAdd(&p.ws.header[kHdrDone], 1) == (int)gridDim.x - 1) {
           atomicExch(&p.ws.header[kHdrNext], 0);
           atomicExch(&p.ws.header[kHdrDone], 0);
+          if constexpr (FP) {
+            // The merge list: empty the previous step's count (its merge has
+            // finished: this kernel started after it) and flip the parity,
+            // so the next step appends there.  Every CTA read the parity
+            // before its producer started, so none reads the new value.
+            const int e = *s_parity;
+            atomicExch(&p.ws.header[kHdrListCount + (e ^ 1)], 0);
+            atomicExch(&p.ws.header[kHdrParity], e ^ 1);
+          }
         }
       }
     }
@@ -612,8 +623,21 @@ __global__ void __launch_bounds__(kThreads, CPS)
       // In-kernel plan: the segment descriptors the merge reads, shared out
       // over the CTAs, and (CTA 0) the plan fields of the header.
       const int S = p.B * p.Hkv;
-      for (int sg = blockIdx.x * 32 + lane; sg < S; sg += gridDim.x * 32)
-        p.ws.seg_desc[sg] = dyn_seg_desc(dg, ts, p.Hkv, sg);
+      // Each split segment (more than one piece) also goes on the merge
+      // list: one atomic per warp batch reserves its entries.
+      for (int sg0 = blockIdx.x * 32; sg0 < S; sg0 += gridDim.x * 32) {
+        const int sg = sg0 + lane;
+        const int2 sd = sg < S ? dyn_seg_desc(dg, ts, p.Hkv, sg) : make_int2(-1, 0);
+        if (sg < S) p.ws.seg_desc[sg] = sd;
+        const unsigned split = __ballot_sync(0xffffffffu, sd.y > 1);
+        if (split) {
+          int base = 0;
+          if (lane == 0) base = atomicAdd(&p.ws.header[kHdrListCount + *s_parity], __popc(split));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const int at = base + __popc(split & ((1u << lane) - 1u));
+          if (sd.y > 1 && at >= 0 && at < S) p.ws.mlist[at] = sg;  // (a stale count is flagged by the merge)
+        }
+      }
       if (blockIdx.x == 0 && lane == 0) {
         int32_t* h = p.ws.header;
         h[kHdrUnits] = (int32_t)dg.U;
@@ -1154,16 +1178,34 @@ struct MergeParams {
   int T, GT;                 // query tokens per sequence; rows per segment = G * T
 };
 
-template <int D, bool OUT_F32>
+// LIST: the plan was made inside the decode kernel, which also listed the
+// split segments (Ws::mlist, its count in the header under the step's
+// parity); only those are visited.  Otherwise every segment is.
+template <int D, bool OUT_F32, bool LIST>
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergeParams p) {
   constexpr int kVec = D / 32;                 // output elements per lane
   constexpr int kBatch = D == 128 ? 24 : 32;   // pieces loaded together (<= 32)
   pdl_wait();                                  // the partials of the decode kernel
   const int G = p.GT, lane = threadIdx.x & 31;  // rows per segment
-  const int jobs = p.S * G;
+  int nseg = p.S;
+  if constexpr (LIST) {
+    // the decode kernel before this merge flipped the parity on its way out
+    const int e = (__ldcg(&p.ws.header[kHdrParity]) & 1) ^ 1;
+    nseg = __ldcg(&p.ws.header[kHdrListCount + e]);
+    if (nseg < 0 || nseg > p.S) {
+      if (threadIdx.x == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
+      nseg = 0;
+    }
+  }
+  const int jobs = nseg * G;
   for (int job = blockIdx.x * kMergeWarps + (threadIdx.x >> 5); job < jobs;
        job += gridDim.x * kMergeWarps) {
-    const int s = job / G, h = job - s * G;
+    const int k = job / G, h = job - k * G;
+    const int s = LIST ? __ldcg(&p.ws.mlist[k]) : k;
+    if (s < 0 || s >= p.S) {
+      if (lane == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
+      continue;
+    }
     const int2 sd = __ldcg(&p.ws.seg_desc[s]);
     const int ns = sd.y;
     if (ns <= 1) continue;
@@ -1504,7 +1546,10 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   mp.slots = (int)(2 * plan_ranges_ll(kind, grid));
   cudaLaunchConfig_t cfg = {};
   const long long merge_ctas = ((long long)mp.S * GT + kMergeWarps - 1) / kMergeWarps;
-  cfg.gridDim = dim3((unsigned)std::min<long long>(merge_ctas, (long long)std::max(1, sms) * 16));
+  // with the split segments listed (in-kernel plan), fewer CTAs: most
+  // segments need no merge
+  const long long cap = (long long)std::max(1, sms) * (plan_lens ? 8 : 16);
+  cfg.gridDim = dim3((unsigned)std::min<long long>(merge_ctas, cap));
   cfg.blockDim = dim3(kMergeWarps * 32);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1513,12 +1558,21 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (head_dim == 128)
-    e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<128, true>, mp)
-            : cudaLaunchKernelEx(&cfg, merge_kernel<128, false>, mp);
-  else
-    e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<64, true>, mp)
-            : cudaLaunchKernelEx(&cfg, merge_kernel<64, false>, mp);
+  if (plan_lens) {
+    if (head_dim == 128)
+      e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<128, true, true>, mp)
+              : cudaLaunchKernelEx(&cfg, merge_kernel<128, false, true>, mp);
+    else
+      e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<64, true, true>, mp)
+              : cudaLaunchKernelEx(&cfg, merge_kernel<64, false, true>, mp);
+  } else {
+    if (head_dim == 128)
+      e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<128, true, false>, mp)
+              : cudaLaunchKernelEx(&cfg, merge_kernel<128, false, false>, mp);
+    else
+      e = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<64, true, false>, mp)
+              : cudaLaunchKernelEx(&cfg, merge_kernel<64, false, false>, mp);
+  }
   if (e != cudaSuccess) {
     set_cuda_error(e, "hpa_decode_run merge launch");
     return HPA_ERR_CUDA;

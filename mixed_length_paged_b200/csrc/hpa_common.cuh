@@ -18,8 +18,11 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
-//   header      int32[16]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next, done,
-//                          tail_den, tail_chunks
+//   header      int32[32]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next, done,
+//                          tail_den, tail_chunks, 0, split segments listed
+//                          (two counts, by step parity), the step parity (the
+//                          run-time counters sit in the header, at the same
+//                          offset for every layout)
 //   lens        int32[B]     clamped lengths
 //   tile_start  int32[B+1]   exclusive prefix sum of tiles per sequence
 //   cta_desc    int4[2*V]    per range v: (u_begin, u_end, b0, g0), (t0, n0,
@@ -31,6 +34,12 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 //   seg_desc    int2[B*Hkv]  per segment: (first partial slot, ranges holding
 //                            its units); a segment held by one range has no
 //                            partials.
+//   mlist       int32[B*Hkv] in-kernel plan: the ids of the split segments (in
+//                            no particular order; their count is in the
+//                            header); the merge kernel visits only them.  A
+//                            step appends to the count of its parity; its last
+//                            CTA zeroes the other count (the previous step's,
+//                            whose merge has finished) and flips the parity
 //   part_ml     float2[2V][G]     (m, l) of each partial, log2 units
 //   part_acc    float[2V][G][D]   un-normalised partial outputs
 //   trace       uint64[grid][4]   per run-kernel CTA: %globaltimer (ns) at its
@@ -51,7 +60,9 @@ enum HeaderField {
   kHdrDone = 12,    // in-kernel plan: CTAs of the current step that finished
   kHdrTailDen = 13,     // dynamic plans: the tail parameters the plan was made with
   kHdrTailChunks = 14,
-  kHdrWords = 16
+  kHdrListCount = 16,   // in-kernel plan: split segments on the merge list (2 words: by parity)
+  kHdrParity = 18,      // in-kernel plan: parity of the current step
+  kHdrWords = 32
 };
 
 // The dynamic plan gives each of its P persistent CTAs one primary range and
@@ -78,7 +89,7 @@ HPA_HD inline long long plan_ranges_ll(int kind, int grid) {
 }
 
 struct WsLayout {
-  size_t header, lens, tile_start, cta_desc, seg_desc, part_ml, part_acc, trace, total;
+  size_t header, lens, tile_start, cta_desc, seg_desc, mlist, part_ml, part_acc, trace, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -96,6 +107,7 @@ inline bool ws_layout(int kind, int B, int Hkv, int Hq, int D, int grid, WsLayou
   L->tile_start = off;  off = align256(off + (size_t(B) + 1) * 4);
   L->cta_desc = off;    off = align256(off + V * 32);
   L->seg_desc = off;    off = align256(off + S * 8);
+  L->mlist = off;       off = align256(off + S * 4);
   L->part_ml = off;     off = align256(off + slots * G * 8);
   L->part_acc = off;    off = align256(off + slots * G * size_t(D) * 4);
   L->trace = off;       off = align256(off + size_t(grid) * 32);
@@ -110,6 +122,7 @@ struct Ws {
   int32_t* tile_start;
   int4* cta_desc;
   int2* seg_desc;
+  int32_t* mlist;
   float2* part_ml;
   float* part_acc;
   unsigned long long* trace;
@@ -119,7 +132,8 @@ inline Ws ws_view(void* base, const WsLayout& L) {
   char* p = static_cast<char*>(base);
   return Ws{reinterpret_cast<int32_t*>(p + L.header), reinterpret_cast<int32_t*>(p + L.lens),
             reinterpret_cast<int32_t*>(p + L.tile_start), reinterpret_cast<int4*>(p + L.cta_desc),
-            reinterpret_cast<int2*>(p + L.seg_desc), reinterpret_cast<float2*>(p + L.part_ml),
+            reinterpret_cast<int2*>(p + L.seg_desc), reinterpret_cast<int32_t*>(p + L.mlist),
+            reinterpret_cast<float2*>(p + L.part_ml),
             reinterpret_cast<float*>(p + L.part_acc),
             reinterpret_cast<unsigned long long*>(p + L.trace)};
 }

@@ -115,10 +115,10 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
                                                 head_dim, ctas);
   if (need == 0) return HPA_ERR_INVALID_ARG;
   if (need > HPA_NOALLOC_SCRATCH_BYTES) return HPA_ERR_WORKSPACE;
-  // Up to 512 sequences the plan is made inside the decode kernel (the
-  // static array starts zero-filled, and every dynamic run leaves its
-  // run-time counters at zero); larger batches take the plan kernel.
-  if (batch <= 512)
+  // Up to kMaxFusedBatch (512) sequences the plan is made inside the decode
+  // kernel (the static array starts zero-filled, and every dynamic run leaves
+  // its run-time counters at zero); larger batches take the plan kernel.
+  if (batch <= hpa::kMaxFusedBatch)
     return hpa_decode_step(seq_lens, q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table,
                            pt_stride, num_pages, out, out_dtype, batch, 1, num_q_heads,
                            num_kv_heads, head_dim, softmax_scale, ctas, scratch,
@@ -132,4 +132,22 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
                         num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,
                         softmax_scale, HPA_PLAN_DYNAMIC, grid, scratch,
                         HPA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" hpa_status hpa_noalloc_read_status(int32_t* status_out, int clear, void* stream) {
+  if (!status_out) return HPA_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  void* scratch = nullptr;
+  hpa_status st = device_setup(&dev, &scratch, &sms);
+  if (st != HPA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* word = static_cast<int32_t*>(scratch) + hpa::kHdrStatus;
+  cudaError_t e = cudaMemcpyAsync(status_out, word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(word, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    hpa::set_cuda_error(e, "hpa_noalloc_read_status");
+    return HPA_ERR_CUDA;
+  }
+  return HPA_OK;
 }

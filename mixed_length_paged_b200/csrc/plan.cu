@@ -182,6 +182,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrRanges] = (int32_t)V;
     h[kHdrNext] = 0;
     h[kHdrDone] = 0;
+    h[kHdrListCount] = 0;  // the in-kernel plan's merge list starts empty
+    h[kHdrListCount + 1] = 0;
+    h[kHdrParity] = 0;
     h[kHdrTailDen] = dyn ? p.tail_den : 0;
     h[kHdrTailChunks] = dyn ? p.tail_chunks : 0;
     // (no fence before the magic word: the run kernel reads the plan only
