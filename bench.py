@@ -73,6 +73,9 @@ def _args():
                          "page-sharded shares, separate prologue) and the e2e leg")
     ap.add_argument("--no-workloads", action="store_true",
                     help="measure the headline workload only (no per-configuration records)")
+    ap.add_argument("--ncu", action="store_true",
+                    help="profiler mode: run --warmup then --steps eager steps of --workload and "
+                         "exit (no timing, no JSON line), so a capture sees only decode steps")
     return ap.parse_args()
 
 
@@ -865,6 +868,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # 1. the headline workload: its record, then K back-to-back steps (the value)
     case = Case(args.workload, dev, args.num_ctas, local_rank)
+    if args.ncu:
+        for _ in range(args.warmup + args.steps):
+            case.step()
+        torch.cuda.synchronize()
+        print(f"ncu mode: {args.warmup + args.steps} steps of {case.name}, device status "
+              f"{case.dec.status()}", flush=True)
+        return
     rec, step = measure_case(case, args, world, dev, stream, peak, clock_rows, headline=True)
     K = args.steps
     barrier()
