@@ -446,7 +446,14 @@ HPA_API hpa_status hpa_decode_step_lse(const int32_t* seq_lens, const void* q,
  *                [rows][head_dim], 16-byte aligned (hpa_decode_step_lse with
  *                HPA_OUT_F32).  A pointer may address a peer GPU's memory
  *                mapped into the current context: the kernel reads it with
- *                plain global loads.
+ *                plain global loads.  Every buffer (states, out, lse_out) must
+ *                be reachable from the current device -- its own memory,
+ *                managed memory, mapped pinned host memory, or a peer's
+ *                memory with peer access enabled; a pageable host pointer or
+ *                an unknown address returns HPA_ERR_INVALID_ARG (a failed
+ *                driver query, HPA_ERR_CUDA) before anything is enqueued.  The
+ *                check is a driver query per new pointer, remembered per host
+ *                thread; it cannot tell whether peer access was enabled.
  *   lse_parts    HOST array of num_states device pointers, each fp32 [rows].
  *   num_states   1 .. 16 (HPA_ERR_UNSUPPORTED beyond).
  *   rows         >= 0; 0 enqueues nothing.

@@ -116,6 +116,53 @@ int device_sms() {
   return n;
 }
 
+// Whether this device's kernels can reach `ptr`, as far as the driver can
+// tell: memory of the current device, managed memory, pinned host memory
+// mapped into the address space, or memory of a peer device this one can
+// access (the caller must have enabled that access).  A pageable host pointer
+// or an address the driver does not know is refused.  Pointers found
+// reachable are remembered per host thread (the same state buffers come back
+// every step), so a step pays the driver query once.
+hpa_status check_reachable(const void* ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_cuda_error(e, "hpa_merge_states cudaGetDevice");
+    return HPA_ERR_CUDA;
+  }
+  constexpr int kSeen = 64;
+  thread_local const void* seen[kSeen] = {};
+  thread_local int seen_dev[kSeen] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kSeen; ++i)
+    if (seen[i] == ptr && seen_dev[i] == dev) return HPA_OK;
+  cudaPointerAttributes a;
+  e = cudaPointerGetAttributes(&a, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    set_cuda_error(e, "hpa_merge_states cudaPointerGetAttributes");
+    return HPA_ERR_CUDA;
+  }
+  bool ok = false;
+  if (a.type == cudaMemoryTypeManaged) {
+    ok = true;
+  } else if (a.type == cudaMemoryTypeHost) {
+    ok = a.devicePointer == ptr;  // mapped pinned memory at the same address
+  } else if (a.type == cudaMemoryTypeDevice) {
+    int can = a.device == dev;
+    if (!can && cudaDeviceCanAccessPeer(&can, dev, a.device) != cudaSuccess) {
+      cudaGetLastError();
+      can = 0;
+    }
+    ok = can != 0;
+  }
+  if (!ok) return HPA_ERR_INVALID_ARG;
+  seen[next] = ptr;
+  seen_dev[next] = dev;
+  next = (next + 1) % kSeen;
+  return HPA_OK;
+}
+
 }  // namespace
 }  // namespace hpa
 
@@ -141,6 +188,18 @@ extern "C" hpa_status hpa_merge_states(const float* const* o_parts, const float*
   if (reinterpret_cast<uintptr_t>(out) & (f32 ? 15 : 7)) return HPA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(lse_out) & 3) return HPA_ERR_INVALID_ARG;
   if (rows == 0) return HPA_OK;
+  // every buffer must be reachable from this device before anything is
+  // enqueued (a pageable host pointer would fault the kernel)
+  for (int i = 0; i < num_states; ++i)
+    for (const void* q : {static_cast<const void*>(o_parts[i]), static_cast<const void*>(lse_parts[i])}) {
+      const hpa_status st = check_reachable(q);
+      if (st != HPA_OK) return st;
+    }
+  for (const void* q : {static_cast<const void*>(out), static_cast<const void*>(lse_out)}) {
+    if (!q) continue;
+    const hpa_status st = check_reachable(q);
+    if (st != HPA_OK) return st;
+  }
   p.n = num_states;
   p.rows = rows;
   p.out = out;

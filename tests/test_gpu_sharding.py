@@ -272,3 +272,31 @@ def test_page_sharded_skewed_workload_full_size():
     ref = oracle_decode(compact_rows(batch, rows))
     mx, mn = errors(out[rows], ref)
     assert mx <= MAX_ABS and mn <= MEAN_ABS, (mx, mn)
+
+
+def test_merge_states_refuses_unreachable_pointers():
+    """A pageable host buffer passed as a state or as the output is refused
+    on the host with HPA_ERR_INVALID_ARG and nothing is launched; device and
+    mapped pinned buffers are accepted."""
+    import ctypes as C
+    rows, D = 8, 64
+    o = torch.randn(rows, D, device="cuda")
+    lse = torch.randn(rows, device="cuda")
+    out = torch.empty(rows, D, device="cuda")
+    host_o = torch.randn(rows, D)                       # pageable host memory
+    host_out = torch.empty(rows, D)
+    L = hpa.lib()
+
+    def call(o_ptrs, lse_ptrs, out_ptr):
+        op = (C.c_void_p * len(o_ptrs))(*o_ptrs)
+        lp = (C.c_void_p * len(lse_ptrs))(*lse_ptrs)
+        return L.hpa_merge_states(op, lp, len(o_ptrs), rows, D, out_ptr, 1, None, None)
+
+    assert call([o.data_ptr(), host_o.data_ptr()], [lse.data_ptr()] * 2, out.data_ptr()) == 1
+    assert call([o.data_ptr()], [lse.data_ptr()], host_out.data_ptr()) == 1
+    pinned = torch.randn(rows, D).pin_memory()
+    assert call([o.data_ptr(), pinned.data_ptr()], [lse.data_ptr()] * 2, out.data_ptr()) == 0
+    torch.cuda.synchronize()
+    assert call([o.data_ptr()], [lse.data_ptr()], out.data_ptr()) == 0
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy(), o.cpu().numpy())  # one state: identity
