@@ -259,7 +259,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
   using C = Cfg<D, NT, FP8, CPS, PRO, FP>;
   static_assert(!(PRO && FP8), "the fused prologue writes bf16 caches");
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned in the shared window (the 128-byte swizzle needs it),
+  // derived by offsetting smem_raw so that every pointer below stays a
+  // shared-memory pointer to the compiler
+  const uint32_t smem_raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((smem_raw_s + 1023u) & ~1023u) - smem_raw_s);
   uint8_t* stages = smem;
   uint8_t* qslots = smem + C::kStages * C::kStageBytes;
   uint8_t* deps = qslots + C::kStages * C::kSlotBytes;  // kDepBufs deposit slots
@@ -845,14 +849,18 @@ __global__ void __launch_bounds__(kThreads, CPS)
         ldsm_x4_t(vb + voff[ip], r0, r1, r2, r3);
         // r0/r1: tokens [0,8)/[8,16) of chunk 2ip; r2/r3: same for chunk 2ip+1.
         // Each holds bytes {V(t,d), V(t,d+1), V(t+1,d), V(t+1,d+1)}.
-        va[2 * ip][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0020));
-        va[2 * ip][1] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r0, 0, 0x0031));
-        va[2 * ip][2] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r1, 0, 0x0020));
-        va[2 * ip][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r1, 0, 0x0031));
-        va[2 * ip + 1][0] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r2, 0, 0x0020));
-        va[2 * ip + 1][1] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r2, 0, 0x0031));
-        va[2 * ip + 1][2] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0020));
-        va[2 * ip + 1][3] = e4m3x2_to_f16x2((uint16_t)__byte_perm(r3, 0, 0x0031));
+        // one byte permutation per register: {b0, b2} in the low half, {b1, b3}
+        // in the high half
+        const uint32_t t0 = __byte_perm(r0, 0, 0x3120), t1 = __byte_perm(r1, 0, 0x3120);
+        const uint32_t t2 = __byte_perm(r2, 0, 0x3120), t3 = __byte_perm(r3, 0, 0x3120);
+        va[2 * ip][0] = e4m3x2_to_f16x2((uint16_t)(t0 & 0xffffu));
+        va[2 * ip][1] = e4m3x2_to_f16x2((uint16_t)(t0 >> 16));
+        va[2 * ip][2] = e4m3x2_to_f16x2((uint16_t)(t1 & 0xffffu));
+        va[2 * ip][3] = e4m3x2_to_f16x2((uint16_t)(t1 >> 16));
+        va[2 * ip + 1][0] = e4m3x2_to_f16x2((uint16_t)(t2 & 0xffffu));
+        va[2 * ip + 1][1] = e4m3x2_to_f16x2((uint16_t)(t2 >> 16));
+        va[2 * ip + 1][2] = e4m3x2_to_f16x2((uint16_t)(t3 & 0xffffu));
+        va[2 * ip + 1][3] = e4m3x2_to_f16x2((uint16_t)(t3 >> 16));
       }
     }
   };
