@@ -491,11 +491,22 @@ def _time_iters(fn, n, stream, flush=None):
     return [a.elapsed_time(b) for a, b in evs]
 
 
+class ABTotals(dict):
+    """Total ms per side of an interleaved A/B, with each block's mean step
+    time (us) per side in `.blocks` for the spread."""
+
+    def spread(self, k):
+        xs = sorted(self.blocks[k])
+        return {"block_median_us": statistics.median(xs), "block_p90_us": _pct(xs, 0.9),
+                "block_min_us": xs[0], "block_max_us": xs[-1]}
+
+
 def _interleaved_ab(fns, stream, blocks=AB_BLOCKS, per=AB_PER):
     """Total ms of each function over `blocks` alternating blocks of `per`
     calls, so that clock and power drift over the run falls on all alike."""
     import torch
-    tot = {k: 0.0 for k in fns}
+    tot = ABTotals({k: 0.0 for k in fns})
+    tot.blocks = {k: [] for k in fns}
     for _ in range(blocks):
         for k, fn in fns.items():
             a = torch.cuda.Event(enable_timing=True)
@@ -505,7 +516,9 @@ def _interleaved_ab(fns, stream, blocks=AB_BLOCKS, per=AB_PER):
                 fn()
             b.record(stream)
             torch.cuda.synchronize()
-            tot[k] += a.elapsed_time(b)
+            ms = a.elapsed_time(b)
+            tot[k] += ms
+            tot.blocks[k].append(1e3 * ms / per)
     return tot
 
 
@@ -719,6 +732,7 @@ def measure_case(case, args, world, dev, stream, peak, sampler_rows, headline):
                 "us_per_step": 1e3 * tot["static"] / n, "grid": sd.grid,
                 "dynamic_us_per_step_same_blocks": 1e3 * tot["dynamic"] / n,
                 "dynamic_speedup": tot["static"] / tot["dynamic"],
+                "static_blocks": tot.spread("static"), "dynamic_blocks": tot.spread("dynamic"),
                 "method": f"interleaved A/B, {AB_BLOCKS} x {AB_PER} graph replays each, no flush"}
             del s_graph
         rec["static_splitkv"]["dynamic_speedup_vs_best_static"] = min(
@@ -765,6 +779,7 @@ def _headline_extras(case, args, world, dev, stream, step):
             "us_per_step": 1e3 * ab["plan_run"] / n,
             "in_kernel_plan_us_per_step_same_blocks": 1e3 * ab["step"] / n,
             "in_kernel_plan_speedup": ab["plan_run"] / ab["step"],
+            "plan_run_blocks": ab.spread("plan_run"), "step_blocks": ab.spread("step"),
             "method": f"interleaved A/B, {blocks} x {per} steps each"}
         # the length-aware plan (cut points moved off segment ends, smallest
         # end piece m tiles) against the dynamic plan, both as plan kernel + run
@@ -784,6 +799,7 @@ def _headline_extras(case, args, world, dev, stream, step):
                 "us_per_step": 1e3 * ab["length_aware"] / n,
                 "dynamic_plan_run_us_same_blocks": 1e3 * ab["dynamic"] / n,
                 "speedup_vs_dynamic": ab["dynamic"] / ab["length_aware"],
+                "length_aware_blocks": ab.spread("length_aware"),
                 "method": f"plan kernel + run each, interleaved A/B, {blocks} x {per} steps"}
     if case.prologue:
         # the prologue as its own kernel before plan + run, against the fused step
@@ -804,6 +820,7 @@ def _headline_extras(case, args, world, dev, stream, step):
             "us_per_step": 1e3 * ab["separate"] / n,
             "fused_us_per_step_same_blocks": 1e3 * ab["fused"] / n,
             "fused_speedup": ab["separate"] / ab["fused"],
+            "separate_blocks": ab.spread("separate"), "fused_blocks": ab.spread("fused"),
             "method": f"interleaved A/B, {blocks} x {per} steps each"}
     if case.use_step and not case.prologue and not case.fp8 and case.T == 1:
         # The batch spread by page range over R ranks (sharding.page_shard),

@@ -95,3 +95,12 @@ def test_percentile_and_config_samples():
     assert bench._cpu_rows("fp8", 256)[0] == list(range(0, 256, 4))
     assert bench._cpu_rows("uniform", 64)[0] == list(range(64))
     assert bench.ClockSampler.summarize([None])["sm_mhz"] is None
+
+
+def test_ab_spread_summary():
+    import bench
+    t = bench.ABTotals({"x": 0.0})
+    t.blocks = {"x": [5.0, 1.0, 4.0, 2.0, 3.0]}
+    sp = t.spread("x")
+    assert sp == {"block_median_us": 3.0, "block_p90_us": 5.0, "block_min_us": 1.0,
+                  "block_max_us": 5.0}
