@@ -866,3 +866,73 @@ def test_cta_times_account_for_every_unit(name, lens, kind):
     assert int(t[:, 3].sum()) == U
     ti = hpa.tail_idle(t)
     assert 0.0 <= ti["idle_fraction"] < 1.0 and ti["span_us"] > 0
+
+
+# ---------------------------------------------------------------- random sweep
+
+def _random_case(seed):
+    rng = np.random.default_rng(1000 + seed)
+    D = int(rng.choice([64, 128]))
+    fp8 = D == 128 and rng.random() < 0.3
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.integers(1, 17))
+    T = int(rng.integers(1, 16 // G + 1)) if rng.random() < 0.4 else 1
+    B = int(rng.integers(1, 12))
+    lens = [int(x) for x in rng.choice([0, 1, 63, 64, 65, 127, 129, 700, 2000, 5000], B)]
+    lens = [L + int(rng.integers(0, 3)) for L in lens]
+    lens = [max(L, T) if rng.random() < 0.9 else L for L in lens]
+    kind = int(rng.choice([0, 0, 1, 2, 3]))
+    param = int(rng.integers(0, 5)) if kind else 0
+    tail = [(8, 4), (0, 1), (3, 2), (16, 4)][int(rng.integers(0, 4))] if kind in (0, 3) else None
+    num_ctas = int(rng.choice([1, 5, 37, 148, 296]))
+    out_dtype = torch.float32 if rng.random() < 0.5 else torch.bfloat16
+    return dict(D=D, fp8=fp8, Hkv=Hkv, G=G, T=T, lens=lens, kind=kind, param=param, tail=tail,
+                num_ctas=num_ctas, out_dtype=out_dtype)
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_configurations_match_oracle(seed):
+    """Seeded random shapes through plan + run (plan kinds, tail shapes, CTA
+    counts, group sizes 1..16, head_dim 64/128, 1..16 query tokens per
+    sequence, bf16 or FP8 KV, bf16 or fp32 output) against the oracle."""
+    c = _random_case(seed)
+    D, Hkv, G, T = c["D"], c["Hkv"], c["G"], c["T"]
+    Hq = G * Hkv
+    shape = W.DecodeShape(f"rnd{seed}", Hq, Hkv, D, kv_dtype="fp8_e4m3" if c["fp8"] else "bf16",
+                          q_tokens=T)
+    batch = W.make_batch(shape, c["lens"], seed=2000 + seed)
+    fp8 = quantize_fp8(batch) if c["fp8"] else None
+    if T == 1:
+        ref = oracle_decode(batch, fp8=fp8)
+    else:
+        kc, vc = (bits16(batch.k_cache), bits16(batch.v_cache)) if fp8 is None else (fp8[0], fp8[2])
+        kw = {} if fp8 is None else dict(kv_fp8=True, k_scale=fp8[1], v_scale=fp8[3])
+        ref = oracle.paged_decode_multi(bits16(batch.q), kc, vc, batch.page_table.numpy(),
+                                        batch.seq_lens.numpy(), Hkv, 1 / math.sqrt(D), **kw)
+    to_device(batch)
+    B = batch.batch
+    maxlen = max(max(c["lens"]), 1)
+    grid = hpa.plan_grid(c["kind"], B, Hkv, c["num_ctas"], c["param"], maxlen)
+    ws = torch.zeros(hpa.decode_workspace_size(c["kind"], B, Hkv, Hq * T, D, grid),
+                     dtype=torch.uint8, device="cuda")
+    g = hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq * T, head_dim=D,
+                        pt_stride=batch.pt_stride, workspace=ws, kind=c["kind"],
+                        num_ctas=c["num_ctas"], param=c["param"], max_seq_len=maxlen,
+                        tail=c["tail"])
+    out = torch.full(batch.q.shape, float("nan"), dtype=c["out_dtype"], device="cuda")
+    kw = {}
+    kc, vc = batch.k_cache, batch.v_cache
+    if fp8 is not None:
+        kc, ks, vc, vs = (torch.from_numpy(x).cuda() for x in fp8)
+        kw = dict(k_scale=ks, v_scale=vs)
+    if T == 1:
+        hpa.decode_run(batch.q, kc, vc, batch.page_table, out, ws, g, 1 / math.sqrt(D),
+                       kind=c["kind"], **kw)
+    else:
+        hpa.decode_run_multi(batch.q, kc, vc, batch.page_table, out, ws, g, 1 / math.sqrt(D),
+                             kind=c["kind"], **kw)
+    torch.cuda.synchronize()
+    assert hpa.read_status(ws) == 0, c
+    assert torch.isfinite(out.float()).all(), c
+    mx, mn = errors(out, ref)
+    assert mx <= (FP8_MAX_ABS if fp8 is not None else MAX_ABS) and mn <= MEAN_ABS, (c, mx, mn)
