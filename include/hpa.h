@@ -97,17 +97,22 @@ typedef enum {
 } hpa_plan_kind;
 
 /* Shape of the run-time tail of the DYNAMIC and LENGTH_AWARE plans (see
- * hpa_decode_plan): the last Ut = min(floor(U / tail_den), U - P) units
- * (none if tail_den = 0) are cut into M = min(tail_chunks * P, Ut) chunks.
+ * hpa_decode_plan), for U units over P persistent CTAs: if tail_den > 0 and
+ * U >= tail_min * P, the last Ut = min(floor(U / tail_den), U - P) units are
+ * cut into M = min(tail_chunks * P, Ut) chunks; otherwise there is no tail.
  * These are this library's tuning choices, not part of the method: the pages
  * fix only that the global tile list is spread as evenly as possible over the
- * persistent CTAs, which every (tail_den, tail_chunks) does, and tail_den = 0
- * is that even spread with nothing left to run time.  hpa_decode_plan, the
- * in-kernel plans (hpa_decode_step*) and hpa_decode_noalloc use the defaults;
- * hpa_decode_plan_tail takes both as arguments.  HPA_TAIL_CHUNKS_MAX bounds
- * tail_chunks (the workspace has room for that many chunks per CTA). */
+ * persistent CTAs, which every shape does, and no tail is that even spread
+ * with nothing left to run time.  A tail evens out the CTAs' unequal shares
+ * of HBM bandwidth, which matters once each CTA streams many tiles; on a
+ * batch of a few tiles per CTA its one-tile chunks cost more in partials and
+ * merge work than they save, hence tail_min.  hpa_decode_plan, the in-kernel
+ * plans (hpa_decode_step*) and hpa_decode_noalloc use the defaults;
+ * hpa_decode_plan_tail takes all three as arguments.  HPA_TAIL_CHUNKS_MAX
+ * bounds tail_chunks (the workspace has room for that many chunks per CTA). */
 #define HPA_TAIL_DEN_DEFAULT 8
 #define HPA_TAIL_CHUNKS_DEFAULT 4
+#define HPA_TAIL_MIN_DEFAULT 32
 #define HPA_TAIL_CHUNKS_MAX 4
 
 /* Bits of the device status word (hpa_read_status). */
@@ -155,7 +160,7 @@ HPA_API size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_
 /* Byte offsets of the workspace regions, for inspection by tests and tools:
  * offsets[0..6] = header (int32[32]: magic, status, units, grid, kind, batch,
  * kv heads, group, head_dim, tiles, ranges V, next tail chunk, finished CTAs,
- * tail_den, tail_chunks (0, 0 for the static kinds), 0, split segments
+ * tail_den, tail_chunks, tail_min (0 for the static kinds), split segments
  * listed for the merge (two counts, by step parity), the step parity, then
  * zeros), lens,
  * tile_start, range descriptors (int32 x8 per range: u_begin, u_end, then
@@ -178,7 +183,7 @@ HPA_API hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_k
  * and the plan cuts it into contiguous ranges.  DYNAMIC (P = num_ctas
  * persistent CTAs, U units): if U <= P, CTA c < U takes unit c; otherwise the
  * last Ut units (Ut from the tail shape above: min(floor(U/8), U - P) by
- * default) form M tail chunks (min(4P, Ut) by default)
+ * default when U >= 32 P, else 0) form M tail chunks (min(4P, Ut) by default)
  * [U1 + floor(jUt/M), U1 + floor((j+1)Ut/M)) and the first U1 = U - Ut units
  * the P primary ranges [floor(cU1/P), floor((c+1)U1/P)).  CTA c runs primary
  * range c, then takes tail chunks in order from a counter as it finishes, so
@@ -228,17 +233,20 @@ HPA_API hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int num_k
  *                partition of all U units).
  *   tail_chunks  1 .. HPA_TAIL_CHUNKS_MAX: the tail is cut into
  *                min(tail_chunks * P, Ut) chunks (ignored if the tail is empty).
+ *   tail_min     0 .. 2^20: no tail unless U >= tail_min * P.
  *   the rest     as for hpa_decode_plan (max_seq_len is not needed).
  * Any other kind, or a parameter out of range, returns HPA_ERR_INVALID_ARG.
  * The workspace size and hpa_decode_run's arguments do not depend on the
  * tail shape.  hpa_decode_plan(kind, ...) equals hpa_decode_plan_tail(kind,
- * ..., HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT, ...).
+ * ..., HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT, HPA_TAIL_MIN_DEFAULT,
+ * ...).
  */
 HPA_API hpa_status hpa_decode_plan_tail(const int32_t* seq_lens, int batch, int num_kv_heads,
                                         int num_q_heads, int head_dim, int pt_stride,
                                         hpa_plan_kind kind, int num_ctas, int param,
-                                        int tail_den, int tail_chunks, void* workspace,
-                                        size_t ws_bytes, int* grid_out, void* stream);
+                                        int tail_den, int tail_chunks, int tail_min,
+                                        void* workspace, size_t ws_bytes, int* grid_out,
+                                        void* stream);
 
 /*
  * hpa_decode_run -- persistent paged GQA decode attention with split-KV

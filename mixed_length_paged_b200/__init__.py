@@ -28,7 +28,7 @@ import torch
 __all__ = [
     "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
     "PLAN_STATIC_CHUNK", "PLAN_LENGTH_AWARE", "TAIL_DEN_DEFAULT", "TAIL_CHUNKS_DEFAULT",
-    "TAIL_CHUNKS_MAX", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
+    "TAIL_MIN_DEFAULT", "TAIL_CHUNKS_MAX", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
     "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run",
     "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
@@ -44,7 +44,7 @@ DEVICE_LEN_CLAMPED, DEVICE_BAD_PAGE, DEVICE_BAD_PLAN = 0x1, 0x2, 0x4
 DEVICE_BAD_POSITION, DEVICE_TIMEOUT = 0x8, 0x10
 PAGE_SIZE = 64
 # run-time tail of the dynamic plans (hpa.h: HPA_TAIL_DEN_DEFAULT, ...)
-TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT, TAIL_CHUNKS_MAX = 8, 4, 4
+TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT, TAIL_MIN_DEFAULT, TAIL_CHUNKS_MAX = 8, 4, 32, 4
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -94,8 +94,8 @@ def lib():
         L.hpa_decode_plan.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V, _Z,
                                       C.POINTER(_I), _V]
         L.hpa_decode_plan_tail.restype = _I
-        L.hpa_decode_plan_tail.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V, _Z,
-                                           C.POINTER(_I), _V]
+        L.hpa_decode_plan_tail.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V,
+                                           _Z, C.POINTER(_I), _V]
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
                                      _F, _I, _I, _V, _Z, _V]
@@ -212,12 +212,13 @@ def workspace_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid) -> 
 def decode_plan(seq_lens: torch.Tensor, *, num_kv_heads: int, num_q_heads: int, head_dim: int,
                 pt_stride: int, workspace: torch.Tensor, kind: int = PLAN_DYNAMIC,
                 num_ctas: int | None = None, param: int = 0, max_seq_len: int = 0,
-                tail: tuple[int, int] | None = None, stream=None) -> int:
+                tail: tuple[int, int, int] | None = None, stream=None) -> int:
     """Enqueue the tile plan; returns the grid to pass to decode_run.
 
-    ``tail = (tail_den, tail_chunks)`` sets the run-time tail of a DYNAMIC or
-    LENGTH_AWARE plan (hpa_decode_plan_tail; (0, 1): no tail); None keeps the
-    library's default (TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT)."""
+    ``tail = (tail_den, tail_chunks, tail_min)`` sets the run-time tail of a
+    DYNAMIC or LENGTH_AWARE plan (hpa_decode_plan_tail; (0, 1, 0): no tail);
+    None keeps the library's default (TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT,
+    TAIL_MIN_DEFAULT)."""
     _dev(seq_lens, "seq_lens", (torch.int32,), 1)
     _dev(workspace, "workspace", (torch.uint8,))
     if num_ctas is None:
@@ -226,7 +227,8 @@ def decode_plan(seq_lens: torch.Tensor, *, num_kv_heads: int, num_q_heads: int, 
     if tail is not None:
         rc = lib().hpa_decode_plan_tail(_ptr(seq_lens), seq_lens.shape[0], num_kv_heads,
                                         num_q_heads, head_dim, pt_stride, kind, num_ctas, param,
-                                        int(tail[0]), int(tail[1]), _ptr(workspace),
+                                        int(tail[0]), int(tail[1]), int(tail[2]),
+                                        _ptr(workspace),
                                         workspace.numel(), C.byref(grid), _stream(stream))
         _check(rc, "hpa_decode_plan_tail")
         return grid.value

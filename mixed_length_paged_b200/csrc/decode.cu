@@ -136,7 +136,7 @@ struct RunParams {
   int T, GT;                // query tokens per sequence; rows per kv head = G * T
   const int32_t* seq_lens;  // in-kernel plan: the step's lengths (else the plan's)
   int capacity;             // in-kernel plan: pt_stride * 64 tokens
-  int tail_den, tail_chunks;  // in-kernel plan: the run-time tail's shape
+  int tail_den, tail_chunks, tail_min;  // in-kernel plan: the run-time tail's shape
   float scale_log2;         // softmax_scale * log2(e)
   Ws ws;
   int grid, kind;
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
   DynGeom dg{};
   if constexpr (FP) {
     if (warp >= kConsumerWarps) {
-      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x, p.tail_den, p.tail_chunks);
+      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x, p.tail_den, p.tail_chunks, p.tail_min);
       double rc[4];
       dyn_reciprocals(dg, rc);
       dg.init_div(rc);
@@ -655,6 +655,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
         h[kHdrRanges] = (int32_t)dg.ranges();
         h[kHdrTailDen] = p.tail_den;
         h[kHdrTailChunks] = p.tail_chunks;
+        h[kHdrTailMin] = p.tail_min;
         h[kHdrMagic] = kPlanMagic;
       }
     }
@@ -1520,6 +1521,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.capacity = pt_stride * kPageSize;
   p.tail_den = HPA_TAIL_DEN_DEFAULT;
   p.tail_chunks = HPA_TAIL_CHUNKS_DEFAULT;
+  p.tail_min = HPA_TAIL_MIN_DEFAULT;
   const int nt = GT > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;

@@ -19,7 +19,7 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
 //   header      int32[32]: magic, status, U, grid, kind, B, Hkv, G, D, T, V, next, done,
-//                          tail_den, tail_chunks, 0, split segments listed
+//                          tail_den, tail_chunks, tail_min, split segments listed
 //                          (two counts, by step parity), the step parity (the
 //                          run-time counters sit in the header, at the same
 //                          offset for every layout)
@@ -60,6 +60,7 @@ enum HeaderField {
   kHdrDone = 12,    // in-kernel plan: CTAs of the current step that finished
   kHdrTailDen = 13,     // dynamic plans: the tail parameters the plan was made with
   kHdrTailChunks = 14,
+  kHdrTailMin = 15,
   kHdrListCount = 16,   // in-kernel plan: split segments on the merge list (2 words: by parity)
   kHdrParity = 18,      // in-kernel plan: parity of the current step
   kHdrWords = 32

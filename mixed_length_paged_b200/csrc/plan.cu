@@ -47,7 +47,7 @@ struct PlanParams {
   int B, Hkv, G, D, capacity;  // capacity = pt_stride * 64 tokens
   int kind, num_ctas, grid;
   long long chunk;             // STATIC_CHUNK: tiles per split; LENGTH_AWARE: smallest piece
-  int tail_den, tail_chunks;   // DYNAMIC / LENGTH_AWARE: the run-time tail's shape
+  int tail_den, tail_chunks, tail_min;  // DYNAMIC / LENGTH_AWARE: the run-time tail's shape
   Ws ws;
 };
 
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
   const bool la = p.kind == HPA_PLAN_LENGTH_AWARE;
   const int per = dyn ? 0 : p.grid / S;  // static: CTAs per segment
   DynGeom dg;
-  dg.init(U, p.num_ctas, p.tail_den, p.tail_chunks);
+  dg.init(U, p.num_ctas, p.tail_den, p.tail_chunks, p.tail_min);
   const LaGeom lg{&dg, ts, p.B, p.Hkv, la ? p.chunk : 1};
   if (tid < 4) {
     const long long d = dg.divisor(tid);
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrParity] = 0;
     h[kHdrTailDen] = dyn ? p.tail_den : 0;
     h[kHdrTailChunks] = dyn ? p.tail_chunks : 0;
+    h[kHdrTailMin] = dyn ? p.tail_min : 0;
     // (no fence before the magic word: the run kernel reads the plan only
     // after griddepcontrol.wait, i.e. after this whole grid has completed)
     h[kHdrMagic] = kPlanMagic;
@@ -212,8 +213,8 @@ namespace hpa {
 static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads,
                             int num_q_heads, int head_dim, int pt_stride, hpa_plan_kind kind,
                             int num_ctas, int param, int max_seq_len, int tail_den,
-                            int tail_chunks, void* workspace, size_t ws_bytes, int* grid_out,
-                            void* stream) {
+                            int tail_chunks, int tail_min, void* workspace, size_t ws_bytes,
+                            int* grid_out, void* stream) {
   if (!seq_lens || !workspace || !grid_out) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || pt_stride <= 0 || num_ctas <= 0 ||
       param < 0 || max_seq_len < 0)
@@ -222,7 +223,8 @@ static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads
   if (kind != HPA_PLAN_DYNAMIC && kind != HPA_PLAN_STATIC_NSPLIT && kind != HPA_PLAN_STATIC_CHUNK &&
       kind != HPA_PLAN_LENGTH_AWARE)
     return HPA_ERR_INVALID_ARG;
-  if (tail_den < 0 || tail_den > (1 << 20) || tail_chunks < 1 || tail_chunks > HPA_TAIL_CHUNKS_MAX)
+  if (tail_den < 0 || tail_den > (1 << 20) || tail_chunks < 1 || tail_chunks > HPA_TAIL_CHUNKS_MAX ||
+      tail_min < 0 || tail_min > (1 << 20))
     return HPA_ERR_INVALID_ARG;
   if ((long long)pt_stride * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
   if (batch > kMaxPlanBatch) return HPA_ERR_UNSUPPORTED;
@@ -254,6 +256,7 @@ static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads
   p.chunk = chunk;
   p.tail_den = tail_den;
   p.tail_chunks = tail_chunks;
+  p.tail_min = tail_min;
   p.ws = ws_view(workspace, L);
 
   const size_t smem = (size_t(batch) + 1) * sizeof(int32_t);
@@ -305,16 +308,17 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
                                       int* grid_out, void* stream) {
   return plan_impl(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride, kind,
                    num_ctas, param, max_seq_len, HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT,
-                   workspace, ws_bytes, grid_out, stream);
+                   HPA_TAIL_MIN_DEFAULT, workspace, ws_bytes, grid_out, stream);
 }
 
 extern "C" hpa_status hpa_decode_plan_tail(const int32_t* seq_lens, int batch, int num_kv_heads,
                                            int num_q_heads, int head_dim, int pt_stride,
                                            hpa_plan_kind kind, int num_ctas, int param,
-                                           int tail_den, int tail_chunks, void* workspace,
-                                           size_t ws_bytes, int* grid_out, void* stream) {
+                                           int tail_den, int tail_chunks, int tail_min,
+                                           void* workspace, size_t ws_bytes, int* grid_out,
+                                           void* stream) {
   if (!plan_is_dynamic(kind)) return HPA_ERR_INVALID_ARG;
   return plan_impl(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride, kind,
-                   num_ctas, param, 0, tail_den, tail_chunks, workspace, ws_bytes, grid_out,
-                   stream);
+                   num_ctas, param, 0, tail_den, tail_chunks, tail_min, workspace, ws_bytes,
+                   grid_out, stream);
 }

@@ -41,24 +41,26 @@ struct FloorDiv {
 // Dynamic plan geometry.  P persistent CTAs; U units.  If U <= P each active
 // CTA takes one unit.  Otherwise the first U1 = U - Ut units are spread over
 // the P primary ranges and the last Ut units over M tail chunks, handed out at
-// run time to whichever CTA is free, where for the tail parameters (den, k)
-// Ut = min(floor(U/den), U - P) (0 if den = 0) and M = min(kP, Ut).  The
-// parameters are the library's tuning (HPA_TAIL_DEN_DEFAULT,
-// HPA_TAIL_CHUNKS_DEFAULT unless the caller gives others); den = 0 is the
-// plain even partition of all U units over the P CTAs.  For n units spread
+// run time to whichever CTA is free, where for the tail parameters (den, k,
+// mn) Ut = min(floor(U/den), U - P) if den > 0 and U >= mn P, else 0, and M =
+// min(kP, Ut).  The parameters are the library's tuning (HPA_TAIL_*_DEFAULT
+// unless the caller gives others); no tail is the plain even partition of
+// all U units over the P CTAs.  For n units spread
 // over m ranges as [floor(cn/m), floor((c+1)n/m)), the range holding unit u is
 // the largest c with floor(cn/m) <= u, i.e. floor(((u+1)m - 1) / n).
 struct DynGeom {
   long long U, P, Pd, U1, Ut, M;
   FloorDiv by_Pd, by_M, by_U1, by_Ut;
-  __device__ void init(long long units, long long ctas, int tail_den, int tail_chunks) {
+  __device__ void init(long long units, long long ctas, int tail_den, int tail_chunks,
+                       int tail_min) {
     U = units;
     P = ctas;
     if (U <= P) {
       Pd = U; U1 = U; Ut = 0; M = 0;
     } else {
       Pd = P;
-      Ut = tail_den > 0 ? std::min<long long>(U / tail_den, U - P) : 0;
+      const bool tail = tail_den > 0 && U >= (long long)tail_min * P;
+      Ut = tail ? std::min<long long>(U / tail_den, U - P) : 0;
       U1 = U - Ut;
       M = std::min<long long>((long long)tail_chunks * P, Ut);
     }

@@ -425,9 +425,10 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  *     at run time as they finish (bitbyai.com "vLLM x HPC-Ops", Attention
  *     Backend: progress is evaluated dynamically).  The pages fix the even
  *     spread but not the size of the tail, so this is a FAMILY of plans with
- *     two parameters given by the caller: the tail divisor den and the chunks
- *     per CTA k.  Ut = min(floor(U / den), U - P) (every primary range keeps
- *     at least one unit; den = 0 means no tail, Ut = 0), M = min(k P, Ut).
+ *     three parameters given by the caller: the tail divisor den, the chunks
+ *     per CTA k and the least units per CTA mn for a tail.  If den > 0 and
+ *     U >= mn P, Ut = min(floor(U / den), U - P) (every primary range keeps
+ *     at least one unit); otherwise there is no tail, Ut = 0.  M = min(k P, Ut).
  *     With U1 = U - Ut, range c < P is [floor(c U1 / P), floor((c+1) U1 / P))
  *     and range P + j is [U1 + floor(j Ut / M), U1 + floor((j+1) Ut / M)).
  *     With den = 0 the ranges are the plain even partition
@@ -496,13 +497,13 @@ static long snap_cut(long x, long U, long m, const int32_t* unit_seg, const int3
 
 int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capacity_tokens,
                 int kind, int num_ctas, int param, int max_seq_len, int tail_den,
-                int tail_chunks, int32_t* lens_out,
+                int tail_chunks, int tail_min, int32_t* lens_out,
                 int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][2] */,
                 int32_t* split_count /* [B*Hkv] */, int32_t* first_slot /* [B*Hkv] */,
                 int32_t* n_units_out, int32_t* n_ranges_out) {
   if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 3)
     return ORC_BAD_ARG;
-  if (tail_den < 0 || tail_chunks < 1) return ORC_BAD_ARG;
+  if (tail_den < 0 || tail_chunks < 1 || tail_min < 0) return ORC_BAD_ARG;
   long grid = oracle_plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len, page_size);
   int S = B * Hkv;
   /* 1. lengths clamped to [0, capacity], tiles per sequence, tile offsets */
@@ -544,8 +545,8 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
         end[c] = c < U ? c + 1 : U;
       }
     } else {
-      long Ut = 0; /* tail units: none when den = 0 */
-      if (tail_den > 0) Ut = U / tail_den < U - P ? U / tail_den : U - P;
+      long Ut = 0; /* tail units: none when den = 0 or U < mn P */
+      if (tail_den > 0 && U >= (long)tail_min * P) Ut = U / tail_den < U - P ? U / tail_den : U - P;
       long U1 = U - Ut;
       long M = (long)tail_chunks * P < Ut ? (long)tail_chunks * P : Ut;
       for (long c = 0; c < P; ++c) {

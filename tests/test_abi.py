@@ -120,14 +120,14 @@ def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
 
 def _plan_tail(L, **kw):
     a = dict(seq_lens=1, batch=2, num_kv_heads=2, num_q_heads=8, head_dim=64, pt_stride=4,
-             kind=0, num_ctas=148, param=0, tail_den=8, tail_chunks=4, workspace=256,
-             ws_bytes=1 << 20)
+             kind=0, num_ctas=148, param=0, tail_den=8, tail_chunks=4, tail_min=32,
+             workspace=256, ws_bytes=1 << 20)
     a.update(kw)
     g = C.c_int(-7)
     rc = L.hpa_decode_plan_tail(a["seq_lens"], a["batch"], a["num_kv_heads"], a["num_q_heads"],
                                 a["head_dim"], a["pt_stride"], a["kind"], a["num_ctas"],
-                                a["param"], a["tail_den"], a["tail_chunks"], a["workspace"],
-                                a["ws_bytes"], C.byref(g), None)
+                                a["param"], a["tail_den"], a["tail_chunks"], a["tail_min"],
+                                a["workspace"], a["ws_bytes"], C.byref(g), None)
     return rc, g.value
 
 
@@ -135,7 +135,7 @@ def _plan_tail(L, **kw):
     (dict(kind=1), 1), (dict(kind=2), 1),           # the static kinds have no tail
     (dict(tail_den=-1), 1), (dict(tail_den=(1 << 20) + 1), 1),
     (dict(tail_chunks=0), 1), (dict(tail_chunks=hpa.TAIL_CHUNKS_MAX + 1), 1),
-    (dict(tail_den=0, tail_chunks=0), 1),
+    (dict(tail_den=0, tail_chunks=0), 1), (dict(tail_min=-1), 1), (dict(tail_min=(1 << 20) + 1), 1),
     (dict(seq_lens=None), 1), (dict(ws_bytes=16), 3), (dict(num_ctas=65537), 2),
 ])
 def test_plan_tail_rejects_bad_arguments_without_launching(L, bad, expect):
@@ -148,6 +148,7 @@ def test_tail_defaults_match_the_header():
     src = open(HEADER).read()
     for name, val in [("HPA_TAIL_DEN_DEFAULT", hpa.TAIL_DEN_DEFAULT),
                       ("HPA_TAIL_CHUNKS_DEFAULT", hpa.TAIL_CHUNKS_DEFAULT),
+                      ("HPA_TAIL_MIN_DEFAULT", hpa.TAIL_MIN_DEFAULT),
                       ("HPA_TAIL_CHUNKS_MAX", hpa.TAIL_CHUNKS_MAX)]:
         assert re.search(rf"#define {name} {val}\b", src), name
 

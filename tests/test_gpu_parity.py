@@ -63,7 +63,7 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
 
 # The library's member of the dynamic plan family (hpa.h: HPA_TAIL_DEN_DEFAULT,
 # HPA_TAIL_CHUNKS_DEFAULT), and other members called with hpa_decode_plan_tail.
-LIB_TAIL = (8, 4)
+LIB_TAIL = (8, 4, 32)
 
 
 @pytest.mark.parametrize("lens,Hkv,P", [
@@ -77,11 +77,11 @@ LIB_TAIL = (8, 4)
 @pytest.mark.parametrize("kind,param,tail", [
     (0, 0, None), (1, 0, None), (1, 3, None), (2, 0, None), (2, 5, None), (3, 0, None),
     (3, 2, None), (3, 9, None),
-    (0, 0, (0, 1)), (0, 0, (3, 1)), (0, 0, (16, 2)), (0, 0, (1, 4)), (3, 4, (0, 1)),
-    (3, 2, (5, 3))])
+    (0, 0, (0, 1, 0)), (0, 0, (8, 4, 0)), (0, 0, (3, 1, 0)), (0, 0, (16, 2, 3)),
+    (0, 0, (1, 4, 0)), (3, 4, (0, 1, 0)), (3, 2, (5, 3, 0))])
 def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail):
     """tail None: hpa_decode_plan (the library's default tail, LIB_TAIL);
-    else hpa_decode_plan_tail with that tail shape (0, 1 = no tail)."""
+    else hpa_decode_plan_tail with that tail shape ((0, 1, 0) = no tail)."""
     B, Hq, D = len(lens), Hkv * 2, 64
     cap = max(64, max(lens))
     pts = (cap + 63) // 64
@@ -120,8 +120,8 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail):
     h = got["header"]
     assert h[2] == ref["n_units"] and h[3] == grid and h[1] == 0
     # the tail shape the plan was made with, recorded in the header
-    want = (LIB_TAIL if tail is None else tail) if kind in (0, 3) else (0, 0)
-    assert (int(h[13]), int(h[14])) == want
+    want = (LIB_TAIL if tail is None else tail) if kind in (0, 3) else (0, 0, 0)
+    assert (int(h[13]), int(h[14]), int(h[15])) == want
 
 
 def test_plan_flags_clamped_lengths():
@@ -883,7 +883,8 @@ def _random_case(seed):
     lens = [max(L, T) if rng.random() < 0.9 else L for L in lens]
     kind = int(rng.choice([0, 0, 1, 2, 3]))
     param = int(rng.integers(0, 5)) if kind else 0
-    tail = [(8, 4), (0, 1), (3, 2), (16, 4)][int(rng.integers(0, 4))] if kind in (0, 3) else None
+    tail = [(8, 4, 32), (0, 1, 0), (3, 2, 0), (16, 4, 4)][int(rng.integers(0, 4))] \
+        if kind in (0, 3) else None
     num_ctas = int(rng.choice([1, 5, 37, 148, 296]))
     out_dtype = torch.float32 if rng.random() < 0.5 else torch.bfloat16
     return dict(D=D, fp8=fp8, Hkv=Hkv, G=G, T=T, lens=lens, kind=kind, param=param, tail=tail,

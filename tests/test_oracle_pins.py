@@ -517,12 +517,13 @@ def _even_ranges(n, m):
 
 
 def _check_dynamic_family(p, U, tail):
-    """A dynamic plan of the family (den, k): the primary ranges are the even
-    partition of the first U1 units over P CTAs and the tail chunks the even
-    partition of the last Ut units over M chunks, where Ut is the largest tail
-    with Ut <= U / den that still leaves every primary range a unit (no tail
-    for den = 0) and M the largest chunk count with M <= k P and M <= Ut."""
-    den, k = tail
+    """A dynamic plan of the family (den, k, mn): the primary ranges are the
+    even partition of the first U1 units over P CTAs and the tail chunks the
+    even partition of the last Ut units over M chunks, where Ut is the largest
+    tail with Ut <= U / den that still leaves every primary range a unit (no
+    tail for den = 0 or when U < mn P) and M the largest chunk count with
+    M <= k P and M <= Ut."""
+    den, k, mn = tail
     P = p["grid"]
     R = p["ranges"]
     cta = [(int(a), int(e)) for a, e in p["cta"]]
@@ -532,7 +533,7 @@ def _check_dynamic_family(p, U, tail):
         return
     M = R - P
     Ut = U - cta[P - 1][1] if M else 0
-    if den == 0:
+    if den == 0 or U < mn * P:
         assert Ut == 0 and M == 0
     else:
         assert Ut * den <= U and U - Ut >= P
@@ -555,8 +556,9 @@ def _check_dynamic_family(p, U, tail):
     ([1], 1, 148),
     ([0, 0], 2, 5),
 ])
-@pytest.mark.parametrize("kind,tail", [(0, (8, 4)), (0, (0, 1)), (0, (3, 1)), (0, (16, 2)),
-                                       (0, (1, 4)), (1, (8, 4)), (2, (8, 4))])
+@pytest.mark.parametrize("kind,tail", [(0, (8, 4, 32)), (0, (8, 4, 0)), (0, (0, 1, 0)),
+                                       (0, (3, 1, 0)), (0, (16, 2, 5)), (0, (1, 4, 0)),
+                                       (1, (8, 4, 32)), (2, (8, 4, 32))])
 def test_planner_invariants(lens, Hkv, P, kind, tail):
     p = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P,
                     max_seq_len=max(lens), capacity_tokens=max(64, max(lens)), tail=tail)
@@ -579,11 +581,11 @@ def test_dynamic_plan_without_tail_is_the_even_partition(U, P):
     [floor(cU/P), floor((c+1)U/P))."""
     # U units as one sequence of U tiles with one kv head
     p = oracle.plan(np.array([64 * U], dtype=np.int32), 1, kind=0, num_ctas=P,
-                    capacity_tokens=64 * U, tail=(0, 1))
+                    capacity_tokens=64 * U, tail=(0, 1, 0))
     assert p["ranges"] == P
     assert [(int(a), int(e)) for a, e in p["cta"]] == _even_ranges(U, P)
     # one split count and consecutive slots, recounted
-    _check_plan_invariants(p, [64 * U], 1, 0, (0, 1))
+    _check_plan_invariants(p, [64 * U], 1, 0, (0, 1, 0))
 
 
 @pytest.mark.parametrize("lens,Hkv,P", [
@@ -601,8 +603,8 @@ def test_length_aware_planner(lens, Hkv, P, m):
     leave a piece of fewer than m tiles at a segment's end moves to that end."""
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
-    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4))
-    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4))
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4, 0))
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4, 0))
     _check_plan_invariants(la, lens, Hkv, 3)
     assert la["grid"] == P and la["ranges"] == dyn["ranges"]
     units = _units(lens, Hkv)
@@ -645,30 +647,30 @@ def test_length_aware_planner_hand_cases():
     # with m = 2 the cut after tile 1 leaves 1 tile on each side (a tie) and
     # moves to the segment's start, so the second range holds the whole segment
     p = oracle.plan(np.array([128], dtype=np.int32), 1, kind=3, num_ctas=2, param=2,
-                    capacity_tokens=128, tail=(8, 4))
+                    capacity_tokens=128, tail=(8, 4, 0))
     np.testing.assert_array_equal(p["cta"], [[0, 0], [0, 2]])
     assert p["split_count"][0] == 1 and p["first_slot"][0] == -1
     # 3 tiles, 3 CTAs, m = 2: the cut after tile 1 (a=1, r=2) moves to the
     # start, the cut after tile 2 (a=2, r=1) to the end: one whole range
     p = oracle.plan(np.array([192], dtype=np.int32), 1, kind=3, num_ctas=3, param=2,
-                    capacity_tokens=192, tail=(8, 4))
+                    capacity_tokens=192, tail=(8, 4, 0))
     np.testing.assert_array_equal(p["cta"], [[0, 0], [0, 3], [3, 3]])
-    # 8 tiles, 2 CTAs, tail (8, 4): the dynamic plan has primary ranges
+    # 8 tiles, 2 CTAs, tail (8, 4, 0): the dynamic plan has primary ranges
     # [0, 3), [3, 7) and one tail chunk [7, 8).  m = 2 keeps the cut at 3 (a=3, r=5) and moves
     # the one at 7 (r=1) to the end; m = 4 also moves the cut at 3 (a=3 < 4)
     for m, want in ((2, [[0, 3], [3, 8], [8, 8]]), (4, [[0, 0], [0, 8], [8, 8]])):
         p = oracle.plan(np.array([512], dtype=np.int32), 1, kind=3, num_ctas=2, param=m,
-                        capacity_tokens=512, tail=(8, 4))
+                        capacity_tokens=512, tail=(8, 4, 0))
         np.testing.assert_array_equal(p["cta"], want)
 
 
 def test_planner_static_shapes():
     lens = [131072] + [4096] * 31
     pA = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=1, num_ctas=148, max_seq_len=131072,
-                     capacity_tokens=131072, tail=(8, 4))
+                     capacity_tokens=131072, tail=(8, 4, 0))
     assert pA["grid"] == 32 * 8  # ceil(148 / 256) = 1 split per (seq, kv head)
     pB = oracle.plan(np.array(lens, dtype=np.int32), 8, kind=2, num_ctas=148, max_seq_len=131072,
-                     capacity_tokens=131072, tail=(8, 4))
+                     capacity_tokens=131072, tail=(8, 4, 0))
     # chunk = ceil(2048 / ceil(148 / 8)) = 108 tiles; 19 chunks per segment
     assert pB["grid"] == 32 * 8 * 19
     sizes = pB["cta"][:, 1] - pB["cta"][:, 0]
@@ -677,7 +679,7 @@ def test_planner_static_shapes():
 
 def test_planner_clamps_lengths_to_capacity():
     p = oracle.plan(np.array([-5, 1000, 64], dtype=np.int32), 2, kind=0, num_ctas=4,
-                    capacity_tokens=128, tail=(8, 4))
+                    capacity_tokens=128, tail=(8, 4, 0))
     np.testing.assert_array_equal(p["lens"], [0, 128, 64])
     np.testing.assert_array_equal(p["tile_start"], [0, 0, 2, 3])
 
@@ -735,3 +737,17 @@ def test_multi_token_last_query_equals_single_token_decode():
     multi = oracle.paged_decode_multi(bits16(batch.q), *args)
     single = oracle.paged_decode(np.ascontiguousarray(bits16(batch.q)[:, -1]), *args)
     np.testing.assert_array_equal(multi[:, -1], single)
+
+
+@pytest.mark.parametrize("U,P,has_tail", [(4096, 296, False), (9471, 296, False),
+                                          (9472, 296, True), (32256, 296, True)])
+def test_tail_needs_enough_units_per_cta(U, P, has_tail):
+    """mn = 32: no run-time tail below 32 units per CTA (U < 32 P), the tail of
+    den = 8 from there on."""
+    p = oracle.plan(np.array([64 * U], dtype=np.int32), 1, kind=0, num_ctas=P,
+                    capacity_tokens=64 * U, tail=(8, 4, 32))
+    assert (p["ranges"] > P) == has_tail
+    if not has_tail:
+        assert [(int(a), int(e)) for a, e in p["cta"]] == _even_ranges(U, P)
+    else:
+        assert int(p["cta"][P][0]) == U - U // 8

@@ -20,8 +20,8 @@ lens_st = st.lists(st.integers(min_value=0, max_value=3000), min_size=1, max_siz
 def test_length_aware_plan_properties(lens, Hkv, P, m):
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
-    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4))
-    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4))
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4, 0))
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4, 0))
     # coverage, contiguity, consecutive holders and partial slots
     _check_plan_invariants(la, lens, Hkv, 3)
     assert la["ranges"] == dyn["ranges"]
@@ -76,17 +76,17 @@ def test_page_shard_properties(lens, N, extra, seed):
 @settings(max_examples=60, deadline=None)
 @given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
        kind=st.sampled_from([0, 1, 2]), param=st.integers(0, 9),
-       den=st.integers(0, 40), k=st.integers(1, 4))
-def test_plan_kinds_properties(lens, Hkv, P, kind, param, den, k):
+       den=st.integers(0, 40), k=st.integers(1, 4), mn=st.integers(0, 40))
+def test_plan_kinds_properties(lens, Hkv, P, kind, param, den, k, mn):
     """Every plan kind covers each unit exactly once with contiguous ranges,
     consecutive holders per segment and distinct partial slots; a dynamic plan
-    of any tail shape (den, k) has the even primary ranges and the even tail
-    chunks of that shape."""
+    of any tail shape (den, k, mn) has the even primary ranges and the even
+    tail chunks of that shape."""
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
     p = oracle.plan(sl, Hkv, kind=kind, num_ctas=P, param=param if kind else 0,
-                    max_seq_len=max(lens), capacity_tokens=cap, tail=(den, k))
-    _check_plan_invariants(p, lens, Hkv, kind, (den, k))
+                    max_seq_len=max(lens), capacity_tokens=cap, tail=(den, k, mn))
+    _check_plan_invariants(p, lens, Hkv, kind, (den, k, mn))
     assert p["n_units"] == len(_units(lens, Hkv))
 
 
@@ -99,7 +99,7 @@ def test_dynamic_tail_covers_the_last_units_evenly(lens, Hkv, P, den, k):
     units before them, also within one unit of each other."""
     sl = np.array(lens, dtype=np.int32)
     p = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=max(64, max(lens)),
-                    tail=(den, k))
+                    tail=(den, k, 0))
     U, R = p["n_units"], p["ranges"]
     if U <= P:
         return
