@@ -354,6 +354,7 @@ CONFIGS = ["tiny", "uniform", "skewed", "mix_prologue", "fp8"]
 ITER_WARMUP, ITERS = 10, 50        # per-config timing: 10 untimed + 50 timed steps
 CPU_CONFIG_SECONDS = 3.0           # CPU baseline of each config but the headline
 AB_BLOCKS, AB_PER = 5, 10          # interleaved A/B: blocks x steps on each side
+CHAIN, CHAIN_REPLAYS = 8, 10       # steps per graph and replays of the chained measurement
 
 
 class Case:
@@ -710,6 +711,29 @@ def measure_case(case, args, world, dev, stream, peak, sampler_rows, headline):
                               "step's launches), mean",
                      "algorithmic_bytes_per_launch": case.run_bytes},
     }
+    # The same steps as a model's graph would hold them: CHAIN consecutive
+    # steps captured in one graph, each step's decode kernel chained to the
+    # merge before it by programmatic dependent launch, so its CTAs are
+    # resident before that merge ends (one graph launch per CHAIN steps).
+    # Only where the batch is well above the L2: consecutive steps of a
+    # smaller batch would find it in the L2.
+    rec["chained_us_per_step"] = None
+    if flush is None:
+        chain, cgraph = _graphed(lambda: [case.step() for _ in range(CHAIN)], dev, args.eager)
+        for _ in range(2):
+            chain()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(CHAIN_REPLAYS):
+            chain()
+        b.record(stream)
+        torch.cuda.synchronize()
+        rec["chained_us_per_step"] = 1e3 * a.elapsed_time(b) / (CHAIN * CHAIN_REPLAYS)
+        rec["chained_method"] = (f"{CHAIN} steps captured in one CUDA graph (each decode kernel "
+                                 f"PDL-chained to the merge before it), {CHAIN_REPLAYS} replays")
+        del cgraph
     # load balance of one step, from the run kernel's per-CTA timeline
     case.step()
     torch.cuda.synchronize()
@@ -952,6 +976,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "us_per_step": 1e3 * ms_per_step,
         "us_per_step_median": rec["us_per_step"]["median"],
         "us_per_step_p90": rec["us_per_step"]["p90"],
+        "us_per_step_chained_in_graph": rec.get("chained_us_per_step"),
         "pct_of_hbm_peak": 100.0 * (head["kv_bytes"] / (ms_per_step * 1e-3) / 1e9) / peak,
         "config": {
             "workload": WORKLOAD_DESC.get(head["name"], head["name"]),
