@@ -102,6 +102,8 @@ WORKLOAD_DESC = {
     "fp8_quarter": "the first 64 sequences of the FP8 batch (profiler captures)",
     "skewed_mtp2": "multi-token decode on the skewed batch: 2 query tokens per sequence "
                    "(causal among themselves), 64 q heads, 8 kv heads, head_dim 128, bf16",
+    "skewed_mtp4": "multi-token decode on the skewed batch: 4 query tokens per sequence "
+                   "(32 query rows per kv head), 64 q heads, 8 kv heads, head_dim 128, bf16",
 }
 
 

@@ -27,7 +27,8 @@
  *     which never trap: they skip the offending access and set a bit in a
  *     device status word (HPA_DEVICE_*), read back with hpa_read_status.
  *   - Shapes: head_dim D in {64, 128}; page (tile) size 64 tokens; GQA group
- *     G = num_q_heads / num_kv_heads in 1 .. 16 (rows padded to whole MMA n-tiles of 8).
+ *     G = num_q_heads / num_kv_heads in 1 .. 32 (G x query tokens <= 32 rows per
+ *     kv head, padded to whole MMA n-tiles of 8; the fused prologue G <= 16).
  *
  * Tensor layouts (row-major, innermost last):
  *   q, q_raw, out        [batch][num_q_heads][D]
@@ -140,9 +141,10 @@ HPA_API int hpa_default_num_ctas(int device);
 /* Persistent CTA count (num_ctas of hpa_decode_plan) that matches how many
  * run-kernel CTAs fit at once for this head geometry; a dynamic plan for more
  * CTAs than fit would leave part of its primary ranges to a second wave.
- * Every supported geometry (G * q_tokens <= 16) fits two per SM, so this is
- * hpa_default_num_ctas for valid arguments.  Returns -1 on invalid arguments
- * or if the device cannot be queried. */
+ * Up to 16 query rows per kv head (G * q_tokens) two fit per SM, and this is
+ * hpa_default_num_ctas; 17 .. 32 rows run one CTA per SM (the SM count).
+ * Returns -1 on invalid arguments (more than 32 rows) or if the device cannot
+ * be queried. */
 HPA_API int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads, int q_tokens);
 
 /* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC and
@@ -298,9 +300,10 @@ HPA_API hpa_status hpa_decode_run(const void* q, const void* k_cache, const void
  *
  *   q, out       device [batch][q_tokens][num_q_heads][D] (bf16 q; bf16 or
  *                fp32 out).
- *   q_tokens     1 .. 16 with (num_q_heads / num_kv_heads) * q_tokens <= 16:
+ *   q_tokens     1 .. 16 with (num_q_heads / num_kv_heads) * q_tokens <= 32:
  *                the G * T query rows of a kv head share one pass over its
- *                tiles (HPA_ERR_UNSUPPORTED otherwise).
+ *                tiles (HPA_ERR_UNSUPPORTED otherwise).  Above 16 rows the
+ *                kernel runs one CTA per SM (hpa_decode_num_ctas).
  *   kind, grid, workspace  from hpa_decode_plan called with num_q_heads *
  *                q_tokens in place of num_q_heads (the plan and the workspace
  *                count G * T rows per kv head); size the workspace the same way.

@@ -97,12 +97,16 @@ struct Cfg {
   // every tile and all 8 rows.  Two n-tiles (9..16 rows): warp w owns n-tile
   // w / 2 and tokens [32 (w % 2), + 32), as two 16-token blocks -- the same
   // MMA work with the registers of the one-n-tile kernel, so two CTAs still
-  // fit an SM.
-  static constexpr bool kSplit = NT == 2;
+  // fit an SM.  Four n-tiles (17..32 rows): warp w owns n-tile w and all 64
+  // tokens, as four 16-token blocks (one CTA per SM: the 32 query rows of a
+  // stage take 8 KiB more shared memory).
+  static constexpr bool kSplit = NT >= 2;
+  static constexpr int kWarpsPerTile = kSplit ? kConsumerWarps / NT : kConsumerWarps;
   static constexpr int kWarpTiles = kSplit ? 1 : NT;   // n-tiles per warp
-  static constexpr int kBlocks = kSplit ? 2 : 1;       // 16-token blocks per warp
+  static constexpr int kBlocks = kSplit ? NT : 1;      // 16-token blocks per warp
   static constexpr int kWarpRows = 8 * kWarpTiles;     // rows each warp deposits
-  static constexpr int kRowWarps = kSplit ? 2 : kConsumerWarps;  // warps holding a row
+  static constexpr int kRowWarps = kSplit ? kWarpsPerTile : kConsumerWarps;  // warps holding a row
+  static_assert(NT == 1 || NT == 2 || NT == 4, "one, two or four n-tiles");
   // one deposit: acc[warp][row of the warp][D + 4] floats, then (m, l)[warp][row]
   static constexpr int kDepAccFloats = kConsumerWarps * kWarpRows * kAccStride;
   static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kWarpRows * 8;
@@ -679,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
       // their shared-memory latencies overlap
       constexpr int R = C::kRowWarps;
       auto load_row = [&](int h, float2 (&ml)[R], float (&a)[R][V]) {
-        const int w0 = C::kSplit ? 2 * (h >> 3) : 0;  // first warp holding row h
+        const int w0 = C::kSplit ? R * (h >> 3) : 0;  // first warp holding row h
         const int lr = C::kSplit ? (h & 7) : h;       // its row inside those warps
 #pragma unroll
         for (int k = 0; k < R; ++k) {
@@ -752,8 +756,9 @@ __global__ void __launch_bounds__(kThreads, CPS)
   constexpr int W = C::kWarpTiles, MB = C::kBlocks;
   const int r = lane >> 2, c = lane & 3;          // MMA fragment coordinates
   const int lm = lane >> 3, lr = lane & 7;        // ldmatrix address lane roles
-  const int nt0 = C::kSplit ? (warp >> 1) : 0;    // this warp's first n-tile
-  const int tok0 = C::kSplit ? 32 * (warp & 1) : 16 * warp;  // its first token
+  const int nt0 = C::kSplit ? warp / C::kWarpsPerTile : 0;  // this warp's first n-tile
+  const int tok0 = C::kSplit ? (kPageSize / C::kWarpsPerTile) * (warp % C::kWarpsPerTile)
+                             : 16 * warp;                   // its first token
   // ldmatrix row (token) for the QK A operand and the PV A operand
   const int k_tok = tok0 + (lm & 1) * 8 + lr;
   const int k_chk = lm >> 1;
@@ -1118,9 +1123,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
     for (int mb = 0; mb < MB; ++mb) {
       if (mb > 0) {
         load_v(vt, mb, va);
-        // all shared-memory reads of this stage are issued: hand it back
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
+        if (mb == MB - 1) {
+          // all shared-memory reads of this stage are issued: hand it back
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
+        }
       }
       const int vb = valid - 16 * mb;
       if (vb < 16) {  // warp-uniform: some V row of the block is past the end
@@ -1386,6 +1393,10 @@ hpa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const RunParams&
 template <int D, bool FP8, bool OUT_F32, bool PRO, bool FP>
 hpa_status launch_nt(int nt, int cps, const CUtensorMap& tk, const CUtensorMap& tv,
                      const RunParams& p, int grid, cudaStream_t s) {
+  if constexpr (!PRO) {
+    // 17..32 rows (multi-token only): one CTA per SM whatever the grid
+    if (nt == 4) return launch<D, 4, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s);
+  }
   if (cps == 1)
     return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s)
                    : launch<D, 2, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s);
@@ -1444,11 +1455,12 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   const bool fp8 = kv_dtype == HPA_KV_FP8_E4M3;
   if (fp8 && (!k_scale || !v_scale)) return HPA_ERR_INVALID_ARG;
   const int G = num_q_heads / num_kv_heads;
-  if (G > 16) return HPA_ERR_UNSUPPORTED;  // a kv head's rows fill at most two MMA n-tiles
+  if (G > 32) return HPA_ERR_UNSUPPORTED;  // a kv head's rows fill at most four MMA n-tiles
   if (q_tokens < 1) return HPA_ERR_INVALID_ARG;
-  // the G * T rows of a kv head ride on the MMA N dimension: at most 16
-  if (q_tokens > kMaxQTokens || G * q_tokens > 16) return HPA_ERR_UNSUPPORTED;
-  if (pro && q_tokens != 1) return HPA_ERR_UNSUPPORTED;
+  // the G * T rows of a kv head ride on the MMA N dimension: at most 32
+  if (q_tokens > kMaxQTokens || G * q_tokens > 32) return HPA_ERR_UNSUPPORTED;
+  // the fused prologue: one query token, at most two n-tiles
+  if (pro && (q_tokens != 1 || G > 16)) return HPA_ERR_UNSUPPORTED;
   if (plan_lens) {
     // in-kernel plan: the dynamic plan for `grid` persistent CTAs, with the
     // plan kernel's limits and the tile offsets in shared memory
@@ -1522,7 +1534,7 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.tail_den = HPA_TAIL_DEN_DEFAULT;
   p.tail_chunks = HPA_TAIL_CHUNKS_DEFAULT;
   p.tail_min = HPA_TAIL_MIN_DEFAULT;
-  const int nt = GT > 8 ? 2 : 1;
+  const int nt = GT > 16 ? 4 : GT > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -92,7 +92,7 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
     return HPA_ERR_INVALID_ARG;
   {
     const int G = num_q_heads / num_kv_heads;
-    if (G > 16) return HPA_ERR_UNSUPPORTED;  // a kv head's rows fill at most two MMA n-tiles
+    if (G > 32) return HPA_ERR_UNSUPPORTED;  // a kv head's rows fill at most four MMA n-tiles
     if (head_dim != 64 && head_dim != 128) return HPA_ERR_UNSUPPORTED;
     if (kv_dtype == HPA_KV_FP8_E4M3 && head_dim != 128) return HPA_ERR_UNSUPPORTED;
     if ((long long)num_pages * num_kv_heads * 64 > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;

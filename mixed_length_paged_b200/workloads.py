@@ -62,6 +62,8 @@ SHAPES = {
     # the skewed batch with two query tokens per sequence (a draft token to
     # verify, or a multi-token-prediction head): 8 heads x 2 tokens per kv head
     "skewed_mtp2": DecodeShape("skewed_mtp2", 64, 8, 128, q_tokens=2),
+    # four query tokens per sequence: 32 query rows per kv head (four MMA n-tiles)
+    "skewed_mtp4": DecodeShape("skewed_mtp4", 64, 8, 128, q_tokens=4),
 }
 
 
@@ -77,7 +79,7 @@ def cache_lengths(name: str, seed: int = 0) -> np.ndarray:
         return np.array([37, 200], dtype=np.int64)
     if name == "uniform":
         return np.full(64, 512, dtype=np.int64)
-    if name in ("skewed", "skewed_mtp2"):
+    if name in ("skewed", "skewed_mtp2", "skewed_mtp4"):
         return np.array([131072] + [4096] * 31, dtype=np.int64)
     if name == "skewed_quarter":
         return np.array([32768] + [1024] * 31, dtype=np.int64)
@@ -228,7 +230,7 @@ def make_batch(shape: DecodeShape, cache_lens, *, seed: int = 0, device="cpu",
 
 def build(name: str, *, seed: int = 0, device="cpu", **kw) -> DecodeBatch:
     """One of the named workloads (tiny, uniform, skewed, skewed_quarter, mix_prologue, fp8,
-    fp8_quarter, skewed_mtp2)."""
+    fp8_quarter, skewed_mtp2, skewed_mtp4)."""
     return make_batch(SHAPES[name], cache_lengths(name, seed), seed=seed, device=device, **kw)
 
 

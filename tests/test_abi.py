@@ -166,8 +166,8 @@ def _run(L, **kw):
     (dict(q=None), 1), (dict(k=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
     (dict(B=0), 1), (dict(Hq=6, Hkv=4), 1), (dict(kvd=5), 1), (dict(outd=2), 1),
     (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(kvd=1), 1),  # fp8 w/o scales
-    (dict(Hq=34, Hkv=2), 2),   # G = 17
-    (dict(Hq=64, Hkv=2), 2),   # G = 32
+    (dict(Hq=66, Hkv=2), 2),   # G = 33: more rows than four MMA n-tiles
+    (dict(Hq=128, Hkv=2), 2),  # G = 64
     (dict(D=96), 2), (dict(D=256), 2), (dict(kvd=1, ks=256, vs=256), 2),  # fp8 needs D = 128
     (dict(pages=1 << 26, Hkv=8, Hq=8), 2),  # rows overflow int32 TMA coordinates
     (dict(k=256 + 8), 1), (dict(q=256 + 2), 1), (dict(q=256 + 8), 1), (dict(out=256 + 2), 1),
@@ -190,8 +190,9 @@ def _run_multi(L, **kw):
 
 @pytest.mark.parametrize("bad,expect", [
     (dict(T=0), 1), (dict(T=-3), 1), (dict(T=17, Hq=2, Hkv=2), 2),
-    (dict(T=3, Hq=64, Hkv=8), 2),    # G * T = 24 rows > 16
-    (dict(T=2, Hq=16, Hkv=1), 2),    # G = 16: no room for a second token
+    (dict(T=5, Hq=64, Hkv=8), 2),    # G * T = 40 rows > 32
+    (dict(T=3, Hq=16, Hkv=1), 2),    # G = 16: room for two tokens, not three
+    (dict(T=2, Hq=32, Hkv=1), 2),    # G = 32: no room for a second token
     (dict(q=None), 1), (dict(q=256 + 8), 1), (dict(wsb=64), 3), (dict(kind=9), 1),
 ])
 def test_run_multi_rejects_bad_arguments_without_launching(L, bad, expect):
@@ -223,7 +224,8 @@ def _run_pro(L, **kw):
     (dict(gk=None), 1), (dict(kc=None), 1), (dict(out=None), 1), (dict(ws=None), 1),
     (dict(kr=256 + 8), 1), (dict(vr=256 + 4), 1), (dict(qr=256 + 8), 1), (dict(qo=256 + 1), 1),
     (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1), (dict(theta=0.0), 1),
-    (dict(theta=float("nan")), 1), (dict(scale=0.0), 1), (dict(D=96), 2), (dict(Hq=34, Hkv=2), 2),
+    (dict(theta=float("nan")), 1), (dict(scale=0.0), 1), (dict(D=96), 2),
+    (dict(Hq=34, Hkv=2), 2),  # G = 17: the fused prologue takes at most 16 rows per kv head
     (dict(wsb=64), 3), (dict(kind=9), 1),
 ])
 def test_run_prologue_rejects_bad_arguments_without_launching(L, bad, expect):
@@ -275,6 +277,8 @@ def test_decode_num_ctas_rejects_bad_geometry(L):
     assert L.hpa_decode_num_ctas(0, 64, 0, 1) == -1
     assert L.hpa_decode_num_ctas(0, 64, 8, 0) == -1
     assert L.hpa_decode_num_ctas(0, 60, 8, 1) == -1  # Hq not a multiple of Hkv
+    assert L.hpa_decode_num_ctas(0, 64, 8, 5) == -1  # 40 rows per kv head
+    assert L.hpa_decode_num_ctas(0, 33, 1, 1) == -1
 
 
 def test_num_ctas_environment_override():
@@ -305,7 +309,7 @@ def _step_call(L, **kw):
 @pytest.mark.parametrize("bad,expect", [
     (dict(sl=None), 1), (dict(q=None), 1), (dict(B=0), 1), (dict(n=0), 1),
     (dict(B=513), 2),                  # tile offsets of at most 512 sequences in shared memory
-    (dict(n=65537), 2), (dict(T=3, Hq=64, Hkv=8), 2), (dict(wsb=64), 3), (dict(D=96), 2),
+    (dict(n=65537), 2), (dict(T=5, Hq=64, Hkv=8), 2), (dict(wsb=64), 3), (dict(D=96), 2),
 ])
 def test_step_rejects_bad_arguments_without_launching(L, bad, expect):
     assert _step_call(L, **bad) == expect

@@ -471,11 +471,46 @@ def test_multi_token_decode_matches_oracle(Hq, Hkv, D, T, kind, num_ctas):
     _check(out, ref)
 
 
+@pytest.mark.parametrize("Hq,Hkv,D,T,fp8", [
+    (64, 8, 128, 4, False),   # G = 8, four query tokens: 32 rows
+    (32, 2, 128, 2, False),   # G = 16, two tokens
+    (24, 2, 64, 2, False),    # 24 rows: padded to four n-tiles
+    (64, 8, 128, 3, True),    # 24 rows, FP8 KV
+    (32, 1, 128, 1, False),   # one kv head for 32 query heads, single token
+    (24, 1, 64, 1, False),
+])
+@pytest.mark.parametrize("kind,num_ctas", [(0, None), (0, 7), (1, None), (2, None), (3, None)])
+def test_wide_query_groups_match_oracle(Hq, Hkv, D, T, fp8, kind, num_ctas):
+    """17..32 query rows per kv head (G x T): one warp per MMA n-tile over the
+    whole tile, one CTA per SM, against the oracle on every plan kind."""
+    shape = W.DecodeShape("wide", Hq, Hkv, D, kv_dtype="fp8_e4m3" if fp8 else "bf16",
+                          q_tokens=T)
+    batch = W.make_batch(shape, MT_LENS, seed=35)
+    q8 = quantize_fp8(batch) if fp8 else None
+    kc, vc = (bits16(batch.k_cache), bits16(batch.v_cache)) if q8 is None else (q8[0], q8[2])
+    kw = {} if q8 is None else dict(kv_fp8=True, k_scale=q8[1], v_scale=q8[3])
+    if T == 1:
+        ref = oracle.paged_decode(bits16(batch.q), kc, vc, batch.page_table.numpy(),
+                                  batch.seq_lens.numpy(), Hkv, 1 / math.sqrt(D), **kw)
+        to_device(batch)
+        out = gpu_decode(batch, kind=kind, num_ctas=num_ctas, out_dtype=torch.float32, fp8=q8)
+    else:
+        ref = oracle.paged_decode_multi(bits16(batch.q), kc, vc, batch.page_table.numpy(),
+                                        batch.seq_lens.numpy(), Hkv, 1 / math.sqrt(D), **kw)
+        out = gpu_decode_multi(batch, kind=kind, num_ctas=num_ctas, out_dtype=torch.float32,
+                               fp8=q8)
+    _check(out, ref, max_abs=FP8_MAX_ABS if fp8 else MAX_ABS)
+
+
 def test_decode_num_ctas_matches_residency():
     two = hpa.default_num_ctas()
     # 8 rows per kv head, and 16 (two n-tiles, warps split by n-tile): 2 CTAs / SM
     for args in ((64, 8, 1), (64, 8, 2), (32, 2, 1), (8, 2, 2)):
         assert hpa.decode_num_ctas(*args) == two, args
+    # 17..32 rows per kv head: one CTA per SM
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for args in ((64, 8, 3), (64, 8, 4), (32, 1, 1), (24, 2, 2)):
+        assert hpa.decode_num_ctas(*args) == sms, args
 
 
 def test_multi_token_fp8_and_bf16_out():
@@ -683,6 +718,8 @@ STEP_CASES = [
     ("mt4_d64", [130, 64, 1000], 16, 4, 64, 4, 5),
     ("max_batch", [int(x) for x in np.random.default_rng(7).integers(0, 400, 512)], 8, 2, 64, 1,
      None),
+    ("g32", [129, 2000, 5, 64], 32, 1, 128, 1, None),      # 32 rows: four n-tiles
+    ("mt4_g8", [65, 300, 2, 4097], 64, 8, 128, 4, None),  # 32 rows of four query tokens
 ]
 
 
@@ -875,8 +912,8 @@ def _random_case(seed):
     D = int(rng.choice([64, 128]))
     fp8 = D == 128 and rng.random() < 0.3
     Hkv = int(rng.choice([1, 2, 4, 8]))
-    G = int(rng.integers(1, 17))
-    T = int(rng.integers(1, 16 // G + 1)) if rng.random() < 0.4 else 1
+    G = int(rng.integers(1, 33))
+    T = int(rng.integers(1, 32 // G + 1)) if rng.random() < 0.4 else 1
     B = int(rng.integers(1, 12))
     lens = [int(x) for x in rng.choice([0, 1, 63, 64, 65, 127, 129, 700, 2000, 5000], B)]
     lens = [L + int(rng.integers(0, 3)) for L in lens]
@@ -894,8 +931,8 @@ def _random_case(seed):
 @pytest.mark.parametrize("seed", range(24))
 def test_random_configurations_match_oracle(seed):
     """Seeded random shapes through plan + run (plan kinds, tail shapes, CTA
-    counts, group sizes 1..16, head_dim 64/128, 1..16 query tokens per
-    sequence, bf16 or FP8 KV, bf16 or fp32 output) against the oracle."""
+    counts, group sizes 1..32, head_dim 64/128, up to 32 query rows per kv
+    head, bf16 or FP8 KV, bf16 or fp32 output) against the oracle."""
     c = _random_case(seed)
     D, Hkv, G, T = c["D"], c["Hkv"], c["G"], c["T"]
     Hq = G * Hkv
