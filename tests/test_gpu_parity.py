@@ -796,13 +796,15 @@ def test_step_flags_clamped_lengths():
 
 # ---------------------------------------------------------------- canaries
 
-@pytest.mark.parametrize("kind,num_ctas,T", [(0, None, 1), (0, 5, 1), (1, None, 1),
-                                             (2, 7, 1), (0, None, 2)])
-def test_writes_stay_inside_out_and_workspace(kind, num_ctas, T):
+@pytest.mark.parametrize("kind,num_ctas,T,Hq", [(0, None, 1, 32), (0, 5, 1, 32), (1, None, 1, 32),
+                                                (2, 7, 1, 32), (0, None, 2, 32),
+                                                (0, None, 4, 64), (1, None, 1, 256)])
+def test_writes_stay_inside_out_and_workspace(kind, num_ctas, T, Hq):
     """Guard bytes around the output and the workspace, and the whole KV
     cache, are unchanged by plan + run (compute-sanitizer is not available,
-    so out-of-range writes are looked for this way)."""
-    Hq, Hkv, D = 32, 8, 128
+    so out-of-range writes are looked for this way); the last two cases run
+    the four-n-tile kernel (32 query rows per kv head)."""
+    Hkv, D = 8, 128
     batch = W.make_batch(W.DecodeShape("canary", Hq, Hkv, D, q_tokens=T),
                          [0, 1, 64, 65, 4000, 300], seed=41)
     to_device(batch)
