@@ -8,15 +8,17 @@ it raises ``HpaLibraryMissing`` -- there is no fallback implementation.
 
 The functions mirror the C ABI in ``include/hpa.h``:
 
-    decode_workspace_size, plan_grid, default_num_ctas, workspace_layout,
-    decode_plan, decode_run, decode_step, decode_run_multi, decode_run_prologue, kv_prologue,
-    merge_states, read_status,
-    decode_noalloc
+    decode_workspace_size, plan_grid, default_num_ctas, decode_num_ctas,
+    workspace_layout, decode_plan (with ``tail=`` for hpa_decode_plan_tail),
+    decode_run, decode_step (+ ``lse=``: hpa_decode_step_lse), decode_step_prologue,
+    decode_run_multi, decode_run_prologue, kv_prologue, merge_states,
+    read_status, read_cta_times, decode_noalloc, noalloc_read_status
 
-and ``PagedDecoder`` bundles a workspace with plan + run for callers who do
-not want to manage it.  ``mixed_length_paged_b200.sharding`` spreads a batch
-over the ranks of a process group (by kv head, or by page range with a
-log-sum-exp merge of the ranks' states).
+plus ``tail_idle`` (a summary of read_cta_times), and ``PagedDecoder``
+bundles a workspace with plan + run for callers who do not want to manage
+it.  ``mixed_length_paged_b200.sharding`` spreads a batch over the ranks of a
+process group (by kv head, or by page with a log-sum-exp merge of the ranks'
+states).
 """
 from __future__ import annotations
 
