@@ -69,7 +69,7 @@ def _declare(L):
     L.oracle_plan_grid.restype = _L
     L.oracle_plan_grid.argtypes = [_I, _I, _I, _I, _I, _I, _I]
     L.oracle_plan.restype = _I
-    L.oracle_plan.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
+    L.oracle_plan.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                               _P, _P, _P]
     L.oracle_num_threads.restype = _I
     L.oracle_num_threads.argtypes = []
@@ -316,12 +316,15 @@ def plan_grid(kind, batch, num_kv_heads, num_ctas, param=0, max_seq_len=0, page_
 
 def plan(seq_lens, num_kv_heads: int, *, kind: int = 0, num_ctas: int, param: int = 0,
          max_seq_len: int = 0, capacity_tokens: int, tail: tuple[int, int, int],
-         page_size: int = 64) -> dict:
+         cost: tuple[int, int] = (1, 0), page_size: int = 64) -> dict:
     """The plan of ``kind`` (oracle.c, oracle_plan).  ``tail = (den, k, mn)``
-    picks the member of the dynamic family (kinds 0 and 3): if U >= mn P, the
-    last min(U // den, U - P) units in min(k P, that) run-time chunks;
-    (0, 1, 0) is the plain even partition.  It is required, so that every
-    caller states which member it checks."""
+    and ``cost = (q, e)`` pick the member of the dynamic family (kinds 0 and
+    3): if U >= mn P, the last min(U // den, U - P) units in min(k P, that)
+    run-time chunks; the primary ranges split the cost of the other units
+    evenly, q per unit and e more per segment end.  tail = (0, 1, 0) with
+    cost = (1, 0) is the plain even partition.  The tail is required, so that
+    every caller states which member it checks; cost (1, 0) -- the units
+    themselves split evenly -- is the default."""
     sl = _c(seq_lens, np.int32)
     B = sl.shape[0]
     grid = plan_grid(kind, B, num_kv_heads, num_ctas, param, max_seq_len, page_size)
@@ -335,7 +338,7 @@ def plan(seq_lens, num_kv_heads: int, *, kind: int = 0, num_ctas: int, param: in
     n_ranges = C.c_int32()
     rc = lib().oracle_plan(_ptr(sl), B, num_kv_heads, page_size, capacity_tokens, kind,
                            num_ctas, param, max_seq_len, int(tail[0]), int(tail[1]),
-                           int(tail[2]),
+                           int(tail[2]), int(cost[0]), int(cost[1]),
                            _ptr(lens), _ptr(tile_start),
                            _ptr(cta), _ptr(split_count), _ptr(first_slot), C.byref(n_units),
                            C.byref(n_ranges))

@@ -429,10 +429,18 @@ void oracle_lse_merge(const double* acc, const double* m, const double* l, int n
  *     per CTA k and the least units per CTA mn for a tail.  If den > 0 and
  *     U >= mn P, Ut = min(floor(U / den), U - P) (every primary range keeps
  *     at least one unit); otherwise there is no tail, Ut = 0.  M = min(k P, Ut).
- *     With U1 = U - Ut, range c < P is [floor(c U1 / P), floor((c+1) U1 / P))
- *     and range P + j is [U1 + floor(j Ut / M), U1 + floor((j+1) Ut / M)).
- *     With den = 0 the ranges are the plain even partition
- *     [floor(c U / P), floor((c+1) U / P)).  Grid = P; V = P + M ranges.
+ *     With U1 = U - Ut, range P + j is [U1 + floor(j Ut / M),
+ *     U1 + floor((j+1) Ut / M)).  The P primary ranges split the first U1
+ *     units so that each carries an even share of their cost, two more
+ *     parameters of the family: every unit costs q (unit_cost) and the last
+ *     unit of each segment e (end_cost) more.  With K(x) the summed cost of
+ *     units [0, x), primary range c starts at the largest x <= U1 with
+ *     P K(x) <= c K(U1), and ends where range c + 1 starts (range P - 1 at
+ *     U1).  The weights apply only if K(U1) >= (q + e) P, so that no primary
+ *     range is empty; otherwise, and always with e = 0, range c is
+ *     [floor(c U1 / P), floor((c+1) U1 / P)) -- with den = 0 too, the plain
+ *     even partition [floor(c U / P), floor((c+1) U / P)).  Grid = P;
+ *     V = P + M ranges.
  *   kind 1, static fixed split count S (param, default ceil(P / (B Hkv))):
  *     one CTA per (segment, split i); each segment's n tiles cut into
  *     chunks of ceil(n / S) tiles, chunk i = [i C, min((i+1) C, n)).
@@ -497,13 +505,14 @@ static long snap_cut(long x, long U, long m, const int32_t* unit_seg, const int3
 
 int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capacity_tokens,
                 int kind, int num_ctas, int param, int max_seq_len, int tail_den,
-                int tail_chunks, int tail_min, int32_t* lens_out,
+                int tail_chunks, int tail_min, int unit_cost, int end_cost, int32_t* lens_out,
                 int32_t* tile_start, int32_t* cta_desc /* [<= 5*grid][2] */,
                 int32_t* split_count /* [B*Hkv] */, int32_t* first_slot /* [B*Hkv] */,
                 int32_t* n_units_out, int32_t* n_ranges_out) {
   if (B <= 0 || Hkv <= 0 || page_size <= 0 || num_ctas <= 0 || kind < 0 || kind > 3)
     return ORC_BAD_ARG;
-  if (tail_den < 0 || tail_chunks < 1 || tail_min < 0) return ORC_BAD_ARG;
+  if (tail_den < 0 || tail_chunks < 1 || tail_min < 0 || unit_cost < 1 || end_cost < 0)
+    return ORC_BAD_ARG;
   long grid = oracle_plan_grid(kind, B, Hkv, num_ctas, param, max_seq_len, page_size);
   int S = B * Hkv;
   /* 1. lengths clamped to [0, capacity], tiles per sequence, tile offsets */
@@ -549,10 +558,29 @@ int oracle_plan(const int32_t* seq_lens, int B, int Hkv, int page_size, int capa
       if (tail_den > 0 && U >= (long)tail_min * P) Ut = U / tail_den < U - P ? U / tail_den : U - P;
       long U1 = U - Ut;
       long M = (long)tail_chunks * P < Ut ? (long)tail_chunks * P : Ut;
-      for (long c = 0; c < P; ++c) {
-        beg[c] = c * U1 / P;
-        end[c] = (c + 1) * U1 / P;
+      /* K[x] = cost of units [0, x): q per unit, e more for a segment's last */
+      long* K = malloc(sizeof(long) * (U1 + 1));
+      K[0] = 0;
+      for (long x = 0; x < U1; ++x) {
+        int last = (x + 1 == U) || unit_seg[x + 1] != unit_seg[x];
+        K[x + 1] = K[x] + unit_cost + (last ? end_cost : 0);
       }
+      if (end_cost > 0 && K[U1] >= (long)(unit_cost + end_cost) * P) {
+        /* start of range c: the largest x <= U1 with P K[x] <= c K[U1]; the
+         * starts do not decrease in c, so one forward scan finds them all */
+        long x = 0;
+        for (long c = 0; c <= P; ++c) {
+          while (x < U1 && P * K[x + 1] <= c * K[U1]) ++x;
+          if (c < P) beg[c] = x;
+          if (c > 0) end[c - 1] = x;
+        }
+      } else {
+        for (long c = 0; c < P; ++c) {
+          beg[c] = c * U1 / P;
+          end[c] = (c + 1) * U1 / P;
+        }
+      }
+      free(K);
       for (long j = 0; j < M; ++j) {
         beg[P + j] = U1 + j * Ut / M;
         end[P + j] = U1 + (j + 1) * Ut / M;

@@ -442,7 +442,7 @@ def _units(lens, Hkv):
     return out
 
 
-def _check_plan_invariants(p, lens, Hkv, kind, tail=None):
+def _check_plan_invariants(p, lens, Hkv, kind, tail=None, cost=(1, 0)):
     units = _units(lens, Hkv)
     U = len(units)
     assert p["n_units"] == U
@@ -495,7 +495,7 @@ def _check_plan_invariants(p, lens, Hkv, kind, tail=None):
     used = [x for ps in pieces.values() for x in ps]
     assert len(used) == len(set(used)) and all(0 <= x < 2 * R for x in used)
     if kind == 0:
-        _check_dynamic_family(p, U, tail)
+        _check_dynamic_family(p, U, tail, _unit_costs(units, cost))
 
 
 def _even_ranges(n, m):
@@ -516,13 +516,50 @@ def _even_ranges(n, m):
     return out
 
 
-def _check_dynamic_family(p, U, tail):
-    """A dynamic plan of the family (den, k, mn): the primary ranges are the
-    even partition of the first U1 units over P CTAs and the tail chunks the
-    even partition of the last Ut units over M chunks, where Ut is the largest
-    tail with Ut <= U / den that still leaves every primary range a unit (no
-    tail for den = 0 or when U < mn P) and M the largest chunk count with
-    M <= k P and M <= Ut."""
+def _unit_costs(units, cost):
+    """Cost of every unit of the list under cost weights (q, e): q, plus e
+    for the last unit of its (sequence, kv head) segment."""
+    q, e = cost
+    out = []
+    for i, (b, g, t) in enumerate(units):
+        last = i + 1 == len(units) or units[i + 1][:2] != (b, g)
+        out.append(q + (e if last else 0))
+    return out
+
+
+def _cost_ranges(costs, m):
+    """Units with the given costs cut into m contiguous ranges of even cost,
+    enumerated from scratch: lay the units end to end on a line, each as long
+    as its cost, scale the line onto m equal ranges and give unit u the range
+    in which its right end falls, each range closed on the right (with unit
+    costs this is _even_ranges).  Exact rational arithmetic."""
+    right, acc = [], 0
+    for c in costs:
+        acc += c
+        right.append(acc)
+    owner = [math.ceil(Fraction(r * m, acc)) - 1 for r in right]
+    out = []
+    for c in range(m):
+        us = [u for u in range(len(costs)) if owner[u] == c]
+        if us:
+            assert us == list(range(us[0], us[-1] + 1))
+            out.append((us[0], us[-1] + 1))
+        else:
+            b = out[-1][1] if out else 0
+            out.append((b, b))
+    return out
+
+
+def _check_dynamic_family(p, U, tail, costs=None):
+    """A dynamic plan of the family (den, k, mn; q, e): the primary ranges
+    cut the first U1 units into P ranges of even cost (every unit q, a
+    segment's last unit e more: `costs`, None = all equal) if that cost is at
+    least the largest unit cost times P, else of even unit count (so that no
+    primary range is empty), and the tail chunks
+    are the even partition of the last Ut units over M chunks, where Ut is the
+    largest tail with Ut <= U / den that still leaves every primary range a
+    unit (no tail for den = 0 or when U < mn P) and M the largest chunk count
+    with M <= k P and M <= Ut."""
     den, k, mn = tail
     P = p["grid"]
     R = p["ranges"]
@@ -543,7 +580,12 @@ def _check_dynamic_family(p, U, tail):
             assert M == k * P or M == Ut
         else:
             assert M == 0
-    assert cta[:P] == _even_ranges(U - Ut, P)
+    prim = costs[:U - Ut] if costs is not None else None
+    if prim is None or sum(prim) < max(costs) * P:
+        assert cta[:P] == _even_ranges(U - Ut, P)
+    else:
+        assert cta[:P] == _cost_ranges(prim, P)
+    assert all(a < e for a, e in cta[:P])  # no primary range is empty
     assert [(a - (U - Ut), e - (U - Ut)) for a, e in cta[P:]] == (_even_ranges(Ut, M) if M else [])
 
 
@@ -571,6 +613,100 @@ def test_even_ranges_enumerator_hand_cases():
     assert _even_ranges(3, 5) == [(0, 0), (0, 1), (1, 1), (1, 2), (2, 3)]
     assert _even_ranges(6, 3) == [(0, 2), (2, 4), (4, 6)]
     assert _even_ranges(10, 4) == [(0, 2), (2, 5), (5, 7), (7, 10)]
+    # with costs: unit costs give the even ranges; costs (1, 1, 3, 1) over 2
+    # ranges: right ends 1, 2, 5, 6 scaled by 2/6 -> 1/3, 2/3, 5/3, 2
+    assert _cost_ranges([1] * 7, 3) == _even_ranges(7, 3)
+    assert _cost_ranges([1, 1, 3, 1], 2) == [(0, 2), (2, 4)]
+    # (5, 1, 1, 1): right ends 5..8 of 8 all lie past the midpoint 4, so
+    # every unit goes to range 1 and range 0 is empty
+    assert _cost_ranges([5, 1, 1, 1], 2) == [(0, 0), (0, 4)]
+
+
+# A batch worked by hand: lens (5, 64, 700, 0, 1, 3000, 130) tokens are
+# (1, 1, 11, 0, 1, 47, 3) tiles; with 2 kv heads the 128 units form 12
+# segments whose last units are 0, 1, 2, 3, 14, 25, 26, 27, 74, 121, 124,
+# 127.  Seven CTAs, no tail.
+#   cost (1, 1): K(x) = x + (segment ends before x), K(128) = 140; cut c is
+#     the largest x with K(x) <= 20 c: K(15) = 15 + 5 = 20, K(32) = 32 + 8 =
+#     40, K(52) = 60, K(72) = 80, K(91) = 91 + 9 = 100, K(111) = 120.
+#   cost (2, 1): K(x) = 2x + ends, K(128) = 268, cut c at K(x) <= floor(268
+#     c / 7) = 38, 76, 114, 153, 191, 229: x = 16 (K 37), 34 (76), 53 (114),
+#     72 (152), 91 (191), 110 (229).
+_HAND_LENS = [5, 64, 700, 0, 1, 3000, 130]
+_HAND_CUTS = {
+    (1, 0): [0, 18, 36, 54, 73, 91, 109, 128],
+    (1, 1): [0, 15, 32, 52, 72, 91, 111, 128],
+    (2, 1): [0, 16, 34, 53, 72, 91, 110, 128],
+}
+
+
+@pytest.mark.parametrize("cost", sorted(_HAND_CUTS))
+def test_cost_weighted_cuts_hand_case(cost):
+    p = oracle.plan(np.array(_HAND_LENS, dtype=np.int32), 2, kind=0, num_ctas=7,
+                    capacity_tokens=4096, tail=(0, 1, 0), cost=cost)
+    cuts = _HAND_CUTS[cost]
+    assert p["n_units"] == 128 and p["ranges"] == 7
+    assert [(int(a), int(e)) for a, e in p["cta"]] == list(zip(cuts[:-1], cuts[1:]))
+
+
+@pytest.mark.parametrize("lens,Hkv,P", [
+    ([131072] + [4096] * 31, 8, 148),
+    ([512] * 64, 8, 148),
+    ([37, 200], 2, 3),
+    ([0, 5, 0, 64, 65, 3000, 1], 4, 7),
+    ([1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7] * 3, 8, 296),
+    ([64] * 40 + [6400] * 3, 2, 37),
+])
+@pytest.mark.parametrize("tail,cost", [((0, 1, 0), (1, 1)), ((0, 1, 0), (2, 1)),
+                                       ((8, 4, 0), (4, 3)), ((8, 4, 32), (1, 4)),
+                                       ((3, 2, 0), (3, 2))])
+def test_cost_weighted_plan_invariants(lens, Hkv, P, tail, cost):
+    """Cost-weighted primary ranges: coverage, slots and split counts as for
+    any plan, and the primary cuts those of the from-scratch enumerator."""
+    p = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=0, num_ctas=P,
+                    capacity_tokens=max(64, max(lens)), tail=tail, cost=cost)
+    _check_plan_invariants(p, lens, Hkv, 0, tail, cost)
+
+
+@pytest.mark.parametrize("lens,Hkv,P", [([64] * 500, 4, 148), ([1, 30, 64] * 70, 2, 37),
+                                        ([10] * 7, 1, 3)])
+@pytest.mark.parametrize("cost", [(1, 1), (2, 1), (3, 4)])
+def test_cost_weights_do_not_move_cuts_when_all_units_cost_the_same(lens, Hkv, P, cost):
+    """Every segment a single tile: every unit costs q + e, so the cost split
+    is the even split of the units, the plan of cost (1, 0)."""
+    kw = dict(kind=0, num_ctas=P, capacity_tokens=64, tail=(8, 4, 0))
+    a = oracle.plan(np.array(lens, dtype=np.int32), Hkv, cost=cost, **kw)
+    b = oracle.plan(np.array(lens, dtype=np.int32), Hkv, cost=(1, 0), **kw)
+    np.testing.assert_array_equal(a["cta"], b["cta"])
+
+
+@pytest.mark.parametrize("q", [1, 2, 3, 4])
+def test_end_cost_zero_is_the_even_split_for_any_unit_cost(q):
+    lens = [1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7]
+    kw = dict(kind=0, num_ctas=37, capacity_tokens=5056, tail=(8, 4, 0))
+    a = oracle.plan(np.array(lens, dtype=np.int32), 8, cost=(q, 0), **kw)
+    b = oracle.plan(np.array(lens, dtype=np.int32), 8, cost=(1, 0), **kw)
+    np.testing.assert_array_equal(a["cta"], b["cta"])
+
+
+def test_cost_weighted_ranges_are_balanced_in_cost():
+    """Each primary range's cost is within one unit's largest cost (q + e) of
+    the mean, and a range of many short segments holds fewer units than one
+    inside a long segment."""
+    lens = [64] * 300 + [64 * 900]
+    q, e = 2, 3
+    P = 50
+    p = oracle.plan(np.array(lens, dtype=np.int32), 1, kind=0, num_ctas=P, capacity_tokens=64 * 900,
+                    tail=(0, 1, 0), cost=(q, e))
+    costs = _unit_costs(_units(lens, 1), (q, e))
+    K1 = sum(costs)
+    sizes = []
+    for a, b in p["cta"]:
+        c = sum(costs[int(a):int(b)])
+        assert abs(c - K1 / P) < q + e
+        sizes.append(int(b - a))
+    # 300 single-tile segments cost 5 each (1500), the long one 2 per unit (1803)
+    assert sizes[0] < sizes[-1]
 
 
 @pytest.mark.parametrize("U,P", [(5, 5), (6, 5), (7, 3), (100, 7), (32256, 148), (4096, 296),

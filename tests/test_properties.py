@@ -76,17 +76,18 @@ def test_page_shard_properties(lens, N, extra, seed):
 @settings(max_examples=60, deadline=None)
 @given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
        kind=st.sampled_from([0, 1, 2]), param=st.integers(0, 9),
-       den=st.integers(0, 40), k=st.integers(1, 4), mn=st.integers(0, 40))
-def test_plan_kinds_properties(lens, Hkv, P, kind, param, den, k, mn):
+       den=st.integers(0, 40), k=st.integers(1, 4), mn=st.integers(0, 40),
+       q=st.integers(1, 4), e=st.integers(0, 4))
+def test_plan_kinds_properties(lens, Hkv, P, kind, param, den, k, mn, q, e):
     """Every plan kind covers each unit exactly once with contiguous ranges,
     consecutive holders per segment and distinct partial slots; a dynamic plan
-    of any tail shape (den, k, mn) has the even primary ranges and the even
-    tail chunks of that shape."""
+    of any tail shape (den, k, mn) and cost weights (q, e) has the primary
+    ranges of even cost and the even tail chunks of that shape."""
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
     p = oracle.plan(sl, Hkv, kind=kind, num_ctas=P, param=param if kind else 0,
-                    max_seq_len=max(lens), capacity_tokens=cap, tail=(den, k, mn))
-    _check_plan_invariants(p, lens, Hkv, kind, (den, k, mn))
+                    max_seq_len=max(lens), capacity_tokens=cap, tail=(den, k, mn), cost=(q, e))
+    _check_plan_invariants(p, lens, Hkv, kind, (den, k, mn), (q, e))
     assert p["n_units"] == len(_units(lens, Hkv))
 
 
