@@ -91,7 +91,7 @@ typedef enum { HPA_OUT_BF16 = 0, HPA_OUT_F32 = 1 } hpa_out_dtype;
  * x HPC-Ops", Attention Backend: nearly-finished short requests first, long
  * ones spread over the grid); see hpa_decode_plan. */
 typedef enum {
-  HPA_PLAN_DYNAMIC = 0,        /* param unused; tail shape: hpa_decode_plan_tail */
+  HPA_PLAN_DYNAMIC = 0,        /* param unused; tail and cost weights: hpa_decode_plan_shape */
   HPA_PLAN_STATIC_NSPLIT = 1,  /* param = splits per (seq, kv head); 0 = ceil(num_ctas / (B Hkv)) */
   HPA_PLAN_STATIC_CHUNK = 2,   /* param = tiles per split; 0 = ceil(T_max / ceil(num_ctas / Hkv)) */
   HPA_PLAN_LENGTH_AWARE = 3    /* param = smallest end piece of a cut segment, tiles; 0 = 4 */
@@ -109,12 +109,35 @@ typedef enum {
  * batch of a few tiles per CTA its one-tile chunks cost more in partials and
  * merge work than they save, hence tail_min.  hpa_decode_plan, the in-kernel
  * plans (hpa_decode_step*) and hpa_decode_noalloc use the defaults;
- * hpa_decode_plan_tail takes all three as arguments.  HPA_TAIL_CHUNKS_MAX
+ * hpa_decode_plan_shape takes all three as arguments.  HPA_TAIL_CHUNKS_MAX
  * bounds tail_chunks (the workspace has room for that many chunks per CTA). */
 #define HPA_TAIL_DEN_DEFAULT 8
 #define HPA_TAIL_CHUNKS_DEFAULT 4
 #define HPA_TAIL_MIN_DEFAULT 32
 #define HPA_TAIL_CHUNKS_MAX 4
+
+/* Cost weights of the primary ranges of the DYNAMIC and LENGTH_AWARE plans
+ * (see hpa_decode_plan): every unit costs unit_cost and the last unit of each
+ * (sequence, kv head) segment end_cost more -- the segment's end, where its
+ * state is handed over and combined, takes time of its own, so a range of
+ * many short segments runs longer than one of as many units of a long one.
+ * The primary ranges split the primary units' total cost evenly, provided
+ * that total is at least (unit_cost + end_cost) times the CTA count, so that
+ * no primary range is empty; below that, and always with end_cost = 0, they
+ * split the units themselves evenly.  Like the tail, these are this
+ * library's tuning, not part of the method.  hpa_decode_plan uses
+ * (HPA_COST_UNIT_DEFAULT, HPA_COST_END_DEFAULT) = (1, 0), and so do the
+ * in-kernel plans (hpa_decode_step*, hpa_decode_noalloc) for bf16 caches; for
+ * e4m3 caches, whose 64-token tiles stream in half the time of a bf16 tile so
+ * that a segment end weighs twice as much, they use (1,
+ * HPA_COST_END_DEFAULT_FP8) = (1, 2) (measured: a batch of many short
+ * sequences runs 16 % faster, long ones as before).  hpa_decode_plan_shape
+ * takes any weights, each in 0 .. HPA_COST_MAX (unit_cost >= 1); with (1, 2)
+ * it gives an e4m3 run the in-kernel plan's ranges. */
+#define HPA_COST_UNIT_DEFAULT 1
+#define HPA_COST_END_DEFAULT 0
+#define HPA_COST_END_DEFAULT_FP8 2
+#define HPA_COST_MAX 4
 
 /* Bits of the device status word (hpa_read_status). */
 #define HPA_DEVICE_LEN_CLAMPED 0x1  /* a seq_len < 0 or > pt_stride * 64 was clamped */
@@ -163,8 +186,8 @@ HPA_API size_t hpa_decode_workspace_size(hpa_plan_kind kind, int batch, int num_
  * offsets[0..6] = header (int32[32]: magic, status, units, grid, kind, batch,
  * kv heads, group, head_dim, tiles, ranges V, next tail chunk, finished CTAs,
  * tail_den, tail_chunks, tail_min (0 for the static kinds), split segments
- * listed for the merge (two counts, by step parity), the step parity, then
- * zeros), lens,
+ * listed for the merge (two counts, by step parity), the step parity,
+ * unit_cost, end_cost (0 for the static kinds), then zeros), lens,
  * tile_start, range descriptors (int32 x8 per range: u_begin, u_end, then
  * the sequence, kv head, tile and tile count of its first unit, 0, 0),
  * segment descriptors (int32 x2 per (sequence, kv head): slot of its first
@@ -187,7 +210,11 @@ HPA_API hpa_status hpa_workspace_layout(hpa_plan_kind kind, int batch, int num_k
  * last Ut units (Ut from the tail shape above: min(floor(U/8), U - P) by
  * default when U >= 32 P, else 0) form M tail chunks (min(4P, Ut) by default)
  * [U1 + floor(jUt/M), U1 + floor((j+1)Ut/M)) and the first U1 = U - Ut units
- * the P primary ranges [floor(cU1/P), floor((c+1)U1/P)).  CTA c runs primary
+ * the P primary ranges.  With the cost weights q = unit_cost, e = end_cost
+ * (above) and K(x) = q x + e n(x), n(x) the number of segments whose last
+ * unit comes before unit x, primary range c is [x_c, x_(c+1)) where x_c is
+ * the largest x <= U1 with P K(x) <= c K(U1), if K(U1) >= (q + e) P; else,
+ * and for e = 0, it is [floor(cU1/P), floor((c+1)U1/P)).  CTA c runs primary
  * range c, then takes tail chunks in order from a counter as it finishes, so
  * CTAs that got more HBM bandwidth do more of the tail.  A short sequence
  * lands whole in one range; a long one is spread over many.  The STATIC
@@ -225,10 +252,11 @@ HPA_API hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int num_k
                            size_t ws_bytes, int* grid_out, void* stream);
 
 /*
- * hpa_decode_plan_tail -- hpa_decode_plan for the DYNAMIC or LENGTH_AWARE kind
- * with the run-time tail's shape given explicitly (xiaodao.ai "HPC-Ops TPOT
- * -48.8%", Attention section: the even spread of the tile list; bitbyai.com
- * "vLLM x HPC-Ops", Attention Backend: progress evaluated at run time).
+ * hpa_decode_plan_shape -- hpa_decode_plan for the DYNAMIC or LENGTH_AWARE
+ * kind with the run-time tail's shape and the cost weights of the primary
+ * ranges given explicitly (xiaodao.ai "HPC-Ops TPOT -48.8%", Attention
+ * section: the even spread of the tile list; bitbyai.com "vLLM x HPC-Ops",
+ * Attention Backend: progress evaluated at run time).
  *
  *   tail_den     0 .. 2^20: the tail holds min(floor(U / tail_den), U - P)
  *                units; 0 = no tail (the primary ranges are the even
@@ -236,19 +264,22 @@ HPA_API hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int num_k
  *   tail_chunks  1 .. HPA_TAIL_CHUNKS_MAX: the tail is cut into
  *                min(tail_chunks * P, Ut) chunks (ignored if the tail is empty).
  *   tail_min     0 .. 2^20: no tail unless U >= tail_min * P.
+ *   unit_cost    1 .. HPA_COST_MAX: cost of one unit.
+ *   end_cost     0 .. HPA_COST_MAX: extra cost of a segment's last unit;
+ *                0 = the primary ranges split the units evenly.
  *   the rest     as for hpa_decode_plan (max_seq_len is not needed).
  * Any other kind, or a parameter out of range, returns HPA_ERR_INVALID_ARG.
  * The workspace size and hpa_decode_run's arguments do not depend on the
- * tail shape.  hpa_decode_plan(kind, ...) equals hpa_decode_plan_tail(kind,
- * ..., HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT, HPA_TAIL_MIN_DEFAULT,
- * ...).
+ * shape.  hpa_decode_plan(kind, ...) equals hpa_decode_plan_shape(kind, ...,
+ * HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT, HPA_TAIL_MIN_DEFAULT,
+ * HPA_COST_UNIT_DEFAULT, HPA_COST_END_DEFAULT, ...).
  */
-HPA_API hpa_status hpa_decode_plan_tail(const int32_t* seq_lens, int batch, int num_kv_heads,
-                                        int num_q_heads, int head_dim, int pt_stride,
-                                        hpa_plan_kind kind, int num_ctas, int param,
-                                        int tail_den, int tail_chunks, int tail_min,
-                                        void* workspace, size_t ws_bytes, int* grid_out,
-                                        void* stream);
+HPA_API hpa_status hpa_decode_plan_shape(const int32_t* seq_lens, int batch, int num_kv_heads,
+                                         int num_q_heads, int head_dim, int pt_stride,
+                                         hpa_plan_kind kind, int num_ctas, int param,
+                                         int tail_den, int tail_chunks, int tail_min,
+                                         int unit_cost, int end_cost, void* workspace,
+                                         size_t ws_bytes, int* grid_out, void* stream);
 
 /*
  * hpa_decode_run -- persistent paged GQA decode attention with split-KV
@@ -326,7 +357,9 @@ HPA_API hpa_status hpa_decode_run_multi(const void* q, const void* k_cache, cons
  * plan; here each persistent CTA scans the lengths itself and derives its own
  * ranges from the same closed forms, so the step needs no plan kernel and no
  * wait for one).  Same partition, same partial slots and merge order, hence
- * the same bits as the two-call path.
+ * the same bits as the two-call path -- for an e4m3 cache that path's plan
+ * is hpa_decode_plan_shape with the cost weights (HPA_COST_UNIT_DEFAULT,
+ * HPA_COST_END_DEFAULT_FP8) (see the cost weights above).
  *
  *   seq_lens     device [batch] int32, as for hpa_decode_plan.
  *   batch        1 .. 512 (the tile offsets live in shared memory;

@@ -9,7 +9,7 @@ it raises ``HpaLibraryMissing`` -- there is no fallback implementation.
 The functions mirror the C ABI in ``include/hpa.h``:
 
     decode_workspace_size, plan_grid, default_num_ctas, decode_num_ctas,
-    workspace_layout, decode_plan (with ``tail=`` for hpa_decode_plan_tail),
+    workspace_layout, decode_plan (with ``tail=`` / ``cost=`` for hpa_decode_plan_shape),
     decode_run, decode_step (+ ``lse=``: hpa_decode_step_lse), decode_step_prologue,
     decode_run_multi, decode_run_prologue, kv_prologue, merge_states,
     read_status, read_cta_times, decode_noalloc, noalloc_read_status
@@ -30,7 +30,9 @@ import torch
 __all__ = [
     "HpaError", "HpaLibraryMissing", "lib", "library_path", "PLAN_DYNAMIC", "PLAN_STATIC_NSPLIT",
     "PLAN_STATIC_CHUNK", "PLAN_LENGTH_AWARE", "TAIL_DEN_DEFAULT", "TAIL_CHUNKS_DEFAULT",
-    "TAIL_MIN_DEFAULT", "TAIL_CHUNKS_MAX", "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
+    "TAIL_MIN_DEFAULT", "TAIL_CHUNKS_MAX", "COST_UNIT_DEFAULT", "COST_END_DEFAULT", "COST_END_DEFAULT_FP8",
+    "COST_MAX",
+    "DEVICE_LEN_CLAMPED", "DEVICE_BAD_PAGE", "DEVICE_BAD_PLAN",
     "DEVICE_BAD_POSITION", "DEVICE_TIMEOUT", "decode_workspace_size", "plan_grid",
     "default_num_ctas", "decode_num_ctas", "workspace_layout", "decode_plan", "decode_run",
     "decode_step", "decode_step_prologue", "MAX_STEP_BATCH", "decode_run_multi",
@@ -47,6 +49,9 @@ DEVICE_BAD_POSITION, DEVICE_TIMEOUT = 0x8, 0x10
 PAGE_SIZE = 64
 # run-time tail of the dynamic plans (hpa.h: HPA_TAIL_DEN_DEFAULT, ...)
 TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT, TAIL_MIN_DEFAULT, TAIL_CHUNKS_MAX = 8, 4, 32, 4
+# cost weights of their primary ranges (hpa.h: HPA_COST_UNIT_DEFAULT, ...); the
+# in-kernel plans use COST_END_DEFAULT_FP8 for e4m3 caches
+COST_UNIT_DEFAULT, COST_END_DEFAULT, COST_END_DEFAULT_FP8, COST_MAX = 1, 0, 2, 4
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,9 +100,9 @@ def lib():
         L.hpa_decode_plan.restype = _I
         L.hpa_decode_plan.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V, _Z,
                                       C.POINTER(_I), _V]
-        L.hpa_decode_plan_tail.restype = _I
-        L.hpa_decode_plan_tail.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _V,
-                                           _Z, C.POINTER(_I), _V]
+        L.hpa_decode_plan_shape.restype = _I
+        L.hpa_decode_plan_shape.argtypes = [_V, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                            _I, _V, _Z, C.POINTER(_I), _V]
         L.hpa_decode_run.restype = _I
         L.hpa_decode_run.argtypes = [_V, _V, _V, _V, _V, _I, _V, _I, _I, _V, _I, _I, _I, _I, _I,
                                      _F, _I, _I, _V, _Z, _V]
@@ -214,25 +219,29 @@ def workspace_layout(kind, batch, num_kv_heads, num_q_heads, head_dim, grid) -> 
 def decode_plan(seq_lens: torch.Tensor, *, num_kv_heads: int, num_q_heads: int, head_dim: int,
                 pt_stride: int, workspace: torch.Tensor, kind: int = PLAN_DYNAMIC,
                 num_ctas: int | None = None, param: int = 0, max_seq_len: int = 0,
-                tail: tuple[int, int, int] | None = None, stream=None) -> int:
+                tail: tuple[int, int, int] | None = None, cost: tuple[int, int] | None = None,
+                stream=None) -> int:
     """Enqueue the tile plan; returns the grid to pass to decode_run.
 
     ``tail = (tail_den, tail_chunks, tail_min)`` sets the run-time tail of a
-    DYNAMIC or LENGTH_AWARE plan (hpa_decode_plan_tail; (0, 1, 0): no tail);
-    None keeps the library's default (TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT,
-    TAIL_MIN_DEFAULT)."""
+    DYNAMIC or LENGTH_AWARE plan ((0, 1, 0): no tail) and ``cost =
+    (unit_cost, end_cost)`` the cost weights of its primary ranges ((1, 0):
+    the units split evenly), both through hpa_decode_plan_shape; None keeps
+    the library's default (TAIL_*_DEFAULT, COST_*_DEFAULT)."""
     _dev(seq_lens, "seq_lens", (torch.int32,), 1)
     _dev(workspace, "workspace", (torch.uint8,))
     if num_ctas is None:
         num_ctas = default_num_ctas(seq_lens.device.index)
     grid = C.c_int(0)
-    if tail is not None:
-        rc = lib().hpa_decode_plan_tail(_ptr(seq_lens), seq_lens.shape[0], num_kv_heads,
-                                        num_q_heads, head_dim, pt_stride, kind, num_ctas, param,
-                                        int(tail[0]), int(tail[1]), int(tail[2]),
-                                        _ptr(workspace),
-                                        workspace.numel(), C.byref(grid), _stream(stream))
-        _check(rc, "hpa_decode_plan_tail")
+    if tail is not None or cost is not None:
+        t = (TAIL_DEN_DEFAULT, TAIL_CHUNKS_DEFAULT, TAIL_MIN_DEFAULT) if tail is None else tail
+        c = (COST_UNIT_DEFAULT, COST_END_DEFAULT) if cost is None else cost
+        rc = lib().hpa_decode_plan_shape(_ptr(seq_lens), seq_lens.shape[0], num_kv_heads,
+                                         num_q_heads, head_dim, pt_stride, kind, num_ctas, param,
+                                         int(t[0]), int(t[1]), int(t[2]), int(c[0]), int(c[1]),
+                                         _ptr(workspace), workspace.numel(), C.byref(grid),
+                                         _stream(stream))
+        _check(rc, "hpa_decode_plan_shape")
         return grid.value
     rc = lib().hpa_decode_plan(_ptr(seq_lens), seq_lens.shape[0], num_kv_heads, num_q_heads,
                                head_dim, pt_stride, kind, num_ctas, param, max_seq_len,

@@ -111,8 +111,11 @@ struct Cfg {
   static constexpr int kDepAccFloats = kConsumerWarps * kWarpRows * kAccStride;
   static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kWarpRows * 8;
   static constexpr int kMisc = 2048;                   // barriers, stage info, flags
-  // in-kernel plan: tile offsets of all sequences
-  static constexpr int kTsBytes = FP ? ((kMaxFusedBatch + 1) * 4 + 15) / 16 * 16 : 0;
+  // in-kernel plan: tile offsets of all sequences, the non-empty mask and
+  // its prefix (SeqIdx), and the scan's per-warp non-empty counts
+  static constexpr int kTsWords = (kMaxFusedBatch + 1) + kMaxFusedBatch / 32 +
+                                  (kMaxFusedBatch / 32 + 1) + kThreads / 32;
+  static constexpr int kTsBytes = FP ? (kTsWords * 4 + 15) / 16 * 16 : 0;
   // CPS CTAs share one SM's 228 KiB (1 KiB of it reserved per CTA)
   static constexpr int kBudget = CPS == 1 ? kSmemLimit : (kSmemPerSm / CPS - 1024);
   static constexpr int kStagesFit =
@@ -141,6 +144,7 @@ struct RunParams {
   const int32_t* seq_lens;  // in-kernel plan: the step's lengths (else the plan's)
   int capacity;             // in-kernel plan: pt_stride * 64 tokens
   int tail_den, tail_chunks, tail_min;  // in-kernel plan: the run-time tail's shape
+  int unit_cost, end_cost;              // in-kernel plan: cost weights of the primary cuts
   float scale_log2;         // softmax_scale * log2(e)
   Ws ws;
   int grid, kind;
@@ -292,9 +296,13 @@ __global__ void __launch_bounds__(kThreads, CPS)
   static_assert(C::kStages * 24 + kDepBufs * 16 + 8 + C::kStages * sizeof(StageInfo) +
                         kDepBufs * sizeof(DepDesc) + 16 + 32 <= C::kMisc / 2,
                 "misc area too small");
-  // in-kernel plan: tile offsets (after the misc area), and per-warp sums of
-  // the scan (behind q_ready)
+  // in-kernel plan: tile offsets, non-empty mask and prefix, per-warp
+  // non-empty counts (after the misc area), and per-warp tile sums of the
+  // scan (behind q_ready)
   int32_t* s_ts = reinterpret_cast<int32_t*>(misc + C::kMisc);
+  uint32_t* s_nzm = reinterpret_cast<uint32_t*>(s_ts + kMaxFusedBatch + 1);
+  int32_t* s_nzp = reinterpret_cast<int32_t*>(s_nzm + kMaxFusedBatch / 32);
+  int* s_wnz = s_nzp + kMaxFusedBatch / 32 + 1;
   int* s_wsum = const_cast<int*>(s_flags) + 4;
   volatile int* s_parity = s_flags + 10;  // in-kernel plan: step parity (after the warp sums)
 
@@ -322,13 +330,14 @@ __global__ void __launch_bounds__(kThreads, CPS)
   const uint64_t t_cta0 = globaltimer();  // this CTA's start, for the trace region
   if constexpr (FP) {
     // In-kernel plan (hpa_decode_step): every CTA turns the step's lengths
-    // into tile offsets in shared memory, as the plan kernel does -- warp w
-    // scans a contiguous slice 32 lengths at a time -- and then derives its
-    // own ranges from the same closed forms.
+    // into tile offsets and the non-empty mask in shared memory, as the plan
+    // kernel does -- warp w scans a contiguous slice (a multiple of 32) 32
+    // lengths at a time -- and then derives its own ranges from the same
+    // closed forms.
     constexpr int kW = kThreads / 32;
-    const int slice = (p.B + kW - 1) / kW;
+    const int slice = ((p.B + kW - 1) / kW + 31) & ~31;
     const int lo = min(p.B, warp * slice), hi = min(p.B, lo + slice);
-    int carry = 0;
+    int carry = 0, carry_nz = 0;
     bool clamped = false;
     for (int i0 = lo; i0 < hi; i0 += 32) {
       const int i = i0 + lane;
@@ -347,21 +356,37 @@ __global__ void __launch_bounds__(kThreads, CPS)
       }
       if (i < hi) s_ts[i] = carry + x - n;
       carry += __shfl_sync(0xffffffffu, x, 31);
+      if constexpr (FP8) {
+        const unsigned bal = __ballot_sync(0xffffffffu, n > 0);
+        if (lane == 0) {
+          s_nzm[i0 >> 5] = bal;
+          s_nzp[i0 >> 5] = carry_nz;
+        }
+        carry_nz += __popc(bal);
+      }
     }
-    if (lane == 0) s_wsum[warp] = carry;
+    if (lane == 0) {
+      s_wsum[warp] = carry;
+      s_wnz[warp] = carry_nz;
+    }
     if (blockIdx.x == 0 && __any_sync(0xffffffffu, clamped) && lane == 0)
       atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_LEN_CLAMPED);
     __syncthreads();
-    int off = 0, T = 0;
+    int off = 0, T = 0, off_nz = 0, T_nz = 0;
 #pragma unroll
     for (int w = 0; w < kW; ++w) {
       off += w < warp ? s_wsum[w] : 0;
       T += s_wsum[w];
+      off_nz += w < warp ? s_wnz[w] : 0;
+      T_nz += s_wnz[w];
     }
     if (off)
       for (int i = lo + lane; i < hi; i += 32) s_ts[i] += off;
+    if (off_nz && lane == 0)
+      for (int i0 = lo; i0 < hi; i0 += 32) s_nzp[i0 >> 5] += off_nz;
     if (threadIdx.x == 0) {
       s_ts[p.B] = T;
+      s_nzp[(p.B + 31) >> 5] = T_nz;
       *s_plan_ok = 1;
       *s_parity = __ldcg(&p.ws.header[kHdrParity]) & 1;  // this step's merge-list count
     }
@@ -396,7 +421,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
   DynGeom dg{};
   if constexpr (FP) {
     if (warp >= kConsumerWarps) {
-      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x, p.tail_den, p.tail_chunks, p.tail_min);
+      // (cost weights only for e4m3 caches: with end cost 0 the cost code
+      // drops out of the bf16 kernels)
+      dg.init((long long)ts[p.B] * p.Hkv, gridDim.x, p.tail_den, p.tail_chunks, p.tail_min,
+              FP8 ? p.unit_cost : 1, FP8 ? p.end_cost : 0, SeqIdx{ts, s_nzm, s_nzp, p.B, p.Hkv},
+              lane);
       double rc[4];
       dyn_reciprocals(dg, rc);
       dg.init_div(rc);
@@ -418,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
     int v = blockIdx.x;
     int4 d0, d1;
     if constexpr (FP) {
-      dyn_range_desc(dg, ts, p.B, p.Hkv, v, &d0, &d1);
+      dyn_range_desc(dg, ts, p.B, p.Hkv, v, &d0, &d1, lane);
     } else {
       d0 = p.ws.cta_desc[2 * v];
       d1 = p.ws.cta_desc[2 * v + 1];
@@ -660,6 +689,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
         h[kHdrTailDen] = p.tail_den;
         h[kHdrTailChunks] = p.tail_chunks;
         h[kHdrTailMin] = p.tail_min;
+        h[kHdrUnitCost] = FP8 ? p.unit_cost : 1;
+        h[kHdrEndCost] = FP8 ? p.end_cost : 0;
         h[kHdrMagic] = kPlanMagic;
       }
     }
@@ -1534,6 +1565,8 @@ hpa_status run_impl(const void* q, const void* k_cache, const void* v_cache, con
   p.tail_den = HPA_TAIL_DEN_DEFAULT;
   p.tail_chunks = HPA_TAIL_CHUNKS_DEFAULT;
   p.tail_min = HPA_TAIL_MIN_DEFAULT;
+  p.unit_cost = HPA_COST_UNIT_DEFAULT;
+  p.end_cost = fp8 ? HPA_COST_END_DEFAULT_FP8 : HPA_COST_END_DEFAULT;
   const int nt = GT > 16 ? 4 : GT > 8 ? 2 : 1;
   const int sms = sm_count();
   const int cps = (sms > 0 && grid > sms) ? 2 : 1;

@@ -63,6 +63,8 @@ enum HeaderField {
   kHdrTailMin = 15,
   kHdrListCount = 16,   // in-kernel plan: split segments on the merge list (2 words: by parity)
   kHdrParity = 18,      // in-kernel plan: parity of the current step
+  kHdrUnitCost = 19,    // dynamic plans: the cost weights of the primary cuts
+  kHdrEndCost = 20,
   kHdrWords = 32
 };
 

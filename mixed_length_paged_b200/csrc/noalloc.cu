@@ -123,10 +123,15 @@ extern "C" hpa_status hpa_decode_noalloc(const void* q, const void* k_cache, con
                            pt_stride, num_pages, out, out_dtype, batch, 1, num_q_heads,
                            num_kv_heads, head_dim, softmax_scale, ctas, scratch,
                            HPA_NOALLOC_SCRATCH_BYTES, stream);
+  // (the plan the in-kernel plan would make: its cost weights depend on the
+  // cache type)
   int grid = 0;
-  st = hpa_decode_plan(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride,
-                       HPA_PLAN_DYNAMIC, ctas, 0, 0, scratch, HPA_NOALLOC_SCRATCH_BYTES, &grid,
-                       stream);
+  st = hpa_decode_plan_shape(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride,
+                             HPA_PLAN_DYNAMIC, ctas, 0, HPA_TAIL_DEN_DEFAULT,
+                             HPA_TAIL_CHUNKS_DEFAULT, HPA_TAIL_MIN_DEFAULT, HPA_COST_UNIT_DEFAULT,
+                             kv_dtype == HPA_KV_FP8_E4M3 ? HPA_COST_END_DEFAULT_FP8
+                                                         : HPA_COST_END_DEFAULT,
+                             scratch, HPA_NOALLOC_SCRATCH_BYTES, &grid, stream);
   if (st != HPA_OK) return st;
   return hpa_decode_run(q, k_cache, v_cache, k_scale, v_scale, kv_dtype, page_table, pt_stride,
                         num_pages, out, out_dtype, batch, num_q_heads, num_kv_heads, head_dim,

@@ -48,12 +48,18 @@ struct PlanParams {
   int kind, num_ctas, grid;
   long long chunk;             // STATIC_CHUNK: tiles per split; LENGTH_AWARE: smallest piece
   int tail_den, tail_chunks, tail_min;  // DYNAMIC / LENGTH_AWARE: the run-time tail's shape
+  int unit_cost, end_cost;              // DYNAMIC / LENGTH_AWARE: cost weights of the primary cuts
   Ws ws;
 };
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
-  extern __shared__ int32_t ts[];  // tile_start[0..B], in shared memory
-  __shared__ int s_warp[kPlanWarps];
+__global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanParams p) {
+  // tile_start[0..B], then the non-empty mask and its prefix (SeqIdx), in
+  // shared memory
+  extern __shared__ int32_t ts[];
+  const int nw = (p.B + 31) / 32;
+  uint32_t* nzm = reinterpret_cast<uint32_t*>(ts + p.B + 1);
+  int32_t* nzp = reinterpret_cast<int32_t*>(nzm + nw);
+  __shared__ int s_warp[kPlanWarps], s_warp_nz[kPlanWarps];
   __shared__ int s_status;
   __shared__ double s_recip[4];
   // The previous step's run kernel may still be reading this workspace.
@@ -63,12 +69,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
   __syncthreads();
 
   // 1. clamped lengths -> tiles per sequence -> exclusive prefix sum, in
-  //    shared memory.  Warp w scans its own contiguous slice 32 entries at a
-  //    time (coalesced loads, shuffle scans); the slices' totals are added
-  //    after one barrier.
-  const int slice = (p.B + kPlanWarps - 1) / kPlanWarps;
+  //    shared memory.  Warp w scans its own contiguous slice (a multiple of
+  //    32 entries) 32 entries at a time (coalesced loads, shuffle scans); the
+  //    slices' totals are added after one barrier.  Alongside: which
+  //    sequences have tiles, one mask word per 32, and the count before each.
+  const int slice = ((p.B + kPlanWarps - 1) / kPlanWarps + 31) & ~31;
   const int lo = min(p.B, warp * slice), hi = min(p.B, lo + slice);
-  int carry = 0;
+  int carry = 0, carry_nz = 0;
   for (int i0 = lo; i0 < hi; i0 += 32) {
     const int i = i0 + lane;
     int n = 0;
@@ -86,26 +93,45 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     }
     if (i < hi) ts[i] = carry + x - n;
     carry += __shfl_sync(0xffffffffu, x, 31);
+    const unsigned bal = __ballot_sync(0xffffffffu, n > 0);
+    if (lane == 0) {
+      nzm[i0 >> 5] = bal;
+      nzp[i0 >> 5] = carry_nz;
+    }
+    carry_nz += __popc(bal);
   }
-  if (lane == 0) s_warp[warp] = carry;
+  if (lane == 0) {
+    s_warp[warp] = carry;
+    s_warp_nz[warp] = carry_nz;
+  }
   __syncthreads();
-  int off = 0, T = 0;
+  int off = 0, T = 0, off_nz = 0, T_nz = 0;
 #pragma unroll
   for (int w = 0; w < kPlanWarps; ++w) {
     off += w < warp ? s_warp[w] : 0;
     T += s_warp[w];
+    off_nz += w < warp ? s_warp_nz[w] : 0;
+    T_nz += s_warp_nz[w];
   }
   if (off)
     for (int i = lo + lane; i < hi; i += 32) ts[i] += off;
-  if (tid == 0) ts[p.B] = T;
+  if (off_nz && lane == 0)
+    for (int i0 = lo; i0 < hi; i0 += 32) nzp[i0 >> 5] += off_nz;
+  if (tid == 0) {
+    ts[p.B] = T;
+    nzp[nw] = T_nz;
+  }
 
   const long long U = (long long)T * p.Hkv;
   const int S = p.B * p.Hkv;
   const bool dyn = plan_is_dynamic(p.kind);
   const bool la = p.kind == HPA_PLAN_LENGTH_AWARE;
   const int per = dyn ? 0 : p.grid / S;  // static: CTAs per segment
+  // (the tile offsets and the mask are complete: K(U1) reads them)
+  __syncthreads();
   DynGeom dg;
-  dg.init(U, p.num_ctas, p.tail_den, p.tail_chunks, p.tail_min);
+  dg.init(U, p.num_ctas, p.tail_den, p.tail_chunks, p.tail_min, p.unit_cost, p.end_cost,
+          SeqIdx{ts, nzm, nzp, p.B, p.Hkv}, lane);
   const LaGeom lg{&dg, ts, p.B, p.Hkv, la ? p.chunk : 1};
   if (tid < 4) {
     const long long d = dg.divisor(tid);
@@ -188,6 +214,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanParams p) {
     h[kHdrTailDen] = dyn ? p.tail_den : 0;
     h[kHdrTailChunks] = dyn ? p.tail_chunks : 0;
     h[kHdrTailMin] = dyn ? p.tail_min : 0;
+    h[kHdrUnitCost] = dyn ? p.unit_cost : 0;
+    h[kHdrEndCost] = dyn ? p.end_cost : 0;
     // (no fence before the magic word: the run kernel reads the plan only
     // after griddepcontrol.wait, i.e. after this whole grid has completed)
     h[kHdrMagic] = kPlanMagic;
@@ -209,12 +237,19 @@ extern "C" int hpa_plan_grid(hpa_plan_kind kind, int batch, int num_kv_heads, in
 
 namespace hpa {
 
-// hpa_decode_plan and hpa_decode_plan_tail: validation, parameters, launch.
+// Shared memory of the plan kernel for `batch` sequences: tile offsets, the
+// non-empty mask and its prefix.
+static size_t plan_smem_bytes(int batch) {
+  const size_t nw = (size_t(batch) + 31) / 32;
+  return (size_t(batch) + 1) * 4 + nw * 4 + (nw + 1) * 4;
+}
+
+// hpa_decode_plan and hpa_decode_plan_shape: validation, parameters, launch.
 static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads,
                             int num_q_heads, int head_dim, int pt_stride, hpa_plan_kind kind,
                             int num_ctas, int param, int max_seq_len, int tail_den,
-                            int tail_chunks, int tail_min, void* workspace, size_t ws_bytes,
-                            int* grid_out, void* stream) {
+                            int tail_chunks, int tail_min, int unit_cost, int end_cost,
+                            void* workspace, size_t ws_bytes, int* grid_out, void* stream) {
   if (!seq_lens || !workspace || !grid_out) return HPA_ERR_INVALID_ARG;
   if (batch <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || pt_stride <= 0 || num_ctas <= 0 ||
       param < 0 || max_seq_len < 0)
@@ -225,6 +260,8 @@ static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads
     return HPA_ERR_INVALID_ARG;
   if (tail_den < 0 || tail_den > (1 << 20) || tail_chunks < 1 || tail_chunks > HPA_TAIL_CHUNKS_MAX ||
       tail_min < 0 || tail_min > (1 << 20))
+    return HPA_ERR_INVALID_ARG;
+  if (unit_cost < 1 || unit_cost > HPA_COST_MAX || end_cost < 0 || end_cost > HPA_COST_MAX)
     return HPA_ERR_INVALID_ARG;
   if ((long long)pt_stride * kPageSize > 0x7fffffffLL) return HPA_ERR_UNSUPPORTED;
   if (batch > kMaxPlanBatch) return HPA_ERR_UNSUPPORTED;
@@ -257,9 +294,11 @@ static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads
   p.tail_den = tail_den;
   p.tail_chunks = tail_chunks;
   p.tail_min = tail_min;
+  p.unit_cost = unit_cost;
+  p.end_cost = end_cost;
   p.ws = ws_view(workspace, L);
 
-  const size_t smem = (size_t(batch) + 1) * sizeof(int32_t);
+  const size_t smem = plan_smem_bytes(batch);
   if (smem > 48 * 1024) {
     // tile offsets above 48 KiB of shared memory need the opt-in, once per device
     static std::atomic<uint64_t> ready_mask{0};
@@ -269,7 +308,7 @@ static hpa_status plan_impl(const int32_t* seq_lens, int batch, int num_kv_heads
     if (!bit || !(ready_mask.load() & bit)) {
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)((size_t(kMaxPlanBatch) + 1) * sizeof(int32_t)));
+                                 (int)plan_smem_bytes(kMaxPlanBatch));
       if (e != cudaSuccess) {
         set_cuda_error(e, "hpa_decode_plan smem attribute");
         return HPA_ERR_CUDA;
@@ -308,17 +347,18 @@ extern "C" hpa_status hpa_decode_plan(const int32_t* seq_lens, int batch, int nu
                                       int* grid_out, void* stream) {
   return plan_impl(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride, kind,
                    num_ctas, param, max_seq_len, HPA_TAIL_DEN_DEFAULT, HPA_TAIL_CHUNKS_DEFAULT,
-                   HPA_TAIL_MIN_DEFAULT, workspace, ws_bytes, grid_out, stream);
+                   HPA_TAIL_MIN_DEFAULT, HPA_COST_UNIT_DEFAULT, HPA_COST_END_DEFAULT, workspace,
+                   ws_bytes, grid_out, stream);
 }
 
-extern "C" hpa_status hpa_decode_plan_tail(const int32_t* seq_lens, int batch, int num_kv_heads,
-                                           int num_q_heads, int head_dim, int pt_stride,
-                                           hpa_plan_kind kind, int num_ctas, int param,
-                                           int tail_den, int tail_chunks, int tail_min,
-                                           void* workspace, size_t ws_bytes, int* grid_out,
-                                           void* stream) {
+extern "C" hpa_status hpa_decode_plan_shape(const int32_t* seq_lens, int batch, int num_kv_heads,
+                                            int num_q_heads, int head_dim, int pt_stride,
+                                            hpa_plan_kind kind, int num_ctas, int param,
+                                            int tail_den, int tail_chunks, int tail_min,
+                                            int unit_cost, int end_cost, void* workspace,
+                                            size_t ws_bytes, int* grid_out, void* stream) {
   if (!plan_is_dynamic(kind)) return HPA_ERR_INVALID_ARG;
   return plan_impl(seq_lens, batch, num_kv_heads, num_q_heads, head_dim, pt_stride, kind,
-                   num_ctas, param, 0, tail_den, tail_chunks, tail_min, workspace, ws_bytes,
-                   grid_out, stream);
+                   num_ctas, param, 0, tail_den, tail_chunks, tail_min, unit_cost, end_cost,
+                   workspace, ws_bytes, grid_out, stream);
 }

@@ -118,16 +118,17 @@ def test_plan_rejects_bad_arguments_without_launching(L, bad, expect):
     assert grid == -7  # nothing reported, nothing enqueued
 
 
-def _plan_tail(L, **kw):
+def _plan_shape(L, **kw):
     a = dict(seq_lens=1, batch=2, num_kv_heads=2, num_q_heads=8, head_dim=64, pt_stride=4,
              kind=0, num_ctas=148, param=0, tail_den=8, tail_chunks=4, tail_min=32,
-             workspace=256, ws_bytes=1 << 20)
+             unit_cost=1, end_cost=0, workspace=256, ws_bytes=1 << 20)
     a.update(kw)
     g = C.c_int(-7)
-    rc = L.hpa_decode_plan_tail(a["seq_lens"], a["batch"], a["num_kv_heads"], a["num_q_heads"],
-                                a["head_dim"], a["pt_stride"], a["kind"], a["num_ctas"],
-                                a["param"], a["tail_den"], a["tail_chunks"], a["tail_min"],
-                                a["workspace"], a["ws_bytes"], C.byref(g), None)
+    rc = L.hpa_decode_plan_shape(a["seq_lens"], a["batch"], a["num_kv_heads"], a["num_q_heads"],
+                                 a["head_dim"], a["pt_stride"], a["kind"], a["num_ctas"],
+                                 a["param"], a["tail_den"], a["tail_chunks"], a["tail_min"],
+                                 a["unit_cost"], a["end_cost"], a["workspace"], a["ws_bytes"],
+                                 C.byref(g), None)
     return rc, g.value
 
 
@@ -137,19 +138,25 @@ def _plan_tail(L, **kw):
     (dict(tail_chunks=0), 1), (dict(tail_chunks=hpa.TAIL_CHUNKS_MAX + 1), 1),
     (dict(tail_den=0, tail_chunks=0), 1), (dict(tail_min=-1), 1), (dict(tail_min=(1 << 20) + 1), 1),
     (dict(seq_lens=None), 1), (dict(ws_bytes=16), 3), (dict(num_ctas=65537), 2),
+    (dict(unit_cost=0), 1), (dict(unit_cost=hpa.COST_MAX + 1), 1), (dict(end_cost=-1), 1),
+    (dict(end_cost=hpa.COST_MAX + 1), 1), (dict(unit_cost=-2, end_cost=3), 1),
 ])
-def test_plan_tail_rejects_bad_arguments_without_launching(L, bad, expect):
-    rc, grid = _plan_tail(L, **bad)
+def test_plan_shape_rejects_bad_arguments_without_launching(L, bad, expect):
+    rc, grid = _plan_shape(L, **bad)
     assert rc == expect
     assert grid == -7
 
 
-def test_tail_defaults_match_the_header():
+def test_plan_shape_defaults_match_the_header():
     src = open(HEADER).read()
     for name, val in [("HPA_TAIL_DEN_DEFAULT", hpa.TAIL_DEN_DEFAULT),
                       ("HPA_TAIL_CHUNKS_DEFAULT", hpa.TAIL_CHUNKS_DEFAULT),
                       ("HPA_TAIL_MIN_DEFAULT", hpa.TAIL_MIN_DEFAULT),
-                      ("HPA_TAIL_CHUNKS_MAX", hpa.TAIL_CHUNKS_MAX)]:
+                      ("HPA_TAIL_CHUNKS_MAX", hpa.TAIL_CHUNKS_MAX),
+                      ("HPA_COST_UNIT_DEFAULT", hpa.COST_UNIT_DEFAULT),
+                      ("HPA_COST_END_DEFAULT", hpa.COST_END_DEFAULT),
+                      ("HPA_COST_END_DEFAULT_FP8", hpa.COST_END_DEFAULT_FP8),
+                      ("HPA_COST_MAX", hpa.COST_MAX)]:
         assert re.search(rf"#define {name} {val}\b", src), name
 
 

@@ -51,7 +51,7 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
         return w[off:off + 4 * n].view(np.int32)
 
     S = B * Hkv
-    header = i32(lay["header"], 16)
+    header = i32(lay["header"], 32)
     V = int(header[10])
     return {
         "header": header, "lens": i32(lay["lens"], B),
@@ -61,9 +61,10 @@ def _read_plan(ws, kind, B, Hkv, Hq, D, grid):
     }
 
 
-# The library's member of the dynamic plan family (hpa.h: HPA_TAIL_DEN_DEFAULT,
-# HPA_TAIL_CHUNKS_DEFAULT), and other members called with hpa_decode_plan_tail.
+# The library's member of the dynamic plan family (hpa.h: HPA_TAIL_*_DEFAULT,
+# HPA_COST_*_DEFAULT); other members are called with hpa_decode_plan_shape.
 LIB_TAIL = (8, 4, 32)
+LIB_COST = (hpa.COST_UNIT_DEFAULT, hpa.COST_END_DEFAULT)
 
 
 @pytest.mark.parametrize("lens,Hkv,P", [
@@ -74,14 +75,20 @@ LIB_TAIL = (8, 4, 32)
     ([int(x) for x in np.random.default_rng(3).integers(0, 300, 20000)], 2, 148),
     ([int(x) for x in np.random.default_rng(4).integers(1, 100, 32768)], 1, 148),  # the maximum
 ])
-@pytest.mark.parametrize("kind,param,tail", [
-    (0, 0, None), (1, 0, None), (1, 3, None), (2, 0, None), (2, 5, None), (3, 0, None),
-    (3, 2, None), (3, 9, None),
-    (0, 0, (0, 1, 0)), (0, 0, (8, 4, 0)), (0, 0, (3, 1, 0)), (0, 0, (16, 2, 3)),
-    (0, 0, (1, 4, 0)), (3, 4, (0, 1, 0)), (3, 2, (5, 3, 0))])
-def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail):
-    """tail None: hpa_decode_plan (the library's default tail, LIB_TAIL);
-    else hpa_decode_plan_tail with that tail shape ((0, 1, 0) = no tail)."""
+@pytest.mark.parametrize("kind,param,tail,cost", [
+    (0, 0, None, None), (1, 0, None, None), (1, 3, None, None), (2, 0, None, None),
+    (2, 5, None, None), (3, 0, None, None), (3, 2, None, None), (3, 9, None, None),
+    (0, 0, (0, 1, 0), None), (0, 0, (8, 4, 0), None), (0, 0, (3, 1, 0), None),
+    (0, 0, (16, 2, 3), None), (0, 0, (1, 4, 0), None), (3, 4, (0, 1, 0), None),
+    (3, 2, (5, 3, 0), None),
+    (0, 0, (0, 1, 0), (1, 0)), (0, 0, (0, 1, 0), (1, 1)), (0, 0, (8, 4, 0), (2, 1)),
+    (0, 0, (8, 4, 32), (4, 3)), (0, 0, (0, 1, 0), (1, 4)), (0, 0, (3, 1, 0), (3, 0)),
+    (0, 0, None, (2, 1)), (3, 2, (8, 4, 0), (2, 1)), (3, 4, (0, 1, 0), (1, 2))])
+def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail, cost):
+    """tail and cost None: hpa_decode_plan (the library's default shape,
+    LIB_TAIL and LIB_COST); else hpa_decode_plan_shape with that tail shape
+    ((0, 1, 0) = no tail) and cost weights ((1, 0) = units split evenly), the
+    default for whichever is None."""
     B, Hq, D = len(lens), Hkv * 2, 64
     cap = max(64, max(lens))
     pts = (cap + 63) // 64
@@ -89,14 +96,15 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail):
     grid = hpa.plan_grid(kind, B, Hkv, P, param, maxlen)
     ref = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=kind, num_ctas=P, param=param,
                       max_seq_len=maxlen, capacity_tokens=pts * 64,
-                      tail=LIB_TAIL if tail is None else tail)
+                      tail=LIB_TAIL if tail is None else tail,
+                      cost=LIB_COST if cost is None else cost)
     assert grid == ref["grid"]
     ws = torch.full((hpa.decode_workspace_size(kind, B, Hkv, Hq, D, grid),), 0xAB,
                     dtype=torch.uint8, device="cuda")
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
     g = hpa.decode_plan(sl, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D, pt_stride=pts,
                         workspace=ws, kind=kind, num_ctas=P, param=param, max_seq_len=maxlen,
-                        tail=tail)
+                        tail=tail, cost=cost)
     torch.cuda.synchronize()
     assert g == grid
     got = _read_plan(ws, kind, B, Hkv, Hq, D, grid)
@@ -122,6 +130,8 @@ def test_plan_is_bit_exact(lens, Hkv, P, kind, param, tail):
     # the tail shape the plan was made with, recorded in the header
     want = (LIB_TAIL if tail is None else tail) if kind in (0, 3) else (0, 0, 0)
     assert (int(h[13]), int(h[14]), int(h[15])) == want
+    want = (LIB_COST if cost is None else cost) if kind in (0, 3) else (0, 0)
+    assert (int(h[19]), int(h[20])) == want
 
 
 def test_plan_flags_clamped_lengths():
@@ -669,7 +679,9 @@ def bits_t(t: torch.Tensor) -> torch.Tensor:
 # ---------------------------------------------------------------- in-kernel plan (decode_step)
 
 def _plan_and_run(batch, num_ctas, out_dtype=torch.float32, fp8=None):
-    """Reference: hpa_decode_plan + hpa_decode_run(_multi) on a fresh workspace."""
+    """Reference: hpa_decode_plan + hpa_decode_run(_multi) on a fresh workspace
+    (for an e4m3 cache hpa_decode_plan_shape with the in-kernel plans' e4m3
+    cost weights)."""
     q = batch.q
     T = q.shape[1] if q.dim() == 4 else 1
     B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
@@ -677,7 +689,8 @@ def _plan_and_run(batch, num_ctas, out_dtype=torch.float32, fp8=None):
     ws = torch.zeros(hpa.decode_workspace_size(0, B, Hkv, Hq * T, D, num_ctas), dtype=torch.uint8,
                      device="cuda")
     hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq * T, head_dim=D,
-                    pt_stride=batch.pt_stride, workspace=ws, num_ctas=num_ctas)
+                    pt_stride=batch.pt_stride, workspace=ws, num_ctas=num_ctas,
+                    cost=None if fp8 is None else (hpa.COST_UNIT_DEFAULT, hpa.COST_END_DEFAULT_FP8))
     out = torch.full(q.shape, float("nan"), dtype=out_dtype, device="cuda")
     kw = {}
     kc, vc = batch.k_cache, batch.v_cache
@@ -747,15 +760,33 @@ def test_step_equals_plan_and_run_bitwise(name, lens, Hq, Hkv, D, T, num_ctas):
     assert hdr_a[11] == 0 and hdr_a[12] == 0  # run-time counters back at zero
 
 
-def test_step_fp8_equals_plan_and_run():
+@pytest.mark.parametrize("lens", [
+    [1, 63, 64, 65, 700, 3000],
+    # many single-tile sequences: the e4m3 cost weights move the cuts
+    [64] * 100 + [4000] * 20 + [1, 130] * 10,
+])
+def test_step_fp8_equals_plan_and_run(lens):
+    """The e4m3 in-kernel plan weighs segment ends (COST_END_DEFAULT_FP8): it
+    equals hpa_decode_plan_shape with those weights, bit for bit, and the plan
+    fields of the header record them."""
     shape = W.DecodeShape("st8", 64, 8, 128, kv_dtype="fp8_e4m3")
-    batch = W.make_batch(shape, [1, 63, 64, 65, 700, 3000], seed=44)
+    batch = W.make_batch(shape, lens, seed=44)
     fp8 = quantize_fp8(batch)
     to_device(batch)
     n = hpa.default_num_ctas()
-    ref, _ = _plan_and_run(batch, n, fp8=fp8)
-    got, _ = _step(batch, n, fp8=fp8)
+    ref, ws_ref = _plan_and_run(batch, n, fp8=fp8)
+    got, ws = _step(batch, n, fp8=fp8)
     assert torch.equal(got, ref)
+    lay = hpa.workspace_layout(0, batch.batch, 8, 64, 128, n)
+    S = batch.batch * 8
+    a, b = ws.cpu().numpy(), ws_ref.cpu().numpy()
+    sd = slice(lay["seg_desc"], lay["seg_desc"] + 8 * S)
+    np.testing.assert_array_equal(a[sd], b[sd])
+    hdr = a[lay["header"]:lay["header"] + 128].view(np.int32)
+    assert (int(hdr[19]), int(hdr[20])) == (hpa.COST_UNIT_DEFAULT, hpa.COST_END_DEFAULT_FP8)
+    ref64 = oracle_decode(batch, fp8=fp8)
+    mx, _ = errors(got, ref64)
+    assert mx <= FP8_MAX_ABS, mx
 
 
 def test_step_repeated_with_changing_lengths_and_mixed_calls():
@@ -926,14 +957,16 @@ def _random_case(seed):
         if kind in (0, 3) else None
     num_ctas = int(rng.choice([1, 5, 37, 148, 296]))
     out_dtype = torch.float32 if rng.random() < 0.5 else torch.bfloat16
+    cost = [None, (1, 0), (1, 1), (2, 1), (4, 4)][int(rng.integers(0, 5))] \
+        if kind in (0, 3) else None
     return dict(D=D, fp8=fp8, Hkv=Hkv, G=G, T=T, lens=lens, kind=kind, param=param, tail=tail,
-                num_ctas=num_ctas, out_dtype=out_dtype)
+                cost=cost, num_ctas=num_ctas, out_dtype=out_dtype)
 
 
 @pytest.mark.parametrize("seed", range(24))
 def test_random_configurations_match_oracle(seed):
-    """Seeded random shapes through plan + run (plan kinds, tail shapes, CTA
-    counts, group sizes 1..32, head_dim 64/128, up to 32 query rows per kv
+    """Seeded random shapes through plan + run (plan kinds, tail shapes, cost
+    weights, CTA counts, group sizes 1..32, head_dim 64/128, up to 32 query rows per kv
     head, bf16 or FP8 KV, bf16 or fp32 output) against the oracle."""
     c = _random_case(seed)
     D, Hkv, G, T = c["D"], c["Hkv"], c["G"], c["T"]
@@ -958,7 +991,7 @@ def test_random_configurations_match_oracle(seed):
     g = hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq * T, head_dim=D,
                         pt_stride=batch.pt_stride, workspace=ws, kind=c["kind"],
                         num_ctas=c["num_ctas"], param=c["param"], max_seq_len=maxlen,
-                        tail=c["tail"])
+                        tail=c["tail"], cost=c["cost"])
     out = torch.full(batch.q.shape, float("nan"), dtype=c["out_dtype"], device="cuda")
     kw = {}
     kc, vc = batch.k_cache, batch.v_cache

@@ -56,8 +56,11 @@ def _reference(batch, out_dtype, fp8=None):
     n = _sms()
     ws = torch.empty(hpa.decode_workspace_size(hpa.PLAN_DYNAMIC, B, Hkv, Hq, D, n),
                      dtype=torch.uint8, device=dev)
+    # (an e4m3 cache: the cost weights noalloc's plan uses for it)
     grid = hpa.decode_plan(batch.seq_lens, num_kv_heads=Hkv, num_q_heads=Hq, head_dim=D,
-                           pt_stride=batch.pt_stride, workspace=ws, num_ctas=n)
+                           pt_stride=batch.pt_stride, workspace=ws, num_ctas=n,
+                           cost=None if fp8 is None
+                           else (hpa.COST_UNIT_DEFAULT, hpa.COST_END_DEFAULT_FP8))
     out = torch.empty(B, Hq, D, dtype=out_dtype, device=dev)
     kc, vc, kw = (batch.k_cache, batch.v_cache, {}) if fp8 is None else _fp8_tensors(fp8)
     hpa.decode_run(batch.q, kc, vc, batch.page_table, out, ws, grid, 1.0 / math.sqrt(D), **kw)
@@ -121,9 +124,14 @@ def test_noalloc_both_plan_forms_in_both_orders(L):
 
 
 @pytest.mark.gpu
-def test_noalloc_fp8_cache(L):
+@pytest.mark.parametrize("lens", [
+    [1, 63, 64, 65, 700, 3000],
+    [64] * 100 + [4000] * 20 + [1, 130] * 10,   # the e4m3 cost weights move the cuts
+    [64] * 500 + [3000] * 20,                    # above 512 sequences: the plan kernel
+])
+def test_noalloc_fp8_cache(L, lens):
     shape = W.DecodeShape("na_f8", 64, 8, 128, kv_dtype="fp8_e4m3")
-    batch = W.make_batch(shape, [1, 63, 64, 65, 700, 3000], seed=26)
+    batch = W.make_batch(shape, lens, seed=26)
     fp8 = quantize_fp8(batch)
     ref64 = oracle_decode(batch, fp8=fp8)
     _on_gpu(batch)
