@@ -281,9 +281,11 @@ __global__ void __launch_bounds__(kThreads, CPS)
   uint64_t* dep_full = empty_bar + C::kStages;
   uint64_t* dep_empty = dep_full + kDepBufs;
   uint64_t* q_full = dep_empty + kDepBufs;  // a stage's small copies (q rows, raw rows) landed
-  // StageInfo / DepDesc are read and written as 16-byte vectors
-  StageInfo* info = reinterpret_cast<StageInfo*>(
-      (reinterpret_cast<uintptr_t>(q_full + C::kStages) + 15) & ~uintptr_t(15));
+  // StageInfo / DepDesc are read and written as 16-byte vectors: the first
+  // 16-byte boundary after the barriers (misc is 16-byte aligned; an offset
+  // from it keeps the pointer in the shared space for the compiler)
+  StageInfo* info =
+      reinterpret_cast<StageInfo*>(misc + ((C::kStages * 24 + kDepBufs * 16 + 15) & ~15));
   DepDesc* dep_desc = reinterpret_cast<DepDesc*>(info + C::kStages);
   volatile int* s_flags = reinterpret_cast<volatile int*>(dep_desc + kDepBufs);
   volatile int* s_abort = s_flags;

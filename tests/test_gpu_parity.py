@@ -764,6 +764,9 @@ def test_step_equals_plan_and_run_bitwise(name, lens, Hq, Hkv, D, T, num_ctas):
     [1, 63, 64, 65, 700, 3000],
     # many single-tile sequences: the e4m3 cost weights move the cuts
     [64] * 100 + [4000] * 20 + [1, 130] * 10,
+    # 480 sequences, a sixth of them empty: the scan's non-empty counts cross
+    # all six warps' slices and the cost prefix skips the empty sequences
+    ([64] * 3 + [0, 1, 2000]) * 80,
 ])
 def test_step_fp8_equals_plan_and_run(lens):
     """The e4m3 in-kernel plan weighs segment ends (COST_END_DEFAULT_FP8): it
