@@ -674,7 +674,9 @@ __global__ void __launch_bounds__(kThreads, CPS)
           if (lane == 0) base = atomicAdd(&p.ws.header[kHdrListCount + *s_parity], __popc(split));
           base = __shfl_sync(0xffffffffu, base, 0);
           const int at = base + __popc(split & ((1u << lane) - 1u));
-          if (sd.y > 1 && at >= 0 && at < S) p.ws.mlist[at] = sg;  // (a stale count is flagged by the merge)
+          // (with its descriptor, so that the merge reads one word less in
+          // its chain of dependent loads; a stale count is flagged by the merge)
+          if (sd.y > 1 && at >= 0 && at < S) p.ws.mlist[at] = make_int4(sg, sd.x, sd.y, 0);
         }
       }
       if (blockIdx.x == 0 && lane == 0) {
@@ -1228,8 +1230,10 @@ struct MergeParams {
 };
 
 // LIST: the plan was made inside the decode kernel, which also listed the
-// split segments (Ws::mlist, its count in the header under the step's
-// parity); only those are visited.  Otherwise every segment is.
+// split segments with their descriptors (Ws::mlist, its count in the header
+// under the step's parity); only those are visited.  Otherwise every segment
+// is.  A job's loads form a chain (list count, list entry, partials), so it
+// is kept short: the counts and the parity come in one 16-byte load.
 template <int D, bool OUT_F32, bool LIST>
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergeParams p) {
   constexpr int kVec = D / 32;                 // output elements per lane
@@ -1238,9 +1242,12 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   const int G = p.GT, lane = threadIdx.x & 31;  // rows per segment
   int nseg = p.S;
   if constexpr (LIST) {
-    // the decode kernel before this merge flipped the parity on its way out
-    const int e = (__ldcg(&p.ws.header[kHdrParity]) & 1) ^ 1;
-    nseg = __ldcg(&p.ws.header[kHdrListCount + e]);
+    // header words kHdrListCount (two counts, by parity) and kHdrParity, at a
+    // 16-byte boundary; the decode kernel before this merge flipped the
+    // parity on its way out
+    static_assert(kHdrListCount % 4 == 0 && kHdrParity == kHdrListCount + 2, "header words");
+    const int4 lc = __ldcg(reinterpret_cast<const int4*>(p.ws.header + kHdrListCount));
+    nseg = (lc.z & 1) ? lc.x : lc.y;
     if (nseg < 0 || nseg > p.S) {
       if (threadIdx.x == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
       nseg = 0;
@@ -1250,12 +1257,18 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   for (int job = blockIdx.x * kMergeWarps + (threadIdx.x >> 5); job < jobs;
        job += gridDim.x * kMergeWarps) {
     const int k = job / G, h = job - k * G;
-    const int s = LIST ? __ldcg(&p.ws.mlist[k]) : k;
+    int s = k;
+    int2 sd;
+    if constexpr (LIST) {
+      const int4 ent = __ldcg(&p.ws.mlist[k]);
+      s = ent.x;
+      sd = make_int2(ent.y, ent.z);
+    }
     if (s < 0 || s >= p.S) {
       if (lane == 0) atomicOr(&p.ws.header[kHdrStatus], HPA_DEVICE_BAD_PLAN);
       continue;
     }
-    const int2 sd = __ldcg(&p.ws.seg_desc[s]);
+    if constexpr (!LIST) sd = __ldcg(&p.ws.seg_desc[s]);
     const int ns = sd.y;
     if (ns <= 1) continue;
     const int r0 = sd.x >> 1;

@@ -34,8 +34,9 @@ constexpr int32_t kPlanMagic = 0x31415048;  // "HPA1"
 //   seg_desc    int2[B*Hkv]  per segment: (first partial slot, ranges holding
 //                            its units); a segment held by one range has no
 //                            partials.
-//   mlist       int32[B*Hkv] in-kernel plan: the ids of the split segments (in
-//                            no particular order; their count is in the
+//   mlist       int4[B*Hkv]  in-kernel plan: the split segments, each as (id,
+//                            first partial slot, ranges holding it, 0), in
+//                            no particular order (their count is in the
 //                            header); the merge kernel visits only them.  A
 //                            step appends to the count of its parity; its last
 //                            CTA zeroes the other count (the previous step's,
@@ -110,7 +111,7 @@ inline bool ws_layout(int kind, int B, int Hkv, int Hq, int D, int grid, WsLayou
   L->tile_start = off;  off = align256(off + (size_t(B) + 1) * 4);
   L->cta_desc = off;    off = align256(off + V * 32);
   L->seg_desc = off;    off = align256(off + S * 8);
-  L->mlist = off;       off = align256(off + S * 4);
+  L->mlist = off;       off = align256(off + S * 16);
   L->part_ml = off;     off = align256(off + slots * G * 8);
   L->part_acc = off;    off = align256(off + slots * G * size_t(D) * 4);
   L->trace = off;       off = align256(off + size_t(grid) * 32);
@@ -125,7 +126,7 @@ struct Ws {
   int32_t* tile_start;
   int4* cta_desc;
   int2* seg_desc;
-  int32_t* mlist;
+  int4* mlist;
   float2* part_ml;
   float* part_acc;
   unsigned long long* trace;
@@ -135,7 +136,7 @@ inline Ws ws_view(void* base, const WsLayout& L) {
   char* p = static_cast<char*>(base);
   return Ws{reinterpret_cast<int32_t*>(p + L.header), reinterpret_cast<int32_t*>(p + L.lens),
             reinterpret_cast<int32_t*>(p + L.tile_start), reinterpret_cast<int4*>(p + L.cta_desc),
-            reinterpret_cast<int2*>(p + L.seg_desc), reinterpret_cast<int32_t*>(p + L.mlist),
+            reinterpret_cast<int2*>(p + L.seg_desc), reinterpret_cast<int4*>(p + L.mlist),
             reinterpret_cast<float2*>(p + L.part_ml),
             reinterpret_cast<float*>(p + L.part_acc),
             reinterpret_cast<unsigned long long*>(p + L.trace)};
