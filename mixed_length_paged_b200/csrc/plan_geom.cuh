@@ -95,7 +95,7 @@ struct SeqIdx {
 struct DynGeom {
   long long U, P, Pd, U1, Ut, M, K1;
   int q, e;
-  bool cost;  // e > 0 and U > P: cut by cost
+  bool cost;  // e > 0, U > P and K1 >= (q + e) P: the primary cuts are by cost
   SeqIdx si;
   FloorDiv by_Pd, by_M, by_K1, by_Ut;
   // (called by whole warps, all lanes with the same arguments)
@@ -273,7 +273,8 @@ __device__ __forceinline__ void dyn_range_desc(const DynGeom& dg, const int32_t*
 // The costs it needs are closed forms in (b, g): K(segment start) = Kseq(b)
 // + g (q n + e), each tile q more, the segment's last e more still.  The
 // segment's first piece opens its range iff the unit before the segment lies
-// in an earlier range (every range of the dynamic plan holds a unit).
+// in an earlier range: every primary range and tail chunk holds a unit when
+// U > P, and for U <= P range c is unit c.
 __device__ __forceinline__ int2 dyn_seg_desc(const DynGeom& dg, const int32_t* ts, int Hkv, int s) {
   const int b = s / Hkv, g = s - b * Hkv;
   const long long n = ts[b + 1] - ts[b];
