@@ -680,6 +680,26 @@ def test_cost_weights_do_not_move_cuts_when_all_units_cost_the_same(lens, Hkv, P
     np.testing.assert_array_equal(a["cta"], b["cta"])
 
 
+@pytest.mark.parametrize("lens,Hkv,P,cost", [
+    ([65, 65], 8, 27, (1, 1)),     # 16 two-unit segments of cost 3: 48 / 27 < 2
+    ([65, 65], 8, 27, (2, 4)),
+    ([1] * 5 + [130], 4, 30, (1, 3)),  # cost 104 < 4 x 30, 32 units
+])
+def test_cost_weights_fall_back_to_the_even_split_when_a_range_could_be_empty(lens, Hkv, P, cost):
+    """When a range's share of the cost, K(U1) / P, is below the largest unit
+    cost q + e, a cut could leave a range empty inside a split segment (and
+    break the consecutive holders the partial slots need): the plan then
+    splits the units evenly.  The first case is the one a random search
+    found before the rule existed."""
+    p = oracle.plan(np.array(lens, dtype=np.int32), Hkv, kind=0, num_ctas=P,
+                    capacity_tokens=max(64, max(lens)), tail=(0, 1, 0), cost=cost)
+    U = p["n_units"]
+    costs = _unit_costs(_units(lens, Hkv), cost)
+    assert sum(costs) < (cost[0] + cost[1]) * P < (cost[0] + cost[1]) * U
+    assert [(int(a), int(e)) for a, e in p["cta"]] == _even_ranges(U, P)
+    _check_plan_invariants(p, lens, Hkv, 0, (0, 1, 0), cost)
+
+
 @pytest.mark.parametrize("q", [1, 2, 3, 4])
 def test_end_cost_zero_is_the_even_split_for_any_unit_cost(q):
     lens = [1, 63, 64, 65, 300, 5000, 129, 4096, 0, 7]
