@@ -71,6 +71,9 @@ LIB_COST = (hpa.COST_UNIT_DEFAULT, hpa.COST_END_DEFAULT)
     ([131072] + [4096] * 31, 8, 148), ([512] * 64, 8, 148), ([37, 200], 2, 148),
     ([37, 200], 2, 3), ([0, 5, 0, 64, 65, 3000, 1], 4, 7), ([1], 1, 148), ([0, 0], 2, 5),
     (list(range(1, 3000, 7)), 2, 148),
+    # cost weights on: a range's share below a segment end's cost, so the
+    # plan falls back to the even split of the units
+    ([65, 65], 8, 27),
     # beyond 12K sequences the tile offsets need more than 48 KiB of shared memory
     ([int(x) for x in np.random.default_rng(3).integers(0, 300, 20000)], 2, 148),
     ([int(x) for x in np.random.default_rng(4).integers(1, 100, 32768)], 1, 148),  # the maximum
@@ -767,6 +770,9 @@ def test_step_equals_plan_and_run_bitwise(name, lens, Hq, Hkv, D, T, num_ctas):
     # 480 sequences, a sixth of them empty: the scan's non-empty counts cross
     # all six warps' slices and the cost prefix skips the empty sequences
     ([64] * 3 + [0, 1, 2000]) * 80,
+    # 320 units over 296 CTAs at cost 640 < 3 x 296: the fallback to the
+    # even split of the units
+    [65] * 20,
 ])
 def test_step_fp8_equals_plan_and_run(lens):
     """The e4m3 in-kernel plan weighs segment ends (COST_END_DEFAULT_FP8): it
