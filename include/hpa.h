@@ -164,10 +164,9 @@ HPA_API int hpa_default_num_ctas(int device);
 /* Persistent CTA count (num_ctas of hpa_decode_plan) that matches how many
  * run-kernel CTAs fit at once for this head geometry; a dynamic plan for more
  * CTAs than fit would leave part of its primary ranges to a second wave.
- * Up to 16 query rows per kv head (G * q_tokens) two fit per SM, and this is
- * hpa_default_num_ctas; 17 .. 32 rows run one CTA per SM (the SM count).
- * Returns -1 on invalid arguments (more than 32 rows) or if the device cannot
- * be queried. */
+ * Up to 32 query rows per kv head (G * q_tokens) two fit per SM, and this is
+ * hpa_default_num_ctas.  Returns -1 on invalid arguments (more than 32 rows)
+ * or if the device cannot be queried. */
 HPA_API int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads, int q_tokens);
 
 /* Grid (CTA count) of the run kernel under a plan: num_ctas for DYNAMIC and
@@ -334,7 +333,8 @@ HPA_API hpa_status hpa_decode_run(const void* q, const void* k_cache, const void
  *   q_tokens     1 .. 16 with (num_q_heads / num_kv_heads) * q_tokens <= 32:
  *                the G * T query rows of a kv head share one pass over its
  *                tiles (HPA_ERR_UNSUPPORTED otherwise).  Above 16 rows the
- *                kernel runs one CTA per SM (hpa_decode_num_ctas).
+ *                kernel keeps one deposit buffer and two stages per CTA so
+ *                that two CTAs still fit an SM (hpa_decode_num_ctas).
  *   kind, grid, workspace  from hpa_decode_plan called with num_q_heads *
  *                q_tokens in place of num_q_heads (the plan and the workspace
  *                count G * T rows per kv head); size the workspace the same way.

@@ -60,18 +60,9 @@ extern "C" int hpa_decode_num_ctas(int device, int num_q_heads, int num_kv_heads
     return -1;
   const long long rows = (long long)(num_q_heads / num_kv_heads) * q_tokens;
   if (rows > 32) return -1;
-  // up to 16 query rows per kv head the run kernel runs two CTAs per SM (the
-  // two-n-tile kernel splits its warps by n-tile); 17..32 rows take one CTA
-  // per SM (the four-n-tile kernel's query rows need the shared memory)
-  if (rows > 16) {
-    int n = 0;
-    const cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
-    if (e != cudaSuccess) {
-      set_cuda_error(e, "hpa_decode_num_ctas");
-      return -1;
-    }
-    return n;
-  }
+  // up to 32 query rows per kv head the run kernel runs two CTAs per SM (the
+  // two-n-tile kernel splits its warps by n-tile; the four-n-tile kernel
+  // then keeps one deposit buffer and two stages)
   return hpa_default_num_ctas(device);
 }
 

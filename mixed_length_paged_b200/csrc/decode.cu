@@ -76,7 +76,7 @@ constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kSmemLimit = 227 * 1024;   // per CTA
 constexpr int kSmemPerSm = 228 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any barrier wait
-constexpr int kDepBufs = 2;              // deposit slots between consumers and epilogue
+constexpr int kDepBufsDefault = 2;              // deposit slots between consumers and epilogue
 constexpr int kMaxQTokens = 16;          // query tokens per sequence (multi-token decode)
 
 template <int D, int NT, bool FP8, int CPS, bool PRO, bool FP>
@@ -98,7 +98,8 @@ struct Cfg {
   // w / 2 and tokens [32 (w % 2), + 32), as two 16-token blocks -- the same
   // MMA work with the registers of the one-n-tile kernel, so two CTAs still
   // fit an SM.  Four n-tiles (17..32 rows): warp w owns n-tile w and all 64
-  // tokens, as four 16-token blocks (one CTA per SM: the 32 query rows of a
+  // tokens, as four 16-token blocks (two CTAs per SM with one deposit buffer
+  // and two stages each, else one CTA per SM: the 32 query rows of a
   // stage take 8 KiB more shared memory).
   static constexpr bool kSplit = NT >= 2;
   static constexpr int kWarpsPerTile = kSplit ? kConsumerWarps / NT : kConsumerWarps;
@@ -110,6 +111,10 @@ struct Cfg {
   // one deposit: acc[warp][row of the warp][D + 4] floats, then (m, l)[warp][row]
   static constexpr int kDepAccFloats = kConsumerWarps * kWarpRows * kAccStride;
   static constexpr int kDepBytes = kDepAccFloats * 4 + kConsumerWarps * kWarpRows * 8;
+  // deposit slots between consumers and epilogue: one for the four-n-tile
+  // kernel at two CTAs per SM (its 8 KiB of query rows per stage leave room
+  // for two stages only then), else two
+  static constexpr int kDepBufs = (NT == 4 && CPS == 2) ? 1 : kDepBufsDefault;
   static constexpr int kMisc = 2048;                   // barriers, stage info, flags
   // in-kernel plan: tile offsets of all sequences, the non-empty mask and
   // its prefix (SeqIdx), and the scan's per-warp non-empty counts
@@ -274,20 +279,20 @@ __global__ void __launch_bounds__(kThreads, CPS)
   uint8_t* smem = smem_raw + (((smem_raw_s + 1023u) & ~1023u) - smem_raw_s);
   uint8_t* stages = smem;
   uint8_t* qslots = smem + C::kStages * C::kStageBytes;
-  uint8_t* deps = qslots + C::kStages * C::kSlotBytes;  // kDepBufs deposit slots
-  uint8_t* misc = deps + kDepBufs * C::kDepBytes;
+  uint8_t* deps = qslots + C::kStages * C::kSlotBytes;  // C::kDepBufs deposit slots
+  uint8_t* misc = deps + C::kDepBufs * C::kDepBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(misc);
   uint64_t* empty_bar = full_bar + C::kStages;
   uint64_t* dep_full = empty_bar + C::kStages;
-  uint64_t* dep_empty = dep_full + kDepBufs;
-  uint64_t* q_full = dep_empty + kDepBufs;  // a stage's small copies (q rows, raw rows) landed
+  uint64_t* dep_empty = dep_full + C::kDepBufs;
+  uint64_t* q_full = dep_empty + C::kDepBufs;  // a stage's small copies (q rows, raw rows) landed
   // StageInfo / DepDesc are read and written as 16-byte vectors: the first
   // 16-byte boundary after the barriers (misc is 16-byte aligned; an offset
   // from it keeps the pointer in the shared space for the compiler)
   StageInfo* info =
-      reinterpret_cast<StageInfo*>(misc + ((C::kStages * 24 + kDepBufs * 16 + 15) & ~15));
+      reinterpret_cast<StageInfo*>(misc + ((C::kStages * 24 + C::kDepBufs * 16 + 15) & ~15));
   DepDesc* dep_desc = reinterpret_cast<DepDesc*>(info + C::kStages);
-  volatile int* s_flags = reinterpret_cast<volatile int*>(dep_desc + kDepBufs);
+  volatile int* s_flags = reinterpret_cast<volatile int*>(dep_desc + C::kDepBufs);
   volatile int* s_abort = s_flags;
   volatile int* s_plan_ok = s_flags + 1;
   uint64_t* q_ready = reinterpret_cast<uint64_t*>(const_cast<int*>(s_flags) + 2);  // fused prologue: q rows done
@@ -295,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
   float* s_qgamma = reinterpret_cast<float*>(misc + C::kMisc / 2);
   float* s_kgamma = s_qgamma + D;
   static_assert(C::kMisc / 2 >= 2 * D * 4, "misc area too small for the weights");
-  static_assert(C::kStages * 24 + kDepBufs * 16 + 8 + C::kStages * sizeof(StageInfo) +
-                        kDepBufs * sizeof(DepDesc) + 16 + 32 <= C::kMisc / 2,
+  static_assert(C::kStages * 24 + C::kDepBufs * 16 + 8 + C::kStages * sizeof(StageInfo) +
+                        C::kDepBufs * sizeof(DepDesc) + 16 + 32 <= C::kMisc / 2,
                 "misc area too small");
   // in-kernel plan: tile offsets, non-empty mask and prefix, per-warp
   // non-empty counts (after the misc area), and per-warp tile sums of the
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, CPS)
       mbar_init(smem_u32(&q_full[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), kConsumerWarps);
     }
-    for (int d = 0; d < kDepBufs; ++d) {
+    for (int d = 0; d < C::kDepBufs; ++d) {
       mbar_init(smem_u32(&dep_full[d]), kConsumerWarps);
       mbar_init(smem_u32(&dep_empty[d]), 1);
     }
@@ -699,8 +704,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
       }
     }
     for (int k = 0;; ++k) {
-      const int db = k % kDepBufs;
-      if (!wait_bar(smem_u32(&dep_full[db]), (k / kDepBufs) & 1, s_abort, status)) break;
+      const int db = k % C::kDepBufs;
+      if (!wait_bar(smem_u32(&dep_full[db]), (k / C::kDepBufs) & 1, s_abort, status)) break;
       DepDesc dd = dep_desc[db];
       if (dd.stop) break;
       // Never trust a deposit as an index without checking it.
@@ -828,8 +833,8 @@ __global__ void __launch_bounds__(kThreads, CPS)
 
   // Hand this warp's state of a finished segment to the epilogue warp.
   auto deposit = [&](const StageInfo* inf) {
-    const int db = nseg % kDepBufs;
-    wait_bar(smem_u32(&dep_empty[db]), ((nseg / kDepBufs) & 1) ^ 1, s_abort, status);
+    const int db = nseg % C::kDepBufs;
+    wait_bar(smem_u32(&dep_empty[db]), ((nseg / C::kDepBufs) & 1) ^ 1, s_abort, status);
     if (inf) {
 #pragma unroll
       for (int nt = 0; nt < W; ++nt)
@@ -1440,8 +1445,10 @@ template <int D, bool FP8, bool OUT_F32, bool PRO, bool FP>
 hpa_status launch_nt(int nt, int cps, const CUtensorMap& tk, const CUtensorMap& tv,
                      const RunParams& p, int grid, cudaStream_t s) {
   if constexpr (!PRO) {
-    // 17..32 rows (multi-token only): one CTA per SM whatever the grid
-    if (nt == 4) return launch<D, 4, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s);
+    // 17..32 rows (multi-token only)
+    if (nt == 4)
+      return cps == 2 ? launch<D, 4, FP8, OUT_F32, 2, PRO, FP>(tk, tv, p, grid, s)
+                      : launch<D, 4, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s);
   }
   if (cps == 1)
     return nt == 1 ? launch<D, 1, FP8, OUT_F32, 1, PRO, FP>(tk, tv, p, grid, s)
