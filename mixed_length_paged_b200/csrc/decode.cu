@@ -98,9 +98,9 @@ struct Cfg {
   // w / 2 and tokens [32 (w % 2), + 32), as two 16-token blocks -- the same
   // MMA work with the registers of the one-n-tile kernel, so two CTAs still
   // fit an SM.  Four n-tiles (17..32 rows): warp w owns n-tile w and all 64
-  // tokens, as four 16-token blocks (two CTAs per SM with one deposit buffer
-  // and two stages each, else one CTA per SM: the 32 query rows of a
-  // stage take 8 KiB more shared memory).
+  // tokens, as four 16-token blocks.  The 32 query rows of a stage take 8 KiB
+  // more shared memory, so at two CTAs per SM this kernel keeps one deposit
+  // buffer (two stages fit then); at one CTA per SM it keeps two.
   static constexpr bool kSplit = NT >= 2;
   static constexpr int kWarpsPerTile = kSplit ? kConsumerWarps / NT : kConsumerWarps;
   static constexpr int kWarpTiles = kSplit ? 1 : NT;   // n-tiles per warp
