@@ -16,12 +16,18 @@ lens_st = st.lists(st.integers(min_value=0, max_value=3000), min_size=1, max_siz
 
 @settings(max_examples=60, deadline=None)
 @given(lens=lens_st, Hkv=st.sampled_from([1, 2, 4, 8]), P=st.integers(1, 300),
-       m=st.integers(1, 12))
-def test_length_aware_plan_properties(lens, Hkv, P, m):
+       m=st.integers(1, 12), q=st.integers(1, 4), e=st.integers(0, 4))
+def test_length_aware_plan_properties(lens, Hkv, P, m, q, e):
+    """The length-aware plan moves each cut of the dynamic plan of the same
+    shape (tail and cost weights) by less than m units, keeps segments of
+    fewer than 2m tiles whole, and leaves the end pieces of a cut segment at
+    least m tiles long."""
     sl = np.array(lens, dtype=np.int32)
     cap = max(64, max(lens))
-    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4, 0))
-    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4, 0))
+    la = oracle.plan(sl, Hkv, kind=3, num_ctas=P, param=m, capacity_tokens=cap, tail=(8, 4, 0),
+                     cost=(q, e))
+    dyn = oracle.plan(sl, Hkv, kind=0, num_ctas=P, capacity_tokens=cap, tail=(8, 4, 0),
+                      cost=(q, e))
     # coverage, contiguity, consecutive holders and partial slots
     _check_plan_invariants(la, lens, Hkv, 3)
     assert la["ranges"] == dyn["ranges"]
